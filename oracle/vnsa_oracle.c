@@ -1,0 +1,396 @@
+/*
+ * vnsa_oracle.c -- plain fp64 CPU oracle of the VideoNSA hybrid sparse-attention
+ * layer prefill.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load
+ * this file: it exists so that the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark have an independent, obviously correct answer to compare with.
+ * It shares no code, header, table or constant with the CUDA library.
+ *
+ * Sources (page title, then the section it falls in):
+ *   [M]  "VideoNSA: Native Sparse Attention Scales Video Understanding" (paper
+ *        notes), section "Method": 28 query heads / 4 KV heads (GQA); tokens split
+ *        into vision and text sets by position IDs; vision tokens go through
+ *        compression (blocks of 64 averaged into block keys/values, then a
+ *        learnable projection), selection (top-k blocks by importance) and a
+ *        sliding window; a per-head sigmoid gate combines the three branch
+ *        outputs; text tokens use standard GQA; outputs are written back at the
+ *        original positions.
+ *   [A]  "VideoNSA: Native Sparse Attention for Video Understanding" (model card),
+ *        section "Model Architecture": three branches (mean of each frame's
+ *        key/value block; a subset of blocks ranked as most useful; a local
+ *        window), mixed with weights that are learned separately per head.
+ *   [K]  same paper notes, section "Key claims": the vision/text split by
+ *        position ID is taken at every layer; dense attention is kept for text.
+ *
+ * Readings of points the pages leave open (each is repeated in the design notes):
+ *   R1  Vision queries see only the vision subsequence; blocks are formed over
+ *       vision order (index i = rank of the token among vision tokens).
+ *   R2  A compressed block j is visible to vision query i iff its last token is
+ *       at or before i, i.e. j < floor((i+1)/B).  No visible block -> the branch
+ *       output is 0 and the block importances are 0.
+ *   R3  The projection is a d x d linear map per tensor (W_K, W_V), applied to
+ *       the block mean as a row vector: K_cmp = mean(K_block) . W_K.  In bf16
+ *       runs K_cmp / V_cmp are rounded to bf16 (round-to-nearest-even) after the
+ *       exact computation, because the kernel stores them in bf16.
+ *   R4  Block importance = the normalised compression softmax probability,
+ *       summed over the query heads of one GQA group.
+ *   R5  Block 0 and the query's own block floor(i/B) are always selected and
+ *       count within top_k; the other top_k - #forced blocks are the best by
+ *       importance among visible, non-forced blocks, ties going to the lower
+ *       block index.  Fewer candidates than slots -> all are taken, the rest
+ *       of the index row is -1.  Indices are stored ascending.
+ *   R6  Selection attends to every token of the selected blocks that is at or
+ *       before the query (causal mask inside the query's own block).
+ *   R7  The window holds the w most recent vision tokens including the query:
+ *       [i-w+1, i].
+ *   R8  out = sig(g_cmp) o_cmp + sig(g_slc) o_slc + sig(g_swa) o_swa with the
+ *       logistic sigmoid and no normalisation; text rows ignore gate logits.
+ *   R9  Every branch uses the same softmax scale (default 1/sqrt(d)).
+ *   R10 A text token at global position t attends to every token u <= t,
+ *       vision or text, with KV head floor(h / (H_q/H_kv)).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+typedef struct {
+    int n;              /* tokens in the sequence                        */
+    int h_q, h_kv, d;   /* query heads, KV heads (= groups), head dim     */
+    int block;          /* compression block = stride = selection block  */
+    int top_k;          /* selected blocks per (group, query)            */
+    int window;         /* sliding-window length in vision tokens        */
+    int force_first;    /* always keep block 0                           */
+    int force_local;    /* always keep the query's own block             */
+    double scale;       /* softmax scale                                 */
+    int round_cmp_bf16; /* round K_cmp / V_cmp to bf16 (R3)              */
+} vnsa_oracle_cfg;
+
+enum { ORACLE_OK = 0, ORACLE_EINVAL = 1, ORACLE_ENOMEM = 2 };
+
+/* Round to the nearest bfloat16 value (8 significant bits), ties to even.  */
+double vnsa_oracle_round_bf16(double x)
+{
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e = ilogb(x);                 /* x = m * 2^e, 1 <= |m| < 2 */
+    if (e < -126) e = -126;           /* bf16 subnormal spacing 2^-133 */
+    double quantum = ldexp(1.0, e - 7);
+    return rint(x / quantum) * quantum; /* rint: round half to even */
+}
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/*
+ * One softmax attention of query q (d values, already fp64) over a key list.
+ * Key u of the list has its key at kb + keys[u]*stride and its value at
+ * vb + keys[u]*stride.  Computes s_u = scale * q.k_u, p = softmax(s),
+ * o = sum_u p_u v_u; returns log(sum exp(s)) (or -inf for an empty list, with
+ * o = 0).  If p_out is given, p_u is written there in list order.
+ */
+static double attend(const double *q, const double *kb, const double *vb,
+                     size_t stride, const int *keys, int nk, int d, double scale,
+                     double *o, double *p_out, double *s)
+{
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    if (nk == 0) return -INFINITY;
+    double m = -INFINITY;
+    for (int u = 0; u < nk; ++u) {
+        const double *k = kb + (size_t)keys[u] * stride;
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += q[e] * k[e];
+        s[u] = scale * acc;
+        if (s[u] > m) m = s[u];
+    }
+    double z = 0.0;
+    for (int u = 0; u < nk; ++u) z += exp(s[u] - m);
+    for (int u = 0; u < nk; ++u) {
+        double p = exp(s[u] - m) / z;
+        if (p_out) p_out[u] = p;
+        const double *v = vb + (size_t)keys[u] * stride;
+        for (int e = 0; e < d; ++e) o[e] += p * v[e];
+    }
+    return m + log(z);
+}
+
+/* Vision / text partition [M], [K]: vis[i] = global position of the i-th
+ * vision token; returns the vision count. */
+static int partition(const uint8_t *is_vision, int n, int *vis)
+{
+    int nv = 0;
+    for (int t = 0; t < n; ++t)
+        if (is_vision[t]) vis[nv++] = t;
+    return nv;
+}
+
+static int check_cfg(const vnsa_oracle_cfg *c)
+{
+    if (!c || c->n < 0 || c->h_q <= 0 || c->h_kv <= 0 || c->d <= 0) return 0;
+    if (c->h_q % c->h_kv != 0) return 0;
+    if (c->block <= 0 || c->window <= 0 || c->top_k <= 0) return 0;
+    int forced = (c->force_first ? 1 : 0) + (c->force_local ? 1 : 0);
+    if (c->top_k < forced) return 0;
+    return 1;
+}
+
+/*
+ * Compression keys/values [M], [A]: each block of B consecutive vision tokens
+ * is averaged, and the mean is mapped to one block key / block value:
+ *   Kbar_j = (1/B) sum_{u<B} K[vis[jB+u]],   K_cmp_j = Kbar_j . W_K   (R3),
+ * per KV head, for the nb = floor(N_v/B) complete blocks.  Same for V.
+ * k_cmp, v_cmp: [nb][h_kv][d].  Kd, Vd: fp64 copies of K, V [n][h_kv][d].
+ */
+static void pool_proj(const vnsa_oracle_cfg *c, const double *Kd, const double *Vd,
+                      const int *vis, int nb, const double *wk, const double *wv,
+                      double *k_cmp, double *v_cmp)
+{
+    const int d = c->d, hk = c->h_kv, B = c->block;
+    #pragma omp parallel for schedule(static)
+    for (int j = 0; j < nb; ++j) {
+        double *kbar = malloc(sizeof(double) * 2 * d);
+        double *vbar = kbar + d;
+        for (int g = 0; g < hk; ++g) {
+            for (int e = 0; e < d; ++e) { kbar[e] = 0.0; vbar[e] = 0.0; }
+            for (int u = 0; u < B; ++u) {
+                size_t row = ((size_t)vis[j * B + u] * hk + g) * d;
+                for (int e = 0; e < d; ++e) { kbar[e] += Kd[row + e]; vbar[e] += Vd[row + e]; }
+            }
+            for (int e = 0; e < d; ++e) { kbar[e] /= B; vbar[e] /= B; }
+            double *ko = k_cmp + ((size_t)j * hk + g) * d;
+            double *vo = v_cmp + ((size_t)j * hk + g) * d;
+            for (int col = 0; col < d; ++col) {
+                double ak = 0.0, av = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    ak += kbar[e] * wk[(size_t)e * d + col];
+                    av += vbar[e] * wv[(size_t)e * d + col];
+                }
+                if (c->round_cmp_bf16) { ak = vnsa_oracle_round_bf16(ak); av = vnsa_oracle_round_bf16(av); }
+                ko[col] = ak;
+                vo[col] = av;
+            }
+        }
+        free(kbar);
+    }
+}
+
+/*
+ * Top-k block selection [M]: the blocks with the highest importance are kept
+ * (32 in the paper's setting), with the forced blocks and tie rule of R5.
+ * imp: importance of the nvis visible blocks 0..nvis-1 of query i.
+ * Writes k entries to out (ascending, -1 padded); returns the count selected.
+ */
+static int select_blocks(const double *imp, int nvis, int i, int B, int k,
+                         int force_first, int force_local, int *out, char *taken)
+{
+    int cnt = 0;
+    int own = i / B;
+    if (force_first) out[cnt++] = 0;
+    if (force_local && !(force_first && own == 0)) out[cnt++] = own;
+    for (int j = 0; j < nvis; ++j) taken[j] = 0;
+    for (int f = 0; f < cnt; ++f)
+        if (out[f] < nvis) taken[out[f]] = 1;
+    while (cnt < k) {
+        int best = -1;
+        for (int j = 0; j < nvis; ++j) {
+            if (taken[j]) continue;
+            /* strict total order: larger importance first, lower j on ties */
+            if (best < 0 || imp[j] > imp[best]) best = j;
+        }
+        if (best < 0) break;
+        taken[best] = 1;
+        out[cnt++] = best;
+    }
+    int nsel = cnt;
+    /* ascending order (insertion sort), then -1 padding */
+    for (int a = 1; a < nsel; ++a) {
+        int x = out[a], b = a - 1;
+        while (b >= 0 && out[b] > x) { out[b + 1] = out[b]; --b; }
+        out[b + 1] = x;
+    }
+    for (int a = nsel; a < k; ++a) out[a] = -1;
+    return nsel;
+}
+
+/* K_cmp / V_cmp only (for the pooling parity checks). Outputs [nb][h_kv][d]. */
+int vnsa_oracle_pool_proj(const vnsa_oracle_cfg *c, const float *k, const float *v,
+                          const uint8_t *is_vision, const float *w_k, const float *w_v,
+                          double *k_cmp, double *v_cmp)
+{
+    if (!check_cfg(c)) return ORACLE_EINVAL;
+    const int n = c->n, d = c->d, hk = c->h_kv;
+    int *vis = malloc(sizeof(int) * (n > 0 ? n : 1));
+    double *Kd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
+    double *Vd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
+    double *wk = malloc(sizeof(double) * (size_t)d * d);
+    double *wv = malloc(sizeof(double) * (size_t)d * d);
+    if (!vis || !Kd || !Vd || !wk || !wv) { free(vis); free(Kd); free(Vd); free(wk); free(wv); return ORACLE_ENOMEM; }
+    for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
+    for (size_t x = 0; x < (size_t)d * d; ++x) { wk[x] = w_k[x]; wv[x] = w_v[x]; }
+    int nv = partition(is_vision, n, vis);
+    pool_proj(c, Kd, Vd, vis, nv / c->block, wk, wv, k_cmp, v_cmp);
+    free(vis); free(Kd); free(Vd); free(wk); free(wv);
+    return ORACLE_OK;
+}
+
+/*
+ * Full layer prefill for a list of query rows (global positions).
+ *
+ * Inputs (row-major, values already exact in fp32: bf16 inputs are widened):
+ *   q [n][h_q][d], k, v [n][h_kv][d], is_vision [n], gate [n][h_q][3]
+ *   (cmp, slc, swa), w_k, w_v [d][d].
+ *   rows[n_rows]: global positions to compute (NULL with n_rows = n: all).
+ *   forced_idx: optional [n_rows][h_kv][top_k]; when given, vision rows use these
+ *   selected blocks instead of computing the top-k (used to compare a branch
+ *   when the kernel legitimately swapped near-tied blocks).
+ * Outputs (each optional except out), row r of the list:
+ *   out [n_rows][h_q][d]                gated vision output / dense text output
+ *   o_cmp, o_slc, o_swa [n_rows][h_q][d] ungated branch outputs (vision rows)
+ *   lse_cmp [n_rows][h_q]               compression log-sum-exp (-inf if empty)
+ *   idx [n_rows][h_kv][top_k]           selected blocks (-1 for text rows)
+ *   imp [n_rows][h_kv][nb]              block importance (0 beyond visibility)
+ *   nb_out                              number of complete blocks
+ */
+int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k,
+                        const float *v, const uint8_t *is_vision, const float *gate,
+                        const float *w_k, const float *w_v, int n_rows, const int *rows,
+                        const int *forced_idx, double *out, double *o_cmp, double *o_slc,
+                        double *o_swa, double *lse_cmp, int *idx, double *imp, int *nb_out)
+{
+    if (!check_cfg(c) || !q || !k || !v || !is_vision || !gate || !w_k || !w_v || !out) return ORACLE_EINVAL;
+    if (n_rows < 0 || (!rows && n_rows != c->n)) return ORACLE_EINVAL;
+    const int n = c->n, d = c->d, hq = c->h_q, hk = c->h_kv, B = c->block, K = c->top_k;
+    const int r = hq / hk;
+    const size_t nn = (size_t)(n > 0 ? n : 1);
+
+    int *vis = malloc(sizeof(int) * nn);
+    int *vpos = malloc(sizeof(int) * nn);
+    double *Kd = malloc(sizeof(double) * nn * hk * d);
+    double *Vd = malloc(sizeof(double) * nn * hk * d);
+    double *wk = malloc(sizeof(double) * (size_t)d * d);
+    double *wv = malloc(sizeof(double) * (size_t)d * d);
+    if (!vis || !vpos || !Kd || !Vd || !wk || !wv) {
+        free(vis); free(vpos); free(Kd); free(Vd); free(wk); free(wv);
+        return ORACLE_ENOMEM;
+    }
+    for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
+    for (size_t x = 0; x < (size_t)d * d; ++x) { wk[x] = w_k[x]; wv[x] = w_v[x]; }
+    const int nv = partition(is_vision, n, vis);
+    for (int t = 0; t < n; ++t) vpos[t] = -1;
+    for (int i = 0; i < nv; ++i) vpos[vis[i]] = i;
+    const int nb = nv / B;
+    if (nb_out) *nb_out = nb;
+    double *k_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
+    double *v_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
+    pool_proj(c, Kd, Vd, vis, nb, wk, wv, k_cmp, v_cmp);
+
+    #pragma omp parallel
+    {
+        /* per-thread scratch: key lists, scores, probabilities, row buffers */
+        int *keys = malloc(sizeof(int) * 2 * nn); /* selection list + window list */
+        double *s = malloc(sizeof(double) * nn);
+        double *p = malloc(sizeof(double) * nn);
+        double *impg = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
+        char *taken = malloc((size_t)(nb > 0 ? nb : 1));
+        int *sel = malloc(sizeof(int) * (size_t)K);
+        double *qd = malloc(sizeof(double) * d);
+        double *oc = malloc(sizeof(double) * d);
+        double *os = malloc(sizeof(double) * d);
+        double *ow = malloc(sizeof(double) * d);
+
+        #pragma omp for schedule(dynamic, 1)
+        for (int rr = 0; rr < n_rows; ++rr) {
+            const int t = rows ? rows[rr] : rr;
+            const int i = vpos[t];
+            double *orow = out + (size_t)rr * hq * d;
+            if (i < 0) {
+                /* R10: dense causal GQA over every token u <= t [M], [K]. */
+                for (int u = 0; u <= t; ++u) keys[u] = u;
+                for (int h = 0; h < hq; ++h) {
+                    const int g = h / r;
+                    for (int e = 0; e < d; ++e) qd[e] = q[((size_t)t * hq + h) * d + e];
+                    attend(qd, Kd + (size_t)g * d, Vd + (size_t)g * d, (size_t)hk * d,
+                           keys, t + 1, d, c->scale, orow + (size_t)h * d, NULL, s);
+                    if (o_cmp) memset(o_cmp + ((size_t)rr * hq + h) * d, 0, sizeof(double) * d);
+                    if (o_slc) memset(o_slc + ((size_t)rr * hq + h) * d, 0, sizeof(double) * d);
+                    if (o_swa) memset(o_swa + ((size_t)rr * hq + h) * d, 0, sizeof(double) * d);
+                    if (lse_cmp) lse_cmp[(size_t)rr * hq + h] = -INFINITY;
+                }
+                if (idx) for (int x = 0; x < hk * K; ++x) idx[(size_t)rr * hk * K + x] = -1;
+                if (imp) for (int x = 0; x < hk * nb; ++x) imp[(size_t)rr * hk * nb + x] = 0.0;
+                continue;
+            }
+            /* R2: visible compressed blocks of vision query i. */
+            int nvis = (i + 1) / B;
+            if (nvis > nb) nvis = nb;
+            for (int g = 0; g < hk; ++g) {
+                /* Compression branch and importance (R4). */
+                for (int j = 0; j < nb; ++j) impg[j] = 0.0;
+                for (int j = 0; j < nvis; ++j) keys[j] = j;
+                for (int hl = 0; hl < r; ++hl) {
+                    const int h = g * r + hl;
+                    for (int e = 0; e < d; ++e) qd[e] = q[((size_t)t * hq + h) * d + e];
+                    double lse = attend(qd, k_cmp + (size_t)g * d, v_cmp + (size_t)g * d,
+                                        (size_t)hk * d, keys, nvis, d, c->scale, oc, p, s);
+                    for (int j = 0; j < nvis; ++j) impg[j] += p[j];
+                    if (lse_cmp) lse_cmp[(size_t)rr * hq + h] = lse;
+                    memcpy(orow + (size_t)h * d, oc, sizeof(double) * d); /* park o_cmp */
+                    if (o_cmp) memcpy(o_cmp + ((size_t)rr * hq + h) * d, oc, sizeof(double) * d);
+                }
+                if (imp) memcpy(imp + ((size_t)rr * hk + g) * nb, impg, sizeof(double) * nb);
+                /* Selection of blocks (R5), or the caller's forced indices. */
+                if (forced_idx) {
+                    for (int x = 0; x < K; ++x) sel[x] = forced_idx[((size_t)rr * hk + g) * K + x];
+                } else {
+                    select_blocks(impg, nvis, i, B, K, c->force_first, c->force_local, sel, taken);
+                }
+                if (idx) memcpy(idx + ((size_t)rr * hk + g) * K, sel, sizeof(int) * K);
+                /* Selection key list (R6): tokens of the chosen blocks, u <= i. */
+                int nk = 0;
+                for (int x = 0; x < K; ++x) {
+                    const int j = sel[x];
+                    if (j < 0) continue;
+                    for (int u = j * B; u < (j + 1) * B && u < nv && u <= i; ++u) keys[nk++] = vis[u];
+                }
+                /* Sliding-window key list (R7): vision tokens [i-w+1, i]. */
+                int *wkeys = keys + nk;
+                int nkw = 0;
+                int lo = i - c->window + 1;
+                if (lo < 0) lo = 0;
+                for (int u = lo; u <= i; ++u) wkeys[nkw++] = vis[u];
+                for (int hl = 0; hl < r; ++hl) {
+                    const int h = g * r + hl;
+                    for (int e = 0; e < d; ++e) qd[e] = q[((size_t)t * hq + h) * d + e];
+                    attend(qd, Kd + (size_t)g * d, Vd + (size_t)g * d, (size_t)hk * d,
+                           keys, nk, d, c->scale, os, NULL, s);
+                    attend(qd, Kd + (size_t)g * d, Vd + (size_t)g * d, (size_t)hk * d,
+                           wkeys, nkw, d, c->scale, ow, NULL, s);
+                    /* Gate (R8) [M], [A]: per-head sigmoid weights of the branches. */
+                    const float *gl = gate + ((size_t)t * hq + h) * 3;
+                    const double gc = sigmoid(gl[0]), gs = sigmoid(gl[1]), gw = sigmoid(gl[2]);
+                    double *o = orow + (size_t)h * d;
+                    for (int e = 0; e < d; ++e) o[e] = gc * o[e] + gs * os[e] + gw * ow[e];
+                    if (o_slc) memcpy(o_slc + ((size_t)rr * hq + h) * d, os, sizeof(double) * d);
+                    if (o_swa) memcpy(o_swa + ((size_t)rr * hq + h) * d, ow, sizeof(double) * d);
+                }
+            }
+        }
+        free(keys); free(s); free(p); free(impg); free(taken); free(sel);
+        free(qd); free(oc); free(os); free(ow);
+    }
+    free(vis); free(vpos); free(Kd); free(Vd); free(wk); free(wv); free(k_cmp); free(v_cmp);
+    return ORACLE_OK;
+}
+
+/* Threads the OpenMP runtime will use (for the CPU-baseline report). */
+int vnsa_oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
