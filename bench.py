@@ -1,0 +1,411 @@
+"""Benchmark of the hybrid sparse-attention layer prefill (one decoder layer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long_128k]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, bounded sample
+
+One step = one vnsa_forward over the whole layer (partition, pooling +
+projection, compression attention + importance, top-k, selection, window + gate,
+text GQA) on inputs already resident in HBM.  The inputs are larger than L2
+(Q 0.94 GB, K and V 0.13 GB each at 128K), so no flush is needed between steps.
+With N > 1 (torchrun) every rank runs its own independent prefill (its own
+seeded sequence): weak scaling, no data-path collective; the time is the max
+over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_long_block_b200.inputs import WORKLOADS, generate  # noqa: E402
+
+METRIC = "layer_prefill_tokens_per_s"
+UNIT = "tokens/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def algorithmic_work(wl, is_vision):
+    """Algorithmic FLOPs per branch (4 d H_q per attended (query, key) pair)
+    and the bytes of the HBM-bound pooling step, from the mask and config."""
+    vis = np.nonzero(is_vision)[0]
+    txt = np.nonzero(is_vision == 0)[0]
+    nv = len(vis)
+    B = wl.block
+    i = np.arange(nv, dtype=np.int64)
+    nb = nv // B
+    c = np.minimum((i + 1) // B, nb)
+    own = i // B
+    n_sel = np.minimum(wl.top_k, c + (own >= c).astype(np.int64))
+    slc_tokens = B * (n_sel - 1) + (i % B + 1)
+    swa_tokens = np.minimum(wl.window, i + 1)
+    f = 4.0 * wl.d * wl.h_q
+    es = 2 if wl.dtype == "bf16" else 4
+    return {
+        "cmp": f * float(c.sum()),
+        "slc": f * float(slc_tokens.sum()),
+        "swa": f * float(swa_tokens.sum()),
+        "text": f * float((txt.astype(np.int64) + 1).sum()),
+        "pool_bytes": float(2 * nb * B * wl.h_kv * wl.d * es + 2 * nb * wl.h_kv * wl.d * es),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = str(index)
+        self.proc = None
+        self.path = os.path.join("/tmp", f"vnsa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for _, _, fl in rows for k, v in enumerate(fl)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def smi_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return local_rank
+
+
+def cpu_baseline(wl, x, target_s=12.0, max_rows=None):
+    """The fp64 oracle as it stands, timed on a bounded sample of rows in the
+    workload's vision/text proportion.  Returns (tokens/s, cores, sample text)."""
+    import oracle
+    p = oracle.OracleParams(h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                            top_k=wl.top_k, window=wl.window,
+                            round_cmp_bf16=(wl.dtype == "bf16"))
+    vis = np.nonzero(x["is_vision"])[0]
+    txt = np.nonzero(x["is_vision"] == 0)[0]
+    rng = np.random.default_rng(1)
+
+    def sample(nrows):
+        nt = int(round(nrows * len(txt) / wl.n))
+        nvr = nrows - nt
+        rows = np.concatenate([rng.choice(vis, size=min(nvr, len(vis)), replace=False),
+                               rng.choice(txt, size=min(nt, len(txt)), replace=False)
+                               if nt and len(txt) else np.array([], int)])
+        return np.sort(rows).astype(np.int32)
+
+    rows = sample(min(wl.n, 128))
+    t0 = time.perf_counter()
+    oracle.forward(p, x["q"], x["k"], x["v"], x["is_vision"], x["gate"], x["w_k"], x["w_v"],
+                   rows=rows)
+    dt = time.perf_counter() - t0
+    nrows = int(min(wl.n, max(len(rows), len(rows) * target_s / max(dt, 1e-3))))
+    if max_rows:
+        nrows = min(nrows, max_rows)
+    rows = sample(nrows)
+    t0 = time.perf_counter()
+    oracle.forward(p, x["q"], x["k"], x["v"], x["is_vision"], x["gate"], x["w_k"], x["w_v"],
+                   rows=rows)
+    dt = time.perf_counter() - t0
+    nt = int((~x["is_vision"][rows].astype(bool)).sum())
+    return (len(rows) / dt, oracle.threads(),
+            f"{len(rows)} of {wl.n} query rows ({len(rows) - nt} vision, {nt} text), "
+            f"same inputs, {dt:.1f} s wall, rate = rows / s")
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle, rank 0 only."""
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    x = generate(wl)
+    import oracle
+    p = oracle.OracleParams(h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                            top_k=wl.top_k, window=wl.window,
+                            round_cmp_bf16=(wl.dtype == "bf16"))
+    vis = np.nonzero(x["is_vision"])[0]
+    txt = np.nonzero(x["is_vision"] == 0)[0]
+    rng = np.random.default_rng(2)
+    per_step = max(16, int(args.ref_rows))
+    nt = max(1, int(round(per_step * len(txt) / wl.n))) if len(txt) else 0
+
+    def step():
+        rows = np.sort(np.concatenate([rng.choice(vis, per_step - nt, replace=False),
+                                       rng.choice(txt, nt, replace=False) if nt else
+                                       np.array([], int)])).astype(np.int32)
+        oracle.forward(p, x["q"], x["k"], x["v"], x["is_vision"], x["gate"], x["w_k"],
+                       x["w_v"], rows=rows)
+        return len(rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    done = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    val = done / dt
+    sample = (f"{per_step} of {wl.n} query rows per step ({per_step - nt} vision, {nt} text), "
+              "rate = rows / s")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": wl.n, "n_vision": wl.n_vision,
+                       "n_text": wl.n_text, "top_k": wl.top_k, "window": wl.window},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="long_128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="vnsa", choices=["vnsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=96)
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from sparse_attention_long_block_b200 import binding
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dist_on = world > 1
+    if dist_on:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    wl = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    x = generate(wl)
+    td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dev = torch.device("cuda", local_rank)
+    q = torch.from_numpy(x["q"]).to(dev, td)
+    k = torch.from_numpy(x["k"]).to(dev, td)
+    v = torch.from_numpy(x["v"]).to(dev, td)
+    isv = torch.from_numpy(x["is_vision"]).to(dev)
+    gate = torch.from_numpy(x["gate"]).to(dev)
+    out = torch.empty_like(q)
+    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
+                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(q, k, v, isv, gate, out=out, stream=stream)
+
+    def barrier():
+        if dist_on:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise SystemExit("device status error during warm-up")
+    launches_per_step = layer.launches()
+
+    sampler = ClockSampler(smi_index(local_rank)) if rank == 0 else None
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = ev0.elapsed_time(ev1) / max(args.steps, 1)
+    if dist_on:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if layer.device_status() != 0:
+        raise SystemExit("device status error in the timed region")
+
+    # per-stage times (library events on the same stream), outside the timed region
+    layer.set_timing(True)
+    stage_ms = {}
+    reps = 3
+    for _ in range(reps):
+        step()
+        for kname, val in layer.timing().items():
+            stage_ms[kname] = stage_ms.get(kname, 0.0) + val / reps
+    layer.set_timing(False)
+    torch.cuda.synchronize()
+
+    # end to end through the C ABI with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(x["q"]).to(td).pin_memory()
+        hk = torch.from_numpy(x["k"]).to(td).pin_memory()
+        hv = torch.from_numpy(x["v"]).to(td).pin_memory()
+        hi = torch.from_numpy(x["is_vision"]).pin_memory()
+        hg = torch.from_numpy(x["gate"]).pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        layer.forward_host(hq, hk, hv, hi, hg, ho, stream=stream)
+        e_steps = max(2, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            layer.forward_host(hq, hk, hv, hi, hg, ho, stream=stream)
+        b.record(stream)
+        b.synchronize()
+        e_ms = a.elapsed_time(b) / e_steps
+        if dist_on:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hi, hg))
+        e2e = {"value": world * wl.n / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": e_ms}
+
+    work = algorithmic_work(wl, x["is_vision"])
+    flops = work["cmp"] + work["slc"] + work["swa"] + work["text"]
+    peaks = load_peaks()
+    branch_ms = {"partition": stage_ms.get("partition", 0.0), "pool": stage_ms.get("pool", 0.0),
+                 "cmp": stage_ms.get("cmp", 0.0), "topk": stage_ms.get("topk", 0.0),
+                 "slc": stage_ms.get("slc", 0.0), "swa": stage_ms.get("swa", 0.0),
+                 "text": stage_ms.get("text", 0.0)}
+    flop_of = {"cmp": work["cmp"], "slc": work["slc"], "swa": work["swa"], "text": work["text"]}
+    # the vision kernel of the SIMT path does selection + window in one stage
+    if branch_ms["slc"] == 0.0 and branch_ms["swa"] > 0.0:
+        flop_of["swa"] = work["slc"] + work["swa"]
+        flop_of["slc"] = 0.0
+    dom = max(flop_of, key=lambda s: branch_ms.get(s, 0.0))
+    dom_ms = branch_ms[dom]
+    achieved = flop_of[dom] / (dom_ms * 1e-3) / 1e12 if dom_ms > 0 else 0.0
+    traffic = None
+    try:
+        with open(args.traffic_json) as f:
+            tj = json.load(f)
+        ent = tj.get(wl.name, {}).get(dom)
+        if ent and ent.get("kernel_build") == layer_build_id():
+            traffic = ent["bytes_per_launch"]
+    except Exception:
+        pass
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": peaks["source"] + " burst bf16"}
+    pool_gbs = work["pool_bytes"] / (branch_ms["pool"] * 1e-3) / 1e9 if branch_ms["pool"] else 0
+    value = world * wl.n / (ms / 1e3)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = cpu_baseline(wl, x)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if dist_on:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": wl.n, "n_vision": wl.n_vision,
+                       "n_text": wl.n_text, "h_q": wl.h_q, "h_kv": wl.h_kv, "d": wl.d,
+                       "block": wl.block, "top_k": wl.top_k, "window": wl.window,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "tensor_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "algorithmic_gflop": {kk: vv / 1e9 for kk, vv in flop_of.items()},
+            "branch_ms": branch_ms,
+            "pool_hbm": {"achieved_gbs": pool_gbs, "peak_gbs": peaks["hbm_gbs"],
+                         "frac": pool_gbs / peaks["hbm_gbs"]},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if dist_on:
+        dist.destroy_process_group()
+
+
+def layer_build_id():
+    """Identity of the built kernels (library mtime and size) for traffic records."""
+    from sparse_attention_long_block_b200 import binding
+    st = os.stat(binding.LIB_PATH)
+    return f"{st.st_size}"
+
+
+if __name__ == "__main__":
+    main()

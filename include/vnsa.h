@@ -1,0 +1,176 @@
+/*
+ * vnsa.h -- C ABI of the VideoNSA hybrid sparse-attention layer prefill on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes ("VideoNSA: Native Sparse Attention Scales Video
+ * Understanding", paper notes, section "Method"; "VideoNSA: Native Sparse
+ * Attention for Video Understanding", model card, section "Model
+ * Architecture"): the attention of one decoder layer over a prompt of n tokens.
+ * A per-token flag splits the tokens into a vision set and a text set.  Vision
+ * tokens attend through three branches over the vision subsequence, each
+ * weighted by a per-head sigmoid gate:
+ *   compression  mean of each block of `block` vision keys/values, projected
+ *                by W_K / W_V, attended causally at block granularity;
+ *   selection    the top_k blocks ranked by the compression probabilities
+ *                summed over each GQA group (block 0 and the query's own block
+ *                always kept), attended token by token;
+ *   window       the `window` most recent vision tokens.
+ * Text tokens attend densely and causally to every earlier token (GQA).  The
+ * outputs are written at the tokens' original positions.
+ *
+ * Layouts (row-major, contiguous, all device pointers unless stated):
+ *   q, out        [n][h_q][d]        dtype (bf16 or fp32)
+ *   k, v          [n][h_kv][d]       dtype
+ *   is_vision     [n]                uint8, nonzero = vision token
+ *   gate_logits   [n][h_q][3]        fp32, branch order (cmp, slc, swa);
+ *                                    ignored for text rows
+ *   w_k, w_v      [d][d]             dtype; block key = mean(K_block) . W_K
+ * Query head h uses KV head h / (h_q / h_kv).
+ *
+ * Ownership: the caller owns every tensor it passes and the stream.  The handle
+ * owns its workspace (sized for n_max tokens at create time) and a copy of
+ * W_K, W_V.  One handle must not run two forwards concurrently.
+ *
+ * Errors: every call returns a vnsa_status.  Argument errors are found on the
+ * host before anything is launched.  vnsa_forward is asynchronous on `stream`
+ * and never synchronises; a failed launch returns VNSA_ERR_CUDA.  Conditions
+ * the kernels detect (a bounded wait that gave up, an index out of range) set a
+ * device status word, read and cleared by vnsa_get_device_status.
+ */
+#ifndef VNSA_H
+#define VNSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vnsa_status {
+    VNSA_OK = 0,
+    VNSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer    */
+    VNSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128) */
+    VNSA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed             */
+    VNSA_ERR_TIMEOUT = 4,      /* device: a bounded wait gave up                */
+    VNSA_ERR_BOUNDS = 5,       /* device: an index fell outside its tensor      */
+    VNSA_ERR_NO_DEVICE = 6     /* no CUDA device is visible                     */
+} vnsa_status;
+
+typedef enum vnsa_dtype { VNSA_BF16 = 0, VNSA_FP32 = 1 } vnsa_dtype;
+
+typedef struct vnsa_config {
+    int n_max;        /* largest n a forward will see (sizes the workspace)     */
+    int h_q, h_kv;    /* query heads, KV heads; h_q % h_kv == 0, h_q/h_kv <= 16  */
+    int d;            /* head dim: 64 or 128                                    */
+    int block;        /* compression block = stride = selection block: 64       */
+    int top_k;        /* blocks kept per (group, query), 1..64, >= #forced      */
+    int window;       /* sliding window in vision tokens, >= 1                  */
+    int force_first;  /* 1: block 0 is always selected (default 1)              */
+    int force_local;  /* 1: the query's own block is always selected (def. 1)   */
+    float scale;      /* softmax scale; 0 -> 1/sqrt(d)                          */
+    vnsa_dtype dtype; /* storage type of q, k, v, w, out                        */
+} vnsa_config;
+
+typedef struct vnsa_handle vnsa_handle;
+
+/*
+ * Optional per-step exports and an optional selection override, all device
+ * pointers, each may be NULL.  N_v = number of vision tokens, nb = N_v / block.
+ * Per-vision-token arrays are indexed by vision rank (0..N_v-1) and sized for
+ * n rows (the forward's token count); rows N_v..n-1 are left untouched.
+ */
+typedef struct vnsa_debug {
+    float *o_cmp;            /* [n][h_q][d] ungated compression output, by position  */
+    float *o_slc;            /* [n][h_q][d] ungated selection output, by position    */
+    float *o_swa;            /* [n][h_q][d] ungated window output, by position       */
+    float *lse_cmp;          /* [n][h_q] compression log-sum-exp (natural log), rank */
+    int32_t *idx;            /* [h_kv][n][top_k] selected blocks, ascending, -1 pad  */
+    float *imp;              /* [h_kv][n][imp_stride] importance; only the visible
+                                blocks j < (i+1)/block of row i are written          */
+    int imp_stride;          /* row stride of imp in floats (>= n / block)           */
+    void *k_cmp;             /* [nb][h_kv][d] dtype block keys                       */
+    void *v_cmp;             /* [nb][h_kv][d] dtype block values                     */
+    const int32_t *forced_idx; /* input [h_kv][n][top_k]: used instead of the top-k  */
+} vnsa_debug;
+
+/* Stages timed by vnsa_get_timing, in launch order. */
+typedef enum vnsa_stage {
+    VNSA_STAGE_PARTITION = 0, /* vision/text split                                  */
+    VNSA_STAGE_POOL = 1,      /* block mean-pool + projection -> K_cmp, V_cmp       */
+    VNSA_STAGE_CMP = 2,       /* compression attention + importance                 */
+    VNSA_STAGE_TOPK = 3,      /* block selection                                    */
+    VNSA_STAGE_SLC = 4,       /* selection attention                                */
+    VNSA_STAGE_SWA = 5,       /* sliding window + gate combine + vision output      */
+    VNSA_STAGE_TEXT = 6,      /* dense text GQA                                     */
+    VNSA_NUM_STAGES = 7
+} vnsa_stage;
+
+/* Human-readable text of a status code (static storage). */
+const char *vnsa_status_string(vnsa_status s);
+
+/* Name of a stage ("partition", "pool", ...), or NULL if out of range. */
+const char *vnsa_stage_name(int stage);
+
+/* Bytes of device workspace vnsa_create would allocate for cfg. */
+vnsa_status vnsa_workspace_bytes(const vnsa_config *cfg, size_t *bytes);
+
+/*
+ * Validate cfg, allocate the workspace on the current device and copy the
+ * projections w_k, w_v ([d][d], dtype, device pointers) into it.  Synchronous.
+ * On success *out holds the handle; on failure *out is NULL and nothing leaks.
+ */
+vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v,
+                        vnsa_handle **out);
+
+/*
+ * One layer prefill of n (1..n_max) tokens, enqueued on `stream` (a
+ * cudaStream_t; NULL = the legacy default stream).  Pointers must be device
+ * pointers, 16-byte aligned, in the layouts above.  `dbg` may be NULL.
+ * Returns after enqueueing; errors found by the kernels are reported by
+ * vnsa_get_device_status.
+ */
+vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k,
+                         const void *v, const uint8_t *is_vision,
+                         const float *gate_logits, void *out, const vnsa_debug *dbg,
+                         void *stream);
+
+/*
+ * The same layer prefill from HOST buffers (same layouts): copies the inputs
+ * to handle-owned device staging buffers, runs vnsa_forward on `stream`, copies
+ * `out` back and synchronises the stream before returning.  Page-locked host
+ * buffers give the fastest copies.  Allocates nothing per call.
+ */
+vnsa_status vnsa_forward_host(vnsa_handle *h, int n, const void *q, const void *k,
+                              const void *v, const uint8_t *is_vision,
+                              const float *gate_logits, void *out, void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear the handle's device status word.
+ * *code receives VNSA_OK or the first device-detected error (TIMEOUT, BOUNDS).
+ */
+vnsa_status vnsa_get_device_status(vnsa_handle *h, void *stream, uint32_t *code);
+
+/*
+ * Vision / text counts of the last forward (synchronises `stream`).
+ */
+vnsa_status vnsa_get_counts(vnsa_handle *h, void *stream, int *n_vision, int *n_text);
+
+/*
+ * Per-stage timing.  With timing on, each forward records CUDA events between
+ * its stages on its stream; vnsa_get_timing synchronises on the last event and
+ * writes VNSA_NUM_STAGES milliseconds (0 for a stage that did not run).
+ */
+vnsa_status vnsa_set_timing(vnsa_handle *h, int enable);
+vnsa_status vnsa_get_timing(vnsa_handle *h, float *ms);
+
+/* Kernel launches the last forward enqueued (for launch accounting). */
+vnsa_status vnsa_get_launch_count(vnsa_handle *h, int *launches);
+
+/* Free the workspace and the handle (synchronises the device first). */
+vnsa_status vnsa_destroy(vnsa_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VNSA_H */

@@ -1,0 +1,289 @@
+// prep.cu -- vision/text partition, block mean-pool + projection, top-k block
+// selection.
+//
+// Method: "VideoNSA: Native Sparse Attention Scales Video Understanding" (paper
+// notes), section "Method": tokens are split into vision and text sets by their
+// position IDs; the compression branch averages each 64-token vision block into
+// one block key and value through a learned projection (a d x d linear map
+// here); the selection branch keeps the top-k blocks ranked by importance.
+#include "kernels.h"
+
+namespace vnsa {
+
+// ---------------------------------------------------------------------------
+// Partition: one CTA of 1024 threads scans the flags.  vis[i] = position of
+// the i-th vision token, txt[x] = position of the x-th text token.
+__global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restrict__ isv,
+                                                         int n, int block,
+                                                         int32_t *__restrict__ vis,
+                                                         int32_t *__restrict__ txt,
+                                                         Counts *counts) {
+    __shared__ int s_cnt[1024];
+    const int tid = threadIdx.x;
+    const int per = (n + 1023) / 1024;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int c = 0;
+    for (int t = lo; t < hi; ++t) c += isv[t] != 0;
+    s_cnt[tid] = c;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+        int add = tid >= off ? s_cnt[tid - off] : 0;
+        __syncthreads();
+        s_cnt[tid] += add;
+        __syncthreads();
+    }
+    int vb = s_cnt[tid] - c;
+    int tb = lo - vb;
+    for (int t = lo; t < hi; ++t) {
+        if (isv[t]) vis[vb++] = t;
+        else txt[tb++] = t;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int nv = s_cnt[1023];
+        Counts cn;
+        cn.n_vision = nv;
+        cn.n_text = n - nv;
+        cn.nb = nv / block;
+        cn.vis_base = nv > 0 ? vis[0] : 0;
+        cn.contiguous = (nv == 0) || (vis[nv - 1] - vis[0] == nv - 1);
+        cn.pad[0] = cn.pad[1] = cn.pad[2] = 0;
+        *counts = cn;
+    }
+}
+
+cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t *vis,
+                             int32_t *txt, Counts *counts, cudaStream_t s) {
+    partition_kernel<<<1, 1024, 0, s>>>(is_vision, n, block, vis, txt, counts);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Pool + projection.  CTA (tile of JB blocks, KV head g, K or V): mean of each
+// block's `block` vision rows in fp32, then mean . W (d x d) and one rounding
+// to the storage type.  Rows are read with vector loads, one row per warp step.
+template <typename T, int PER>
+__device__ __forceinline__ void load_row_part(const T *p, float (&x)[PER]) {
+    if constexpr (sizeof(T) == 2 && PER == 4) {
+        uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    } else if constexpr (sizeof(T) == 2 && PER == 2) {
+        float2 a = __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p)));
+        x[0] = a.x; x[1] = a.y;
+    } else if constexpr (sizeof(T) == 4 && PER == 4) {
+        float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    } else {
+        float2 a = __ldg(reinterpret_cast<const float2 *>(p));
+        x[0] = a.x; x[1] = a.y;
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) pool_proj_kernel(
+    const T *__restrict__ k, const T *__restrict__ v, const int32_t *__restrict__ vis,
+    const Counts *__restrict__ counts, const T *__restrict__ w_k, const T *__restrict__ w_v,
+    T *__restrict__ k_cmp, T *__restrict__ v_cmp, int h_kv, int block) {
+    constexpr int JB = 16;             // blocks per CTA
+    constexpr int PER = D / 32;        // elements per lane in a row
+    constexpr int NPART = 256 / D;     // threads per output column
+    constexpr int JBP = JB / NPART;    // blocks per thread in the projection
+    __shared__ float mean[JB][D];
+    const int nb = counts->nb;
+    const int j0 = blockIdx.x * JB;
+    if (j0 >= nb) return;
+    const int g = blockIdx.y;
+    const bool is_v = blockIdx.z != 0;
+    const T *src = is_v ? v : k;
+    const T *W = is_v ? w_v : w_k;
+    T *dst = is_v ? v_cmp : k_cmp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float inv = 1.0f / (float)block;
+    for (int jb = warp; jb < JB; jb += 8) {
+        const int j = j0 + jb;
+        float acc[PER];
+#pragma unroll
+        for (int c = 0; c < PER; ++c) acc[c] = 0.f;
+        if (j < nb) {
+            const int32_t *rows = vis + (size_t)j * block;
+#pragma unroll 8
+            for (int u = 0; u < block; ++u) {
+                const T *p = src + ((size_t)rows[u] * h_kv + g) * D + lane * PER;
+                float x[PER];
+                load_row_part<T, PER>(p, x);
+#pragma unroll
+                for (int c = 0; c < PER; ++c) acc[c] += x[c];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < PER; ++c) mean[jb][lane * PER + c] = acc[c] * inv;
+    }
+    __syncthreads();
+    const int col = threadIdx.x % D, part = threadIdx.x / D;
+    float o[JBP];
+#pragma unroll
+    for (int x = 0; x < JBP; ++x) o[x] = 0.f;
+    for (int e = 0; e < D; ++e) {
+        const float w = to_f(W[(size_t)e * D + col]);
+#pragma unroll
+        for (int x = 0; x < JBP; ++x) o[x] = fmaf(mean[part * JBP + x][e], w, o[x]);
+    }
+#pragma unroll
+    for (int x = 0; x < JBP; ++x) {
+        const int j = j0 + part * JBP + x;
+        if (j < nb) dst[((size_t)j * h_kv + g) * D + col] = from_f<T>(o[x]);
+    }
+}
+
+cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
+                             const int32_t *vis, const Counts *counts, const void *w_k,
+                             const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
+                             int nb_max, cudaStream_t s) {
+    if (nb_max <= 0) return cudaSuccess;
+    dim3 grid((nb_max + 15) / 16, h_kv, 2);
+#define VNSA_POOL(T, D)                                                                  \
+    pool_proj_kernel<T, D><<<grid, 256, 0, s>>>(                                         \
+        (const T *)k, (const T *)v, vis, counts, (const T *)w_k, (const T *)w_v,         \
+        (T *)k_cmp, (T *)v_cmp, h_kv, block)
+    if (dtype == VNSA_BF16 && d == 128) VNSA_POOL(__nv_bfloat16, 128);
+    else if (dtype == VNSA_BF16 && d == 64) VNSA_POOL(__nv_bfloat16, 64);
+    else if (dtype == VNSA_FP32 && d == 128) VNSA_POOL(float, 128);
+    else if (dtype == VNSA_FP32 && d == 64) VNSA_POOL(float, 64);
+    else return cudaErrorInvalidValue;
+#undef VNSA_POOL
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Top-k block selection: one warp per (group g, vision query i).
+// Forced blocks: 0 and the query's own block i/B (when enabled) count within
+// top_k.  The remaining slots take the visible, non-forced blocks with the
+// largest importance, ties to the lower block index.  Output ascending, -1
+// padded.  Importance values are probabilities (>= 0): a taken block is marked
+// with -1 in the shared copy of its row.
+__global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
+    extern __shared__ float s_imp[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 8 + warp;
+    const int g = blockIdx.y;
+    const Counts cn = *p.counts;
+    if (i >= cn.n_vision) return;
+    float *s = s_imp + (size_t)warp * p.nb_max;
+    const int B = p.block;
+    const int own = i / B;
+    int c = (i + 1) / B;
+    if (c > cn.nb) c = cn.nb;
+    const float *row = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
+    for (int j = lane; j < c; j += 32) s[j] = row[j];
+    __syncwarp();
+    int nforced = 0;
+    if (p.force_first) {
+        ++nforced;
+        if (c > 0 && lane == 0) s[0] = -1.f;
+    }
+    if (p.force_local && !(p.force_first && own == 0)) {
+        ++nforced;
+        if (own < c && lane == 0) s[own] = -1.f;
+    }
+    __syncwarp();
+    const bool extra = (p.force_local && own >= c) || (p.force_first && c == 0);
+    const int m = p.top_k - nforced;
+    for (int round = 0; round < m; ++round) {
+        float bv = -1.f;
+        int bj = 0x7fffffff;
+        for (int j = lane; j < c; j += 32) {
+            const float x = s[j];
+            if (x > bv) { bv = x; bj = j; }  // lanes scan ascending j: ties keep lower j
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+            if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
+        }
+        if (bv < 0.f) break;  // no candidate left
+        if (lane == 0) s[bj] = -1.f;
+        __syncwarp();
+    }
+    int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
+    int cnt = 0;
+    for (int base = 0; base < c; base += 32) {
+        const int j = base + lane;
+        const bool f = j < c && s[j] < 0.f;
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (f && pos < p.top_k) out[pos] = j;
+        cnt += __popc(bal);
+    }
+    if (extra) {
+        if (lane == 0 && cnt < p.top_k) out[cnt] = own;
+        ++cnt;
+    }
+    for (int x = cnt + lane; x < p.top_k; x += 32) out[x] = -1;
+    if (cnt > p.top_k && lane == 0) report(p.status, VNSA_ERR_BOUNDS);
+}
+
+cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {
+    const size_t smem = (size_t)8 * p.nb_max * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((p.n_max + 7) / 8, p.h_kv);
+    topk_kernel<<<grid, 256, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace vnsa
+
+namespace vnsa {
+
+// ---------------------------------------------------------------------------
+// Debug exports: copies of workspace tensors into caller buffers, sized by the
+// device-side vision count (so the host never has to synchronise for it).
+__global__ void export_kernel(LayerParams p, int esize, float *lse_out, int32_t *idx_out,
+                              float *imp_out, size_t imp_stride_out, uint32_t *kc_out,
+                              uint32_t *vc_out) {
+    const Counts cn = *p.counts;
+    const size_t nv = (size_t)cn.n_vision, nb = (size_t)cn.nb;
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t step = (size_t)gridDim.x * blockDim.x;
+    if (lse_out)
+        for (size_t x = tid; x < nv * p.h_q; x += step) lse_out[x] = p.lse[x];
+    if (idx_out) {
+        const size_t k = (size_t)p.top_k;
+        for (size_t x = tid; x < (size_t)p.h_kv * nv * k; x += step) {
+            const size_t g = x / (nv * k), rem = x % (nv * k);
+            const size_t i = rem / k, c = rem % k;
+            idx_out[(g * p.n + i) * k + c] = p.idx_src[(g * p.idx_rows + i) * k + c];
+        }
+    }
+    if (imp_out && nb > 0) {
+        for (size_t x = tid; x < (size_t)p.h_kv * nv * nb; x += step) {
+            const size_t j = x % nb, gi = x / nb;
+            const size_t g = gi / nv, i = gi % nv;
+            if ((int)j < (int)((i + 1) / p.block))
+                imp_out[(g * p.n + i) * imp_stride_out + j] =
+                    p.imp[(g * p.n_max + i) * p.imp_stride + j];
+        }
+    }
+    const size_t words = nb * p.h_kv * p.d * esize / 4;
+    if (kc_out)
+        for (size_t x = tid; x < words; x += step) kc_out[x] = ((const uint32_t *)p.k_cmp)[x];
+    if (vc_out)
+        for (size_t x = tid; x < words; x += step) vc_out[x] = ((const uint32_t *)p.v_cmp)[x];
+}
+
+cudaError_t launch_export(const LayerParams &p, int esize, float *lse_out, int32_t *idx_out,
+                          float *imp_out, size_t imp_stride_out, void *kc_out, void *vc_out,
+                          cudaStream_t s) {
+    export_kernel<<<592, 256, 0, s>>>(p, esize, lse_out, idx_out, imp_out, imp_stride_out,
+                                      (uint32_t *)kc_out, (uint32_t *)vc_out);
+    return cudaGetLastError();
+}
+
+}  // namespace vnsa

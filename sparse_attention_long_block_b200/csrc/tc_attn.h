@@ -1,0 +1,28 @@
+// tc_attn.h -- tensor-core (tcgen05 / TMEM / TMA) attention path of the bf16
+// layer prefill, behind the C ABI of vnsa_api.cu.
+#pragma once
+
+#include "kernels.h"
+
+namespace vnsa {
+
+struct TcState;
+
+// True if the bf16 tensor-core path handles this configuration.
+bool tc_supported(const vnsa_config &c);
+
+// Extra workspace bytes the tensor-core path needs for n_max tokens.
+size_t tc_workspace_bytes(const vnsa_config &c);
+
+// Set up the path (tensor maps are rebuilt per forward); ws is its workspace.
+cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out);
+
+// Compression, top-k, selection, window + gate, text: enqueued on s.  `ev`
+// (nullable) holds the per-stage timing events (begin, end) of vnsa_api.cu;
+// `ran` marks the stages that ran; `launches` counts kernel launches.
+cudaError_t tc_forward(TcState *st, const LayerParams &p, cudaStream_t s, cudaEvent_t *ev,
+                       int *ran, int *launches, bool forced);
+
+void tc_destroy(TcState *st);
+
+}  // namespace vnsa

@@ -1,0 +1,405 @@
+// vnsa_api.cu -- the C ABI declared in include/vnsa.h: argument validation,
+// workspace ownership, and the launch sequence of one layer prefill.
+//
+// One forward enqueues, on the caller's stream and without host syncs:
+//   partition -> pool+projection -> compression attention (+ importance)
+//   -> top-k -> vision branches + gate -> text GQA.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+
+#include "kernels.h"
+#include "tc_attn.h"
+
+using namespace vnsa;
+
+namespace {
+
+constexpr int kMaxTokens = 262144;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+    size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, idx, o_cmp, tc;
+    size_t total;
+    size_t imp_stride;
+};
+
+Layout make_layout(const vnsa_config &c) {
+    const size_t es = c.dtype == VNSA_BF16 ? 2 : 4;
+    const size_t n = (size_t)c.n_max;
+    const size_t nb = (size_t)(c.n_max / c.block);
+    Layout L;
+    L.imp_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes > 0 ? bytes : 1); return o; };
+    L.vis = take(n * 4);
+    L.txt = take(n * 4);
+    L.counts = take(sizeof(Counts));
+    L.status = take(16);
+    L.w_k = take((size_t)c.d * c.d * es);
+    L.w_v = take((size_t)c.d * c.d * es);
+    L.k_cmp = take(nb * c.h_kv * c.d * es);
+    L.v_cmp = take(nb * c.h_kv * c.d * es);
+    L.lse = take(n * c.h_q * 4);
+    L.imp = take((size_t)c.h_kv * n * L.imp_stride * 4);
+    L.idx = take((size_t)c.h_kv * n * c.top_k * 4);
+    L.o_cmp = take(n * c.h_q * c.d * 4);
+    L.tc = take(tc_workspace_bytes(c));
+    L.total = off;
+    return L;
+}
+
+vnsa_status check_config(const vnsa_config *c) {
+    if (!c) return VNSA_ERR_INVALID_ARG;
+    if (c->n_max < 1 || c->h_q < 1 || c->h_kv < 1 || c->d < 1) return VNSA_ERR_INVALID_ARG;
+    if (c->h_q % c->h_kv != 0) return VNSA_ERR_INVALID_ARG;
+    if (c->top_k < 1 || c->window < 1 || c->block < 1) return VNSA_ERR_INVALID_ARG;
+    if ((c->force_first != 0 && c->force_first != 1) ||
+        (c->force_local != 0 && c->force_local != 1))
+        return VNSA_ERR_INVALID_ARG;
+    if (c->top_k < c->force_first + c->force_local) return VNSA_ERR_INVALID_ARG;
+    if (!(c->scale >= 0.f) || isinf(c->scale)) return VNSA_ERR_INVALID_ARG;
+    if (c->dtype != VNSA_BF16 && c->dtype != VNSA_FP32) return VNSA_ERR_INVALID_ARG;
+    if (c->n_max > kMaxTokens) return VNSA_ERR_UNSUPPORTED;
+    if (c->d != 64 && c->d != 128) return VNSA_ERR_UNSUPPORTED;
+    if (c->block != 64) return VNSA_ERR_UNSUPPORTED;
+    if (c->h_q / c->h_kv > 16) return VNSA_ERR_UNSUPPORTED;
+    if (c->top_k > 64) return VNSA_ERR_UNSUPPORTED;
+    return VNSA_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+struct vnsa_handle {
+    vnsa_config cfg;
+    int device;
+    int r, nb_max;
+    size_t esize;
+    Layout L;
+    char *ws;
+    Counts *counts;
+    uint32_t *status;
+    char *stage;  // staging buffers of vnsa_forward_host (allocated on first use)
+    size_t stage_bytes;
+    TcState *tc;
+    int timing;
+    cudaEvent_t ev[2 * VNSA_NUM_STAGES];
+    int ran[VNSA_NUM_STAGES];
+    int launches;
+};
+
+extern "C" {
+
+const char *vnsa_status_string(vnsa_status s) {
+    switch (s) {
+        case VNSA_OK: return "ok";
+        case VNSA_ERR_INVALID_ARG: return "invalid argument";
+        case VNSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case VNSA_ERR_CUDA: return "CUDA error";
+        case VNSA_ERR_TIMEOUT: return "device wait timed out";
+        case VNSA_ERR_BOUNDS: return "device index out of bounds";
+        case VNSA_ERR_NO_DEVICE: return "no CUDA device";
+    }
+    return "unknown status";
+}
+
+const char *vnsa_stage_name(int stage) {
+    static const char *names[VNSA_NUM_STAGES] = {"partition", "pool", "cmp", "topk",
+                                                 "slc", "swa", "text"};
+    if (stage < 0 || stage >= VNSA_NUM_STAGES) return nullptr;
+    return names[stage];
+}
+
+vnsa_status vnsa_workspace_bytes(const vnsa_config *cfg, size_t *bytes) {
+    if (!bytes) return VNSA_ERR_INVALID_ARG;
+    vnsa_status st = check_config(cfg);
+    if (st != VNSA_OK) return st;
+    *bytes = make_layout(*cfg).total;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v,
+                        vnsa_handle **out) {
+    if (!out) return VNSA_ERR_INVALID_ARG;
+    *out = nullptr;
+    vnsa_status st = check_config(cfg);
+    if (st != VNSA_OK) return st;
+    if (!w_k || !w_v || !aligned16(w_k) || !aligned16(w_v)) return VNSA_ERR_INVALID_ARG;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return VNSA_ERR_NO_DEVICE;
+    }
+    vnsa_handle *h = new (std::nothrow) vnsa_handle();
+    if (!h) return VNSA_ERR_CUDA;
+    h->cfg = *cfg;
+    if (h->cfg.scale == 0.f) h->cfg.scale = 1.0f / sqrtf((float)cfg->d);
+    cudaGetDevice(&h->device);
+    h->r = cfg->h_q / cfg->h_kv;
+    h->nb_max = cfg->n_max / cfg->block;
+    h->esize = cfg->dtype == VNSA_BF16 ? 2 : 4;
+    h->L = make_layout(h->cfg);
+    if (cudaMalloc(&h->ws, h->L.total) != cudaSuccess) {
+        cudaGetLastError();
+        delete h;
+        return VNSA_ERR_CUDA;
+    }
+    h->counts = (Counts *)(h->ws + h->L.counts);
+    h->status = (uint32_t *)(h->ws + h->L.status);
+    const size_t wbytes = (size_t)cfg->d * cfg->d * h->esize;
+    bool ok = cudaMemset(h->ws + h->L.status, 0, 16) == cudaSuccess &&
+              cudaMemset(h->ws + h->L.counts, 0, sizeof(Counts)) == cudaSuccess &&
+              cudaMemcpy(h->ws + h->L.w_k, w_k, wbytes, cudaMemcpyDefault) == cudaSuccess &&
+              cudaMemcpy(h->ws + h->L.w_v, w_v, wbytes, cudaMemcpyDefault) == cudaSuccess;
+    if (ok) ok = tc_create(h->cfg, h->ws + h->L.tc, &h->tc) == cudaSuccess;
+    for (int e = 0; ok && e < 2 * VNSA_NUM_STAGES; ++e)
+        ok = cudaEventCreate(&h->ev[e]) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        vnsa_destroy(h);
+        return VNSA_ERR_CUDA;
+    }
+    *out = h;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, const void *v,
+                         const uint8_t *is_vision, const float *gate_logits, void *out,
+                         const vnsa_debug *dbg, void *stream) {
+    if (!h || !q || !k || !v || !is_vision || !gate_logits || !out) return VNSA_ERR_INVALID_ARG;
+    if (n < 1 || n > h->cfg.n_max) return VNSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(gate_logits))
+        return VNSA_ERR_INVALID_ARG;
+    if (dbg && dbg->imp && dbg->imp_stride < n / h->cfg.block) return VNSA_ERR_INVALID_ARG;
+    const vnsa_config &c = h->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return VNSA_ERR_CUDA;
+
+    LayerParams p;
+    memset(&p, 0, sizeof(p));
+    p.n = n;
+    p.n_max = c.n_max;
+    p.h_q = c.h_q;
+    p.h_kv = c.h_kv;
+    p.d = c.d;
+    p.r = h->r;
+    p.block = c.block;
+    p.top_k = c.top_k;
+    p.window = c.window;
+    p.force_first = c.force_first;
+    p.force_local = c.force_local;
+    p.nb_max = h->nb_max;
+    p.scale_log2 = c.scale * kLog2e;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.is_vision = is_vision;
+    p.gate = gate_logits;
+    p.out = out;
+    p.vis = (const int32_t *)(h->ws + h->L.vis);
+    p.txt = (const int32_t *)(h->ws + h->L.txt);
+    p.counts = h->counts;
+    p.status = h->status;
+    p.k_cmp = h->ws + h->L.k_cmp;
+    p.v_cmp = h->ws + h->L.v_cmp;
+    p.lse = (float *)(h->ws + h->L.lse);
+    p.imp = (float *)(h->ws + h->L.imp);
+    p.imp_stride = h->L.imp_stride;
+    p.idx = (int32_t *)(h->ws + h->L.idx);
+    p.idx_src = p.idx;
+    p.idx_rows = (size_t)c.n_max;
+    p.o_cmp_ws = (float *)(h->ws + h->L.o_cmp);
+    const bool forced = dbg && dbg->forced_idx;
+    if (forced) {
+        p.idx_src = dbg->forced_idx;
+        p.idx_rows = (size_t)n;  // caller layout [h_kv][n][top_k]
+    }
+    if (dbg) {
+        p.dbg_o_cmp = dbg->o_cmp;
+        p.dbg_o_slc = dbg->o_slc;
+        p.dbg_o_swa = dbg->o_swa;
+    }
+
+    const int dt = (int)c.dtype;
+    const bool use_tc = tc_supported(c);
+    h->launches = 0;
+    for (int x = 0; x < VNSA_NUM_STAGES; ++x) h->ran[x] = 0;
+    cudaError_t e = cudaSuccess;
+    auto begin = [&](int stg) {
+        if (h->timing) cudaEventRecord(h->ev[2 * stg], s);
+        h->ran[stg] = 1;
+    };
+    auto end = [&](int stg) {
+        if (h->timing) cudaEventRecord(h->ev[2 * stg + 1], s);
+    };
+#define VNSA_RUN(call)                                \
+    do {                                              \
+        if (e == cudaSuccess) {                       \
+            e = (call);                               \
+            ++h->launches;                            \
+        }                                             \
+    } while (0)
+
+    begin(VNSA_STAGE_PARTITION);
+    VNSA_RUN(launch_partition(is_vision, n, c.block, (int32_t *)p.vis, (int32_t *)p.txt,
+                              h->counts, s));
+    end(VNSA_STAGE_PARTITION);
+    begin(VNSA_STAGE_POOL);
+    VNSA_RUN(launch_pool_proj(dt, c.d, k, v, p.vis, h->counts, h->ws + h->L.w_k,
+                              h->ws + h->L.w_v, (void *)p.k_cmp, (void *)p.v_cmp, c.h_kv,
+                              c.block, h->nb_max, s));
+    end(VNSA_STAGE_POOL);
+    if (use_tc) {
+        VNSA_RUN(tc_forward(h->tc, p, s, h->timing ? h->ev : nullptr, h->ran, &h->launches,
+                            forced));
+    } else {
+        begin(VNSA_STAGE_CMP);
+        VNSA_RUN(launch_cmp_simt(dt, p, s));
+        end(VNSA_STAGE_CMP);
+        if (!forced) {
+            begin(VNSA_STAGE_TOPK);
+            VNSA_RUN(launch_topk(p, s));
+            end(VNSA_STAGE_TOPK);
+        }
+        begin(VNSA_STAGE_SWA);
+        VNSA_RUN(launch_vision_simt(dt, p, s));
+        end(VNSA_STAGE_SWA);
+        begin(VNSA_STAGE_TEXT);
+        VNSA_RUN(launch_text_simt(dt, p, s));
+        end(VNSA_STAGE_TEXT);
+    }
+    if (dbg && (dbg->lse_cmp || dbg->idx || dbg->imp || dbg->k_cmp || dbg->v_cmp))
+        VNSA_RUN(launch_export(p, (int)h->esize, dbg->lse_cmp, dbg->idx, dbg->imp,
+                               (size_t)dbg->imp_stride, dbg->k_cmp, dbg->v_cmp, s));
+#undef VNSA_RUN
+    if (cur != h->device && cur >= 0) cudaSetDevice(cur);
+    if (e != cudaSuccess) {
+        fprintf(stderr, "vnsa_forward: %s\n", cudaGetErrorString(e));
+        return VNSA_ERR_CUDA;
+    }
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_forward_host(vnsa_handle *h, int n, const void *q, const void *k,
+                              const void *v, const uint8_t *is_vision,
+                              const float *gate_logits, void *out, void *stream) {
+    if (!h || !q || !k || !v || !is_vision || !gate_logits || !out) return VNSA_ERR_INVALID_ARG;
+    if (n < 1 || n > h->cfg.n_max) return VNSA_ERR_INVALID_ARG;
+    const vnsa_config &c = h->cfg;
+    const size_t nm = (size_t)c.n_max;
+    const size_t bq = align_up(nm * c.h_q * c.d * h->esize);
+    const size_t bk = align_up(nm * c.h_kv * c.d * h->esize);
+    const size_t bg = align_up(nm * c.h_q * 3 * 4);
+    const size_t bi = align_up(nm);
+    const size_t need = 2 * bq + 2 * bk + bg + bi;
+    if (!h->stage) {
+        if (cudaMalloc(&h->stage, need) != cudaSuccess) {
+            cudaGetLastError();
+            h->stage = nullptr;
+            return VNSA_ERR_CUDA;
+        }
+        h->stage_bytes = need;
+    }
+    char *dq = h->stage, *dk = dq + bq, *dv = dk + bk, *dg = dv + bk, *di = dg + bg,
+         *dout = di + bi;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t nq = (size_t)n * c.h_q * c.d * h->esize;
+    const size_t nk = (size_t)n * c.h_kv * c.d * h->esize;
+    bool ok = cudaMemcpyAsync(dq, q, nq, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(dk, k, nk, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(dv, v, nk, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(dg, gate_logits, (size_t)n * c.h_q * 3 * 4,
+                              cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(di, is_vision, (size_t)n, cudaMemcpyHostToDevice, s) ==
+                  cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    vnsa_status st = vnsa_forward(h, n, dq, dk, dv, (const uint8_t *)di, (const float *)dg,
+                                  dout, nullptr, stream);
+    if (st != VNSA_OK) return st;
+    if (cudaMemcpyAsync(out, dout, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_get_device_status(vnsa_handle *h, void *stream, uint32_t *code) {
+    if (!h || !code) return VNSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpy(&v, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(h->status, 0, 4) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    *code = v;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_get_counts(vnsa_handle *h, void *stream, int *n_vision, int *n_text) {
+    if (!h || !n_vision || !n_text) return VNSA_ERR_INVALID_ARG;
+    Counts cn;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess ||
+        cudaMemcpy(&cn, h->counts, sizeof(cn), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    *n_vision = cn.n_vision;
+    *n_text = cn.n_text;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_set_timing(vnsa_handle *h, int enable) {
+    if (!h) return VNSA_ERR_INVALID_ARG;
+    h->timing = enable ? 1 : 0;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_get_timing(vnsa_handle *h, float *ms) {
+    if (!h || !ms) return VNSA_ERR_INVALID_ARG;
+    for (int x = 0; x < VNSA_NUM_STAGES; ++x) {
+        ms[x] = 0.f;
+        if (!h->timing || !h->ran[x]) continue;
+        if (cudaEventSynchronize(h->ev[2 * x + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&ms[x], h->ev[2 * x], h->ev[2 * x + 1]) != cudaSuccess) {
+            cudaGetLastError();
+            return VNSA_ERR_CUDA;
+        }
+    }
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_get_launch_count(vnsa_handle *h, int *launches) {
+    if (!h || !launches) return VNSA_ERR_INVALID_ARG;
+    *launches = h->launches;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_destroy(vnsa_handle *h) {
+    if (!h) return VNSA_ERR_INVALID_ARG;
+    cudaDeviceSynchronize();
+    tc_destroy(h->tc);
+    for (int e = 0; e < 2 * VNSA_NUM_STAGES; ++e)
+        if (h->ev[e]) cudaEventDestroy(h->ev[e]);
+    if (h->stage) cudaFree(h->stage);
+    if (h->ws) cudaFree(h->ws);
+    cudaGetLastError();
+    delete h;
+    return VNSA_OK;
+}
+
+}  // extern "C"

@@ -73,10 +73,14 @@ WORKLOADS = {
 
 def bf16_round(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 value (ties to even), in float32."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
+    a = np.array(a, dtype=np.float32, copy=True, order="C")
     u = a.view(np.uint32)
-    bias = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    return ((u + bias) & np.uint32(0xFFFF0000)).view(np.float32)
+    t = u >> np.uint32(16)
+    t &= np.uint32(1)
+    t += np.uint32(0x7FFF)
+    u += t
+    u &= np.uint32(0xFFFF0000)
+    return a
 
 
 def _frame_tokens(rng, n_vision, h, d, ar1):

@@ -1,0 +1,90 @@
+"""The C ABI on the host: the library loads, exports every symbol include/vnsa.h
+declares, and rejects bad configurations before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_block_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "vnsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vnsa_[a-z_]+)\s*\(", text)))
+
+
+def cfg(**kw):
+    base = dict(n_max=8448, h_q=28, h_kv=4, d=128, block=64, top_k=16, window=256,
+                force_first=1, force_local=1, scale=0.0, dtype=binding.VNSA_BF16)
+    base.update(kw)
+    return binding.vnsa_config(**base)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = binding.load()
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(binding.EXPORTED) == names
+
+
+def test_status_and_stage_strings():
+    assert binding.status_string(0) == "ok"
+    assert "invalid" in binding.status_string(1)
+    assert binding.status_string(99) == "unknown status"
+    assert [binding.stage_name(i) for i in range(binding.NUM_STAGES)] == [
+        "partition", "pool", "cmp", "topk", "slc", "swa", "text"]
+    assert binding.stage_name(7) is None
+
+
+def test_workspace_bytes_valid_config():
+    b = binding.vnsa_workspace_bytes(cfg())
+    # imp alone is [h_kv][n_max][nb] fp32
+    assert b > 4 * 8448 * (8448 // 64) * 4
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(h_q=28, h_kv=3), binding.VNSA_ERR_INVALID_ARG),
+    (dict(top_k=1), binding.VNSA_ERR_INVALID_ARG),
+    (dict(window=0), binding.VNSA_ERR_INVALID_ARG),
+    (dict(n_max=0), binding.VNSA_ERR_INVALID_ARG),
+    (dict(force_first=2), binding.VNSA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), binding.VNSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.VNSA_ERR_INVALID_ARG),
+    (dict(dtype=7), binding.VNSA_ERR_INVALID_ARG),
+    (dict(d=96), binding.VNSA_ERR_UNSUPPORTED),
+    (dict(block=32), binding.VNSA_ERR_UNSUPPORTED),
+    (dict(top_k=65), binding.VNSA_ERR_UNSUPPORTED),
+    (dict(n_max=262145), binding.VNSA_ERR_UNSUPPORTED),
+    (dict(h_q=34, h_kv=2), binding.VNSA_ERR_UNSUPPORTED),
+])
+def test_bad_configs_rejected_on_host(bad, code):
+    with pytest.raises(binding.VnsaError) as e:
+        binding.vnsa_workspace_bytes(cfg(**bad))
+    assert e.value.code == code
+
+
+def test_create_rejects_null_weights_and_handles_missing_device():
+    lib = binding.load()
+    h = ctypes.c_void_p(0)
+    c = cfg()
+    rc = lib.vnsa_create(ctypes.byref(c), None, None, ctypes.byref(h))
+    assert rc == binding.VNSA_ERR_INVALID_ARG and not h.value
+    import torch
+    if not torch.cuda.is_available():
+        fake = ctypes.c_void_p(4096)  # aligned, never dereferenced without a device
+        rc = lib.vnsa_create(ctypes.byref(c), fake, fake, ctypes.byref(h))
+        assert rc == binding.VNSA_ERR_NO_DEVICE and not h.value
+
+
+def test_forward_rejects_null_handle_and_bad_n():
+    lib = binding.load()
+    rc = lib.vnsa_forward(None, 10, None, None, None, None, None, None, None, None)
+    assert rc == binding.VNSA_ERR_INVALID_ARG
+    rc = lib.vnsa_destroy(None)
+    assert rc == binding.VNSA_ERR_INVALID_ARG
