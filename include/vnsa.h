@@ -170,6 +170,37 @@ vnsa_status vnsa_get_launch_count(vnsa_handle *h, int *launches);
 /* Free the workspace and the handle (synchronises the device first). */
 vnsa_status vnsa_destroy(vnsa_handle *h);
 
+/*
+ * Block selection without any device allocation (the paper has no counterpart:
+ * this is a library-only entry point).  For callers that cannot call
+ * cudaMalloc -- code under CUDA stream capture, plugins that must draw all
+ * device memory from a host framework's own pool, latency-critical paths that
+ * cannot take the allocator's synchronisation -- it runs the selection chain
+ * of one layer: vision/text split, block mean-pool + projection, compression
+ * attention with group importance, top-k.  No handle is needed.
+ *
+ * Inputs (device, 16-byte aligned, layouts as above): q, k, v, is_vision for
+ * n tokens, w_k, w_v [d][d]; cfg as for vnsa_create (n_max is ignored).
+ * Outputs (device, caller-owned): o_cmp [n][h_q][d] fp32, the ungated
+ * compression output of each vision token by vision rank; idx
+ * [h_kv][n][top_k], the selected blocks by vision rank, ascending, -1 padded.
+ * Rows N_v..n-1 of both are left untouched.
+ *
+ * Scratch: every intermediate lives in one 8 MiB array in device global
+ * memory that the library declares statically; each GPU that loads the library
+ * holds it until the process exits.  A call whose intermediates do not fit
+ * returns VNSA_ERR_UNSUPPORTED before launching anything (for 28/4 heads, d 128
+ * this allows about 5,000 tokens).  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls on a device share the
+ * one array and it keeps the previous call's contents, so calls that overlap
+ * on the GPU (different streams, or concurrent host threads) race and must be
+ * serialised by the caller.  Asynchronous on `stream` (a cudaStream_t).
+ */
+vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const void *q, const void *k,
+                                const void *v, const uint8_t *is_vision, const void *w_k,
+                                const void *w_v, float *o_cmp, int32_t *idx, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,8 @@ NUM_STAGES = 7
 
 EXPORTED = ("vnsa_status_string", "vnsa_stage_name", "vnsa_workspace_bytes", "vnsa_create",
             "vnsa_forward", "vnsa_forward_host", "vnsa_get_device_status", "vnsa_get_counts",
-            "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy")
+            "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy",
+            "vnsa_select_noalloc")
 
 
 class vnsa_config(ctypes.Structure):
@@ -75,6 +76,7 @@ def load(path: str = LIB_PATH):
     lib.vnsa_get_timing.argtypes = [P, ctypes.POINTER(ctypes.c_float)]
     lib.vnsa_get_launch_count.argtypes = [P, ctypes.POINTER(I)]
     lib.vnsa_destroy.argtypes = [P]
+    lib.vnsa_select_noalloc.argtypes = [ctypes.POINTER(vnsa_config), I, P, P, P, P, P, P, P, P, P]
     for name in EXPORTED:
         if name not in ("vnsa_status_string", "vnsa_stage_name"):
             getattr(lib, name).restype = I
@@ -148,6 +150,13 @@ def vnsa_get_launch_count(h) -> int:
 
 def vnsa_destroy(h):
     _check("vnsa_destroy", load().vnsa_destroy(h))
+
+
+def vnsa_select_noalloc(cfg: vnsa_config, n, q, k, v, is_vision, w_k, w_v, o_cmp, idx,
+                        stream=0):
+    """Selection chain with no device allocation (static library scratch)."""
+    _check("vnsa_select_noalloc", load().vnsa_select_noalloc(
+        ctypes.byref(cfg), n, q, k, v, is_vision, w_k, w_v, o_cmp, idx, stream))
 
 
 # --- torch-facing convenience -------------------------------------------------
