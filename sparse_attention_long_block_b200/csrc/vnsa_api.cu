@@ -259,8 +259,9 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
                               c.block, h->nb_max, s));
     end(VNSA_STAGE_POOL);
     if (use_tc) {
-        VNSA_RUN(tc_forward(h->tc, p, s, h->timing ? h->ev : nullptr, h->ran, &h->launches,
-                            forced));
+        // counts its own launches
+        if (e == cudaSuccess)
+            e = tc_forward(h->tc, p, s, h->timing ? h->ev : nullptr, h->ran, &h->launches, forced);
     } else {
         begin(VNSA_STAGE_CMP);
         VNSA_RUN(launch_cmp_simt(dt, p, s));
