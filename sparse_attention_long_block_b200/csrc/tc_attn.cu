@@ -70,9 +70,9 @@ enum Mode { MODE_CMP = 0, MODE_VIS = 1, MODE_TEXT = 2 };
 enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
 
 struct TcParams {
-    CUtensorMap tm_k, tm_v;    // original K, V: [n rows][h_kv*d]
-    CUtensorMap tm_kc, tm_vc;  // compacted vision K, V (used if not contiguous)
-    CUtensorMap tm_kb, tm_vb;  // K_cmp, V_cmp: [nb_max rows][h_kv*d]
+    CUtensorMap tm_k, tm_v;    // K (bf16, the caller's) and V (fp16 copy): [n rows][h_kv*d]
+    CUtensorMap tm_kc, tm_vc;  // compacted vision K (bf16), V (fp16), if not contiguous
+    CUtensorMap tm_kb, tm_vb;  // K_cmp (bf16), V_cmp (fp16): [nb_max rows][h_kv*d]
     LayerParams L;
     const int32_t *plan;       // VIS: [item][1 + 2*plan_max]
     int plan_max;
@@ -278,8 +278,10 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
 __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
-    constexpr uint32_t idesc_s = ptx::idesc_bf16(kRows, kKeys, 0, 0);
-    constexpr uint32_t idesc_pv = ptx::idesc_bf16(kRows, kD, 0, 1);
+    // S = Q K^T with bf16 operands; O += P V with fp16 operands (P and V in
+    // fp16: 11-bit significands keep the probability rounding small)
+    constexpr uint32_t idesc_s = ptx::idesc_f16kind(kRows, kKeys, 0, 0, 1u);
+    constexpr uint32_t idesc_pv = ptx::idesc_f16kind(kRows, kD, 0, 1, 0u);
     const uint32_t q_addr = sm.base_u32 + SM_Q;
     const uint32_t p_addr = sm.base_u32 + SM_P;
     uint32_t gt = 0, nitems = 0;
@@ -374,15 +376,17 @@ __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool
     ok = __all_sync(0xffffffffu, r && ok);
 }
 
-__device__ __forceinline__ void store_p_bf16(const Smem &sm, int rho, const float (&p)[64]) {
+// P row (fp16) into the 128-byte swizzled K-major layout: 16-byte chunk c8 of
+// row rho goes to chunk c8 ^ (rho % 8).
+__device__ __forceinline__ void store_p_f16(const Smem &sm, int rho, const float (&p)[64]) {
     uint8_t *row = sm.base + SM_P + rho * 128;
 #pragma unroll
     for (int c8 = 0; c8 < 8; ++c8) {
         uint4 v;
-        __nv_bfloat162 a = __floats2bfloat162_rn(p[8 * c8 + 0], p[8 * c8 + 1]);
-        __nv_bfloat162 b = __floats2bfloat162_rn(p[8 * c8 + 2], p[8 * c8 + 3]);
-        __nv_bfloat162 c = __floats2bfloat162_rn(p[8 * c8 + 4], p[8 * c8 + 5]);
-        __nv_bfloat162 d = __floats2bfloat162_rn(p[8 * c8 + 6], p[8 * c8 + 7]);
+        __half2 a = __floats2half2_rn(p[8 * c8 + 0], p[8 * c8 + 1]);
+        __half2 b = __floats2half2_rn(p[8 * c8 + 2], p[8 * c8 + 3]);
+        __half2 c = __floats2half2_rn(p[8 * c8 + 4], p[8 * c8 + 5]);
+        __half2 d = __floats2half2_rn(p[8 * c8 + 6], p[8 * c8 + 7]);
         v.x = *reinterpret_cast<uint32_t *>(&a);
         v.y = *reinterpret_cast<uint32_t *>(&b);
         v.z = *reinterpret_cast<uint32_t *>(&c);
@@ -579,7 +583,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     ok = __all_sync(0xffffffffu, r3 && ok);
                     if (!ok) break;
                 }
-                store_p_bf16(sm, rho, pv);
+                store_p_f16(sm, rho, pv);
                 ptx::fence_proxy_async();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(sm.bar(B_P_FULL + b));
@@ -766,22 +770,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Vision K/V in vision order when the vision tokens are not one contiguous run
-// of positions (the TMA tiles need consecutive rows).
-__global__ void compact_kv_kernel(LayerParams p, __nv_bfloat16 *kc, __nv_bfloat16 *vc) {
-    const Counts cn = *p.counts;
-    if (cn.contiguous) return;
-    const size_t row_vec = (size_t)p.h_kv * kD / 8;  // 16-byte pieces per row
-    const size_t total = (size_t)cn.n_vision * row_vec;
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const size_t u = e / row_vec, c = e % row_vec;
-        const size_t src = (size_t)p.vis[u] * row_vec + c;
-        reinterpret_cast<uint4 *>(kc)[u * row_vec + c] =
-            __ldg(reinterpret_cast<const uint4 *>(p.k) + src);
-        reinterpret_cast<uint4 *>(vc)[u * row_vec + c] =
-            __ldg(reinterpret_cast<const uint4 *>(p.v) + src);
+// Operand preparation for the tensor-core kernels:
+//  * fp16 copies of V (all positions) and of V_cmp for the P V products.  A
+//    bf16 value converts to fp16 exactly when its magnitude lies in the fp16
+//    normal range; a value beyond the fp16 range is reported as a bounds error.
+//  * vision K (bf16) and V (fp16) in vision order when the vision tokens are
+//    not one contiguous run of positions (the TMA tiles need consecutive rows).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u, bool &overflow) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    uint4 r;
+    __half2 *h = reinterpret_cast<__half2 *>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(b[i]);
+        h[i] = __floats2half2_rn(f.x, f.y);
+        if (fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f) overflow = true;
     }
+    return r;
+}
+
+__global__ void prepare_kernel(LayerParams p, __nv_bfloat16 *kc, __half *vhc, __half *vh,
+                               __half *vh_cmp) {
+    const Counts cn = *p.counts;
+    const size_t row_vec = (size_t)p.h_kv * kD / 8;  // 16-byte pieces per row
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t step = (size_t)gridDim.x * blockDim.x;
+    bool overflow = false;
+    const uint4 *v = reinterpret_cast<const uint4 *>(p.v);
+    for (size_t e = tid; e < (size_t)p.n * row_vec; e += step)
+        reinterpret_cast<uint4 *>(vh)[e] = bf16x8_to_f16x8(__ldg(v + e), overflow);
+    const uint4 *vb = reinterpret_cast<const uint4 *>(p.v_cmp);
+    for (size_t e = tid; e < (size_t)cn.nb * row_vec; e += step)
+        reinterpret_cast<uint4 *>(vh_cmp)[e] = bf16x8_to_f16x8(vb[e], overflow);
+    if (!cn.contiguous) {
+        for (size_t e = tid; e < (size_t)cn.n_vision * row_vec; e += step) {
+            const size_t u = e / row_vec, c = e % row_vec;
+            const size_t src = (size_t)p.vis[u] * row_vec + c;
+            reinterpret_cast<uint4 *>(kc)[e] = __ldg(reinterpret_cast<const uint4 *>(p.k) + src);
+            reinterpret_cast<uint4 *>(vhc)[e] = bf16x8_to_f16x8(__ldg(v + src), overflow);
+        }
+    }
+    if (overflow) report(p.status, VNSA_ERR_BOUNDS);
 }
 
 // ---------------------------------------------------------------------------
@@ -904,6 +933,15 @@ __global__ void text_combine_kernel(LayerParams p, const float *part, int part_i
     const int qt = kRows / p.r;
     const int n_tt = (cn.n_text + qt - 1) / qt;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    if (cn.n_text == 0) return;
+    {
+        // with a single key split the attention kernel wrote the rows itself
+        const int span = p.txt[cn.n_text - 1] + 1;
+        const int tiles = p.h_kv * n_tt;
+        const int ns = max(1, min((span + kTextSplitKeys - 1) / kTextSplitKeys,
+                                  max(1, part_items / tiles)));
+        if (ns == 1) return;
+    }
     for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < cn.n_text * p.h_q;
          wi += nwarps)
         text_combine_row(p, part, part_items, n_tt, qt, wi / p.h_q, wi % p.h_q, lane);
@@ -929,15 +967,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D map over [rows][h_kv*128] bf16 with 64 x 64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int h_kv, long long rows) {
+// 2-D map over [rows][h_kv*128] 16-bit elements with 64 x 64 boxes, 128-byte
+// swizzle.
+bool make_map(CUtensorMap *m, const void *base, int h_kv, long long rows, bool f16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || rows < 1) return false;
     cuuint64_t dims[2] = {(cuuint64_t)h_kv * kD, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)h_kv * kD * 2};
     cuuint32_t box[2] = {64, 64};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+    return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void *>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
@@ -952,7 +992,10 @@ struct TcState {
     int num_sms;
     int plan_max;
     int part_items;
-    __nv_bfloat16 *kc, *vc;
+    __nv_bfloat16 *kc;  // vision K in vision order (non-contiguous vision only)
+    __half *vhc;        // vision V (fp16) in vision order (non-contiguous vision only)
+    __half *vh;         // V in fp16, all positions
+    __half *vh_cmp;     // V_cmp in fp16
     int32_t *plan;
     float *part;
 };
@@ -971,7 +1014,8 @@ static size_t plan_bytes(const vnsa_config &c) {
 size_t tc_workspace_bytes(const vnsa_config &c) {
     if (c.dtype != VNSA_BF16 || c.d != kD || c.block != kKeys) return 0;
     const size_t kv = (size_t)c.n_max * c.h_kv * kD * 2;
-    return up256(kv) * 2 + up256(plan_bytes(c)) + kTextPartBytes;
+    const size_t kvb = (size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2;
+    return up256(kv) * 3 + up256(kvb) + up256(plan_bytes(c)) + kTextPartBytes;
 }
 
 cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
@@ -987,10 +1031,13 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     st->part_items = (int)(kTextPartBytes / ((size_t)kRows * kPartStride * 4));
     char *p = (char *)ws;
     const size_t kv = up256((size_t)c.n_max * c.h_kv * kD * 2);
+    const size_t kvb = up256((size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2);
     st->kc = (__nv_bfloat16 *)p;
-    st->vc = (__nv_bfloat16 *)(p + kv);
-    st->plan = (int32_t *)(p + 2 * kv);
-    st->part = (float *)(p + 2 * kv + up256(plan_bytes(c)));
+    st->vhc = (__half *)(p + kv);
+    st->vh = (__half *)(p + 2 * kv);
+    st->vh_cmp = (__half *)(p + 3 * kv);
+    st->plan = (int32_t *)(p + 3 * kv + kvb);
+    st->part = (float *)(p + 3 * kv + kvb + up256(plan_bytes(c)));
     cudaError_t e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) {
@@ -1013,11 +1060,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     P.part = st->part;
     P.part_items = st->part_items;
     const int nb_rows = c.n_max / c.block > 0 ? c.n_max / c.block : 1;
-    if (!make_map(&P.tm_k, L.k, c.h_kv, L.n) || !make_map(&P.tm_v, L.v, c.h_kv, L.n) ||
-        !make_map(&P.tm_kc, st->kc, c.h_kv, c.n_max) ||
-        !make_map(&P.tm_vc, st->vc, c.h_kv, c.n_max) ||
-        !make_map(&P.tm_kb, L.k_cmp, c.h_kv, nb_rows) ||
-        !make_map(&P.tm_vb, L.v_cmp, c.h_kv, nb_rows))
+    if (!make_map(&P.tm_k, L.k, c.h_kv, L.n, false) ||
+        !make_map(&P.tm_v, st->vh, c.h_kv, L.n, true) ||
+        !make_map(&P.tm_kc, st->kc, c.h_kv, c.n_max, false) ||
+        !make_map(&P.tm_vc, st->vhc, c.h_kv, c.n_max, true) ||
+        !make_map(&P.tm_kb, L.k_cmp, c.h_kv, nb_rows, false) ||
+        !make_map(&P.tm_vb, st->vh_cmp, c.h_kv, nb_rows, true))
         return cudaErrorInvalidValue;
     auto begin = [&](int stg) {
         if (ev) cudaEventRecord(ev[2 * stg], s);
@@ -1029,7 +1077,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     const int grid = st->num_sms;
     cudaError_t e;
     // compression (vision K/V compaction first, for the later window/selection)
-    compact_kv_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vc);
+    prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vhc, st->vh, st->vh_cmp);
     ++*launches;
     begin(VNSA_STAGE_CMP);
     P.mode = MODE_CMP;

@@ -192,12 +192,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation:
-// D format F32 (bit 4), A bf16 (bits 7-9 = 1), B bf16 (bits 10-12 = 1),
-// A/B major (bits 15/16: 0 K-major, 1 MN-major), N >> 3 at bit 17, M >> 4 at
-// bit 24.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
+// Instruction descriptor of kind::f16 with fp32 accumulation: D format F32
+// (bit 4), A and B format in bits 7-9 and 10-12 (0 = f16, 1 = bf16; both the
+// same type), A/B major (bits 15/16: 0 K-major, 1 MN-major), N >> 3 at bit 17,
+// M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int m, int n, int a_mn_major, int b_mn_major,
+                                                     uint32_t bf16) {
+    return (1u << 4) | (bf16 << 7) | (bf16 << 10) | ((uint32_t)a_mn_major << 15) |
            ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(m >> 4) << 24);
 }
