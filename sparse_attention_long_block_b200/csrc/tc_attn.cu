@@ -53,16 +53,19 @@ constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
 constexpr uint32_t SM_KV = 32768;                             // stages x (K, V)
 constexpr uint32_t KV_BYTES = 32768;
-constexpr uint32_t SM_P = SM_KV + kStages * KV_BYTES;         // [128][64] bf16
-constexpr uint32_t SM_P32 = SM_P + 16384;                     // [128][65] fp32
+constexpr uint32_t SM_P = SM_KV + kStages * KV_BYTES;         // 2 x [128][64] fp16
+constexpr uint32_t P_BYTES = 16384;
+constexpr uint32_t SM_P32 = SM_P + 2 * P_BYTES;               // [128][65] fp32
 constexpr uint32_t P32_STRIDE = 65;
-constexpr uint32_t SM_BAR = SM_P32 + kRows * P32_STRIDE * 4;  // barriers
+constexpr int kPlanSmem = 1152;                               // selection tiles per item
+constexpr uint32_t SM_PLAN = SM_P32 + kRows * P32_STRIDE * 4; // [2][kPlanSmem] int32
+constexpr uint32_t SM_BAR = SM_PLAN + 2 * kPlanSmem * 4;      // barriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment slack
 
 // barrier slots (8 bytes each) after SM_BAR
 constexpr int B_KV_FULL = 0, B_KV_EMPTY = 3, B_S_FULL = 6, B_P_FULL = 8, B_PV_DONE = 10,
-              B_Q_FULL = 11, B_GRP = 12, B_FINAL = 13, B_COUNT = 14;
+              B_Q_FULL = 12, B_GRP = 13, B_FINAL = 14, B_COUNT = 15;
 
 constexpr uint32_t TM_S0 = 0, TM_O0 = 128, TM_O1 = 256, TM_COLS = 512;
 
@@ -283,8 +286,8 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
     constexpr uint32_t idesc_s = ptx::idesc_f16kind(kRows, kKeys, 0, 0, 1u);
     constexpr uint32_t idesc_pv = ptx::idesc_f16kind(kRows, kD, 0, 1, 0u);
     const uint32_t q_addr = sm.base_u32 + SM_Q;
-    const uint32_t p_addr = sm.base_u32 + SM_P;
     uint32_t gt = 0, nitems = 0;
+    uint32_t npv = 0;  // P V products issued; P buffer and PV-done barrier = npv & 1
     bool ok = true;
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
@@ -321,13 +324,15 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
                                         L.status)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t vb = sm.base_u32 + SM_KV + pend_st * KV_BYTES + 16384;
+                    const uint32_t pa = sm.base_u32 + SM_P + (npv & 1) * P_BYTES;
 #pragma unroll
                     for (int k = 0; k < kKeys / 16; ++k)
-                        ptx::mma_ss(tmem + pend_col, desc_kmajor(p_addr + (uint32_t)k * 32u),
+                        ptx::mma_ss(tmem + pend_col, desc_kmajor(pa + (uint32_t)k * 32u),
                                     desc_vmajor(vb + (uint32_t)k * 2048u), idesc_pv,
                                     (k > 0 || pend_acc) ? 1u : 0u);
-                    ptx::mma_commit(sm.bar(B_PV_DONE));
+                    ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
                     ptx::mma_commit(sm.bar(B_KV_EMPTY + pend_st));
+                    ++npv;
                     pending = false;
                 }
                 if (kind_has_pv(kind)) {
@@ -344,13 +349,15 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
                                 L.status)) { ok = false; break; }
             ptx::tc_fence_after();
             const uint32_t vb = sm.base_u32 + SM_KV + pend_st * KV_BYTES + 16384;
+            const uint32_t pa = sm.base_u32 + SM_P + (npv & 1) * P_BYTES;
 #pragma unroll
             for (int k = 0; k < kKeys / 16; ++k)
-                ptx::mma_ss(tmem + pend_col, desc_kmajor(p_addr + (uint32_t)k * 32u),
+                ptx::mma_ss(tmem + pend_col, desc_kmajor(pa + (uint32_t)k * 32u),
                             desc_vmajor(vb + (uint32_t)k * 2048u), idesc_pv,
                             (k > 0 || pend_acc) ? 1u : 0u);
-            ptx::mma_commit(sm.bar(B_PV_DONE));
+            ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
             ptx::mma_commit(sm.bar(B_KV_EMPTY + pend_st));
+            ++npv;
         }
     }
     // every MMA this thread issued has completed once this barrier flips
@@ -378,8 +385,9 @@ __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool
 
 // P row (fp16) into the 128-byte swizzled K-major layout: 16-byte chunk c8 of
 // row rho goes to chunk c8 ^ (rho % 8).
-__device__ __forceinline__ void store_p_f16(const Smem &sm, int rho, const float (&p)[64]) {
-    uint8_t *row = sm.base + SM_P + rho * 128;
+__device__ __forceinline__ void store_p_f16(const Smem &sm, uint32_t buf, int rho,
+                                            const float (&p)[64]) {
+    uint8_t *row = sm.base + SM_P + buf * P_BYTES + rho * 128;
 #pragma unroll
     for (int c8 = 0; c8 < 8; ++c8) {
         uint4 v;
@@ -453,35 +461,51 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         ptx::fence_proxy_async();
         ptx::mbar_arrive(sm.bar(B_Q_FULL));
 
+        // VIS: the item's selection tiles (first key, query mask) into shared
+        // memory, once every thread is done with the previous item's copy
+        const int32_t *plan_s = (const int32_t *)(sm.base + SM_PLAN);
+        if (P.mode == MODE_VIS) {
+            group_sync(sm, gphase, ok, L);
+            if (!ok) break;
+            int32_t *dst = (int32_t *)(sm.base + SM_PLAN);
+            const int32_t *src = P.plan + (size_t)item * (1 + 2 * P.plan_max);
+            for (int x = rho; x < it.seg_tiles[0]; x += 128) {
+                dst[x] = src[1 + x] * kKeys;
+                dst[kPlanSmem + x] = src[1 + P.plan_max + x];
+            }
+            group_sync(sm, gphase, ok, L);
+            if (!ok) break;
+        }
+
         float lse2 = -INFINITY;                 // CMP: from the stats segment
         float m_s = -INFINITY, l_s = 0.f;       // segment 0 running max / sum
         float l_w = 0.f;                        // segment 1 (VIS window) sum
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
             float m_run = -INFINITY, l_run = 0.f;
-            uint32_t qmask_bit = 0;
             const uint32_t ocol = (kind == K_SWA) ? TM_O1 : TM_O0;
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
                 const uint32_t b = gt & 1;
-                const int key0 = tile_key0(P, it, item, kind, x);
+                const int key0 = kind == K_SLC ? plan_s[x] : tile_key0(P, it, item, kind, x);
                 // column range [lo, hi] of valid keys for this row
                 int lo = 1, hi = 0;
                 if (rc.valid) {
                     switch (kind) {
                         case K_STATS:
                         case K_EXACT: lo = 0; hi = rc.c_vis - 1 - key0; break;
-                        case K_SLC: {
-                            qmask_bit = (uint32_t)P.plan[(size_t)item * (1 + 2 * P.plan_max) + 1 +
-                                                         P.plan_max + x];
-                            if ((qmask_bit >> rc.qi) & 1u) { lo = 0; hi = rc.i - key0; }
+                        case K_SLC:
+                            if (((uint32_t)plan_s[kPlanSmem + x] >> rc.qi) & 1u) {
+                                lo = 0;
+                                hi = rc.i - key0;
+                            }
                             break;
-                        }
                         case K_SWA: lo = rc.i - L.window + 1 - key0; hi = rc.i - key0; break;
                         default: lo = 0; hi = rc.t - key0; break;
                     }
                     lo = max(lo, 0);
                     hi = min(hi, kKeys - 1);
                 }
+                const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kKeys - 1);
                 bool r = ptx::mbar_wait(sm.bar(B_S_FULL + b), (gt >> 1) & 1, abort, L.status);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
@@ -495,18 +519,31 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
 #pragma unroll
                     for (int k = 0; k < 32; ++k) { sv[k] = a[k]; sv[32 + k] = c[k]; }
                 }
-                float mx = -INFINITY;
+                if (full) {
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    sv[k] = (k >= lo && k <= hi) ? sv[k] * sc : -INFINITY;
-                    mx = fmaxf(mx, sv[k]);
+                    for (int k = 0; k < 64; ++k) sv[k] *= sc;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] * sc : -INFINITY;
+                }
+                float mx;
+                {
+                    float m8[8];
+#pragma unroll
+                    for (int z = 0; z < 8; ++z) m8[z] = sv[z];
+#pragma unroll
+                    for (int k = 8; k < 64; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
+                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
                 }
                 if (kind == K_STATS) {
                     const float mn = fmaxf(m_run, mx);
                     const float mu = mn == -INFINITY ? 0.f : mn;
-                    float acc = 0.f;
+                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) acc += ptx::ex2(sv[k] - mu);
+                    for (int k = 0; k < 64; ++k) a8[k & 7] += ptx::ex2(sv[k] - mu);
+                    const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) +
+                                      ((a8[4] + a8[5]) + (a8[6] + a8[7]));
                     l_run = l_run * ptx::ex2(m_run - mu) + acc;
                     m_run = mn;
                     ptx::tc_fence_before();
@@ -548,18 +585,19 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                         m_run = mn;
                     }
                     const float mu = m_run == -INFINITY ? 0.f : m_run;
-                    float acc = 0.f;
+                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int k = 0; k < 64; ++k) {
                         pv[k] = ptx::ex2(sv[k] - mu);
-                        acc += pv[k];
+                        a8[k & 7] += pv[k];
                     }
-                    l_run += acc;
+                    l_run += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
                     const bool resc = __any_sync(0xffffffffu, need && x > 0);
                     if (resc) {
+                        // O may only be rescaled once every earlier P V has landed
                         if (npv > 0) {
-                            bool r2 = ptx::mbar_wait(sm.bar(B_PV_DONE), (npv - 1) & 1, abort,
-                                                     L.status);
+                            bool r2 = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)),
+                                                     ((npv - 1) >> 1) & 1, abort, L.status);
                             ok = __all_sync(0xffffffffu, r2 && ok);
                             if (!ok) break;
                         }
@@ -577,13 +615,14 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                         ptx::tmem_wait_st();
                     }
                 }
-                // P into shared memory once the previous P V has consumed it
-                if (npv > 0) {
-                    bool r3 = ptx::mbar_wait(sm.bar(B_PV_DONE), (npv - 1) & 1, abort, L.status);
+                // P into buffer npv & 1 once the P V that last read it (#npv-2) is done
+                if (npv > 1) {
+                    bool r3 = ptx::mbar_wait(sm.bar(B_PV_DONE + (npv & 1)), ((npv - 2) >> 1) & 1,
+                                             abort, L.status);
                     ok = __all_sync(0xffffffffu, r3 && ok);
                     if (!ok) break;
                 }
-                store_p_f16(sm, rho, pv);
+                store_p_f16(sm, npv & 1, rho, pv);
                 ptx::fence_proxy_async();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(sm.bar(B_P_FULL + b));
@@ -600,9 +639,10 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             }
         }
         if (!ok) break;
-        // ---- epilogue: wait for the item's last P V
+        // ---- epilogue: wait for the item's last P V (#npv-1)
         {
-            bool r = ptx::mbar_wait(sm.bar(B_PV_DONE), (npv - 1) & 1, abort, L.status);
+            bool r = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)), ((npv - 1) >> 1) & 1,
+                                    abort, L.status);
             ok = __all_sync(0xffffffffu, r && ok);
             if (!ok) break;
             ptx::tc_fence_after();
@@ -736,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             ptx::mbar_init(sm.bar(B_P_FULL + b), 128);
         }
         ptx::mbar_init(sm.bar(B_PV_DONE), 1);
+        ptx::mbar_init(sm.bar(B_PV_DONE + 1), 1);
         ptx::mbar_init(sm.bar(B_Q_FULL), 128);
         ptx::mbar_init(sm.bar(B_GRP), 128);
         ptx::mbar_init(sm.bar(B_FINAL), 1);
@@ -1001,8 +1042,9 @@ struct TcState {
 };
 
 bool tc_supported(const vnsa_config &c) {
+    const int qt = kRows / (c.h_q / c.h_kv);
     return c.dtype == VNSA_BF16 && c.d == kD && c.block == kKeys && c.h_q / c.h_kv <= 16 &&
-           encode_fn() != nullptr;
+           qt * c.top_k <= kPlanSmem && encode_fn() != nullptr;
 }
 
 static size_t plan_bytes(const vnsa_config &c) {
