@@ -1,5 +1,5 @@
 // tc_attn.cu -- tensor-core path of the bf16 layer prefill (head dim 128):
-// compression attention + importance, selection + sliding window + gate, and
+// compression attention + importance, selection, sliding window + gate, and
 // dense text GQA, on tcgen05 MMAs with TMEM accumulators fed by TMA.
 //
 // Method: "VideoNSA: Native Sparse Attention Scales Video Understanding" (paper
@@ -7,28 +7,28 @@
 // selection and a sliding window mixed by per-head sigmoid gates; text tokens
 // attend densely (GQA).
 //
-// One persistent kernel template serves three modes.  A CTA (8 warps, one per
-// SM) walks work items; an item is an M tile of 128 MMA rows, row = (query,
-// head of one GQA group): 128 / (h_q/h_kv) consecutive queries times the
-// group's heads, so the heads of a group share every K/V tile (18 queries x 7
-// heads = 126 rows for 28/4 heads).  Per item the CTA streams 64-key tiles:
-//   warp 0   TMA loads of K (and V) tiles into a 3-stage ring;
-//   warp 1   one thread issues S = Q K^T (M 128, N 64, K 128) into one of two
-//            TMEM S buffers, then O += P V (M 128, N 128, K 64) into TMEM;
-//   warps 4-7  one thread per row: S row from TMEM, mask, softmax, P (bf16)
-//            into shared memory in the 128-byte swizzled K-major layout,
-//            lazy O rescaling, epilogue.
+// One persistent kernel serves four modes; two CTAs share each SM so that one
+// CTA's softmax overlaps the other's tensor-core work.  A CTA (6 warps) walks
+// work items; an item is an M tile of 128 MMA rows, row = (query, head of one
+// GQA group): consecutive queries times the group's heads, so every K/V tile
+// serves the whole group.  Per item the CTA streams 64-key tiles:
+//   warp 0     TMA loads of K (and V) tiles into a 2-stage ring;
+//   warp 1     one thread issues S = Q K^T (M 128, N 64, K 128, bf16) into TMEM
+//              and O += P V (M 128, N 128, K 64, fp16, P read from TMEM);
+//   warps 2-5  one thread per row: S row from TMEM (released at once so the
+//              next S overlaps), mask, softmax, P (fp16) into TMEM, lazy O
+//              rescaling, epilogue.
 // Modes:
-//   CMP   items over vision queries; keys = compressed blocks (K_cmp, V_cmp).
-//         Segment 1 computes each row's log-sum-exp; segment 2 recomputes S,
-//         forms exact probabilities, sums them over the group's heads into
-//         the block importance, and accumulates O = P V (already normalised).
-//   VIS   items over vision queries; segment 1 = the union of the blocks the
-//         item's queries selected (a query's row masks blocks it did not
-//         select), segment 2 = the window keys; the epilogue adds the three
-//         gated branch outputs and writes the final vision rows.
-//   TEXT  items = (text query tile, key split); partial O, max and sum go to a
-//         buffer that a small combine kernel reduces.
+//   CMP   keys = compressed blocks.  Segment 1: each row's log-sum-exp.
+//         Segment 2: exact probabilities, their sum over the group's heads
+//         (the block importance, a warp reduce-scatter: rows are 16 queries x
+//         8 head slots) and O = P V, already normalised.
+//   SLC   the union of the blocks the item's queries selected; a row masks the
+//         blocks its query did not select.  Epilogue: partial = sig(g_cmp) o_cmp
+//         + sig(g_slc) o_slc, kept in fp32 in the workspace.
+//   SWA   the window keys; epilogue: out = partial + sig(g_swa) o_swa (bf16).
+//   TEXT  items = (text query tile, key split); partial O, max and sum to a
+//         buffer that a small combine kernel reduces (or the row directly).
 #include <cuda.h>
 #include <math.h>
 #include <string.h>
@@ -40,11 +40,11 @@ namespace vnsa {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 192;
 constexpr int kRows = 128;        // MMA M
 constexpr int kKeys = 64;         // keys per tile
 constexpr int kD = 128;           // head dim of this path
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 constexpr int kTextSplitKeys = 8192;
 constexpr size_t kTextPartBytes = 256ull << 20;
@@ -53,23 +53,20 @@ constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
 constexpr uint32_t SM_KV = 32768;                             // stages x (K, V)
 constexpr uint32_t KV_BYTES = 32768;
-constexpr uint32_t SM_P = SM_KV + kStages * KV_BYTES;         // 2 x [128][64] fp16
-constexpr uint32_t P_BYTES = 16384;
-constexpr uint32_t SM_P32 = SM_P + 2 * P_BYTES;               // [128][65] fp32
-constexpr uint32_t P32_STRIDE = 65;
 constexpr int kPlanSmem = 1152;                               // selection tiles per item
-constexpr uint32_t SM_PLAN = SM_P32 + kRows * P32_STRIDE * 4; // [2][kPlanSmem] int32
+constexpr uint32_t SM_PLAN = SM_KV + kStages * KV_BYTES;      // [2][kPlanSmem] int32
 constexpr uint32_t SM_BAR = SM_PLAN + 2 * kPlanSmem * 4;      // barriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment slack
 
 // barrier slots (8 bytes each) after SM_BAR
-constexpr int B_KV_FULL = 0, B_KV_EMPTY = 3, B_S_FULL = 6, B_P_FULL = 8, B_PV_DONE = 10,
-              B_Q_FULL = 12, B_GRP = 13, B_FINAL = 14, B_COUNT = 15;
+constexpr int B_KV_FULL = 0, B_KV_EMPTY = 2, B_S_FULL = 4, B_S_FREE = 5, B_P_FULL = 6,
+              B_PV_DONE = 8, B_Q_FULL = 10, B_GRP = 11, B_FINAL = 12, B_COUNT = 13;
 
-constexpr uint32_t TM_S0 = 0, TM_O0 = 128, TM_O1 = 256, TM_COLS = 512;
+// TMEM columns: S (fp32, 64), P buffers (fp16 pairs, 32 each), O (fp32, 128)
+constexpr uint32_t TM_S = 0, TM_P = 64, TM_O = 128, TM_COLS = 256;
 
-enum Mode { MODE_CMP = 0, MODE_VIS = 1, MODE_TEXT = 2 };
+enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3 };
 enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
 
 struct TcParams {
@@ -77,18 +74,24 @@ struct TcParams {
     CUtensorMap tm_kc, tm_vc;  // compacted vision K (bf16), V (fp16), if not contiguous
     CUtensorMap tm_kb, tm_vb;  // K_cmp (bf16), V_cmp (fp16): [nb_max rows][h_kv*d]
     LayerParams L;
-    const int32_t *plan;       // VIS: [item][1 + 2*plan_max]
+    const int32_t *plan;       // SLC: [item][1 + 2*plan_max]
     int plan_max;
     float *part;               // TEXT partials: [item][128][kPartStride]
     int part_items;
     int mode;
 };
 
+__host__ __device__ __forceinline__ int pow2_at_least(int r) {
+    int p = 1;
+    while (p < r) p <<= 1;
+    return p;
+}
+
 // ---------------------------------------------------------------------------
 // Work decomposition shared by every role (all compute the same values).
 struct Work {
+    int rpad;      // MMA rows per query (>= heads per group)
     int qt;        // queries per item
-    int rows;      // used MMA rows = qt * r
     int n_q;       // queries of the item kind (N_v or N_t)
     int n_tiles_q; // query tiles per group
     int nsplit;    // text key splits
@@ -101,8 +104,8 @@ struct Work {
 __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
     Work w;
     const LayerParams &L = P.L;
-    w.qt = kRows / L.r;
-    w.rows = w.qt * L.r;
+    w.rpad = P.mode == MODE_CMP ? pow2_at_least(L.r) : L.r;
+    w.qt = kRows / w.rpad;
     w.nb = cn.nb;
     w.contiguous = cn.contiguous;
     w.vis_base = cn.vis_base;
@@ -129,12 +132,10 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
 
 struct Item {
     int g, q0, nq, split;
-    int last_pos;   // TEXT: position of the item's last query; else its vision rank
     int nseg;
     int seg_kind[2];
     int seg_tiles[2];
-    int key_lo;     // VIS window start (vision rank) / TEXT split start (position)
-    int key_hi;     // VIS: last query rank; TEXT: last key (inclusive)
+    int key_lo;     // SWA window start (vision rank) / TEXT split start (position)
 };
 
 __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int item) {
@@ -156,34 +157,31 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     it.nq = min(w.qt, w.n_q - it.q0);
     const int ql = it.q0 + it.nq - 1;
     it.key_lo = 0;
-    it.key_hi = 0;
+    it.seg_tiles[1] = 0;
+    it.seg_kind[1] = K_EXACT;
     if (P.mode == MODE_CMP) {
-        it.last_pos = ql;
         const int c_last = min((ql + 1) / L.block, w.nb);
         const int t = (c_last + kKeys - 1) / kKeys;
         it.nseg = 2;
         it.seg_kind[0] = K_STATS;
-        it.seg_kind[1] = K_EXACT;
         it.seg_tiles[0] = t;
         it.seg_tiles[1] = t;
-    } else if (P.mode == MODE_VIS) {
-        it.last_pos = ql;
-        it.nseg = 2;
+    } else if (P.mode == MODE_SLC) {
+        it.nseg = 1;
         it.seg_kind[0] = K_SLC;
-        it.seg_kind[1] = K_SWA;
         it.seg_tiles[0] = P.plan[(size_t)item * (1 + 2 * P.plan_max)];
+    } else if (P.mode == MODE_SWA) {
+        it.nseg = 1;
+        it.seg_kind[0] = K_SWA;
         it.key_lo = max(0, it.q0 - L.window + 1);
-        it.key_hi = ql;
-        it.seg_tiles[1] = (ql - it.key_lo + kKeys) / kKeys;
+        it.seg_tiles[0] = (ql - it.key_lo + kKeys) / kKeys;
     } else {
-        it.last_pos = L.txt[ql];
+        const int last_pos = L.txt[ql];
         it.nseg = 1;
         it.seg_kind[0] = K_TEXT;
-        it.seg_kind[1] = K_TEXT;
         it.key_lo = it.split * w.split_len;
-        it.key_hi = min(it.key_lo + w.split_len, it.last_pos + 1) - 1;
-        it.seg_tiles[0] = it.key_hi >= it.key_lo ? (it.key_hi - it.key_lo + kKeys) / kKeys : 0;
-        it.seg_tiles[1] = 0;
+        const int key_hi = min(it.key_lo + w.split_len, last_pos + 1) - 1;
+        it.seg_tiles[0] = key_hi >= it.key_lo ? (key_hi - it.key_lo + kKeys) / kKeys : 0;
     }
     return it;
 }
@@ -194,18 +192,6 @@ __device__ __forceinline__ int item_tiles(const Item &it) {
 
 __device__ __forceinline__ bool kind_has_pv(int kind) { return kind != K_STATS; }
 
-// First key of tile x of a segment: a vision rank (SLC, SWA), a compressed
-// block (STATS, EXACT) or a position (TEXT).
-__device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int item, int kind,
-                                         int x) {
-    switch (kind) {
-        case K_SLC: return P.plan[(size_t)item * (1 + 2 * P.plan_max) + 1 + x] * kKeys;
-        case K_SWA: return it.key_lo + x * kKeys;
-        case K_TEXT: return it.key_lo + x * kKeys;
-        default: return x * kKeys;
-    }
-}
-
 // ---------------------------------------------------------------------------
 struct Smem {
     uint8_t *base;
@@ -214,6 +200,9 @@ struct Smem {
     __device__ uint32_t *tmem_slot() const { return (uint32_t *)(base + SM_BAR + 8 * B_COUNT); }
     __device__ volatile int *abort_flag() const {
         return (volatile int *)(base + SM_BAR + 8 * B_COUNT + 8);
+    }
+    __device__ uint32_t *failed_flag() const {
+        return (uint32_t *)(base + SM_BAR + 8 * B_COUNT + 16);
     }
 };
 
@@ -224,27 +213,36 @@ __device__ __forceinline__ uint64_t desc_vmajor(uint32_t addr) {
     return ptx::sdesc_sw128(addr, 8192, 1024);
 }
 
+// First key of tile x: a vision rank (SLC, SWA), a compressed block (STATS,
+// EXACT) or a position (TEXT).  SLC reads the item's plan.
+__device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int item, int kind,
+                                         int x) {
+    switch (kind) {
+        case K_SLC: return P.plan[(size_t)item * (1 + 2 * P.plan_max) + 1 + x] * kKeys;
+        case K_SWA:
+        case K_TEXT: return it.key_lo + x * kKeys;
+        default: return x * kKeys;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Producer: TMA loads of the K (and V) tiles of every item, in order.
 __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
     uint32_t gt = 0;
-    const CUtensorMap *mk, *mv;
+    const CUtensorMap *mk = &P.tm_k, *mv = &P.tm_v;
+    int vbase = 0;
+    if (P.mode == MODE_CMP) {
+        mk = &P.tm_kb;
+        mv = &P.tm_vb;
+    } else if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+        mk = w.contiguous ? &P.tm_k : &P.tm_kc;
+        mv = w.contiguous ? &P.tm_v : &P.tm_vc;
+        vbase = w.contiguous ? w.vis_base : 0;
+    }
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
-        int vbase = 0;
-        if (P.mode == MODE_CMP) {
-            mk = &P.tm_kb;
-            mv = &P.tm_vb;
-        } else if (P.mode == MODE_VIS) {
-            mk = w.contiguous ? &P.tm_k : &P.tm_kc;
-            mv = w.contiguous ? &P.tm_v : &P.tm_vc;
-            vbase = w.contiguous ? w.vis_base : 0;
-        } else {
-            mk = &P.tm_k;
-            mv = &P.tm_v;
-        }
         for (int s = 0; s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
@@ -268,7 +266,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
             }
         }
     }
-    // make sure no load is still landing in shared memory when the CTA ends
+    // no load may still be landing in shared memory when the CTA ends
     for (uint32_t back = 1; back <= (uint32_t)kStages && back <= gt; ++back) {
         const uint32_t t = gt - back;
         if (!ptx::mbar_wait(sm.bar(B_KV_FULL + t % kStages), (t / kStages) & 1, abort, L.status))
@@ -281,14 +279,28 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
 __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
-    // S = Q K^T with bf16 operands; O += P V with fp16 operands (P and V in
-    // fp16: 11-bit significands keep the probability rounding small)
+    // S = Q K^T: bf16 operands, both K-major.  O += P V: fp16 operands, P from
+    // TMEM, V as an MN-major shared-memory operand.
     constexpr uint32_t idesc_s = ptx::idesc_f16kind(kRows, kKeys, 0, 0, 1u);
     constexpr uint32_t idesc_pv = ptx::idesc_f16kind(kRows, kD, 0, 1, 0u);
     const uint32_t q_addr = sm.base_u32 + SM_Q;
-    uint32_t gt = 0, nitems = 0;
-    uint32_t npv = 0;  // P V products issued; P buffer and PV-done barrier = npv & 1
+    uint32_t gt = 0, nitems = 0, npv = 0;
     bool ok = true;
+    auto issue_pv = [&](uint32_t pst, uint32_t acc) -> bool {
+        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (npv & 1)), (npv >> 1) & 1, abort, L.status))
+            return false;
+        ptx::tc_fence_after();
+        const uint32_t vb = sm.base_u32 + SM_KV + pst * KV_BYTES + 16384;
+        const uint32_t pa = tmem + TM_P + (npv & 1) * 32;
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k)
+            ptx::mma_ts(tmem + TM_O, pa + (uint32_t)k * 8u, desc_vmajor(vb + (uint32_t)k * 2048u),
+                        idesc_pv, (k > 0 || acc) ? 1u : 0u);
+        ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
+        ptx::mma_commit(sm.bar(B_KV_EMPTY + pst));
+        ++npv;
+        return true;
+    };
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
         if (item_tiles(it) == 0) continue;
@@ -296,15 +308,13 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         ++nitems;
         ptx::tc_fence_after();
         bool pending = false;
-        uint32_t pend_st = 0, pend_col = 0, pend_acc = 0, pend_gt = 0;
+        uint32_t pend_st = 0, pend_acc = 0;
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
-            const uint32_t ocol = (kind == K_SWA) ? TM_O1 : TM_O0;
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
-                const uint32_t st = gt % kStages, b = gt & 1;
-                if (gt >= 2 && !ptx::mbar_wait(sm.bar(B_P_FULL + b), ((gt - 2) >> 1) & 1, abort,
-                                               L.status)) { ok = false; break; }
-                if (!ptx::mbar_wait(sm.bar(B_KV_FULL + st), (gt / kStages) & 1, abort, L.status)) {
+                const uint32_t st = gt % kStages;
+                if (!ptx::mbar_wait(sm.bar(B_KV_FULL + st), (gt / kStages) & 1, abort, L.status) ||
+                    (gt > 0 && !ptx::mbar_wait(sm.bar(B_S_FREE), (gt - 1) & 1, abort, L.status))) {
                     ok = false;
                     break;
                 }
@@ -314,51 +324,23 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t off = (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u;
                     const uint32_t koff = (uint32_t)(k >> 2) * 8192u + (uint32_t)(k & 3) * 32u;
-                    ptx::mma_ss(tmem + TM_S0 + b * kKeys, desc_kmajor(q_addr + off),
-                                desc_kmajor(kv + koff), idesc_s, k > 0 ? 1u : 0u);
+                    ptx::mma_ss(tmem + TM_S, desc_kmajor(q_addr + off), desc_kmajor(kv + koff),
+                                idesc_s, k > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(sm.bar(B_S_FULL + b));
+                ptx::mma_commit(sm.bar(B_S_FULL));
                 if (!kind_has_pv(kind)) ptx::mma_commit(sm.bar(B_KV_EMPTY + st));
                 if (pending) {
-                    if (!ptx::mbar_wait(sm.bar(B_P_FULL + (pend_gt & 1)), (pend_gt >> 1) & 1, abort,
-                                        L.status)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t vb = sm.base_u32 + SM_KV + pend_st * KV_BYTES + 16384;
-                    const uint32_t pa = sm.base_u32 + SM_P + (npv & 1) * P_BYTES;
-#pragma unroll
-                    for (int k = 0; k < kKeys / 16; ++k)
-                        ptx::mma_ss(tmem + pend_col, desc_kmajor(pa + (uint32_t)k * 32u),
-                                    desc_vmajor(vb + (uint32_t)k * 2048u), idesc_pv,
-                                    (k > 0 || pend_acc) ? 1u : 0u);
-                    ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
-                    ptx::mma_commit(sm.bar(B_KV_EMPTY + pend_st));
-                    ++npv;
+                    if (!issue_pv(pend_st, pend_acc)) { ok = false; break; }
                     pending = false;
                 }
                 if (kind_has_pv(kind)) {
                     pending = true;
                     pend_st = st;
-                    pend_col = ocol;
                     pend_acc = x > 0 ? 1u : 0u;
-                    pend_gt = gt;
                 }
             }
         }
-        if (ok && pending) {
-            if (!ptx::mbar_wait(sm.bar(B_P_FULL + (pend_gt & 1)), (pend_gt >> 1) & 1, abort,
-                                L.status)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const uint32_t vb = sm.base_u32 + SM_KV + pend_st * KV_BYTES + 16384;
-            const uint32_t pa = sm.base_u32 + SM_P + (npv & 1) * P_BYTES;
-#pragma unroll
-            for (int k = 0; k < kKeys / 16; ++k)
-                ptx::mma_ss(tmem + pend_col, desc_kmajor(pa + (uint32_t)k * 32u),
-                            desc_vmajor(vb + (uint32_t)k * 2048u), idesc_pv,
-                            (k > 0 || pend_acc) ? 1u : 0u);
-            ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
-            ptx::mma_commit(sm.bar(B_KV_EMPTY + pend_st));
-            ++npv;
-        }
+        if (ok && pending && !issue_pv(pend_st, pend_acc)) ok = false;
     }
     // every MMA this thread issued has completed once this barrier flips
     ptx::mma_commit(sm.bar(B_FINAL));
@@ -366,13 +348,13 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
 }
 
 // ---------------------------------------------------------------------------
-// Softmax / epilogue warpgroup (warps 4-7): thread rho owns MMA row rho.
+// Softmax / epilogue warps 2-5: thread rho owns MMA row rho = TMEM lane rho.
 struct RowCtx {
     bool valid;
     int qi, hl, h;
-    int i;      // vision rank (CMP/VIS) or text rank (TEXT)
+    int i;      // vision rank (CMP/SLC/SWA) or text rank (TEXT)
     int t;      // position of the query token
-    int c_vis;  // CMP: visible compressed blocks
+    int c_vis;  // visible compressed blocks
 };
 
 __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool &ok,
@@ -383,61 +365,89 @@ __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool
     ok = __all_sync(0xffffffffu, r && ok);
 }
 
-// P row (fp16) into the 128-byte swizzled K-major layout: 16-byte chunk c8 of
-// row rho goes to chunk c8 ^ (rho % 8).
-__device__ __forceinline__ void store_p_f16(const Smem &sm, uint32_t buf, int rho,
-                                            const float (&p)[64]) {
-    uint8_t *row = sm.base + SM_P + buf * P_BYTES + rho * 128;
+// Block importance of one S tile: the sum over the RPAD rows (head slots) of a
+// query of its 64 probabilities, as a reduce-scatter across the RPAD lanes
+// that hold the query's rows: each lane ends with 64/RPAD consecutive column
+// sums starting at column `first`.
+template <int RPAD>
+__device__ __forceinline__ void imp_reduce_store(float (&p)[64], int lane, float *irow, int lim) {
+    int first = 0;
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-        uint4 v;
-        __half2 a = __floats2half2_rn(p[8 * c8 + 0], p[8 * c8 + 1]);
-        __half2 b = __floats2half2_rn(p[8 * c8 + 2], p[8 * c8 + 3]);
-        __half2 c = __floats2half2_rn(p[8 * c8 + 4], p[8 * c8 + 5]);
-        __half2 d = __floats2half2_rn(p[8 * c8 + 6], p[8 * c8 + 7]);
-        v.x = *reinterpret_cast<uint32_t *>(&a);
-        v.y = *reinterpret_cast<uint32_t *>(&b);
-        v.z = *reinterpret_cast<uint32_t *>(&c);
-        v.w = *reinterpret_cast<uint32_t *>(&d);
-        *reinterpret_cast<uint4 *>(row + ((c8 ^ (rho & 7)) << 4)) = v;
+    for (int sh = RPAD / 2, width = 32; sh >= 1; sh >>= 1, width >>= 1) {
+        const bool upper = (lane & sh) != 0;
+#pragma unroll
+        for (int c = 0; c < width; ++c) {
+            const float mine = upper ? p[width + c] : p[c];
+            const float other = upper ? p[c] : p[width + c];
+            p[c] = mine + __shfl_xor_sync(0xffffffffu, other, sh);
+        }
+        if (upper) first += width;
+    }
+    // columns [first, first + 64/RPAD) of the tile, valid below lim
+    constexpr int kCnt = 64 / RPAD;
+    if (irow == nullptr) return;
+    if (first + kCnt <= lim && (kCnt & 3) == 0) {
+#pragma unroll
+        for (int z = 0; z < kCnt; z += 4)
+            *reinterpret_cast<float4 *>(irow + first + z) =
+                make_float4(p[z], p[z + 1], p[z + 2], p[z + 3]);
+    } else {
+#pragma unroll
+        for (int z = 0; z < kCnt; ++z)
+            if (first + z < lim) irow[first + z] = p[z];
     }
 }
 
 __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
-    const int rho = threadIdx.x - 128;          // 0..127
-    const int wq = (threadIdx.x >> 5) & 3;      // TMEM lane quadrant of this warp
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wq = warp & 3;                     // TMEM lane quadrant of this warp
+    const int rho = wq * 32 + lane;              // MMA row / TMEM lane
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const float sc = L.scale_log2;
     const __nv_bfloat16 *Q = (const __nv_bfloat16 *)L.q;
+    const int32_t *plan_s = (const int32_t *)(sm.base + SM_PLAN);
     uint32_t gt = 0, npv = 0, gphase = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
-        // per-row context
         RowCtx rc;
-        rc.qi = rho / L.r;
-        rc.hl = rho % L.r;
-        rc.h = it.g * L.r + rc.hl;
-        rc.valid = rho < w.rows && rc.qi < it.nq;
+        rc.qi = rho / w.rpad;
+        rc.hl = rho % w.rpad;
+        rc.h = it.g * L.r + min(rc.hl, L.r - 1);
+        rc.valid = rc.qi < it.nq && rc.hl < L.r;
         rc.i = it.q0 + min(rc.qi, max(it.nq - 1, 0));
         if (P.mode == MODE_TEXT) rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
         else rc.t = it.nq > 0 ? L.vis[rc.i] : 0;
         rc.c_vis = min((rc.i + 1) / L.block, w.nb);
-        const int ntiles = item_tiles(it);
-        if (ntiles == 0) {
+        if (item_tiles(it) == 0) {
             // nothing attended: empty branch outputs
             if (rc.valid) {
                 if (P.mode == MODE_CMP) {
                     float *orow = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                     for (int e = 0; e < kD; e += 4)
                         *reinterpret_cast<float4 *>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (L.dbg_o_cmp)
+                        for (int e = 0; e < kD; ++e)
+                            L.dbg_o_cmp[((size_t)rc.t * L.h_q + rc.h) * kD + e] = 0.f;
                     L.lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
                 } else if (P.mode == MODE_TEXT) {
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
+                } else {
+                    // no selected / window key: the branch output is 0
+                    const float *gl = L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3;
+                    float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+                    const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
+                    float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+                    const float gc = sigmoidf_(gl[0]);
+                    for (int e = 0; e < kD; ++e) {
+                        if (dbg) dbg[prow + e] = 0.f;
+                        if (P.mode == MODE_SLC) part[e] *= gc;
+                        else ((__nv_bfloat16 *)L.out)[prow + e] = __float2bfloat16_rn(part[e]);
+                    }
                 }
             }
             continue;
@@ -445,9 +455,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // ---- Q tile: rows gathered from their positions, 16-byte pieces
         for (int e = rho; e < kRows * 16; e += 128) {
             const int row = e >> 4, c16 = e & 15;
-            const int qi = row / L.r, hl = row % L.r;
+            const int qi = row / w.rpad, hl = row % w.rpad;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (row < w.rows && qi < it.nq) {
+            if (qi < it.nq && hl < L.r) {
                 const int q = it.q0 + qi;
                 const int t = (P.mode == MODE_TEXT) ? L.txt[q] : L.vis[q];
                 const __nv_bfloat16 *src =
@@ -460,11 +470,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(sm.bar(B_Q_FULL));
-
-        // VIS: the item's selection tiles (first key, query mask) into shared
+        // SLC: the item's selection tiles (first key, query mask) into shared
         // memory, once every thread is done with the previous item's copy
-        const int32_t *plan_s = (const int32_t *)(sm.base + SM_PLAN);
-        if (P.mode == MODE_VIS) {
+        if (P.mode == MODE_SLC) {
             group_sync(sm, gphase, ok, L);
             if (!ok) break;
             int32_t *dst = (int32_t *)(sm.base + SM_PLAN);
@@ -478,14 +486,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
 
         float lse2 = -INFINITY;                 // CMP: from the stats segment
-        float m_s = -INFINITY, l_s = 0.f;       // segment 0 running max / sum
-        float l_w = 0.f;                        // segment 1 (VIS window) sum
+        float m_run = -INFINITY, l_run = 0.f;   // running max / sum (log2 units)
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
-            float m_run = -INFINITY, l_run = 0.f;
-            const uint32_t ocol = (kind == K_SWA) ? TM_O1 : TM_O0;
+            m_run = -INFINITY;
+            l_run = 0.f;
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
-                const uint32_t b = gt & 1;
                 const int key0 = kind == K_SLC ? plan_s[x] : tile_key0(P, it, item, kind, x);
                 // column range [lo, hi] of valid keys for this row
                 int lo = 1, hi = 0;
@@ -506,19 +512,22 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     hi = min(hi, kKeys - 1);
                 }
                 const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kKeys - 1);
-                bool r = ptx::mbar_wait(sm.bar(B_S_FULL + b), (gt >> 1) & 1, abort, L.status);
+                bool r = ptx::mbar_wait(sm.bar(B_S_FULL), gt & 1, abort, L.status);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 float sv[64];
                 {
                     float a[32], c[32];
-                    ptx::tmem_ld32(tmem + lane_base + TM_S0 + b * kKeys, a);
-                    ptx::tmem_ld32(tmem + lane_base + TM_S0 + b * kKeys + 32, c);
+                    ptx::tmem_ld32(tmem + lane_base + TM_S, a);
+                    ptx::tmem_ld32(tmem + lane_base + TM_S + 32, c);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 32; ++k) { sv[k] = a[k]; sv[32 + k] = c[k]; }
                 }
+                // S is in registers: let the next Q K^T overwrite it
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(sm.bar(B_S_FREE));
                 if (full) {
 #pragma unroll
                     for (int k = 0; k < 64; ++k) sv[k] *= sc;
@@ -546,39 +555,18 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                                       ((a8[4] + a8[5]) + (a8[6] + a8[7]));
                     l_run = l_run * ptx::ex2(m_run - mu) + acc;
                     m_run = mn;
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(sm.bar(B_P_FULL + b));
                     continue;
                 }
-                float pv[64];
+                bool need = false;
+                float factor = 1.f;
                 if (kind == K_EXACT) {
                     const bool live = lse2 != -INFINITY;
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) pv[k] = live ? ptx::ex2(sv[k] - lse2) : 0.f;
-                    // importance: sum of the group's heads for each (query, block)
-                    float *p32 = (float *)(sm.base + SM_P32);
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) p32[rho * P32_STRIDE + k] = pv[k];
-                    group_sync(sm, gphase, ok, L);
-                    if (!ok) break;
-                    for (int pair = rho; pair < it.nq * 64; pair += 128) {
-                        const int qi = pair >> 6, col = pair & 63;
-                        const int iq = it.q0 + qi;
-                        const int cq = min((iq + 1) / L.block, w.nb);
-                        if (key0 + col < cq) {
-                            float acc = 0.f;
-                            for (int hh = 0; hh < L.r; ++hh)
-                                acc += p32[(qi * L.r + hh) * P32_STRIDE + col];
-                            L.imp[((size_t)it.g * L.n_max + iq) * L.imp_stride + key0 + col] = acc;
-                        }
-                    }
-                    group_sync(sm, gphase, ok, L);
-                    if (!ok) break;
+                    for (int k = 0; k < 64; ++k) sv[k] = live ? ptx::ex2(sv[k] - lse2) : 0.f;
                 } else {
                     // online softmax with lazy rescaling of O
                     const float mn = fmaxf(m_run, mx);
-                    const bool need = mn > m_run + kRescale;
-                    float factor = 1.f;
+                    need = mn > m_run + kRescale;
                     if (need) {
                         factor = ptx::ex2(m_run - mn);  // 0 if m_run = -inf
                         l_run *= factor;
@@ -588,55 +576,73 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int k = 0; k < 64; ++k) {
-                        pv[k] = ptx::ex2(sv[k] - mu);
-                        a8[k & 7] += pv[k];
+                        sv[k] = ptx::ex2(sv[k] - mu);
+                        a8[k & 7] += sv[k];
                     }
                     l_run += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-                    const bool resc = __any_sync(0xffffffffu, need && x > 0);
-                    if (resc) {
-                        // O may only be rescaled once every earlier P V has landed
-                        if (npv > 0) {
-                            bool r2 = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)),
-                                                     ((npv - 1) >> 1) & 1, abort, L.status);
-                            ok = __all_sync(0xffffffffu, r2 && ok);
-                            if (!ok) break;
-                        }
-                        ptx::tc_fence_after();
-                        const float f = (need && x > 0) ? factor : 1.f;
-#pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
-                            float o[32];
-                            ptx::tmem_ld32(tmem + lane_base + ocol + ch * 32, o);
-                            ptx::tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) o[k] *= f;
-                            ptx::tmem_st32(tmem + lane_base + ocol + ch * 32, o);
-                        }
-                        ptx::tmem_wait_st();
-                    }
                 }
-                // P into buffer npv & 1 once the P V that last read it (#npv-2) is done
+                const uint32_t pb = npv & 1;
+                // P buffer pb is free once P V #npv-2 (its last reader) is done
                 if (npv > 1) {
-                    bool r3 = ptx::mbar_wait(sm.bar(B_PV_DONE + (npv & 1)), ((npv - 2) >> 1) & 1,
-                                             abort, L.status);
+                    bool r3 = ptx::mbar_wait(sm.bar(B_PV_DONE + pb), ((npv - 2) >> 1) & 1, abort,
+                                             L.status);
                     ok = __all_sync(0xffffffffu, r3 && ok);
                     if (!ok) break;
                 }
-                store_p_f16(sm, npv & 1, rho, pv);
-                ptx::fence_proxy_async();
+                if (__any_sync(0xffffffffu, need && x > 0)) {
+                    // O may only be rescaled once every earlier P V has landed
+                    if (npv > 0) {
+                        bool r2 = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)),
+                                                 ((npv - 1) >> 1) & 1, abort, L.status);
+                        ok = __all_sync(0xffffffffu, r2 && ok);
+                        if (!ok) break;
+                    }
+                    ptx::tc_fence_after();
+                    const float f = (need && x > 0) ? factor : 1.f;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        float o[32];
+                        ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] *= f;
+                        ptx::tmem_st32(tmem + lane_base + TM_O + ch * 32, o);
+                    }
+                }
+                {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        __half2 h2 = __floats2half2_rn(sv[2 * k], sv[2 * k + 1]);
+                        pk[k] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+                    ptx::tmem_st32u(tmem + lane_base + TM_P + pb * 32, pk);
+                }
+                ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(sm.bar(B_P_FULL + b));
+                ptx::mbar_arrive(sm.bar(B_P_FULL + pb));
                 ++npv;
+                if (kind == K_EXACT) {
+                    // block importance: the sum of the probabilities over the
+                    // query's head slots (P is already handed to the MMA)
+                    const int iq = it.q0 + rc.qi;
+                    const int cq = min((iq + 1) / L.block, w.nb);
+                    float *irow = rc.qi < it.nq
+                                      ? L.imp + ((size_t)it.g * L.n_max + iq) * L.imp_stride + key0
+                                      : nullptr;
+                    const int lim = cq - key0;  // valid columns of this tile for the query
+                    switch (w.rpad) {
+                        case 1: imp_reduce_store<1>(sv, lane, irow, lim); break;
+                        case 2: imp_reduce_store<2>(sv, lane, irow, lim); break;
+                        case 4: imp_reduce_store<4>(sv, lane, irow, lim); break;
+                        case 8: imp_reduce_store<8>(sv, lane, irow, lim); break;
+                        default: imp_reduce_store<16>(sv, lane, irow, lim); break;
+                    }
+                }
             }
             if (!ok) break;
-            if (kind == K_STATS) {
+            if (kind == K_STATS)
                 lse2 = (m_run == -INFINITY || l_run <= 0.f) ? -INFINITY : m_run + log2f(l_run);
-            } else if (s == 0) {
-                m_s = m_run;
-                l_s = l_run;
-            } else {
-                l_w = l_run;
-            }
         }
         if (!ok) break;
         // ---- epilogue: wait for the item's last P V (#npv-1)
@@ -647,81 +653,83 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             if (!ok) break;
             ptx::tc_fence_after();
         }
+        const size_t qrow = ((size_t)rc.i * L.h_q + rc.h) * kD;   // by vision rank
+        const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;   // by position
         if (P.mode == MODE_CMP) {
-            float *orow = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+            float *orow = L.o_cmp_ws + qrow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
-                ptx::tmem_ld32(tmem + lane_base + TM_O0 + ch * 32, o);
+                ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
                 ptx::tmem_wait_ld();
                 if (rc.valid) {
 #pragma unroll
                     for (int k = 0; k < 32; k += 4)
                         *reinterpret_cast<float4 *>(orow + ch * 32 + k) =
                             make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+                    if (L.dbg_o_cmp)
+                        for (int k = 0; k < 32; ++k) L.dbg_o_cmp[prow + ch * 32 + k] = o[k];
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
-        } else if (P.mode == MODE_VIS) {
-            const float *gl = L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3;
-            float gc = 0.f, gs = 0.f, gw = 0.f;
+        } else if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+            float g = 0.f, gc = 0.f;
             if (rc.valid) {
+                const float *gl = L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3;
                 gc = sigmoidf_(gl[0]);
-                gs = sigmoidf_(gl[1]);
-                gw = sigmoidf_(gl[2]);
+                g = sigmoidf_(gl[P.mode == MODE_SLC ? 1 : 2]);
             }
-            const float inv_s = l_s > 0.f ? 1.f / l_s : 0.f;
-            const float inv_w = l_w > 0.f ? 1.f / l_w : 0.f;
-            const float *oc = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
-            __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + ((size_t)rc.t * L.h_q + rc.h) * kD;
-            const size_t drow = ((size_t)rc.t * L.h_q + rc.h) * kD;
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            float *part = L.o_cmp_ws + qrow;
+            float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+            __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                float a[32], c[32];
-                ptx::tmem_ld32(tmem + lane_base + TM_O0 + ch * 32, a);
-                ptx::tmem_ld32(tmem + lane_base + TM_O1 + ch * 32, c);
+                float o[32];
+                ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
 #pragma unroll
-                for (int k = 0; k < 32; k += 8) {
-                    float o8[8];
+                for (int k = 0; k < 32; k += 4) {
+                    float4 pr = *reinterpret_cast<float4 *>(part + ch * 32 + k);
+                    float b4[4];
 #pragma unroll
-                    for (int z = 0; z < 8; ++z) {
-                        const int e = ch * 32 + k + z;
-                        const float os = l_s > 0.f ? a[k + z] * inv_s : 0.f;
-                        const float ow = l_w > 0.f ? c[k + z] * inv_w : 0.f;
-                        const float occ = oc[e];
-                        o8[z] = gc * occ + gs * os + gw * ow;
-                        if (L.dbg_o_cmp) L.dbg_o_cmp[drow + e] = occ;
-                        if (L.dbg_o_slc) L.dbg_o_slc[drow + e] = os;
-                        if (L.dbg_o_swa) L.dbg_o_swa[drow + e] = ow;
+                    for (int z = 0; z < 4; ++z) b4[z] = l_run > 0.f ? o[k + z] * inv : 0.f;
+                    if (dbg)
+                        for (int z = 0; z < 4; ++z) dbg[prow + ch * 32 + k + z] = b4[z];
+                    if (P.mode == MODE_SLC) {
+                        // partial = sig(g_cmp) o_cmp + sig(g_slc) o_slc, in place
+                        pr.x = gc * pr.x + g * b4[0];
+                        pr.y = gc * pr.y + g * b4[1];
+                        pr.z = gc * pr.z + g * b4[2];
+                        pr.w = gc * pr.w + g * b4[3];
+                        *reinterpret_cast<float4 *>(part + ch * 32 + k) = pr;
+                    } else {
+                        __nv_bfloat162 lo2 =
+                            __floats2bfloat162_rn(pr.x + g * b4[0], pr.y + g * b4[1]);
+                        __nv_bfloat162 hi2 =
+                            __floats2bfloat162_rn(pr.z + g * b4[2], pr.w + g * b4[3]);
+                        uint2 v;
+                        v.x = *reinterpret_cast<uint32_t *>(&lo2);
+                        v.y = *reinterpret_cast<uint32_t *>(&hi2);
+                        *reinterpret_cast<uint2 *>(orow + ch * 32 + k) = v;
                     }
-                    uint4 v;
-                    __nv_bfloat162 b0 = __floats2bfloat162_rn(o8[0], o8[1]);
-                    __nv_bfloat162 b1 = __floats2bfloat162_rn(o8[2], o8[3]);
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(o8[4], o8[5]);
-                    __nv_bfloat162 b3 = __floats2bfloat162_rn(o8[6], o8[7]);
-                    v.x = *reinterpret_cast<uint32_t *>(&b0);
-                    v.y = *reinterpret_cast<uint32_t *>(&b1);
-                    v.z = *reinterpret_cast<uint32_t *>(&b2);
-                    v.w = *reinterpret_cast<uint32_t *>(&b3);
-                    *reinterpret_cast<uint4 *>(orow + ch * 32 + k) = v;
                 }
             }
         } else if (w.nsplit == 1) {
             // one key split: the item holds the whole softmax, write the row
-            const float inv = l_s > 0.f ? 1.f / l_s : 0.f;
-            __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + ((size_t)rc.t * L.h_q + rc.h) * kD;
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
-                ptx::tmem_ld32(tmem + lane_base + TM_O0 + ch * 32, o);
+                ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
 #pragma unroll
                 for (int k = 0; k < 32; k += 2) {
-                    const float a = l_s > 0.f ? o[k] * inv : 0.f;
-                    const float c = l_s > 0.f ? o[k + 1] * inv : 0.f;
+                    const float a = l_run > 0.f ? o[k] * inv : 0.f;
+                    const float c = l_run > 0.f ? o[k + 1] * inv : 0.f;
                     *reinterpret_cast<__nv_bfloat162 *>(orow + ch * 32 + k) =
                         __floats2bfloat162_rn(a, c);
                 }
@@ -731,7 +739,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
-                ptx::tmem_ld32(tmem + lane_base + TM_O0 + ch * 32, o);
+                ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
                 ptx::tmem_wait_ld();
                 if (rc.valid) {
 #pragma unroll
@@ -739,22 +747,16 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
             }
             if (rc.valid) {
-                pr[kD] = m_s;
-                pr[kD + 1] = l_s;
+                pr[kD] = m_run;
+                pr[kD + 1] = l_run;
             }
         }
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_constant__ TcParams P) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint32_t s_failed;
     const LayerParams &L = P.L;
-    // skip the work if an earlier kernel already failed (one read, shared by
-    // the whole CTA so that every thread takes the same path)
-    if (threadIdx.x == 0) s_failed = *(volatile uint32_t *)L.status;
-    __syncthreads();
-    if (s_failed != 0) return;
     Smem sm;
     {
         const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -762,6 +764,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
         sm.base = smem_raw + pad;
         sm.base_u32 = raw + pad;
     }
+    // skip the work if an earlier kernel already failed (one read, shared by
+    // the whole CTA so that every thread takes the same path)
+    if (threadIdx.x == 0) *sm.failed_flag() = *(volatile uint32_t *)L.status;
+    __syncthreads();
+    if (*sm.failed_flag() != 0) return;
     const Counts cn = *L.counts;
     const Work w = make_work(P, cn);
     if ((int)blockIdx.x >= w.items) return;
@@ -771,12 +778,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
             ptx::mbar_init(sm.bar(B_KV_FULL + s), 1);
             ptx::mbar_init(sm.bar(B_KV_EMPTY + s), 1);
         }
+        ptx::mbar_init(sm.bar(B_S_FULL), 1);
+        ptx::mbar_init(sm.bar(B_S_FREE), 128);
         for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(sm.bar(B_S_FULL + b), 1);
             ptx::mbar_init(sm.bar(B_P_FULL + b), 128);
+            ptx::mbar_init(sm.bar(B_PV_DONE + b), 1);
         }
-        ptx::mbar_init(sm.bar(B_PV_DONE), 1);
-        ptx::mbar_init(sm.bar(B_PV_DONE + 1), 1);
         ptx::mbar_init(sm.bar(B_Q_FULL), 128);
         ptx::mbar_init(sm.bar(B_GRP), 128);
         ptx::mbar_init(sm.bar(B_FINAL), 1);
@@ -801,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attn_kernel(const __grid_const
     } else if (warp == 1) {
         if (lane == 0) run_mma(P, w, sm, tmem);
         __syncwarp();
-    } else if (warp >= 4) {
+    } else {
         run_softmax(P, w, sm, tmem);
     }
     ptx::tc_fence_before();
@@ -855,7 +862,7 @@ __global__ void prepare_kernel(LayerParams p, __nv_bfloat16 *kc, __half *vhc, __
 }
 
 // ---------------------------------------------------------------------------
-// Union of the blocks selected by the queries of each VIS item, with a mask of
+// Union of the blocks selected by the queries of each SLC item, with a mask of
 // the queries that chose each block.  One warp per item.
 __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int words) {
     extern __shared__ uint32_t sh[];
@@ -929,15 +936,9 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
 
 // ---------------------------------------------------------------------------
 // Text split-KV combine: one warp per (text query, head).
-__device__ void text_combine_row(const LayerParams &p, const float *part, int part_items,
-                                 int n_tt, int qt, int x, int h, int lane) {
-    const Counts &cn = *p.counts;
-    // same split rule as make_work
-    const int span = p.txt[cn.n_text - 1] + 1;
-    int ns = (span + kTextSplitKeys - 1) / kTextSplitKeys;
+__device__ void text_combine_row(const LayerParams &p, const float *part, int ns, int n_tt,
+                                 int qt, int x, int h, int lane) {
     const int tiles = p.h_kv * n_tt;
-    ns = min(ns, max(1, part_items / tiles));
-    ns = max(1, ns);
     const int g = h / p.r, hl = h % p.r;
     const int tt = x / qt, qi = x % qt;
     const int rho = qi * p.r + hl;
@@ -970,22 +971,20 @@ __device__ void text_combine_row(const LayerParams &p, const float *part, int pa
 
 __global__ void text_combine_kernel(LayerParams p, const float *part, int part_items) {
     const Counts cn = *p.counts;
+    if (cn.n_text == 0) return;
     const int lane = threadIdx.x & 31;
     const int qt = kRows / p.r;
     const int n_tt = (cn.n_text + qt - 1) / qt;
+    // the same split rule as make_work
+    const int span = p.txt[cn.n_text - 1] + 1;
+    const int tiles = p.h_kv * n_tt;
+    const int ns = max(1, min((span + kTextSplitKeys - 1) / kTextSplitKeys,
+                              max(1, part_items / tiles)));
+    if (ns == 1) return;  // with a single key split the attention kernel wrote the rows
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    if (cn.n_text == 0) return;
-    {
-        // with a single key split the attention kernel wrote the rows itself
-        const int span = p.txt[cn.n_text - 1] + 1;
-        const int tiles = p.h_kv * n_tt;
-        const int ns = max(1, min((span + kTextSplitKeys - 1) / kTextSplitKeys,
-                                  max(1, part_items / tiles)));
-        if (ns == 1) return;
-    }
     for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < cn.n_text * p.h_q;
          wi += nwarps)
-        text_combine_row(p, part, part_items, n_tt, qt, wi / p.h_q, wi % p.h_q, lane);
+        text_combine_row(p, part, ns, n_tt, qt, wi / p.h_q, wi % p.h_q, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -1018,10 +1017,9 @@ bool make_map(CUtensorMap *m, const void *base, int h_kv, long long rows, bool f
     cuuint32_t box[2] = {64, 64};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-              const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
@@ -1116,18 +1114,19 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     auto end = [&](int stg) {
         if (ev) cudaEventRecord(ev[2 * stg + 1], s);
     };
-    const int grid = st->num_sms;
+    const int grid = 2 * st->num_sms;  // two CTAs per SM
     cudaError_t e;
-    // compression (vision K/V compaction first, for the later window/selection)
+    auto attn = [&](int mode) {
+        P.mode = mode;
+        tc_attn_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(P);
+        ++*launches;
+    };
     prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vhc, st->vh, st->vh_cmp);
     ++*launches;
     begin(VNSA_STAGE_CMP);
-    P.mode = MODE_CMP;
-    tc_attn_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(P);
-    ++*launches;
+    attn(MODE_CMP);
     end(VNSA_STAGE_CMP);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // selection
     begin(VNSA_STAGE_TOPK);
     if (!forced) {
         if ((e = launch_topk(L, s)) != cudaSuccess) return e;
@@ -1147,16 +1146,15 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     }
     end(VNSA_STAGE_TOPK);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    begin(VNSA_STAGE_SLC);
+    attn(MODE_SLC);
+    end(VNSA_STAGE_SLC);
     begin(VNSA_STAGE_SWA);
-    P.mode = MODE_VIS;
-    tc_attn_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(P);
-    ++*launches;
+    attn(MODE_SWA);
     end(VNSA_STAGE_SWA);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TEXT);
-    P.mode = MODE_TEXT;
-    tc_attn_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(P);
-    ++*launches;
+    attn(MODE_TEXT);
     // grid-stride over (text query, head); the kernel reads N_t on the device
     text_combine_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->part, st->part_items);
     ++*launches;
