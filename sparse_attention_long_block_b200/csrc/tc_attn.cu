@@ -54,8 +54,10 @@ constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] b
 constexpr uint32_t SM_KV = 32768;                             // stages x (K, V)
 constexpr uint32_t KV_BYTES = 32768;
 constexpr int kPlanSmem = 1152;                               // selection tiles per item
-constexpr uint32_t SM_PLAN = SM_KV + kStages * KV_BYTES;      // [2][kPlanSmem] int32
-constexpr uint32_t SM_BAR = SM_PLAN + 2 * kPlanSmem * 4;      // barriers
+constexpr int kPrefetch = 4;                                  // tiles prefetched into L2 ahead
+constexpr uint32_t SM_PLAN = SM_KV + kStages * KV_BYTES;      // [2][kPlanSmem] int32 (softmax)
+constexpr uint32_t SM_PPLAN = SM_PLAN + 2 * kPlanSmem * 4;    // [kPlanSmem] int32 (producer)
+constexpr uint32_t SM_BAR = SM_PPLAN + kPlanSmem * 4;         // barriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment slack
 
@@ -226,8 +228,10 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
 }
 
 // ---------------------------------------------------------------------------
-// Producer: TMA loads of the K (and V) tiles of every item, in order.
-__device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
+// Producer (warp 0): TMA loads of the K (and V) tiles of every item, in order,
+// with the tiles kPrefetch ahead prefetched into L2.  The warp copies a
+// selection item's block list into shared memory; lane 0 issues the copies.
+__device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, int lane) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
     uint32_t gt = 0;
@@ -241,31 +245,66 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm) {
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
     }
+    int32_t *pplan = (int32_t *)(sm.base + SM_PPLAN);
+    bool ok = true;
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
-        for (int s = 0; s < it.nseg; ++s) {
-            const int kind = it.seg_kind[s];
-            for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
-                const uint32_t st = gt % kStages;
-                if (gt >= (uint32_t)kStages &&
-                    !ptx::mbar_wait(sm.bar(B_KV_EMPTY + st), ((gt / kStages) - 1) & 1, abort,
-                                    L.status))
-                    return;
+        if (P.mode == MODE_SLC) {
+            const int32_t *src = P.plan + (size_t)item * (1 + 2 * P.plan_max) + 1;
+            for (int x = lane; x < it.seg_tiles[0]; x += 32) pplan[x] = src[x] * kKeys;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            const int xc = it.g * kD;
+            // row coordinate of tile x of segment s (both CMP segments share keys)
+            auto row_of = [&](int kind, int x) {
+                if (kind == K_SLC) return vbase + pplan[x];
                 const int key0 = tile_key0(P, it, item, kind, x);
-                const int y = (kind == K_SLC || kind == K_SWA) ? vbase + key0 : key0;
-                const bool pv = kind_has_pv(kind);
-                const uint32_t kv = sm.base_u32 + SM_KV + st * KV_BYTES;
-                ptx::mbar_expect_tx(sm.bar(B_KV_FULL + st), pv ? 32768u : 16384u);
-                const int xc = it.g * kD;
-                ptx::tma_load_2d(kv, mk, sm.bar(B_KV_FULL + st), xc, y);
-                ptx::tma_load_2d(kv + 8192, mk, sm.bar(B_KV_FULL + st), xc + 64, y);
-                if (pv) {
-                    ptx::tma_load_2d(kv + 16384, mv, sm.bar(B_KV_FULL + st), xc, y);
-                    ptx::tma_load_2d(kv + 16384 + 8192, mv, sm.bar(B_KV_FULL + st), xc + 64, y);
+                return kind == K_SWA ? vbase + key0 : key0;
+            };
+            const int pf0 = min(kPrefetch, it.seg_tiles[0]);
+            for (int x = 0; x < pf0; ++x) {
+                const int y = row_of(it.seg_kind[0], x);
+                ptx::tma_prefetch_2d(mk, xc, y);
+                ptx::tma_prefetch_2d(mk, xc + 64, y);
+                ptx::tma_prefetch_2d(mv, xc, y);
+                ptx::tma_prefetch_2d(mv, xc + 64, y);
+            }
+            for (int s = 0; ok && s < it.nseg; ++s) {
+                const int kind = it.seg_kind[s];
+                for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
+                    const uint32_t st = gt % kStages;
+                    if (gt >= (uint32_t)kStages &&
+                        !ptx::mbar_wait(sm.bar(B_KV_EMPTY + st), ((gt / kStages) - 1) & 1, abort,
+                                        L.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int y = row_of(kind, x);
+                    const bool pv = kind_has_pv(kind);
+                    const uint32_t kv = sm.base_u32 + SM_KV + st * KV_BYTES;
+                    ptx::mbar_expect_tx(sm.bar(B_KV_FULL + st), pv ? 32768u : 16384u);
+                    ptx::tma_load_2d(kv, mk, sm.bar(B_KV_FULL + st), xc, y);
+                    ptx::tma_load_2d(kv + 8192, mk, sm.bar(B_KV_FULL + st), xc + 64, y);
+                    if (pv) {
+                        ptx::tma_load_2d(kv + 16384, mv, sm.bar(B_KV_FULL + st), xc, y);
+                        ptx::tma_load_2d(kv + 16384 + 8192, mv, sm.bar(B_KV_FULL + st), xc + 64,
+                                         y);
+                    }
+                    if (s == 0 && x + kPrefetch < it.seg_tiles[0]) {
+                        const int yp = row_of(kind, x + kPrefetch);
+                        ptx::tma_prefetch_2d(mk, xc, yp);
+                        ptx::tma_prefetch_2d(mk, xc + 64, yp);
+                        ptx::tma_prefetch_2d(mv, xc, yp);
+                        ptx::tma_prefetch_2d(mv, xc + 64, yp);
+                    }
                 }
             }
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);  // also keeps pplan until lane 0 is done
+        if (!ok) return;
     }
+    if (lane != 0) return;
     // no load may still be landing in shared memory when the CTA ends
     for (uint32_t back = 1; back <= (uint32_t)kStages && back <= gt; ++back) {
         const uint32_t t = gt - back;
@@ -512,11 +551,23 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     hi = min(hi, kKeys - 1);
                 }
                 const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kKeys - 1);
+                // every row of this warp masked (common in selection tiles:
+                // most queries did not pick a given block): P = 0, no S read
+                const bool none = __all_sync(0xffffffffu, lo > hi);
                 bool r = ptx::mbar_wait(sm.bar(B_S_FULL), gt & 1, abort, L.status);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 float sv[64];
+                bool need = false;
+                float factor = 1.f;
+                if (none) {
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(sm.bar(B_S_FREE));
+                    if (kind == K_STATS) continue;
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) sv[k] = 0.f;
+                } else {
                 {
                     float a[32], c[32];
                     ptx::tmem_ld32(tmem + lane_base + TM_S, a);
@@ -557,8 +608,6 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     m_run = mn;
                     continue;
                 }
-                bool need = false;
-                float factor = 1.f;
                 if (kind == K_EXACT) {
                     const bool live = lse2 != -INFINITY;
 #pragma unroll
@@ -581,6 +630,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     }
                     l_run += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
                 }
+                }  // !none
                 const uint32_t pb = npv & 1;
                 // P buffer pb is free once P V #npv-2 (its last reader) is done
                 if (npv > 1) {
@@ -622,7 +672,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(sm.bar(B_P_FULL + pb));
                 ++npv;
-                if (kind == K_EXACT) {
+                if (kind == K_EXACT && !none) {
                     // block importance: the sum of the probabilities over the
                     // query's head slots (P is already handed to the MMA)
                     const int iq = it.q0 + rc.qi;
@@ -804,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     const uint32_t tmem = *sm.tmem_slot();
 
     if (warp == 0) {
-        if (lane == 0) run_producer(P, w, sm);
+        run_producer(P, w, sm, lane);
     } else if (warp == 1) {
         if (lane == 0) run_mma(P, w, sm, tmem);
         __syncwarp();
