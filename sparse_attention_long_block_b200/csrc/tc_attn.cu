@@ -51,19 +51,20 @@ constexpr size_t kTextPartBytes = 256ull << 20;
 constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
 
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
-constexpr uint32_t SM_KV = 32768;                             // stages x (K, V)
-constexpr uint32_t KV_BYTES = 32768;
+constexpr uint32_t SM_KV = 32768;                             // K ring, then V ring
+constexpr uint32_t K_BYTES = 16384;                           // one 64-key K or V tile
+constexpr uint32_t KV_BYTES = 2 * K_BYTES;
 constexpr int kPlanSmem = 1152;                               // selection tiles per item
 constexpr int kPrefetch = 4;                                  // tiles prefetched into L2 ahead
 constexpr uint32_t SM_PLAN = SM_KV + kStages * KV_BYTES;      // [2][kPlanSmem] int32 (softmax)
-constexpr uint32_t SM_PPLAN = SM_PLAN + 2 * kPlanSmem * 4;    // [kPlanSmem] int32 (producer)
-constexpr uint32_t SM_BAR = SM_PPLAN + kPlanSmem * 4;         // barriers
+constexpr uint32_t SM_BAR = SM_PLAN + 2 * kPlanSmem * 4;      // barriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment slack
 
 // barrier slots (8 bytes each) after SM_BAR
-constexpr int B_KV_FULL = 0, B_KV_EMPTY = 2, B_S_FULL = 4, B_S_FREE = 5, B_P_FULL = 6,
-              B_PV_DONE = 8, B_Q_FULL = 10, B_GRP = 11, B_FINAL = 12, B_COUNT = 13;
+constexpr int B_K_FULL = 0, B_V_FULL = 2, B_K_EMPTY = 4, B_V_EMPTY = 6, B_S_FULL = 8,
+              B_S_FREE = 9, B_P_FULL = 10, B_PV_DONE = 12, B_Q_FULL = 14, B_GRP = 15,
+              B_FINAL = 16, B_COUNT = 17;
 
 // TMEM columns: S (fp32, 64), P buffers (fp16 pairs, 32 each), O (fp32, 128)
 constexpr uint32_t TM_S = 0, TM_P = 64, TM_O = 128, TM_COLS = 256;
@@ -228,13 +229,19 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
 }
 
 // ---------------------------------------------------------------------------
-// Producer (warp 0): TMA loads of the K (and V) tiles of every item, in order,
-// with the tiles kPrefetch ahead prefetched into L2.  The warp copies a
-// selection item's block list into shared memory; lane 0 issues the copies.
+// Producer (warp 0): TMA loads of the K tiles (lane 0) and V tiles (lane 1) of
+// every item, in order, each lane with its own ring and waits: a K stage is
+// free once its Q K^T is done, a V stage only after its P V, so the K loads
+// run ahead.  Lane 0 also prefetches the tiles kPrefetch ahead into L2.
 __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, int lane) {
+    if (lane > 1) return;
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
-    uint32_t gt = 0;
+    const bool is_k = lane == 0;
+    const int ring_full = is_k ? B_K_FULL : B_V_FULL;
+    const int ring_empty = is_k ? B_K_EMPTY : B_V_EMPTY;
+    const uint32_t ring_base = sm.base_u32 + SM_KV + (is_k ? 0u : kStages * K_BYTES);
+    uint32_t t = 0;  // tiles issued on this lane's ring
     const CUtensorMap *mk = &P.tm_k, *mv = &P.tm_v;
     int vbase = 0;
     if (P.mode == MODE_CMP) {
@@ -245,23 +252,16 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
     }
-    int32_t *pplan = (int32_t *)(sm.base + SM_PPLAN);
-    bool ok = true;
+    const CUtensorMap *mine = is_k ? mk : mv;
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
         const Item it = make_item(P, w, item);
-        if (P.mode == MODE_SLC) {
-            const int32_t *src = P.plan + (size_t)item * (1 + 2 * P.plan_max) + 1;
-            for (int x = lane; x < it.seg_tiles[0]; x += 32) pplan[x] = src[x] * kKeys;
-        }
-        __syncwarp();
-        if (lane == 0) {
-            const int xc = it.g * kD;
-            // row coordinate of tile x of segment s (both CMP segments share keys)
-            auto row_of = [&](int kind, int x) {
-                if (kind == K_SLC) return vbase + pplan[x];
-                const int key0 = tile_key0(P, it, item, kind, x);
-                return kind == K_SWA ? vbase + key0 : key0;
-            };
+        const int xc = it.g * kD;
+        // row coordinate of tile x of a segment (both CMP segments share keys)
+        auto row_of = [&](int kind, int x) {
+            const int key0 = tile_key0(P, it, item, kind, x);
+            return (kind == K_SLC || kind == K_SWA) ? vbase + key0 : key0;
+        };
+        if (is_k) {
             const int pf0 = min(kPrefetch, it.seg_tiles[0]);
             for (int x = 0; x < pf0; ++x) {
                 const int y = row_of(it.seg_kind[0], x);
@@ -270,45 +270,37 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
                 ptx::tma_prefetch_2d(mv, xc, y);
                 ptx::tma_prefetch_2d(mv, xc + 64, y);
             }
-            for (int s = 0; ok && s < it.nseg; ++s) {
-                const int kind = it.seg_kind[s];
-                for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
-                    const uint32_t st = gt % kStages;
-                    if (gt >= (uint32_t)kStages &&
-                        !ptx::mbar_wait(sm.bar(B_KV_EMPTY + st), ((gt / kStages) - 1) & 1, abort,
-                                        L.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const int y = row_of(kind, x);
-                    const bool pv = kind_has_pv(kind);
-                    const uint32_t kv = sm.base_u32 + SM_KV + st * KV_BYTES;
-                    ptx::mbar_expect_tx(sm.bar(B_KV_FULL + st), pv ? 32768u : 16384u);
-                    ptx::tma_load_2d(kv, mk, sm.bar(B_KV_FULL + st), xc, y);
-                    ptx::tma_load_2d(kv + 8192, mk, sm.bar(B_KV_FULL + st), xc + 64, y);
-                    if (pv) {
-                        ptx::tma_load_2d(kv + 16384, mv, sm.bar(B_KV_FULL + st), xc, y);
-                        ptx::tma_load_2d(kv + 16384 + 8192, mv, sm.bar(B_KV_FULL + st), xc + 64,
-                                         y);
-                    }
-                    if (s == 0 && x + kPrefetch < it.seg_tiles[0]) {
-                        const int yp = row_of(kind, x + kPrefetch);
-                        ptx::tma_prefetch_2d(mk, xc, yp);
-                        ptx::tma_prefetch_2d(mk, xc + 64, yp);
-                        ptx::tma_prefetch_2d(mv, xc, yp);
-                        ptx::tma_prefetch_2d(mv, xc + 64, yp);
-                    }
+        }
+        for (int s = 0; s < it.nseg; ++s) {
+            const int kind = it.seg_kind[s];
+            if (!is_k && !kind_has_pv(kind)) continue;
+            int y_next = it.seg_tiles[s] > 0 ? row_of(kind, 0) : 0;
+            for (int x = 0; x < it.seg_tiles[s]; ++x, ++t) {
+                const int y = y_next;
+                if (x + 1 < it.seg_tiles[s]) y_next = row_of(kind, x + 1);
+                const uint32_t st = t % kStages;
+                if (t >= (uint32_t)kStages &&
+                    !ptx::mbar_wait(sm.bar(ring_empty + st), ((t / kStages) - 1) & 1, abort,
+                                    L.status))
+                    return;
+                const uint32_t dst = ring_base + st * K_BYTES;
+                ptx::mbar_expect_tx(sm.bar(ring_full + st), K_BYTES);
+                ptx::tma_load_2d(dst, mine, sm.bar(ring_full + st), xc, y);
+                ptx::tma_load_2d(dst + 8192, mine, sm.bar(ring_full + st), xc + 64, y);
+                if (is_k && s == 0 && x + kPrefetch < it.seg_tiles[0]) {
+                    const int yp = row_of(kind, x + kPrefetch);
+                    ptx::tma_prefetch_2d(mk, xc, yp);
+                    ptx::tma_prefetch_2d(mk, xc + 64, yp);
+                    ptx::tma_prefetch_2d(mv, xc, yp);
+                    ptx::tma_prefetch_2d(mv, xc + 64, yp);
                 }
             }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);  // also keeps pplan until lane 0 is done
-        if (!ok) return;
     }
-    if (lane != 0) return;
     // no load may still be landing in shared memory when the CTA ends
-    for (uint32_t back = 1; back <= (uint32_t)kStages && back <= gt; ++back) {
-        const uint32_t t = gt - back;
-        if (!ptx::mbar_wait(sm.bar(B_KV_FULL + t % kStages), (t / kStages) & 1, abort, L.status))
+    for (uint32_t back = 1; back <= (uint32_t)kStages && back <= t; ++back) {
+        const uint32_t u = t - back;
+        if (!ptx::mbar_wait(sm.bar(ring_full + u % kStages), (u / kStages) & 1, abort, L.status))
             return;
     }
 }
@@ -323,20 +315,22 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
     constexpr uint32_t idesc_s = ptx::idesc_f16kind(kRows, kKeys, 0, 0, 1u);
     constexpr uint32_t idesc_pv = ptx::idesc_f16kind(kRows, kD, 0, 1, 0u);
     const uint32_t q_addr = sm.base_u32 + SM_Q;
-    uint32_t gt = 0, nitems = 0, npv = 0;
+    uint32_t gt = 0, nitems = 0, npv = 0;  // npv: P V products = V tiles consumed
     bool ok = true;
-    auto issue_pv = [&](uint32_t pst, uint32_t acc) -> bool {
-        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (npv & 1)), (npv >> 1) & 1, abort, L.status))
+    auto issue_pv = [&](uint32_t acc) -> bool {
+        const uint32_t sv = npv % kStages;
+        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (npv & 1)), (npv >> 1) & 1, abort, L.status) ||
+            !ptx::mbar_wait(sm.bar(B_V_FULL + sv), (npv / kStages) & 1, abort, L.status))
             return false;
         ptx::tc_fence_after();
-        const uint32_t vb = sm.base_u32 + SM_KV + pst * KV_BYTES + 16384;
+        const uint32_t vb = sm.base_u32 + SM_KV + kStages * K_BYTES + sv * K_BYTES;
         const uint32_t pa = tmem + TM_P + (npv & 1) * 32;
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k)
             ptx::mma_ts(tmem + TM_O, pa + (uint32_t)k * 8u, desc_vmajor(vb + (uint32_t)k * 2048u),
                         idesc_pv, (k > 0 || acc) ? 1u : 0u);
         ptx::mma_commit(sm.bar(B_PV_DONE + (npv & 1)));
-        ptx::mma_commit(sm.bar(B_KV_EMPTY + pst));
+        ptx::mma_commit(sm.bar(B_V_EMPTY + sv));
         ++npv;
         return true;
     };
@@ -347,39 +341,38 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         ++nitems;
         ptx::tc_fence_after();
         bool pending = false;
-        uint32_t pend_st = 0, pend_acc = 0;
+        uint32_t pend_acc = 0;
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
                 const uint32_t st = gt % kStages;
-                if (!ptx::mbar_wait(sm.bar(B_KV_FULL + st), (gt / kStages) & 1, abort, L.status) ||
+                if (!ptx::mbar_wait(sm.bar(B_K_FULL + st), (gt / kStages) & 1, abort, L.status) ||
                     (gt > 0 && !ptx::mbar_wait(sm.bar(B_S_FREE), (gt - 1) & 1, abort, L.status))) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint32_t kv = sm.base_u32 + SM_KV + st * KV_BYTES;
+                const uint32_t kb = sm.base_u32 + SM_KV + st * K_BYTES;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t off = (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u;
                     const uint32_t koff = (uint32_t)(k >> 2) * 8192u + (uint32_t)(k & 3) * 32u;
-                    ptx::mma_ss(tmem + TM_S, desc_kmajor(q_addr + off), desc_kmajor(kv + koff),
+                    ptx::mma_ss(tmem + TM_S, desc_kmajor(q_addr + off), desc_kmajor(kb + koff),
                                 idesc_s, k > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(sm.bar(B_S_FULL));
-                if (!kind_has_pv(kind)) ptx::mma_commit(sm.bar(B_KV_EMPTY + st));
+                ptx::mma_commit(sm.bar(B_K_EMPTY + st));  // K is dead once Q K^T is done
                 if (pending) {
-                    if (!issue_pv(pend_st, pend_acc)) { ok = false; break; }
+                    if (!issue_pv(pend_acc)) { ok = false; break; }
                     pending = false;
                 }
                 if (kind_has_pv(kind)) {
                     pending = true;
-                    pend_st = st;
                     pend_acc = x > 0 ? 1u : 0u;
                 }
             }
         }
-        if (ok && pending && !issue_pv(pend_st, pend_acc)) ok = false;
+        if (ok && pending && !issue_pv(pend_acc)) ok = false;
     }
     // every MMA this thread issued has completed once this barrier flips
     ptx::mma_commit(sm.bar(B_FINAL));
@@ -463,29 +456,26 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         if (item_tiles(it) == 0) {
             // nothing attended: empty branch outputs
             if (rc.valid) {
+                __half *part = (__half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+                const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
                 if (P.mode == MODE_CMP) {
-                    float *orow = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
-                    for (int e = 0; e < kD; e += 4)
-                        *reinterpret_cast<float4 *>(orow + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int e = 0; e < kD; e += 8)
+                        *reinterpret_cast<uint4 *>(part + e) = make_uint4(0u, 0u, 0u, 0u);
                     if (L.dbg_o_cmp)
-                        for (int e = 0; e < kD; ++e)
-                            L.dbg_o_cmp[((size_t)rc.t * L.h_q + rc.h) * kD + e] = 0.f;
+                        for (int e = 0; e < kD; ++e) L.dbg_o_cmp[prow + e] = 0.f;
                     L.lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
                 } else if (P.mode == MODE_TEXT) {
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
                 } else {
-                    // no selected / window key: the branch output is 0
-                    const float *gl = L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3;
-                    float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
-                    const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
+                    // no selected / window key: this branch adds nothing
                     float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
-                    const float gc = sigmoidf_(gl[0]);
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
-                        if (P.mode == MODE_SLC) part[e] *= gc;
-                        else ((__nv_bfloat16 *)L.out)[prow + e] = __float2bfloat16_rn(part[e]);
+                        if (P.mode == MODE_SWA)
+                            ((__nv_bfloat16 *)L.out)[prow + e] =
+                                __float2bfloat16_rn(__half2float(part[e]));
                     }
                 }
             }
@@ -509,6 +499,26 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         ptx::fence_proxy_async();
         ptx::mbar_arrive(sm.bar(B_Q_FULL));
+        // L2 prefetch of this row's epilogue inputs and of its Q row in the
+        // next item, so that neither waits on DRAM when it is needed
+        if (rc.valid) {
+            ptx::prefetch_l2(L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3);
+            if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+                const __half *part = (const __half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+                ptx::prefetch_l2(part);
+                ptx::prefetch_l2(part + 64);
+            }
+        }
+        if (item + (int)gridDim.x < w.items) {
+            const Item nx = make_item(P, w, item + gridDim.x);
+            const int qn = rho / w.rpad, hn = rho % w.rpad;
+            if (qn < nx.nq && hn < L.r) {
+                const int tn = (P.mode == MODE_TEXT) ? L.txt[nx.q0 + qn] : L.vis[nx.q0 + qn];
+                const __nv_bfloat16 *qr = Q + ((size_t)tn * L.h_q + nx.g * L.r + hn) * kD;
+                ptx::prefetch_l2(qr);
+                ptx::prefetch_l2(qr + 64);
+            }
+        }
         // SLC: the item's selection tiles (first key, query mask) into shared
         // memory, once every thread is done with the previous item's copy
         if (P.mode == MODE_SLC) {
@@ -705,8 +715,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         const size_t qrow = ((size_t)rc.i * L.h_q + rc.h) * kD;   // by vision rank
         const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;   // by position
+        // The gated vision partial lives in the workspace as fp16 [N_v][h_q][d]:
+        // CMP writes sig(g_cmp) o_cmp, SLC adds sig(g_slc) o_slc in place, SWA
+        // adds sig(g_swa) o_swa and writes the bf16 output row.
+        __half *part = (__half *)L.o_cmp_ws + qrow;
         if (P.mode == MODE_CMP) {
-            float *orow = L.o_cmp_ws + qrow;
+            const float gc = rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3]) : 0.f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
@@ -714,23 +728,24 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (rc.valid) {
 #pragma unroll
-                    for (int k = 0; k < 32; k += 4)
-                        *reinterpret_cast<float4 *>(orow + ch * 32 + k) =
-                            make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+                    for (int k = 0; k < 32; k += 8) {
+                        uint4 v;
+                        __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+#pragma unroll
+                        for (int z = 0; z < 4; ++z)
+                            h2[z] = __floats2half2_rn(gc * o[k + 2 * z], gc * o[k + 2 * z + 1]);
+                        __stcs(reinterpret_cast<uint4 *>(part + ch * 32 + k), v);
+                    }
                     if (L.dbg_o_cmp)
                         for (int k = 0; k < 32; ++k) L.dbg_o_cmp[prow + ch * 32 + k] = o[k];
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
         } else if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
-            float g = 0.f, gc = 0.f;
-            if (rc.valid) {
-                const float *gl = L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3;
-                gc = sigmoidf_(gl[0]);
-                g = sigmoidf_(gl[P.mode == MODE_SLC ? 1 : 2]);
-            }
+            const float g =
+                rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (P.mode == MODE_SLC ? 1 : 2)])
+                         : 0.f;
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            float *part = L.o_cmp_ws + qrow;
             float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
             __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
@@ -740,29 +755,32 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
 #pragma unroll
-                for (int k = 0; k < 32; k += 4) {
-                    float4 pr = *reinterpret_cast<float4 *>(part + ch * 32 + k);
-                    float b4[4];
+                for (int k = 0; k < 32; k += 8) {
+                    uint4 pv4 = __ldcs(reinterpret_cast<const uint4 *>(part + ch * 32 + k));
+                    const __half2 *ph = reinterpret_cast<const __half2 *>(&pv4);
+                    float b8[8];
 #pragma unroll
-                    for (int z = 0; z < 4; ++z) b4[z] = l_run > 0.f ? o[k + z] * inv : 0.f;
+                    for (int z = 0; z < 8; ++z) b8[z] = l_run > 0.f ? o[k + z] * inv : 0.f;
                     if (dbg)
-                        for (int z = 0; z < 4; ++z) dbg[prow + ch * 32 + k + z] = b4[z];
+                        for (int z = 0; z < 8; ++z) dbg[prow + ch * 32 + k + z] = b8[z];
+                    uint4 v;
                     if (P.mode == MODE_SLC) {
-                        // partial = sig(g_cmp) o_cmp + sig(g_slc) o_slc, in place
-                        pr.x = gc * pr.x + g * b4[0];
-                        pr.y = gc * pr.y + g * b4[1];
-                        pr.z = gc * pr.z + g * b4[2];
-                        pr.w = gc * pr.w + g * b4[3];
-                        *reinterpret_cast<float4 *>(part + ch * 32 + k) = pr;
+                        __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+#pragma unroll
+                        for (int z = 0; z < 4; ++z) {
+                            const float2 f = __half22float2(ph[z]);
+                            h2[z] = __floats2half2_rn(f.x + g * b8[2 * z], f.y + g * b8[2 * z + 1]);
+                        }
+                        __stcs(reinterpret_cast<uint4 *>(part + ch * 32 + k), v);
                     } else {
-                        __nv_bfloat162 lo2 =
-                            __floats2bfloat162_rn(pr.x + g * b4[0], pr.y + g * b4[1]);
-                        __nv_bfloat162 hi2 =
-                            __floats2bfloat162_rn(pr.z + g * b4[2], pr.w + g * b4[3]);
-                        uint2 v;
-                        v.x = *reinterpret_cast<uint32_t *>(&lo2);
-                        v.y = *reinterpret_cast<uint32_t *>(&hi2);
-                        *reinterpret_cast<uint2 *>(orow + ch * 32 + k) = v;
+                        __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+                        for (int z = 0; z < 4; ++z) {
+                            const float2 f = __half22float2(ph[z]);
+                            b2[z] = __floats2bfloat162_rn(f.x + g * b8[2 * z],
+                                                          f.y + g * b8[2 * z + 1]);
+                        }
+                        __stcs(reinterpret_cast<uint4 *>(orow + ch * 32 + k), v);
                     }
                 }
             }
@@ -825,8 +843,10 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(sm.bar(B_KV_FULL + s), 1);
-            ptx::mbar_init(sm.bar(B_KV_EMPTY + s), 1);
+            ptx::mbar_init(sm.bar(B_K_FULL + s), 1);
+            ptx::mbar_init(sm.bar(B_V_FULL + s), 1);
+            ptx::mbar_init(sm.bar(B_K_EMPTY + s), 1);
+            ptx::mbar_init(sm.bar(B_V_EMPTY + s), 1);
         }
         ptx::mbar_init(sm.bar(B_S_FULL), 1);
         ptx::mbar_init(sm.bar(B_S_FREE), 128);
