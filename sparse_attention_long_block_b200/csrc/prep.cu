@@ -159,64 +159,116 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 // ---------------------------------------------------------------------------
 // Top-k block selection: one warp per (group g, vision query i).
 // Forced blocks: 0 and the query's own block i/B (when enabled) count within
-// top_k.  The remaining slots take the visible, non-forced blocks with the
+// top_k.  The remaining m slots take the visible, non-forced blocks with the
 // largest importance, ties to the lower block index.  Output ascending, -1
-// padded.  Importance values are probabilities (>= 0): a taken block is marked
-// with -1 in the shared copy of its row.
+// padded.
+//
+// Importance values are non-negative floats, so their bit patterns order like
+// the values.  The m-th largest key T is found by radix select over four 8-bit
+// digits (a 256-bin histogram per digit, counts added once per group of lanes
+// holding the same digit); the selection is then every candidate above T plus
+// the lowest-indexed candidates equal to T, which is the tie rule.
 __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
-    extern __shared__ float s_imp[];
+    extern __shared__ uint32_t sh_topk[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
     const int g = blockIdx.y;
     const Counts cn = *p.counts;
     if (i >= cn.n_vision) return;
-    float *s = s_imp + (size_t)warp * p.nb_max;
+    uint32_t *key = sh_topk + (size_t)warp * (p.nb_max + 256);  // [nb_max] keys
+    uint32_t *hist = key + p.nb_max;                            // [256]
     const int B = p.block;
     const int own = i / B;
     int c = (i + 1) / B;
     if (c > cn.nb) c = cn.nb;
-    const float *row = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
-    for (int j = lane; j < c; j += 32) s[j] = row[j];
-    __syncwarp();
-    int nforced = 0;
-    if (p.force_first) {
-        ++nforced;
-        if (c > 0 && lane == 0) s[0] = -1.f;
-    }
-    if (p.force_local && !(p.force_first && own == 0)) {
-        ++nforced;
-        if (own < c && lane == 0) s[own] = -1.f;
-    }
-    __syncwarp();
-    const bool extra = (p.force_local && own >= c) || (p.force_first && c == 0);
+    const bool f0 = p.force_first && c > 0;                    // block 0 forced and visible
+    const bool fo = p.force_local && own < c && !(f0 && own == 0);  // own block forced, visible
+    const int nforced = (p.force_first ? 1 : 0) + ((p.force_local && !(p.force_first && own == 0)) ? 1 : 0);
     const int m = p.top_k - nforced;
-    for (int round = 0; round < m; ++round) {
-        float bv = -1.f;
-        int bj = 0x7fffffff;
-        for (int j = lane; j < c; j += 32) {
-            const float x = s[j];
-            if (x > bv) { bv = x; bj = j; }  // lanes scan ascending j: ties keep lower j
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-            if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
-        }
-        if (bv < 0.f) break;  // no candidate left
-        if (lane == 0) s[bj] = -1.f;
-        __syncwarp();
+    const float *row = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
+    // candidates: visible, not forced; keys of non-candidates = 0 with a flag bit
+    // kept apart (a candidate's key is its float bits, always < 0x80000000)
+    int ncand = 0;
+    for (int j = lane; j < c; j += 32) {
+        const bool forced = (f0 && j == 0) || (fo && j == own);
+        key[j] = forced ? 0xFFFFFFFFu : __float_as_uint(fmaxf(row[j], 0.f));
+        ncand += forced ? 0 : 1;
     }
+    ncand = __reduce_add_sync(0xffffffffu, ncand);
+    __syncwarp();
+    uint32_t thr = 0, mask = 0;
+    int need = m;  // candidates still to take at or below the current prefix
+    const bool all = ncand <= m;
+    if (!all && m > 0) {
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int b = lane; b < 256; b += 32) hist[b] = 0u;
+            __syncwarp();
+            for (int base = 0; base < c; base += 32) {
+                const int j = base + lane;
+                const uint32_t kj = j < c ? key[j] : 0xFFFFFFFFu;
+                const bool in = kj != 0xFFFFFFFFu && (kj & mask) == thr;
+                const uint32_t digit = in ? (kj >> shift) & 255u : 256u + lane;
+                const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+                if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+            }
+            __syncwarp();
+            // the digit value holding the need-th largest: scan bins from the top
+            uint32_t h[8];
+            int local = 0;
+#pragma unroll
+            for (int z = 0; z < 8; ++z) {
+                h[z] = hist[255 - (lane * 8 + z)];
+                local += (int)h[z];
+            }
+            int incl = local;  // inclusive prefix over lanes (bins in descending order)
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const int excl = incl - local;
+            int found = -1, above = 0;
+            if (excl < need && incl >= need) {
+                int run = excl;
+#pragma unroll
+                for (int z = 0; z < 8; ++z) {
+                    if (found < 0 && run + (int)h[z] >= need) {
+                        found = 255 - (lane * 8 + z);
+                        above = run;
+                    }
+                    run += (int)h[z];
+                }
+            }
+            const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+            const int src = __ffs(who) - 1;
+            found = __shfl_sync(0xffffffffu, found, src);
+            above = __shfl_sync(0xffffffffu, above, src);
+            thr |= (uint32_t)found << shift;
+            mask |= 255u << shift;
+            need -= above;
+            __syncwarp();
+        }
+    }
+    // ascending output: forced visible blocks, candidates above thr, and the
+    // first `need` candidates equal to thr
     int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
-    int cnt = 0;
+    int cnt = 0, eq_taken = 0;
     for (int base = 0; base < c; base += 32) {
         const int j = base + lane;
-        const bool f = j < c && s[j] < 0.f;
-        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        const uint32_t kj = j < c ? key[j] : 0u;
+        const bool forced = j < c && kj == 0xFFFFFFFFu;
+        const bool cand = j < c && !forced;
+        const bool eq = cand && !all && kj == thr;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = eq_taken + __popc(eqb & ((1u << lane) - 1u));
+        const bool take = forced || (cand && (all || (m > 0 && (kj > thr || (eq && eq_rank < need)))));
+        eq_taken += __popc(eqb);
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
         const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-        if (f && pos < p.top_k) out[pos] = j;
+        if (take && pos < p.top_k) out[pos] = j;
         cnt += __popc(bal);
     }
+    const bool extra = (p.force_local && own >= c) || (p.force_first && c == 0);
     if (extra) {
         if (lane == 0 && cnt < p.top_k) out[cnt] = own;
         ++cnt;
@@ -226,7 +278,7 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
 }
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {
-    const size_t smem = (size_t)8 * p.nb_max * sizeof(float);
+    const size_t smem = (size_t)8 * (p.nb_max + 256) * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -589,39 +589,54 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 // S is in registers: let the next Q K^T overwrite it
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(sm.bar(B_S_FREE));
-                if (full) {
+                // mask on the raw scores (scale > 0 keeps the order)
+                if (!full) {
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) sv[k] *= sc;
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] * sc : -INFINITY;
+                    for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] : -INFINITY;
                 }
-                float mx;
+                float mx;  // row max of this tile, in log2 units
                 {
                     float m8[8];
 #pragma unroll
-                    for (int z = 0; z < 8; ++z) m8[z] = sv[z];
+                    for (int z = 0; z < 8; ++z) m8[z] = ptx::fmax3(sv[z], sv[8 + z], sv[16 + z]);
 #pragma unroll
-                    for (int k = 8; k < 64; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
-                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                    for (int k = 24; k < 64; k += 16)
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) m8[z] = ptx::fmax3(m8[z], sv[k + z], sv[k + 8 + z]);
+                    mx = ptx::fmax3(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], m8[5]),
+                                    fmaxf(m8[6], m8[7])) * sc;
                 }
+                // sv[k] <- 2^(sv[k] * sc - sub) in place, returning the sum
+                auto exp_sum = [&](float sub) {
+                    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 64; k += 4) {
+                        ptx::ffma2(sv[k], sv[k + 1], sv[k], sv[k + 1], sc, sc, -sub, -sub);
+                        ptx::ffma2(sv[k + 2], sv[k + 3], sv[k + 2], sv[k + 3], sc, sc, -sub, -sub);
+                        sv[k] = ptx::ex2(sv[k]);
+                        sv[k + 1] = ptx::ex2(sv[k + 1]);
+                        sv[k + 2] = ptx::ex2(sv[k + 2]);
+                        sv[k + 3] = ptx::ex2(sv[k + 3]);
+                        ptx::fadd2(a0, a1, a0, a1, sv[k], sv[k + 1]);
+                        ptx::fadd2(b0, b1, b0, b1, sv[k + 2], sv[k + 3]);
+                    }
+                    return (a0 + a1) + (b0 + b1);
+                };
                 if (kind == K_STATS) {
                     const float mn = fmaxf(m_run, mx);
                     const float mu = mn == -INFINITY ? 0.f : mn;
-                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) a8[k & 7] += ptx::ex2(sv[k] - mu);
-                    const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) +
-                                      ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+                    const float acc = exp_sum(mu);
                     l_run = l_run * ptx::ex2(m_run - mu) + acc;
                     m_run = mn;
                     continue;
                 }
                 if (kind == K_EXACT) {
-                    const bool live = lse2 != -INFINITY;
+                    if (lse2 != -INFINITY) {
+                        exp_sum(lse2);
+                    } else {
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) sv[k] = live ? ptx::ex2(sv[k] - lse2) : 0.f;
+                        for (int k = 0; k < 64; ++k) sv[k] = 0.f;
+                    }
                 } else {
                     // online softmax with lazy rescaling of O
                     const float mn = fmaxf(m_run, mx);
@@ -631,14 +646,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                         l_run *= factor;
                         m_run = mn;
                     }
-                    const float mu = m_run == -INFINITY ? 0.f : m_run;
-                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int k = 0; k < 64; ++k) {
-                        sv[k] = ptx::ex2(sv[k] - mu);
-                        a8[k & 7] += sv[k];
-                    }
-                    l_run += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+                    l_run += exp_sum(m_run == -INFINITY ? 0.f : m_run);
                 }
                 }  // !none
                 const uint32_t pb = npv & 1;
