@@ -164,10 +164,35 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 // padded.
 //
 // Importance values are non-negative floats, so their bit patterns order like
-// the values.  The m-th largest key T is found by radix select over four 8-bit
-// digits (a 256-bin histogram per digit, counts added once per group of lanes
-// holding the same digit); the selection is then every candidate above T plus
-// the lowest-indexed candidates equal to T, which is the tie rule.
+// the values; a block's sort key is (bits << 32) | ~index, so that the larger
+// key is the block the rule prefers.  Fast path: each lane keeps the two
+// largest candidate bit patterns of its blocks; the m-th largest of those 64
+// values cannot exceed the m-th largest candidate, so only candidates at or
+// above it can be selected.  If at most 128 survive, they are sorted
+// (bitonic, in shared memory) and the first m taken.  Otherwise m rounds of a
+// warp argmax select them exactly.
+__device__ __forceinline__ void warp_sort_desc(uint64_t *v, int n, int lane) {
+    // bitonic sort of n (power of two, <= 256) keys in shared memory, descending
+    for (int size = 2; size <= n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = lane; t < n / 2; t += 32) {
+                const int lo = 2 * t - (t & (stride - 1));
+                const int hi = lo + stride;
+                const bool desc = ((lo & size) == 0);
+                const uint64_t a = v[lo], b = v[hi];
+                if ((a < b) == desc) {
+                    v[lo] = b;
+                    v[hi] = a;
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+constexpr uint32_t kTaken = 0xFFFFFFFEu;   // selected (or forced) marker in key[]
+constexpr uint32_t kForced = 0xFFFFFFFFu;
+
 __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     extern __shared__ uint32_t sh_topk[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -175,94 +200,94 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     const int g = blockIdx.y;
     const Counts cn = *p.counts;
     if (i >= cn.n_vision) return;
-    uint32_t *key = sh_topk + (size_t)warp * (p.nb_max + 256);  // [nb_max] keys
-    uint32_t *hist = key + p.nb_max;                            // [256]
+    const int kstride = (p.nb_max + 1) & ~1;  // keeps buf 8-byte aligned
+    uint32_t *key = sh_topk + (size_t)warp * (kstride + 256);              // [nb_max]
+    uint64_t *buf = reinterpret_cast<uint64_t *>(key + kstride);           // [128]
     const int B = p.block;
     const int own = i / B;
     int c = (i + 1) / B;
     if (c > cn.nb) c = cn.nb;
-    const bool f0 = p.force_first && c > 0;                    // block 0 forced and visible
-    const bool fo = p.force_local && own < c && !(f0 && own == 0);  // own block forced, visible
-    const int nforced = (p.force_first ? 1 : 0) + ((p.force_local && !(p.force_first && own == 0)) ? 1 : 0);
+    const bool f0 = p.force_first && c > 0;
+    const bool fo = p.force_local && own < c && !(f0 && own == 0);
+    const int nforced =
+        (p.force_first ? 1 : 0) + ((p.force_local && !(p.force_first && own == 0)) ? 1 : 0);
     const int m = p.top_k - nforced;
     const float *row = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
-    // candidates: visible, not forced; keys of non-candidates = 0 with a flag bit
-    // kept apart (a candidate's key is its float bits, always < 0x80000000)
     int ncand = 0;
+    uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
     for (int j = lane; j < c; j += 32) {
         const bool forced = (f0 && j == 0) || (fo && j == own);
-        key[j] = forced ? 0xFFFFFFFFu : __float_as_uint(fmaxf(row[j], 0.f));
-        ncand += forced ? 0 : 1;
+        const uint32_t kj = forced ? kForced : __float_as_uint(fmaxf(row[j], 0.f));
+        key[j] = kj;
+        if (!forced) {
+            ++ncand;
+            if (kj > t1) { t2 = t1; t1 = kj; }
+            else if (kj > t2) { t2 = kj; }
+        }
     }
     ncand = __reduce_add_sync(0xffffffffu, ncand);
     __syncwarp();
-    uint32_t thr = 0, mask = 0;
-    int need = m;  // candidates still to take at or below the current prefix
-    const bool all = ncand <= m;
-    if (!all && m > 0) {
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int b = lane; b < 256; b += 32) hist[b] = 0u;
-            __syncwarp();
-            for (int base = 0; base < c; base += 32) {
-                const int j = base + lane;
-                const uint32_t kj = j < c ? key[j] : 0xFFFFFFFFu;
-                const bool in = kj != 0xFFFFFFFFu && (kj & mask) == thr;
-                const uint32_t digit = in ? (kj >> shift) & 255u : 256u + lane;
-                const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-                if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
-            }
-            __syncwarp();
-            // the digit value holding the need-th largest: scan bins from the top
-            uint32_t h[8];
-            int local = 0;
-#pragma unroll
-            for (int z = 0; z < 8; ++z) {
-                h[z] = hist[255 - (lane * 8 + z)];
-                local += (int)h[z];
-            }
-            int incl = local;  // inclusive prefix over lanes (bins in descending order)
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const int excl = incl - local;
-            int found = -1, above = 0;
-            if (excl < need && incl >= need) {
-                int run = excl;
-#pragma unroll
-                for (int z = 0; z < 8; ++z) {
-                    if (found < 0 && run + (int)h[z] >= need) {
-                        found = 255 - (lane * 8 + z);
-                        above = run;
-                    }
-                    run += (int)h[z];
-                }
-            }
-            const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
-            const int src = __ffs(who) - 1;
-            found = __shfl_sync(0xffffffffu, found, src);
-            above = __shfl_sync(0xffffffffu, above, src);
-            thr |= (uint32_t)found << shift;
-            mask |= 255u << shift;
-            need -= above;
-            __syncwarp();
+    if (m > 0 && ncand > m) {
+        // lower bound T0 of the m-th largest candidate value
+        buf[lane] = t1;
+        buf[lane + 32] = t2;
+        __syncwarp();
+        warp_sort_desc(buf, 64, lane);
+        const uint32_t t0 = (uint32_t)buf[min(m, 64) - 1];
+        __syncwarp();
+        // survivors: candidates with bits >= t0
+        int cnt = 0;
+        for (int base = 0; base < c; base += 32) {
+            const int j = base + lane;
+            const bool sv = j < c && key[j] != kForced && key[j] >= t0;
+            const unsigned bal = __ballot_sync(0xffffffffu, sv);
+            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            if (sv && pos < 128) buf[pos] = ((uint64_t)key[j] << 32) | (uint32_t)(~(uint32_t)j);
+            cnt += __popc(bal);
         }
+        __syncwarp();
+        if (cnt <= 128) {
+            int n2 = 32;
+            while (n2 < cnt) n2 <<= 1;
+            for (int x = cnt + lane; x < n2; x += 32) buf[x] = 0ull;  // smallest keys
+            __syncwarp();
+            warp_sort_desc(buf, n2, lane);
+            for (int x = lane; x < m; x += 32) {
+                const int j = (int)(~(uint32_t)buf[x]);
+                key[j] = kTaken;
+            }
+        } else {
+            // exact fallback: m rounds of a warp argmax over the candidates
+            for (int round = 0; round < m; ++round) {
+                uint64_t best = 0;
+                for (int j = lane; j < c; j += 32) {
+                    const uint32_t kj = key[j];
+                    if (kj >= kTaken) continue;
+                    const uint64_t kk = ((uint64_t)kj << 32) | (uint32_t)(~(uint32_t)j);
+                    if (kk > best) best = kk;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+                    if (other > best) best = other;
+                }
+                if (lane == 0) key[(int)(~(uint32_t)best)] = kTaken;
+                __syncwarp();
+            }
+        }
+        __syncwarp();
+    } else if (m > 0) {
+        for (int j = lane; j < c; j += 32)
+            if (key[j] != kForced) key[j] = kTaken;
     }
-    // ascending output: forced visible blocks, candidates above thr, and the
-    // first `need` candidates equal to thr
+    __syncwarp();
+    // ascending output: forced and selected visible blocks, then the own
+    // block when it is forced but not yet complete (it is above every visible one)
     int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
-    int cnt = 0, eq_taken = 0;
+    int cnt = 0;
     for (int base = 0; base < c; base += 32) {
         const int j = base + lane;
-        const uint32_t kj = j < c ? key[j] : 0u;
-        const bool forced = j < c && kj == 0xFFFFFFFFu;
-        const bool cand = j < c && !forced;
-        const bool eq = cand && !all && kj == thr;
-        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-        const int eq_rank = eq_taken + __popc(eqb & ((1u << lane) - 1u));
-        const bool take = forced || (cand && (all || (m > 0 && (kj > thr || (eq && eq_rank < need)))));
-        eq_taken += __popc(eqb);
+        const bool take = j < c && key[j] >= kTaken;
         const unsigned bal = __ballot_sync(0xffffffffu, take);
         const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
         if (take && pos < p.top_k) out[pos] = j;
@@ -278,7 +303,7 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
 }
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {
-    const size_t smem = (size_t)8 * (p.nb_max + 256) * sizeof(uint32_t);
+    const size_t smem = (size_t)8 * (((p.nb_max + 1) & ~1) + 256) * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
