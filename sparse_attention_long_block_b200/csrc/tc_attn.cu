@@ -598,11 +598,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 {
                     float m8[8];
 #pragma unroll
-                    for (int z = 0; z < 8; ++z) m8[z] = ptx::fmax3(sv[z], sv[8 + z], sv[16 + z]);
-#pragma unroll
-                    for (int k = 24; k < 64; k += 16)
-#pragma unroll
-                        for (int z = 0; z < 8; ++z) m8[z] = ptx::fmax3(m8[z], sv[k + z], sv[k + 8 + z]);
+                    for (int z = 0; z < 8; ++z) {
+                        m8[z] = ptx::fmax3(sv[z], sv[8 + z], sv[16 + z]);        // 0..23
+                        m8[z] = ptx::fmax3(m8[z], sv[24 + z], sv[32 + z]);       // 24..39
+                        m8[z] = ptx::fmax3(m8[z], sv[40 + z], sv[48 + z]);       // 40..55
+                        m8[z] = fmaxf(m8[z], sv[56 + z]);                        // 56..63
+                    }
                     mx = ptx::fmax3(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], m8[5]),
                                     fmaxf(m8[6], m8[7])) * sc;
                 }
