@@ -607,24 +607,19 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     mx = ptx::fmax3(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], m8[5]),
                                     fmaxf(m8[6], m8[7])) * sc;
                 }
-                // sv[k] <- 2^(sv[k] * sc - sub) in place, returning the sum; one
-                // pair in four goes through the FMA-pipe polynomial so that the
-                // special-function unit is not the only exponent path
+                // sv[k] <- 2^(sv[k] * sc - sub) in place, returning the sum
                 auto exp_sum = [&](float sub) {
                     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
-                    for (int k = 0; k < 64; k += 8) {
-#pragma unroll
-                        for (int z = 0; z < 8; z += 2)
-                            ptx::ffma2(sv[k + z], sv[k + z + 1], sv[k + z], sv[k + z + 1], sc, sc,
-                                       -sub, -sub);
-#pragma unroll
-                        for (int z = 0; z < 6; ++z) sv[k + z] = ptx::ex2(sv[k + z]);
-                        ptx::ex2_poly2(sv[k + 6], sv[k + 7], sv[k + 6], sv[k + 7]);
+                    for (int k = 0; k < 64; k += 4) {
+                        ptx::ffma2(sv[k], sv[k + 1], sv[k], sv[k + 1], sc, sc, -sub, -sub);
+                        ptx::ffma2(sv[k + 2], sv[k + 3], sv[k + 2], sv[k + 3], sc, sc, -sub, -sub);
+                        sv[k] = ptx::ex2(sv[k]);
+                        sv[k + 1] = ptx::ex2(sv[k + 1]);
+                        sv[k + 2] = ptx::ex2(sv[k + 2]);
+                        sv[k + 3] = ptx::ex2(sv[k + 3]);
                         ptx::fadd2(a0, a1, a0, a1, sv[k], sv[k + 1]);
                         ptx::fadd2(b0, b1, b0, b1, sv[k + 2], sv[k + 3]);
-                        ptx::fadd2(a0, a1, a0, a1, sv[k + 4], sv[k + 5]);
-                        ptx::fadd2(b0, b1, b0, b1, sv[k + 6], sv[k + 7]);
                     }
                     return (a0 + a1) + (b0 + b1);
                 };

@@ -262,32 +262,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for a pair of values on the FMA pipe instead of the special-function
-// unit.  x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial whose
-// coefficients were fitted for this library (weighted least squares on
-// Chebyshev nodes, max relative error 2.7e-6); 2^n is added to the exponent
-// field.  Inputs are clamped to >= -125 so the result stays a positive normal
-// float (the values below that are 0 for every use here, e.g. masked keys).
-__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float x1) {
-    constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
-    float t0, t1, n0, n1, f0, f1;
-    fadd2(t0, t1, x0, x1, kMagic, kMagic);
-    fadd2(n0, n1, t0, t1, -kMagic, -kMagic);
-    ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);  // f = x - n
-    float p0 = 0.009570094756782055f, p1 = 0.009570094756782055f;
-    ffma2(p0, p1, p0, p1, f0, f1, 0.05591785907745361f, 0.05591785907745361f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.240247443318367f, 0.240247443318367f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.6931217908859253f, 0.6931217908859253f);
-    ffma2(p0, p1, p0, p1, f0, f1, 0.9999992847442627f, 0.9999992847442627f);
-    const int e0 = (__float_as_int(t0) - 0x4B400000) << 23;
-    const int e1 = (__float_as_int(t1) - 0x4B400000) << 23;
-    y0 = __int_as_float(__float_as_int(p0) + e0);
-    y1 = __int_as_float(__float_as_int(p1) + e1);
-}
-
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
