@@ -423,10 +423,16 @@ def main():
 
 
 def layer_build_id():
-    """Identity of the built kernels (library mtime and size) for traffic records."""
-    from sparse_attention_long_block_b200 import binding
-    st = os.stat(binding.LIB_PATH)
-    return f"{st.st_size}"
+    """Identity of the kernel sources (hash of csrc) for stored traffic records:
+    a record taken on other kernels is not reported."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_attention_long_block_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
 if __name__ == "__main__":
