@@ -560,10 +560,18 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     lo = max(lo, 0);
                     hi = min(hi, kKeys - 1);
                 }
-                const bool full = __all_sync(0xffffffffu, lo == 0 && hi == kKeys - 1);
+                const bool row_in = lo <= hi;
+                const bool row_full = lo == 0 && hi == kKeys - 1;
+                // every row of the warp either takes the whole tile or none of
+                // it (selection tiles off the diagonal, interior window and
+                // text tiles): rows are masked by their exponent bias alone
+                const bool rowwise = __all_sync(0xffffffffu, row_full || !row_in);
                 // every row of this warp masked (common in selection tiles:
                 // most queries did not pick a given block): P = 0, no S read
-                const bool none = __all_sync(0xffffffffu, lo > hi);
+                const bool none = __all_sync(0xffffffffu, !row_in);
+                // a masked row in a row-wise tile: 2^(s * 0 - inf) = 0 for its
+                // whole row (scores of finite inputs are finite)
+                const bool kill = rowwise && !row_in;
                 bool r = ptx::mbar_wait(sm.bar(B_S_FULL), gt & 1, abort, L.status);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
@@ -590,7 +598,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(sm.bar(B_S_FREE));
                 // mask on the raw scores (scale > 0 keeps the order)
-                if (!full) {
+                if (!rowwise) {
 #pragma unroll
                     for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] : -INFINITY;
                 }
@@ -606,14 +614,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     }
                     mx = ptx::fmax3(ptx::fmax3(m8[0], m8[1], m8[2]), ptx::fmax3(m8[3], m8[4], m8[5]),
                                     fmaxf(m8[6], m8[7])) * sc;
+                    if (kill) mx = -INFINITY;
                 }
                 // sv[k] <- 2^(sv[k] * sc - sub) in place, returning the sum
                 auto exp_sum = [&](float sub) {
+                    const float s_r = kill ? 0.f : sc;
+                    const float b_r = kill ? -INFINITY : -sub;
                     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
                     for (int k = 0; k < 64; k += 4) {
-                        ptx::ffma2(sv[k], sv[k + 1], sv[k], sv[k + 1], sc, sc, -sub, -sub);
-                        ptx::ffma2(sv[k + 2], sv[k + 3], sv[k + 2], sv[k + 3], sc, sc, -sub, -sub);
+                        ptx::ffma2(sv[k], sv[k + 1], sv[k], sv[k + 1], s_r, s_r, b_r, b_r);
+                        ptx::ffma2(sv[k + 2], sv[k + 3], sv[k + 2], sv[k + 3], s_r, s_r, b_r, b_r);
                         sv[k] = ptx::ex2(sv[k]);
                         sv[k + 1] = ptx::ex2(sv[k + 1]);
                         sv[k + 2] = ptx::ex2(sv[k + 2]);
