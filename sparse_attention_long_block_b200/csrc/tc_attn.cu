@@ -13,11 +13,11 @@
 // GQA group): consecutive queries times the group's heads, so every K/V tile
 // serves the whole group.  Per item the CTA streams 64-key tiles:
 //   warp 0     TMA loads of K (and V) tiles into a 2-stage ring;
-//   warp 1     one thread issues S = Q K^T (M 128, N 64, K 128, bf16) into TMEM
-//              and O += P V (M 128, N 128, K 64, fp16, P read from TMEM);
-//   warps 2-5  one thread per row: S row from TMEM (released at once so the
-//              next S overlaps), mask, softmax, P (fp16) into TMEM, lazy O
-//              rescaling, epilogue.
+//   warp 1     one thread issues S = Q K^T (M 128, N 64, K 128, bf16) into one
+//              of two TMEM S buffers, a tile ahead of the softmax, and
+//              O += P V (M 128, N 128, K 64, fp16, P read from TMEM);
+//   warps 2-5  one thread per row: S row from TMEM, mask, softmax, P (fp16)
+//              into the same TMEM buffer, lazy O rescaling, epilogue.
 // Modes:
 //   CMP   keys = compressed blocks.  Segment 1: each row's log-sum-exp.
 //         Segment 2: exact probabilities, their sum over the group's heads
@@ -61,13 +61,16 @@ constexpr uint32_t SM_BAR = SM_PLAN + 2 * kPlanSmem * 4;      // barriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment slack
 
-// barrier slots (8 bytes each) after SM_BAR
+// barrier slots (8 bytes each) after SM_BAR; S_FULL and P_FULL per S buffer
 constexpr int B_K_FULL = 0, B_V_FULL = 2, B_K_EMPTY = 4, B_V_EMPTY = 6, B_S_FULL = 8,
-              B_S_FREE = 9, B_P_FULL = 10, B_PV_DONE = 12, B_Q_FULL = 14, B_GRP = 15,
-              B_FINAL = 16, B_COUNT = 17;
+              B_P_FULL = 10, B_PV_DONE = 12, B_Q_FULL = 14, B_GRP = 15, B_FINAL = 16,
+              B_COUNT = 17;
 
-// TMEM columns: S (fp32, 64), P buffers (fp16 pairs, 32 each), O (fp32, 128)
-constexpr uint32_t TM_S = 0, TM_P = 64, TM_O = 128, TM_COLS = 256;
+// TMEM columns: two S buffers (fp32, 64 each) and O (fp32, 128).  Tile x uses
+// S buffer x & 1; its P (fp16 pairs) overwrites the first 32 columns of that
+// buffer once the row is in registers, and Q K^T of tile x + 2 reuses the
+// buffer after P V of tile x (MMAs of one thread run in issue order).
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;
 
 enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3 };
 enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
@@ -317,14 +320,18 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
     const uint32_t q_addr = sm.base_u32 + SM_Q;
     uint32_t gt = 0, nitems = 0, npv = 0;  // npv: P V products = V tiles consumed
     bool ok = true;
-    auto issue_pv = [&](uint32_t acc) -> bool {
+    // Tile `pg` (global count) is finished once its softmax is done with the S
+    // buffer: wait for that, then issue its P V if the tile has one.
+    auto finish = [&](uint32_t pg, bool has_pv, uint32_t acc) -> bool {
+        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (pg & 1)), (pg >> 1) & 1, abort, L.status))
+            return false;
+        if (!has_pv) return true;
         const uint32_t sv = npv % kStages;
-        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (npv & 1)), (npv >> 1) & 1, abort, L.status) ||
-            !ptx::mbar_wait(sm.bar(B_V_FULL + sv), (npv / kStages) & 1, abort, L.status))
+        if (!ptx::mbar_wait(sm.bar(B_V_FULL + sv), (npv / kStages) & 1, abort, L.status))
             return false;
         ptx::tc_fence_after();
         const uint32_t vb = sm.base_u32 + SM_KV + kStages * K_BYTES + sv * K_BYTES;
-        const uint32_t pa = tmem + TM_P + (npv & 1) * 32;
+        const uint32_t pa = tmem + TM_S + (pg & 1) * 64;
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k)
             ptx::mma_ts(tmem + TM_O, pa + (uint32_t)k * 8u, desc_vmajor(vb + (uint32_t)k * 2048u),
@@ -340,39 +347,37 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         if (!ptx::mbar_wait(sm.bar(B_Q_FULL), nitems & 1, abort, L.status)) { ok = false; break; }
         ++nitems;
         ptx::tc_fence_after();
-        bool pending = false;
+        bool pending = false, pend_pv = false;
         uint32_t pend_acc = 0;
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
                 const uint32_t st = gt % kStages;
-                if (!ptx::mbar_wait(sm.bar(B_K_FULL + st), (gt / kStages) & 1, abort, L.status) ||
-                    (gt > 0 && !ptx::mbar_wait(sm.bar(B_S_FREE), (gt - 1) & 1, abort, L.status))) {
+                if (!ptx::mbar_wait(sm.bar(B_K_FULL + st), (gt / kStages) & 1, abort, L.status)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
                 const uint32_t kb = sm.base_u32 + SM_KV + st * K_BYTES;
+                const uint32_t sd = tmem + TM_S + (gt & 1) * 64;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t off = (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u;
                     const uint32_t koff = (uint32_t)(k >> 2) * 8192u + (uint32_t)(k & 3) * 32u;
-                    ptx::mma_ss(tmem + TM_S, desc_kmajor(q_addr + off), desc_kmajor(kb + koff),
-                                idesc_s, k > 0 ? 1u : 0u);
+                    ptx::mma_ss(sd, desc_kmajor(q_addr + off), desc_kmajor(kb + koff), idesc_s,
+                                k > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(sm.bar(B_S_FULL));
+                ptx::mma_commit(sm.bar(B_S_FULL + (gt & 1)));
                 ptx::mma_commit(sm.bar(B_K_EMPTY + st));  // K is dead once Q K^T is done
-                if (pending) {
-                    if (!issue_pv(pend_acc)) { ok = false; break; }
-                    pending = false;
-                }
-                if (kind_has_pv(kind)) {
-                    pending = true;
-                    pend_acc = x > 0 ? 1u : 0u;
-                }
+                // the previous tile: its P V follows this Q K^T in the pipe, and
+                // its S buffer is free for the next Q K^T after that
+                if (pending && !finish(gt - 1, pend_pv, pend_acc)) { ok = false; break; }
+                pending = true;
+                pend_pv = kind_has_pv(kind);
+                pend_acc = x > 0 ? 1u : 0u;
             }
         }
-        if (ok && pending && !issue_pv(pend_acc)) ok = false;
+        if (ok && pending && !finish(gt - 1, pend_pv, pend_acc)) ok = false;
     }
     // every MMA this thread issued has completed once this barrier flips
     ptx::mma_commit(sm.bar(B_FINAL));
@@ -572,7 +577,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 // a masked row in a row-wise tile: 2^(s * 0 - inf) = 0 for its
                 // whole row (scores of finite inputs are finite)
                 const bool kill = rowwise && !row_in;
-                bool r = ptx::mbar_wait(sm.bar(B_S_FULL), gt & 1, abort, L.status);
+                const uint32_t sbuf = gt & 1;
+                const uint32_t s_col = tmem + lane_base + TM_S + sbuf * 64;
+                bool r = ptx::mbar_wait(sm.bar(B_S_FULL + sbuf), (gt >> 1) & 1, abort, L.status);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -580,23 +587,27 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 bool need = false;
                 float factor = 1.f;
                 if (none) {
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(sm.bar(B_S_FREE));
-                    if (kind == K_STATS) continue;
+                    if (kind == K_STATS) {
+                        ptx::tc_fence_before();
+                        ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
+                        continue;
+                    }
 #pragma unroll
                     for (int k = 0; k < 64; ++k) sv[k] = 0.f;
                 } else {
                 {
                     float a[32], c[32];
-                    ptx::tmem_ld32(tmem + lane_base + TM_S, a);
-                    ptx::tmem_ld32(tmem + lane_base + TM_S + 32, c);
+                    ptx::tmem_ld32(s_col, a);
+                    ptx::tmem_ld32(s_col + 32, c);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 32; ++k) { sv[k] = a[k]; sv[32 + k] = c[k]; }
                 }
-                // S is in registers: let the next Q K^T overwrite it
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(sm.bar(B_S_FREE));
+                if (kind == K_STATS) {
+                    // no P: the S buffer is free as soon as the row is read
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
+                }
                 // mask on the raw scores (scale > 0 keeps the order)
                 if (!rowwise) {
 #pragma unroll
@@ -661,14 +672,6 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     l_run += exp_sum(m_run == -INFINITY ? 0.f : m_run);
                 }
                 }  // !none
-                const uint32_t pb = npv & 1;
-                // P buffer pb is free once P V #npv-2 (its last reader) is done
-                if (npv > 1) {
-                    bool r3 = ptx::mbar_wait(sm.bar(B_PV_DONE + pb), ((npv - 2) >> 1) & 1, abort,
-                                             L.status);
-                    ok = __all_sync(0xffffffffu, r3 && ok);
-                    if (!ok) break;
-                }
                 if (__any_sync(0xffffffffu, need && x > 0)) {
                     // O may only be rescaled once every earlier P V has landed
                     if (npv > 0) {
@@ -696,11 +699,11 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                         __half2 h2 = __floats2half2_rn(sv[2 * k], sv[2 * k + 1]);
                         pk[k] = *reinterpret_cast<uint32_t *>(&h2);
                     }
-                    ptx::tmem_st32u(tmem + lane_base + TM_P + pb * 32, pk);
+                    ptx::tmem_st32u(s_col, pk);
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(sm.bar(B_P_FULL + pb));
+                ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
                 ++npv;
                 if (kind == K_EXACT && !none) {
                     // block importance: the sum of the probabilities over the
@@ -868,9 +871,8 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
             ptx::mbar_init(sm.bar(B_K_EMPTY + s), 1);
             ptx::mbar_init(sm.bar(B_V_EMPTY + s), 1);
         }
-        ptx::mbar_init(sm.bar(B_S_FULL), 1);
-        ptx::mbar_init(sm.bar(B_S_FREE), 128);
         for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(sm.bar(B_S_FULL + b), 1);
             ptx::mbar_init(sm.bar(B_P_FULL + b), 128);
             ptx::mbar_init(sm.bar(B_PV_DONE + b), 1);
         }
