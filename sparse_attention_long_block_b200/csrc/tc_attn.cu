@@ -663,10 +663,14 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 } else {
                     // online softmax with lazy rescaling of O
                     const float mn = fmaxf(m_run, mx);
-                    need = mn > m_run + kRescale;
-                    if (need) {
-                        factor = ptx::ex2(m_run - mn);  // 0 if m_run = -inf
-                        l_run *= factor;
+                    if (mn > m_run + kRescale) {
+                        // a row with no key so far has O = 0 and l = 0 (all its
+                        // earlier P were 0): only a finite running max rescales
+                        if (m_run != -INFINITY) {
+                            need = true;
+                            factor = ptx::ex2(m_run - mn);
+                            l_run *= factor;
+                        }
                         m_run = mn;
                     }
                     l_run += exp_sum(m_run == -INFINITY ? 0.f : m_run);
