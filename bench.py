@@ -182,11 +182,13 @@ def cpu_baseline(wl, x, target_s=12.0, max_rows=None):
     nrows = int(min(wl.n, max(r2, (target_s - fixed) / slope)))
     if max_rows:
         nrows = min(nrows, max_rows)
-    rows = sample(nrows)
-    t0 = time.perf_counter()
-    oracle.forward(p, x["q"], x["k"], x["v"], x["is_vision"], x["gate"], x["w_k"], x["w_v"],
-                   rows=rows)
-    dt = time.perf_counter() - t0
+    rows, dt = timed(nrows)
+    if dt < 0.5 * target_s and nrows < wl.n and (not max_rows or nrows < max_rows):
+        # the two-point estimate undershot: rescale once by the observed rate
+        nrows = int(min(wl.n, nrows * target_s / max(dt, 1e-3)))
+        if max_rows:
+            nrows = min(nrows, max_rows)
+        rows, dt = timed(nrows)
     nt = int((~x["is_vision"][rows].astype(bool)).sum())
     return (len(rows) / dt, oracle.threads(),
             f"{len(rows)} of {wl.n} query rows ({len(rows) - nt} vision, {nt} text), "
