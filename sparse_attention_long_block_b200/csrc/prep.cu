@@ -165,12 +165,14 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 //
 // Importance values are non-negative floats, so their bit patterns order like
 // the values; a block's sort key is (bits << 32) | ~index, so that the larger
-// key is the block the rule prefers.  Fast path: each lane keeps the two
-// largest candidate bit patterns of its blocks; the m-th largest of those 64
-// values cannot exceed the m-th largest candidate, so only candidates at or
-// above it can be selected.  If at most 128 survive, they are sorted
-// (bitonic, in shared memory) and the first m taken.  Otherwise m rounds of a
-// warp argmax select them exactly.
+// key is the block the rule prefers (keys are unique).  Pass 1 (float4 loads
+// of the importance row) keeps each lane's two largest candidate bit
+// patterns; the m-th largest of those 64 values cannot exceed the m-th
+// largest candidate, so only candidates at or above it can be selected.
+// Pass 2 re-reads the row (now in cache) and collects those survivors; if at
+// most 128 survive they are sorted (bitonic, in shared memory) and the first
+// m taken, otherwise m rounds of a warp argmax over keys below the previous
+// pick select them exactly.  Shared memory is 1 KB per warp.
 __device__ __forceinline__ void warp_sort_desc(uint64_t *v, int n, int lane) {
     // bitonic sort of n (power of two, <= 256) keys in shared memory, descending
     for (int size = 2; size <= n; size <<= 1) {
@@ -190,19 +192,16 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t *v, int n, int lane) {
     }
 }
 
-constexpr uint32_t kTaken = 0xFFFFFFFEu;   // selected (or forced) marker in key[]
-constexpr uint32_t kForced = 0xFFFFFFFFu;
+constexpr int kTopkBuf = 128;  // survivors sorted in shared memory, per warp
 
 __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
-    extern __shared__ uint32_t sh_topk[];
+    __shared__ uint64_t sh_buf[8][kTopkBuf];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
     const int g = blockIdx.y;
     const Counts cn = *p.counts;
     if (i >= cn.n_vision) return;
-    const int kstride = (p.nb_max + 1) & ~1;  // keeps buf 8-byte aligned
-    uint32_t *key = sh_topk + (size_t)warp * (kstride + 256);              // [nb_max]
-    uint64_t *buf = reinterpret_cast<uint64_t *>(key + kstride);           // [128]
+    uint64_t *buf = sh_buf[warp];
     const int B = p.block;
     const int own = i / B;
     int c = (i + 1) / B;
@@ -212,23 +211,29 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     const int nforced =
         (p.force_first ? 1 : 0) + ((p.force_local && !(p.force_first && own == 0)) ? 1 : 0);
     const int m = p.top_k - nforced;
-    const float *row = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
-    int ncand = 0;
-    uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
-    for (int j = lane; j < c; j += 32) {
-        const bool forced = (f0 && j == 0) || (fo && j == own);
-        const uint32_t kj = forced ? kForced : __float_as_uint(fmaxf(row[j], 0.f));
-        key[j] = kj;
-        if (!forced) {
-            ++ncand;
-            if (kj > t1) { t2 = t1; t1 = kj; }
-            else if (kj > t2) { t2 = kj; }
-        }
-    }
-    ncand = __reduce_add_sync(0xffffffffu, ncand);
-    __syncwarp();
+    const int ncand = c - (f0 ? 1 : 0) - (fo ? 1 : 0);
+    const float4 *row4 =
+        reinterpret_cast<const float4 *>(p.imp + ((size_t)g * p.n_max + i) * p.imp_stride);
+    const int c4 = (c + 3) / 4;
+    auto is_cand = [&](int j) { return j < c && !(f0 && j == 0) && !(fo && j == own); };
+    auto key_of = [&](float v, int j) {
+        return ((uint64_t)__float_as_uint(fmaxf(v, 0.f)) << 32) | (uint32_t)(~(uint32_t)j);
+    };
+    int sel = 0;  // selected non-forced blocks, their keys in buf[0, sel)
     if (m > 0 && ncand > m) {
-        // lower bound T0 of the m-th largest candidate value
+        uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
+        for (int q = lane; q < c4; q += 32) {
+            const float4 v4 = __ldg(row4 + q);
+            const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (!is_cand(4 * q + e)) continue;
+                const uint32_t kj = __float_as_uint(fmaxf(vv[e], 0.f));
+                if (kj > t1) { t2 = t1; t1 = kj; }
+                else if (kj > t2) { t2 = kj; }
+            }
+        }
+        // lower bound t0 of the m-th largest candidate value
         buf[lane] = t1;
         buf[lane + 32] = t2;
         __syncwarp();
@@ -237,62 +242,93 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
         __syncwarp();
         // survivors: candidates with bits >= t0
         int cnt = 0;
-        for (int base = 0; base < c; base += 32) {
-            const int j = base + lane;
-            const bool sv = j < c && key[j] != kForced && key[j] >= t0;
-            const unsigned bal = __ballot_sync(0xffffffffu, sv);
-            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-            if (sv && pos < 128) buf[pos] = ((uint64_t)key[j] << 32) | (uint32_t)(~(uint32_t)j);
-            cnt += __popc(bal);
+        for (int base = 0; base < c4; base += 32) {
+            const int q = base + lane;
+            float vv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (q < c4) {
+                const float4 v4 = __ldg(row4 + q);
+                vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 4 * q + e;
+                const bool sv = q < c4 && is_cand(j) && __float_as_uint(fmaxf(vv[e], 0.f)) >= t0;
+                const unsigned bal = __ballot_sync(0xffffffffu, sv);
+                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                if (sv && pos < kTopkBuf) buf[pos] = key_of(vv[e], j);
+                cnt += __popc(bal);
+            }
         }
         __syncwarp();
-        if (cnt <= 128) {
+        if (cnt <= kTopkBuf) {
             int n2 = 32;
             while (n2 < cnt) n2 <<= 1;
             for (int x = cnt + lane; x < n2; x += 32) buf[x] = 0ull;  // smallest keys
             __syncwarp();
             warp_sort_desc(buf, n2, lane);
-            for (int x = lane; x < m; x += 32) {
-                const int j = (int)(~(uint32_t)buf[x]);
-                key[j] = kTaken;
-            }
         } else {
-            // exact fallback: m rounds of a warp argmax over the candidates
+            // exact fallback: m rounds of a warp argmax over the keys below the
+            // previous pick
+            uint64_t last = ~0ull;
             for (int round = 0; round < m; ++round) {
                 uint64_t best = 0;
-                for (int j = lane; j < c; j += 32) {
-                    const uint32_t kj = key[j];
-                    if (kj >= kTaken) continue;
-                    const uint64_t kk = ((uint64_t)kj << 32) | (uint32_t)(~(uint32_t)j);
-                    if (kk > best) best = kk;
+                for (int q = lane; q < c4; q += 32) {
+                    const float4 v4 = __ldg(row4 + q);
+                    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * q + e;
+                        if (!is_cand(j)) continue;
+                        const uint64_t kk = key_of(vv[e], j);
+                        if (kk < last && kk > best) best = kk;
+                    }
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
                     if (other > best) best = other;
                 }
-                if (lane == 0) key[(int)(~(uint32_t)best)] = kTaken;
+                __syncwarp();
+                if (lane == 0) buf[round] = best;
+                last = best;
                 __syncwarp();
             }
         }
-        __syncwarp();
+        sel = m;
     } else if (m > 0) {
-        for (int j = lane; j < c; j += 32)
-            if (key[j] != kForced) key[j] = kTaken;
+        // every non-forced visible block is selected
+        int cnt = 0;
+        for (int base = 0; base < c; base += 32) {
+            const int j = base + lane;
+            const bool t = is_cand(j);
+            const unsigned bal = __ballot_sync(0xffffffffu, t);
+            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            if (t && pos < kTopkBuf) buf[pos] = (uint32_t)(~(uint32_t)j);
+            cnt += __popc(bal);
+        }
+        sel = min(cnt, kTopkBuf);
     }
     __syncwarp();
-    // ascending output: forced and selected visible blocks, then the own
-    // block when it is forced but not yet complete (it is above every visible one)
-    int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
-    int cnt = 0;
-    for (int base = 0; base < c; base += 32) {
-        const int j = base + lane;
-        const bool take = j < c && key[j] >= kTaken;
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-        if (take && pos < p.top_k) out[pos] = j;
-        cnt += __popc(bal);
+    // ascending output: the picks and the visible forced blocks sorted by
+    // index (keys ~j, descending), then the own block when it is forced but
+    // not yet complete (it is above every visible one)
+    for (int x = lane; x < sel; x += 32) buf[x] = (uint32_t)buf[x];
+    __syncwarp();
+    int total = sel;
+    if (lane == 0) {
+        if (f0) buf[total] = (uint32_t)(~0u);
+        if (fo) buf[total + (f0 ? 1 : 0)] = (uint32_t)(~(uint32_t)own);
     }
+    total += (f0 ? 1 : 0) + (fo ? 1 : 0);
+    int n2 = 32;
+    while (n2 < total) n2 <<= 1;
+    __syncwarp();
+    for (int x = total + lane; x < n2; x += 32) buf[x] = 0ull;
+    __syncwarp();
+    warp_sort_desc(buf, n2, lane);
+    int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
+    for (int x = lane; x < total && x < p.top_k; x += 32) out[x] = (int)(~(uint32_t)buf[x]);
+    int cnt = total;
     const bool extra = (p.force_local && own >= c) || (p.force_first && c == 0);
     if (extra) {
         if (lane == 0 && cnt < p.top_k) out[cnt] = own;
@@ -303,15 +339,8 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
 }
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {
-    const size_t smem = (size_t)8 * (((p.nb_max + 1) & ~1) + 256) * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(topk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-    }
     dim3 grid((p.n_max + 7) / 8, p.h_kv);
-    topk_kernel<<<grid, 256, smem, s>>>(p);
+    topk_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
