@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     int sel = 0;  // selected non-forced blocks, their keys in buf[0, sel)
     if (m > 0 && ncand > m) {
         uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
+#pragma unroll 4
         for (int q = lane; q < c4; q += 32) {
             const float4 v4 = __ldg(row4 + q);
             const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
         __syncwarp();
         // survivors: candidates with bits >= t0
         int cnt = 0;
+#pragma unroll 2
         for (int base = 0; base < c4; base += 32) {
             const int q = base + lane;
             float vv[4] = {0.f, 0.f, 0.f, 0.f};

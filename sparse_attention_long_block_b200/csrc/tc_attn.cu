@@ -545,8 +545,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             const int kind = it.seg_kind[s];
             m_run = -INFINITY;
             l_run = 0.f;
+            // selection tiles: the plan entry of the next tile is read from
+            // shared memory one tile ahead, off the tile's critical path
+            int nkey0 = 0;
+            uint32_t nmask = 0u;
+            if (kind == K_SLC && it.seg_tiles[s] > 0) {
+                nkey0 = plan_s[0];
+                nmask = (uint32_t)plan_s[kPlanSmem];
+            }
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
-                const int key0 = kind == K_SLC ? plan_s[x] : tile_key0(P, it, item, kind, x);
+                const int key0 = kind == K_SLC ? nkey0 : tile_key0(P, it, item, kind, x);
+                const uint32_t qmask = nmask;
                 // column range [lo, hi] of valid keys for this row
                 int lo = 1, hi = 0;
                 if (rc.valid) {
@@ -554,7 +563,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                         case K_STATS:
                         case K_EXACT: lo = 0; hi = rc.c_vis - 1 - key0; break;
                         case K_SLC:
-                            if (((uint32_t)plan_s[kPlanSmem + x] >> rc.qi) & 1u) {
+                            if ((qmask >> rc.qi) & 1u) {
                                 lo = 0;
                                 hi = rc.i - key0;
                             }
@@ -583,13 +592,18 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                if (kind == K_SLC && x + 1 < it.seg_tiles[s]) {
+                    nkey0 = plan_s[x + 1];
+                    nmask = (uint32_t)plan_s[kPlanSmem + x + 1];
+                }
                 float sv[64];
                 bool need = false;
                 float factor = 1.f;
                 if (none) {
                     if (kind == K_STATS) {
                         ptx::tc_fence_before();
-                        ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
                         continue;
                     }
 #pragma unroll
@@ -606,7 +620,8 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 if (kind == K_STATS) {
                     // no P: the S buffer is free as soon as the row is read
                     ptx::tc_fence_before();
-                    ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
                 }
                 // mask on the raw scores (scale > 0 keeps the order)
                 if (!rowwise) {
@@ -707,7 +722,8 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(sm.bar(B_P_FULL + sbuf));  // one per warp
                 ++npv;
                 if (kind == K_EXACT && !none) {
                     // block importance: the sum of the probabilities over the
@@ -877,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(sm.bar(B_S_FULL + b), 1);
-            ptx::mbar_init(sm.bar(B_P_FULL + b), 128);
+            ptx::mbar_init(sm.bar(B_P_FULL + b), 4);
             ptx::mbar_init(sm.bar(B_PV_DONE + b), 1);
         }
         ptx::mbar_init(sm.bar(B_Q_FULL), 128);
