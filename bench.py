@@ -405,6 +405,7 @@ def main():
             "config": {"workload": wl.name, "tokens": wl.n, "n_vision": wl.n_vision,
                        "n_text": wl.n_text, "h_q": wl.h_q, "h_kv": wl.h_kv, "d": wl.d,
                        "block": wl.block, "top_k": wl.top_k, "window": wl.window,
+                       "attention": "dense (all tokens text)" if wl.dense else "hybrid",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (no flush)"},
             "tensor_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],

@@ -21,6 +21,9 @@ frame-mean model because no video data or trained weights are available:
   round-to-nearest-even; values are kept as float32 arrays holding exact bf16
   values, so the GPU and the oracle read identical numbers.
 * Vision tokens come first and text tokens follow, unless a mask is given.
+* ``dense`` workloads (Dense-NSA: the same tokens under full causal attention)
+  draw the same tensors and mark every token as text, so every query attends
+  to all earlier tokens.
 """
 from __future__ import annotations
 
@@ -45,6 +48,7 @@ class Workload:
     ar1: bool = False            # AR(1) drift of K/V frame means
     seed: int = 0
     block: int = 64
+    dense: bool = False          # Dense-NSA: every token attends densely (no vision set)
 
     @property
     def n(self) -> int:
@@ -68,6 +72,11 @@ WORKLOADS = {
     "sweep_64k_k8_w1024": Workload("sweep_64k_k8_w1024", 65024, 512, top_k=8, window=1024),
     "sweep_64k_k16_w512": Workload("sweep_64k_k16_w512", 65024, 512, top_k=16, window=512),
     "sweep_64k_k32_w128": Workload("sweep_64k_k32_w128", 65024, 512, top_k=32, window=128),
+    # Dense-NSA: the 8K, 36K and 128K token streams under full causal attention.
+    "dense_8k": Workload("dense_8k", 8192, 256, top_k=16, window=256, dense=True),
+    "dense_36k": Workload("dense_36k", 35840, 512, top_k=16, window=256, dense=True),
+    "dense_128k": Workload("dense_128k", 130048, 1024, top_k=32, window=512, ar1=True,
+                           dense=True),
 }
 
 
@@ -111,6 +120,8 @@ def generate(wl: Workload, is_vision: np.ndarray | None = None) -> dict:
     must hold wl.n_vision ones among wl.n entries.
     """
     n = wl.n
+    if wl.dense and is_vision is not None:
+        raise ValueError("a dense workload takes no mask")
     if is_vision is None:
         is_vision = np.zeros(n, np.uint8)
         is_vision[: wl.n_vision] = 1
@@ -137,6 +148,8 @@ def generate(wl: Workload, is_vision: np.ndarray | None = None) -> dict:
         w_k, w_v = bf16_round(w_k), bf16_round(w_v)
     elif wl.dtype != "fp32":
         raise ValueError(f"unknown dtype {wl.dtype}")
+    if wl.dense:
+        is_vision = np.zeros(n, np.uint8)
     return dict(q=tensors["q"], k=tensors["k"], v=tensors["v"], is_vision=is_vision,
                 gate=gate, w_k=w_k, w_v=w_v)
 

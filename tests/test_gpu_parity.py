@@ -53,6 +53,23 @@ def test_long_128k_sampled_rows():
     compare_layer(wl, x, rows=rows, want_branches=False)
 
 
+def test_dense_nsa_8k_full():
+    """Dense-NSA (every token attends densely; the text path over all tokens)."""
+    wl = WORKLOADS["dense_8k"]
+    x = generate(wl)
+    assert int(x["is_vision"].sum()) == 0
+    stats = compare_layer(wl, x, want_branches=False)
+    assert stats["rows"] == wl.n
+
+
+@pytest.mark.parametrize("name,max_text", [("dense_36k", 96), ("dense_128k", 48)])
+def test_dense_nsa_sampled_rows(name, max_text):
+    wl = WORKLOADS[name]
+    x = generate(wl)
+    rows = stratified_rows(x["is_vision"], max_text=max_text)
+    compare_layer(wl, x, rows=rows, want_branches=False)
+
+
 EDGE = [
     # ragged: vision count not a multiple of 64, odd text count
     dict(n_vision=1000, n_text=37),
