@@ -146,6 +146,31 @@ vnsa_status vnsa_forward_host(vnsa_handle *h, int n, const void *q, const void *
                               const float *gate_logits, void *out, void *stream);
 
 /*
+ * One decode step ("VideoNSA: Native Sparse Attention Scales Video
+ * Understanding", paper notes, section "Method", applied to a single new
+ * token): the attention output of token n-1, appended to the token stream that
+ * the previous vnsa_forward or vnsa_decode on this handle processed (that call
+ * must have covered exactly tokens 0..n-2 of the same stream; otherwise
+ * VNSA_ERR_INVALID_ARG).  The result equals row n-1 of vnsa_forward over all n
+ * tokens: a vision token attends through compression (the complete vision
+ * blocks so far), selection and the window with its gates, a text token
+ * densely to every token 0..n-1.
+ *
+ * Inputs (device, 16-byte aligned): k, v [n][h_kv][d] and is_vision [n] hold the
+ * whole stream, the new token last (the caller appends it to its cache);
+ * q_new [h_q][d] and gate_new [h_q][3] (fp32, ignored for a text token) belong
+ * to the new token.  Output: out_new [h_q][d].  sel_out, if not NULL, receives
+ * the selected blocks [h_kv][top_k] (ascending, -1 padded; all -1 for a text
+ * token).  The handle's workspace keeps the stream's vision/text lists and the
+ * block keys/values; the step extends them (pooling the block the token
+ * completes, if any).  n <= n_max.  Asynchronous on `stream`; device-detected
+ * errors go to the status word.
+ */
+vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k, const void *v,
+                        const uint8_t *is_vision, const float *gate_new, void *out_new,
+                        int32_t *sel_out, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device status word.
  * *code receives VNSA_OK or the first device-detected error (TIMEOUT, BOUNDS).
  */

@@ -24,7 +24,7 @@ NUM_STAGES = 7
 EXPORTED = ("vnsa_status_string", "vnsa_stage_name", "vnsa_workspace_bytes", "vnsa_create",
             "vnsa_forward", "vnsa_forward_host", "vnsa_get_device_status", "vnsa_get_counts",
             "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy",
-            "vnsa_select_noalloc")
+            "vnsa_select_noalloc", "vnsa_decode")
 
 
 class vnsa_config(ctypes.Structure):
@@ -70,6 +70,7 @@ def load(path: str = LIB_PATH):
     lib.vnsa_create.argtypes = [ctypes.POINTER(vnsa_config), P, P, ctypes.POINTER(P)]
     lib.vnsa_forward.argtypes = [P, I, P, P, P, P, P, P, ctypes.POINTER(vnsa_debug), P]
     lib.vnsa_forward_host.argtypes = [P, I, P, P, P, P, P, P, P]
+    lib.vnsa_decode.argtypes = [P, I, P, P, P, P, P, P, P, P]
     lib.vnsa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.vnsa_get_counts.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.vnsa_set_timing.argtypes = [P, I]
@@ -118,6 +119,11 @@ def vnsa_forward(h, n, q, k, v, is_vision, gate, out, dbg=None, stream=0):
 
 def vnsa_forward_host(h, n, q, k, v, is_vision, gate, out, stream=0):
     _check("vnsa_forward_host", load().vnsa_forward_host(h, n, q, k, v, is_vision, gate, out, stream))
+
+
+def vnsa_decode(h, n, q_new, k, v, is_vision, gate_new, out_new, sel_out=None, stream=0):
+    _check("vnsa_decode", load().vnsa_decode(h, n, q_new, k, v, is_vision, gate_new, out_new,
+                                             sel_out, stream))
 
 
 def vnsa_get_device_status(h, stream=0) -> int:
@@ -205,6 +211,23 @@ class Layer:
         vnsa_forward(self.handle, n, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                      is_vision.data_ptr(), gate.data_ptr(), out.data_ptr(), dbg,
                      self._stream(stream))
+        return out
+
+    def decode(self, n, q_new, k, v, is_vision, gate_new, out=None, sel_out=None, stream=None):
+        """One decode step: the output of token n-1 of the stream in k, v,
+        is_vision (all n tokens), continuing the previous forward/decode call
+        over tokens 0..n-2.  q_new [h_q][d], gate_new [h_q][3]."""
+        import torch
+        for t in (q_new, k, v, is_vision, gate_new):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("inputs must be contiguous CUDA tensors")
+        if q_new.dtype != self.tdtype or k.dtype != self.tdtype or v.dtype != self.tdtype:
+            raise ValueError("q, k, v must match the layer dtype")
+        if out is None:
+            out = torch.empty_like(q_new)
+        vnsa_decode(self.handle, int(n), q_new.data_ptr(), k.data_ptr(), v.data_ptr(),
+                    is_vision.data_ptr(), gate_new.data_ptr(), out.data_ptr(),
+                    None if sel_out is None else sel_out.data_ptr(), self._stream(stream))
         return out
 
     def forward_host(self, q, k, v, is_vision, gate, out, stream=None):

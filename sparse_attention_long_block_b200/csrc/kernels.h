@@ -39,7 +39,7 @@ cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s);
+                             int nb_max, cudaStream_t s, int from_pad = 0);
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s);
 

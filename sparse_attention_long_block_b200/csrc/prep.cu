@@ -7,6 +7,7 @@
 // one block key and value through a learned projection (a d x d linear map
 // here); the selection branch keeps the top-k blocks ranked by importance.
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace vnsa {
 
@@ -85,14 +86,16 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_proj_kernel(
     const T *__restrict__ k, const T *__restrict__ v, const int32_t *__restrict__ vis,
     const Counts *__restrict__ counts, const T *__restrict__ w_k, const T *__restrict__ w_v,
-    T *__restrict__ k_cmp, T *__restrict__ v_cmp, int h_kv, int block) {
+    T *__restrict__ k_cmp, T *__restrict__ v_cmp, int h_kv, int block, int from_pad) {
     constexpr int JB = 16;             // blocks per CTA
     constexpr int PER = D / 32;        // elements per lane in a row
     constexpr int NPART = 256 / D;     // threads per output column
     constexpr int JBP = JB / NPART;    // blocks per thread in the projection
     __shared__ float mean[JB][D];
     const int nb = counts->nb;
-    const int j0 = blockIdx.x * JB;
+    // from_pad: only the blocks from counts->pad[0] on (the block a decode
+    // step completed, or none)
+    const int j0 = (from_pad ? counts->pad[0] : 0) + blockIdx.x * JB;
     if (j0 >= nb) return;
     const int g = blockIdx.y;
     const bool is_v = blockIdx.z != 0;
@@ -140,13 +143,13 @@ __global__ void __launch_bounds__(256) pool_proj_kernel(
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s) {
+                             int nb_max, cudaStream_t s, int from_pad) {
     if (nb_max <= 0) return cudaSuccess;
-    dim3 grid((nb_max + 15) / 16, h_kv, 2);
+    dim3 grid(from_pad ? 1 : (nb_max + 15) / 16, h_kv, 2);
 #define VNSA_POOL(T, D)                                                                  \
     pool_proj_kernel<T, D><<<grid, 256, 0, s>>>(                                         \
         (const T *)k, (const T *)v, vis, counts, (const T *)w_k, (const T *)w_v,         \
-        (T *)k_cmp, (T *)v_cmp, h_kv, block)
+        (T *)k_cmp, (T *)v_cmp, h_kv, block, from_pad)
     if (dtype == VNSA_BF16 && d == 128) VNSA_POOL(__nv_bfloat16, 128);
     else if (dtype == VNSA_BF16 && d == 64) VNSA_POOL(__nv_bfloat16, 64);
     else if (dtype == VNSA_FP32 && d == 128) VNSA_POOL(float, 128);
@@ -157,43 +160,7 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 }
 
 // ---------------------------------------------------------------------------
-// Top-k block selection: one warp per (group g, vision query i).
-// Forced blocks: 0 and the query's own block i/B (when enabled) count within
-// top_k.  The remaining m slots take the visible, non-forced blocks with the
-// largest importance, ties to the lower block index.  Output ascending, -1
-// padded.
-//
-// Importance values are non-negative floats, so their bit patterns order like
-// the values; a block's sort key is (bits << 32) | ~index, so that the larger
-// key is the block the rule prefers (keys are unique).  Pass 1 (float4 loads
-// of the importance row) keeps each lane's two largest candidate bit
-// patterns; the m-th largest of those 64 values cannot exceed the m-th
-// largest candidate, so only candidates at or above it can be selected.
-// Pass 2 re-reads the row (now in cache) and collects those survivors; if at
-// most 128 survive they are sorted (bitonic, in shared memory) and the first
-// m taken, otherwise m rounds of a warp argmax over keys below the previous
-// pick select them exactly.  Shared memory is 1 KB per warp.
-__device__ __forceinline__ void warp_sort_desc(uint64_t *v, int n, int lane) {
-    // bitonic sort of n (power of two, <= 256) keys in shared memory, descending
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = lane; t < n / 2; t += 32) {
-                const int lo = 2 * t - (t & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = ((lo & size) == 0);
-                const uint64_t a = v[lo], b = v[hi];
-                if ((a < b) == desc) {
-                    v[lo] = b;
-                    v[hi] = a;
-                }
-            }
-            __syncwarp();
-        }
-    }
-}
-
-constexpr int kTopkBuf = 128;  // survivors sorted in shared memory, per warp
-
+// Top-k block selection (topk.cuh): one warp per (group g, vision query i).
 __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     __shared__ uint64_t sh_buf[8][kTopkBuf];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -201,143 +168,11 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     const int g = blockIdx.y;
     const Counts cn = *p.counts;
     if (i >= cn.n_vision) return;
-    uint64_t *buf = sh_buf[warp];
-    const int B = p.block;
-    const int own = i / B;
-    int c = (i + 1) / B;
+    int c = (i + 1) / p.block;
     if (c > cn.nb) c = cn.nb;
-    const bool f0 = p.force_first && c > 0;
-    const bool fo = p.force_local && own < c && !(f0 && own == 0);
-    const int nforced =
-        (p.force_first ? 1 : 0) + ((p.force_local && !(p.force_first && own == 0)) ? 1 : 0);
-    const int m = p.top_k - nforced;
-    const int ncand = c - (f0 ? 1 : 0) - (fo ? 1 : 0);
-    const float4 *row4 =
-        reinterpret_cast<const float4 *>(p.imp + ((size_t)g * p.n_max + i) * p.imp_stride);
-    const int c4 = (c + 3) / 4;
-    auto is_cand = [&](int j) { return j < c && !(f0 && j == 0) && !(fo && j == own); };
-    auto key_of = [&](float v, int j) {
-        return ((uint64_t)__float_as_uint(fmaxf(v, 0.f)) << 32) | (uint32_t)(~(uint32_t)j);
-    };
-    int sel = 0;  // selected non-forced blocks, their keys in buf[0, sel)
-    if (m > 0 && ncand > m) {
-        uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
-#pragma unroll 4
-        for (int q = lane; q < c4; q += 32) {
-            const float4 v4 = __ldg(row4 + q);
-            const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                if (!is_cand(4 * q + e)) continue;
-                const uint32_t kj = __float_as_uint(fmaxf(vv[e], 0.f));
-                if (kj > t1) { t2 = t1; t1 = kj; }
-                else if (kj > t2) { t2 = kj; }
-            }
-        }
-        // lower bound t0 of the m-th largest candidate value
-        buf[lane] = t1;
-        buf[lane + 32] = t2;
-        __syncwarp();
-        warp_sort_desc(buf, 64, lane);
-        const uint32_t t0 = (uint32_t)buf[min(m, 64) - 1];
-        __syncwarp();
-        // survivors: candidates with bits >= t0
-        int cnt = 0;
-#pragma unroll 2
-        for (int base = 0; base < c4; base += 32) {
-            const int q = base + lane;
-            float vv[4] = {0.f, 0.f, 0.f, 0.f};
-            if (q < c4) {
-                const float4 v4 = __ldg(row4 + q);
-                vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 4 * q + e;
-                const bool sv = q < c4 && is_cand(j) && __float_as_uint(fmaxf(vv[e], 0.f)) >= t0;
-                const unsigned bal = __ballot_sync(0xffffffffu, sv);
-                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-                if (sv && pos < kTopkBuf) buf[pos] = key_of(vv[e], j);
-                cnt += __popc(bal);
-            }
-        }
-        __syncwarp();
-        if (cnt <= kTopkBuf) {
-            int n2 = 32;
-            while (n2 < cnt) n2 <<= 1;
-            for (int x = cnt + lane; x < n2; x += 32) buf[x] = 0ull;  // smallest keys
-            __syncwarp();
-            warp_sort_desc(buf, n2, lane);
-        } else {
-            // exact fallback: m rounds of a warp argmax over the keys below the
-            // previous pick
-            uint64_t last = ~0ull;
-            for (int round = 0; round < m; ++round) {
-                uint64_t best = 0;
-                for (int q = lane; q < c4; q += 32) {
-                    const float4 v4 = __ldg(row4 + q);
-                    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * q + e;
-                        if (!is_cand(j)) continue;
-                        const uint64_t kk = key_of(vv[e], j);
-                        if (kk < last && kk > best) best = kk;
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-                    if (other > best) best = other;
-                }
-                __syncwarp();
-                if (lane == 0) buf[round] = best;
-                last = best;
-                __syncwarp();
-            }
-        }
-        sel = m;
-    } else if (m > 0) {
-        // every non-forced visible block is selected
-        int cnt = 0;
-        for (int base = 0; base < c; base += 32) {
-            const int j = base + lane;
-            const bool t = is_cand(j);
-            const unsigned bal = __ballot_sync(0xffffffffu, t);
-            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-            if (t && pos < kTopkBuf) buf[pos] = (uint32_t)(~(uint32_t)j);
-            cnt += __popc(bal);
-        }
-        sel = min(cnt, kTopkBuf);
-    }
-    __syncwarp();
-    // ascending output: the picks and the visible forced blocks sorted by
-    // index (keys ~j, descending), then the own block when it is forced but
-    // not yet complete (it is above every visible one)
-    for (int x = lane; x < sel; x += 32) buf[x] = (uint32_t)buf[x];
-    __syncwarp();
-    int total = sel;
-    if (lane == 0) {
-        if (f0) buf[total] = (uint32_t)(~0u);
-        if (fo) buf[total + (f0 ? 1 : 0)] = (uint32_t)(~(uint32_t)own);
-    }
-    total += (f0 ? 1 : 0) + (fo ? 1 : 0);
-    int n2 = 32;
-    while (n2 < total) n2 <<= 1;
-    __syncwarp();
-    for (int x = total + lane; x < n2; x += 32) buf[x] = 0ull;
-    __syncwarp();
-    warp_sort_desc(buf, n2, lane);
-    int32_t *out = p.idx + ((size_t)g * p.n_max + i) * p.top_k;
-    for (int x = lane; x < total && x < p.top_k; x += 32) out[x] = (int)(~(uint32_t)buf[x]);
-    int cnt = total;
-    const bool extra = (p.force_local && own >= c) || (p.force_first && c == 0);
-    if (extra) {
-        if (lane == 0 && cnt < p.top_k) out[cnt] = own;
-        ++cnt;
-    }
-    for (int x = cnt + lane; x < p.top_k; x += 32) out[x] = -1;
-    if (cnt > p.top_k && lane == 0) report(p.status, VNSA_ERR_BOUNDS);
+    topk_select_row<true>(p.imp + ((size_t)g * p.n_max + i) * p.imp_stride, c, i / p.block,
+                          p.top_k, p.force_first, p.force_local, sh_buf[warp], lane,
+                          p.idx + ((size_t)g * p.n_max + i) * p.top_k, p.status);
 }
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {

@@ -10,6 +10,7 @@
 
 #include <new>
 
+#include "decode.h"
 #include "kernels.h"
 #include "tc_attn.h"
 
@@ -23,7 +24,8 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-    size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, idx, o_cmp, tc;
+    size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, idx, o_cmp, tc, dec,
+        dec_sel, dec_ocmp;
     size_t total;
     size_t imp_stride;
 };
@@ -49,6 +51,9 @@ Layout make_layout(const vnsa_config &c) {
     L.idx = take((size_t)c.h_kv * n * c.top_k * 4);
     L.o_cmp = take(n * c.h_q * c.d * 4);
     L.tc = take(tc_workspace_bytes(c));
+    L.dec = take(decode_workspace_bytes(c.h_kv, c.h_q / c.h_kv, c.d, (int)nb));
+    L.dec_sel = take((size_t)c.h_kv * c.top_k * 4);
+    L.dec_ocmp = take((size_t)c.h_q * c.d * 4);
     L.total = off;
     return L;
 }
@@ -89,6 +94,7 @@ struct vnsa_handle {
     size_t stage_bytes;
     TcState *tc;
     int timing;
+    long long stream_n;  // tokens the last forward / decode step processed (-1: none)
     cudaEvent_t ev[2 * VNSA_NUM_STAGES];
     int ran[VNSA_NUM_STAGES];
     int launches;
@@ -142,6 +148,7 @@ vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v
     if (h->cfg.scale == 0.f) h->cfg.scale = 1.0f / sqrtf((float)cfg->d);
     cudaGetDevice(&h->device);
     h->r = cfg->h_q / cfg->h_kv;
+    h->stream_n = -1;
     h->nb_max = cfg->n_max / cfg->block;
     h->esize = cfg->dtype == VNSA_BF16 ? 2 : 4;
     h->L = make_layout(h->cfg);
@@ -285,8 +292,70 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     if (cur != h->device && cur >= 0) cudaSetDevice(cur);
     if (e != cudaSuccess) {
         fprintf(stderr, "vnsa_forward: %s\n", cudaGetErrorString(e));
+        h->stream_n = -1;
         return VNSA_ERR_CUDA;
     }
+    h->stream_n = n;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k, const void *v,
+                        const uint8_t *is_vision, const float *gate_new, void *out_new,
+                        int32_t *sel_out, void *stream) {
+    if (!h || !q_new || !k || !v || !is_vision || !gate_new || !out_new)
+        return VNSA_ERR_INVALID_ARG;
+    if (n < 2 || n > h->cfg.n_max || h->stream_n != (long long)n - 1) return VNSA_ERR_INVALID_ARG;
+    if (!aligned16(q_new) || !aligned16(k) || !aligned16(v) || !aligned16(out_new) ||
+        !aligned16(gate_new) || (sel_out && !aligned16(sel_out)))
+        return VNSA_ERR_INVALID_ARG;
+    const vnsa_config &c = h->cfg;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return VNSA_ERR_CUDA;
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.n = n;
+    p.h_q = c.h_q;
+    p.h_kv = c.h_kv;
+    p.d = c.d;
+    p.r = h->r;
+    p.block = c.block;
+    p.top_k = c.top_k;
+    p.window = c.window;
+    p.force_first = c.force_first;
+    p.force_local = c.force_local;
+    p.nb_max = h->nb_max;
+    p.scale_log2 = c.scale * kLog2e;
+    p.q = q_new;
+    p.k = k;
+    p.v = v;
+    p.is_vision = is_vision;
+    p.gate = gate_new;
+    p.out = out_new;
+    p.vis = (int32_t *)(h->ws + h->L.vis);
+    p.txt = (int32_t *)(h->ws + h->L.txt);
+    p.counts = h->counts;
+    p.status = h->status;
+    p.k_cmp = h->ws + h->L.k_cmp;
+    p.v_cmp = h->ws + h->L.v_cmp;
+    p.w_k = h->ws + h->L.w_k;
+    p.w_v = h->ws + h->L.w_v;
+    char *dec = h->ws + h->L.dec;
+    p.s_cmp = (float *)dec;
+    p.part = (float *)(dec + (size_t)c.h_kv * h->r * (h->nb_max > 0 ? h->nb_max : 1) * 4);
+    p.sel = (int32_t *)(h->ws + h->L.dec_sel);
+    p.o_cmp = (float *)(h->ws + h->L.dec_ocmp);
+    p.sel_out = sel_out;
+    h->launches = 0;
+    for (int x = 0; x < VNSA_NUM_STAGES; ++x) h->ran[x] = 0;
+    const cudaError_t e = launch_decode((int)c.dtype, p, (cudaStream_t)stream, &h->launches);
+    if (cur != h->device && cur >= 0) cudaSetDevice(cur);
+    if (e != cudaSuccess) {
+        fprintf(stderr, "vnsa_decode: %s\n", cudaGetErrorString(e));
+        h->stream_n = -1;
+        return VNSA_ERR_CUDA;
+    }
+    h->stream_n = n;
     return VNSA_OK;
 }
 
