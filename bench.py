@@ -247,6 +247,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="long_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="vnsa", choices=["vnsa", "reference"])
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"],
+                    help="decode: time single-token steps after a prefill of the rest")
+    ap.add_argument("--decode-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=96)
@@ -258,6 +261,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.mode == "decode":
+        run_decode_bench(args, rank, world, local_rank)
         return
 
     import torch
@@ -423,6 +429,94 @@ def main():
     layer.close()
     if dist_on:
         dist.destroy_process_group()
+
+
+def decode_bytes(wl, i, kind):
+    """Algorithmic HBM bytes of one decode step: block keys/values of the
+    visible blocks, the selected blocks' and the window's K/V rows (vision), or
+    every K/V row (text), plus q, gates and the output row."""
+    es = 2 if wl.dtype == "bf16" else 4
+    row = wl.h_kv * wl.d * es
+    io = 2 * wl.h_q * wl.d * es + wl.h_q * 3 * 4
+    if kind == "text":
+        return 2 * (i + 1) * row + io
+    c = (i + 1) // wl.block
+    sel = min(wl.top_k, c + 1) * wl.block
+    return 2 * c * row + 2 * sel * row + 2 * min(wl.window, i + 1) * row + io
+
+
+def run_decode_bench(args, rank, world, local_rank):
+    """Decode steps of the named workload's stream: the last D tokens are moved
+    to the end of the vision run (so they decode through the sparse branches),
+    the rest is prefilled once, then D single-token steps are timed on the
+    device; the first `warmup` steps of a second pass are untimed."""
+    import torch
+    from sparse_attention_long_block_b200 import binding
+    base = replica_workload(args.workload, rank)
+    D = args.decode_tokens
+    nv, nt = base.n_vision, base.n_text
+    mask = np.concatenate([np.ones(nv - D, np.uint8), np.zeros(nt, np.uint8),
+                           np.ones(D, np.uint8)])
+    wl = base.with_(name=base.name)
+    x = generate(wl, is_vision=mask)
+    torch.cuda.set_device(local_rank)
+    td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dev = torch.device("cuda", local_rank)
+    q = torch.from_numpy(x["q"]).to(dev, td)
+    k = torch.from_numpy(x["k"]).to(dev, td)
+    v = torch.from_numpy(x["v"]).to(dev, td)
+    isv = torch.from_numpy(x["is_vision"]).to(dev)
+    gate = torch.from_numpy(x["gate"]).to(dev)
+    n = wl.n
+    n0 = n - D
+    layer = binding.Layer(n_max=n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
+                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+    qs = [q[t].contiguous() for t in range(n0, n)]
+    gs = [gate[t].contiguous() for t in range(n0, n)]
+    outs = [torch.empty_like(qs[0]) for _ in range(D)]
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        layer.forward(q[:n0].contiguous(), k[:n0].contiguous(), v[:n0].contiguous(),
+                      isv[:n0].contiguous(), gate[:n0].contiguous(), stream=stream)
+
+    def steps(lo, hi):
+        for j in range(lo, hi):
+            layer.decode(n0 + j + 1, qs[j], k, v, isv, gs[j], out=outs[j], stream=stream)
+
+    prefill()
+    steps(0, D)  # warm-up pass
+    prefill()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    steps(0, D)
+    ev1.record(stream)
+    ev1.synchronize()
+    if layer.device_status() != 0:
+        raise SystemExit("device status error in the decode steps")
+    ms = ev0.elapsed_time(ev1) / D
+    launches = layer.launches()
+    peaks = load_peaks()
+    i0 = nv - D
+    nbytes = float(np.mean([decode_bytes(wl, i0 + j, "vision") for j in range(D)]))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "decode_tokens_per_s", "value": world * 1e3 / ms, "unit": "tokens/s",
+            "n_gpus": world, "steps": D, "warmup": D, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "mode": "decode (vision tokens)", "context": n,
+                       "decoded": D, "top_k": wl.top_k, "window": wl.window},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "bytes_per_step": nbytes},
+            "gpu_launches": launches * D,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
 
 
 def layer_build_id():

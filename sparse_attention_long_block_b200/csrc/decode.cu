@@ -34,8 +34,54 @@ constexpr int kWarps = 4;  // warps per CTA of the split kernels
 // Row pieces: lane owns elements [lane * PER, lane * PER + PER) of a d-row.
 template <typename T, int PER>
 __device__ __forceinline__ void load_piece(const T *p, float (&x)[PER]) {
+    if constexpr (sizeof(T) == 2 && PER == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    } else if constexpr (sizeof(T) == 2 && PER == 2) {
+        const float2 a = __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p)));
+        x[0] = a.x; x[1] = a.y;
+    } else if constexpr (sizeof(T) == 4 && PER == 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    } else {
 #pragma unroll
-    for (int e = 0; e < PER; ++e) x[e] = to_f(p[e]);
+        for (int e = 0; e < PER; ++e) x[e] = to_f(p[e]);
+    }
+}
+
+// Split softmax states of one (branch, group): per head the largest split
+// maximum M, the weights f_b = 2^(m_b - M) / L of every split, L = sum l_b f'_b,
+// into shared memory fw [R_max][kSplit] (threads of the CTA cooperate).  The
+// head's output element e is then sum_b o_b[e] fw[hh][b].
+__device__ void split_weights(const float *part, int r, int d, float *fw, float *lse) {
+    for (int hh = threadIdx.x >> 5; hh < r; hh += blockDim.x >> 5) {
+        const int lane = threadIdx.x & 31;
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int b = lane + 32 * z;
+            if (b < kSplit) {
+                const float *w = part + ((size_t)b * r + hh) * (d + 2);
+                m[z] = w[d];
+                l[z] = w[d + 1];
+            }
+        }
+        const float M = warp_max(fmaxf(m[0], m[1]));
+        float L = 0.f;
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+            if (M != -INFINITY && l[z] > 0.f) L += l[z] * exp2f(m[z] - M);
+        L = warp_sum(L);
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int b = lane + 32 * z;
+            if (b < kSplit)
+                fw[hh * kSplit + b] = (L > 0.f && l[z] > 0.f) ? exp2f(m[z] - M) / L : 0.f;
+        }
+        if (lane == 0 && lse) lse[hh] = L > 0.f ? M + log2f(L) : -INFINITY;
+    }
 }
 
 // Online softmax state of one head over this lane's part of d.
@@ -183,7 +229,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_cmp_kernel(DecodeParams p)
 // visible block, and the top-k selection.
 template <int D>
 __global__ void __launch_bounds__(256) decode_select_kernel(DecodeParams p) {
-    extern __shared__ float sm[];  // lse [16], importance [nb_max + 4]
+    extern __shared__ float sm[];  // lse [16], split weights [16][kSplit], importance
     __shared__ uint64_t buf[128];
     const Counts cn = *p.counts;
     if (!cn.pad[1]) return;
@@ -191,25 +237,18 @@ __global__ void __launch_bounds__(256) decode_select_kernel(DecodeParams p) {
     const int c = min((i + 1) / p.block, cn.nb);
     const int g = blockIdx.x, r = p.r;
     float *lse = sm;
-    float *imp = sm + 16;
+    float *fw = sm + 16;                    // [16][kSplit]
+    float *imp = fw + 16 * kSplit + 4;      // 16-byte aligned: 16 + 16 * 37 + 4 floats
     // compression partials -> o_cmp (normalised) and the log2-sum-exp per head
+    const float *part0 = part_of(p, 0, g, 0);
+    split_weights(part0, r, D, fw, lse);
+    __syncthreads();
     for (int x = threadIdx.x; x < r * D; x += blockDim.x) {
         const int hh = x / D, e = x % D;
-        float M = -INFINITY;
-        for (int b = 0; b < kSplit; ++b) M = fmaxf(M, part_of(p, 0, g, b)[(size_t)hh * (D + 2) + D]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-            for (int b = 0; b < kSplit; ++b) {
-                const float *w = part_of(p, 0, g, b) + (size_t)hh * (D + 2);
-                const float f = exp2f(w[D] - M);
-                L += w[D + 1] * f;
-                O += w[e] * f;
-            }
-        }
-        p.o_cmp[(size_t)(g * r + hh) * D + e] = L > 0.f ? O / L : 0.f;
-        if (e == 0) lse[hh] = L > 0.f ? M + log2f(L) : -INFINITY;
+        float O = 0.f;
+        for (int b = 0; b < kSplit; ++b) O += part0[((size_t)b * r + hh) * (D + 2) + e] * fw[hh * kSplit + b];
+        p.o_cmp[(size_t)(g * r + hh) * D + e] = O;
     }
-    __syncthreads();
     // importance: the exact compression probabilities summed over the heads
     for (int j = threadIdx.x; j < c; j += blockDim.x) {
         float s = 0.f;
@@ -307,22 +346,42 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
 // One CTA per query head: the branch partials, the gates, the output row.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
+    __shared__ float fw[2][kSplit];
     const Counts cn = *p.counts;
     const bool vision = cn.pad[1] != 0;
     const int h = blockIdx.x, g = h / p.r, hh = h % p.r, e = threadIdx.x;
-    auto branch = [&](int br) {
-        float M = -INFINITY;
-        for (int b = 0; b < kSplit; ++b) M = fmaxf(M, part_of(p, br, g, b)[(size_t)hh * (D + 2) + D]);
-        float L = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-            for (int b = 0; b < kSplit; ++b) {
-                const float *w = part_of(p, br, g, b) + (size_t)hh * (D + 2);
-                const float f = exp2f(w[D] - M);
-                L += w[D + 1] * f;
-                O += w[e] * f;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // split weights of this head for branch 1 (selection) and 2 (window/text)
+    if (warp < 2) {
+        const float *part = part_of(p, 1 + warp, g, 0);
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int b = lane + 32 * z;
+            if (b < kSplit) {
+                const float *w = part + ((size_t)b * p.r + hh) * (D + 2);
+                m[z] = w[D];
+                l[z] = w[D + 1];
             }
         }
-        return L > 0.f ? O / L : 0.f;
+        const float M = warp_max(fmaxf(m[0], m[1]));
+        float L = 0.f;
+#pragma unroll
+        for (int z = 0; z < 2; ++z)
+            if (M != -INFINITY && l[z] > 0.f) L += l[z] * exp2f(m[z] - M);
+        L = warp_sum(L);
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+            const int b = lane + 32 * z;
+            if (b < kSplit) fw[warp][b] = (L > 0.f && l[z] > 0.f) ? exp2f(m[z] - M) / L : 0.f;
+        }
+    }
+    __syncthreads();
+    auto branch = [&](int br) {
+        const float *part = part_of(p, br, g, 0);
+        float O = 0.f;
+        for (int b = 0; b < kSplit; ++b) O += part[((size_t)b * p.r + hh) * (D + 2) + e] * fw[br - 1][b];
+        return O;
     };
     float o;
     if (vision) {
@@ -344,7 +403,7 @@ cudaError_t launch_typed(const DecodeParams &p, cudaStream_t s, int *launches) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(decode_attn_kernel<T, D, R>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)part_smem);
-    const size_t sel_smem = (16 + (size_t)p.nb_max + 4) * sizeof(float);
+    const size_t sel_smem = (16 + 16 * kSplit + 4 + (size_t)p.nb_max + 4) * sizeof(float);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(decode_select_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem);
