@@ -12,39 +12,53 @@
 namespace vnsa {
 
 // ---------------------------------------------------------------------------
-// Partition: one CTA of 1024 threads scans the flags.  vis[i] = position of
+// Partition: one CTA of 1024 threads walks the flags in stripes of 1024
+// positions; a stripe is compacted with warp ballots and a scan of the 32 warp
+// counts, so every read and most writes are coalesced.  vis[i] = position of
 // the i-th vision token, txt[x] = position of the x-th text token.
 __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restrict__ isv,
                                                          int n, int block,
                                                          int32_t *__restrict__ vis,
                                                          int32_t *__restrict__ txt,
                                                          Counts *counts) {
-    __shared__ int s_cnt[1024];
-    const int tid = threadIdx.x;
-    const int per = (n + 1023) / 1024;
-    const int lo = min(n, tid * per), hi = min(n, lo + per);
-    int c = 0;
-    for (int t = lo; t < hi; ++t) c += isv[t] != 0;
-    s_cnt[tid] = c;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-        int add = tid >= off ? s_cnt[tid - off] : 0;
+    __shared__ int s_warp[32];  // exclusive prefix of the warps' vision counts
+    __shared__ int s_stripe;    // vision tokens of the current stripe
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const unsigned below = (1u << lane) - 1u;
+    int nv = 0, nt = 0;  // totals before the current stripe (same in every thread)
+    for (int base = 0; base < n; base += 1024) {
+        const int t = base + tid;
+        const bool in = t < n;
+        const bool v = in && isv[t] != 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, v);
+        if (lane == 0) s_warp[warp] = __popc(bal);
         __syncthreads();
-        s_cnt[tid] += add;
+        if (warp == 0) {
+            const int x = s_warp[lane];
+            int incl = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            s_warp[lane] = incl - x;
+            if (lane == 31) s_stripe = incl;
+        }
         __syncthreads();
+        const int vbefore = s_warp[warp] + __popc(bal & below);  // vision before t in the stripe
+        if (in) {
+            if (v) vis[nv + vbefore] = t;
+            else txt[nt + (tid - vbefore)] = t;
+        }
+        const int sv = s_stripe;
+        nv += sv;
+        nt += min(1024, n - base) - sv;
+        __syncthreads();  // s_warp / s_stripe are rewritten by the next stripe
     }
-    int vb = s_cnt[tid] - c;
-    int tb = lo - vb;
-    for (int t = lo; t < hi; ++t) {
-        if (isv[t]) vis[vb++] = t;
-        else txt[tb++] = t;
-    }
-    __syncthreads();
     if (tid == 0) {
-        const int nv = s_cnt[1023];
         Counts cn;
         cn.n_vision = nv;
-        cn.n_text = n - nv;
+        cn.n_text = nt;
         cn.nb = nv / block;
         cn.vis_base = nv > 0 ? vis[0] : 0;
         cn.contiguous = (nv == 0) || (vis[nv - 1] - vis[0] == nv - 1);
