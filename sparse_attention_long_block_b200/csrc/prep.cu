@@ -12,47 +12,63 @@
 namespace vnsa {
 
 // ---------------------------------------------------------------------------
-// Partition: one CTA of 1024 threads walks the flags in stripes of 1024
-// positions; a stripe is compacted with warp ballots and a scan of the 32 warp
-// counts, so every read and most writes are coalesced.  vis[i] = position of
-// the i-th vision token, txt[x] = position of the x-th text token.
+// Partition: one CTA of 1024 threads walks the flags in stripes of 4096
+// positions, four consecutive flags per thread; a stripe is compacted with a
+// warp scan of the threads' vision counts and a scan of the 32 warp totals.
+// vis[i] = position of the i-th vision token, txt[x] = position of the x-th
+// text token.
 __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restrict__ isv,
                                                          int n, int block,
                                                          int32_t *__restrict__ vis,
                                                          int32_t *__restrict__ txt,
                                                          Counts *counts) {
+    constexpr int kPer = 4;
+    constexpr int kStripe = 1024 * kPer;
     __shared__ int s_warp[32];  // exclusive prefix of the warps' vision counts
     __shared__ int s_stripe;    // vision tokens of the current stripe
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const unsigned below = (1u << lane) - 1u;
     int nv = 0, nt = 0;  // totals before the current stripe (same in every thread)
-    for (int base = 0; base < n; base += 1024) {
-        const int t = base + tid;
-        const bool in = t < n;
-        const bool v = in && isv[t] != 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, v);
-        if (lane == 0) s_warp[warp] = __popc(bal);
+    for (int base = 0; base < n; base += kStripe) {
+        const int t0 = base + tid * kPer;
+        bool f[kPer];
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            f[e] = t0 + e < n && isv[t0 + e] != 0;
+            c += f[e];
+        }
+        // inclusive scan of c over the warp
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_warp[warp] = incl;
         __syncthreads();
         if (warp == 0) {
             const int x = s_warp[lane];
-            int incl = x;
+            int wi = x;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+                const int y = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += y;
             }
-            s_warp[lane] = incl - x;
-            if (lane == 31) s_stripe = incl;
+            s_warp[lane] = wi - x;
+            if (lane == 31) s_stripe = wi;
         }
         __syncthreads();
-        const int vbefore = s_warp[warp] + __popc(bal & below);  // vision before t in the stripe
-        if (in) {
-            if (v) vis[nv + vbefore] = t;
-            else txt[nt + (tid - vbefore)] = t;
+        int vb = s_warp[warp] + incl - c;  // vision tokens before t0 in the stripe
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int t = t0 + e;
+            if (t >= n) break;
+            if (f[e]) vis[nv + vb++] = t;
+            else txt[nt + (t - base) - vb] = t;
         }
         const int sv = s_stripe;
         nv += sv;
-        nt += min(1024, n - base) - sv;
+        nt += min(kStripe, n - base) - sv;
         __syncthreads();  // s_warp / s_stripe are rewritten by the next stripe
     }
     if (tid == 0) {
