@@ -107,17 +107,18 @@ struct Work {
     int contiguous, vis_base;
 };
 
+template <int MODE>
 __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
     Work w;
     const LayerParams &L = P.L;
-    w.rpad = P.mode == MODE_CMP ? pow2_at_least(L.r) : L.r;
+    w.rpad = MODE == MODE_CMP ? pow2_at_least(L.r) : L.r;
     w.qt = kRows / w.rpad;
     w.nb = cn.nb;
     w.contiguous = cn.contiguous;
     w.vis_base = cn.vis_base;
     w.nsplit = 1;
     w.split_len = 0;
-    if (P.mode == MODE_TEXT) {
+    if (MODE == MODE_TEXT) {
         w.n_q = cn.n_text;
         w.n_tiles_q = (w.n_q + w.qt - 1) / w.qt;
         const int span = w.n_q > 0 ? L.txt[w.n_q - 1] + 1 : 0;
@@ -144,11 +145,12 @@ struct Item {
     int key_lo;     // SWA window start (vision rank) / TEXT split start (position)
 };
 
+template <int MODE>
 __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int item) {
     const LayerParams &L = P.L;
     Item it;
     int tile;
-    if (P.mode == MODE_TEXT) {
+    if (MODE == MODE_TEXT) {
         const int per_split = L.h_kv * w.n_tiles_q;
         it.split = item / per_split;
         const int rem = item % per_split;
@@ -165,18 +167,18 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     it.key_lo = 0;
     it.seg_tiles[1] = 0;
     it.seg_kind[1] = K_EXACT;
-    if (P.mode == MODE_CMP) {
+    if (MODE == MODE_CMP) {
         const int c_last = min((ql + 1) / L.block, w.nb);
         const int t = (c_last + kKeys - 1) / kKeys;
         it.nseg = 2;
         it.seg_kind[0] = K_STATS;
         it.seg_tiles[0] = t;
         it.seg_tiles[1] = t;
-    } else if (P.mode == MODE_SLC) {
+    } else if (MODE == MODE_SLC) {
         it.nseg = 1;
         it.seg_kind[0] = K_SLC;
         it.seg_tiles[0] = P.plan[(size_t)item * (1 + 2 * P.plan_max)];
-    } else if (P.mode == MODE_SWA) {
+    } else if (MODE == MODE_SWA) {
         it.nseg = 1;
         it.seg_kind[0] = K_SWA;
         it.key_lo = max(0, it.q0 - L.window + 1);
@@ -236,6 +238,7 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
 // every item, in order, each lane with its own ring and waits: a K stage is
 // free once its Q K^T is done, a V stage only after its P V, so the K loads
 // run ahead.  Lane 0 also prefetches the tiles kPrefetch ahead into L2.
+template <int MODE>
 __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, int lane) {
     if (lane > 1) return;
     const LayerParams &L = P.L;
@@ -247,17 +250,17 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
     uint32_t t = 0;  // tiles issued on this lane's ring
     const CUtensorMap *mk = &P.tm_k, *mv = &P.tm_v;
     int vbase = 0;
-    if (P.mode == MODE_CMP) {
+    if (MODE == MODE_CMP) {
         mk = &P.tm_kb;
         mv = &P.tm_vb;
-    } else if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+    } else if (MODE == MODE_SLC || MODE == MODE_SWA) {
         mk = w.contiguous ? &P.tm_k : &P.tm_kc;
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
     }
     const CUtensorMap *mine = is_k ? mk : mv;
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
-        const Item it = make_item(P, w, item);
+        const Item it = make_item<MODE>(P, w, item);
         const int xc = it.g * kD;
         // row coordinate of tile x of a segment (both CMP segments share keys)
         auto row_of = [&](int kind, int x) {
@@ -310,6 +313,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
 
 // ---------------------------------------------------------------------------
 // MMA issuer (one thread).
+template <int MODE>
 __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
@@ -342,7 +346,7 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         return true;
     };
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
-        const Item it = make_item(P, w, item);
+        const Item it = make_item<MODE>(P, w, item);
         if (item_tiles(it) == 0) continue;
         if (!ptx::mbar_wait(sm.bar(B_Q_FULL), nitems & 1, abort, L.status)) { ok = false; break; }
         ++nitems;
@@ -435,6 +439,7 @@ __device__ __forceinline__ void imp_reduce_store(float (&p)[64], int lane, float
     }
 }
 
+template <int MODE>
 __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
@@ -448,14 +453,14 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
     uint32_t gt = 0, npv = 0, gphase = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
-        const Item it = make_item(P, w, item);
+        const Item it = make_item<MODE>(P, w, item);
         RowCtx rc;
         rc.qi = rho / w.rpad;
         rc.hl = rho % w.rpad;
         rc.h = it.g * L.r + min(rc.hl, L.r - 1);
         rc.valid = rc.qi < it.nq && rc.hl < L.r;
         rc.i = it.q0 + min(rc.qi, max(it.nq - 1, 0));
-        if (P.mode == MODE_TEXT) rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
+        if (MODE == MODE_TEXT) rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
         else rc.t = it.nq > 0 ? L.vis[rc.i] : 0;
         rc.c_vis = min((rc.i + 1) / L.block, w.nb);
         if (item_tiles(it) == 0) {
@@ -463,22 +468,22 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             if (rc.valid) {
                 __half *part = (__half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                 const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
-                if (P.mode == MODE_CMP) {
+                if (MODE == MODE_CMP) {
                     for (int e = 0; e < kD; e += 8)
                         *reinterpret_cast<uint4 *>(part + e) = make_uint4(0u, 0u, 0u, 0u);
                     if (L.dbg_o_cmp)
                         for (int e = 0; e < kD; ++e) L.dbg_o_cmp[prow + e] = 0.f;
                     L.lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
-                } else if (P.mode == MODE_TEXT) {
+                } else if (MODE == MODE_TEXT) {
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
                 } else {
                     // no selected / window key: this branch adds nothing
-                    float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+                    float *dbg = MODE == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
-                        if (P.mode == MODE_SWA)
+                        if (MODE == MODE_SWA)
                             ((__nv_bfloat16 *)L.out)[prow + e] =
                                 __float2bfloat16_rn(__half2float(part[e]));
                     }
@@ -493,7 +498,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (qi < it.nq && hl < L.r) {
                 const int q = it.q0 + qi;
-                const int t = (P.mode == MODE_TEXT) ? L.txt[q] : L.vis[q];
+                const int t = (MODE == MODE_TEXT) ? L.txt[q] : L.vis[q];
                 const __nv_bfloat16 *src =
                     Q + ((size_t)t * L.h_q + it.g * L.r + hl) * kD + c16 * 8;
                 val = __ldg(reinterpret_cast<const uint4 *>(src));
@@ -508,17 +513,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // next item, so that neither waits on DRAM when it is needed
         if (rc.valid) {
             ptx::prefetch_l2(L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3);
-            if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+            if (MODE == MODE_SLC || MODE == MODE_SWA) {
                 const __half *part = (const __half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                 ptx::prefetch_l2(part);
                 ptx::prefetch_l2(part + 64);
             }
         }
         if (item + (int)gridDim.x < w.items) {
-            const Item nx = make_item(P, w, item + gridDim.x);
+            const Item nx = make_item<MODE>(P, w, item + gridDim.x);
             const int qn = rho / w.rpad, hn = rho % w.rpad;
             if (qn < nx.nq && hn < L.r) {
-                const int tn = (P.mode == MODE_TEXT) ? L.txt[nx.q0 + qn] : L.vis[nx.q0 + qn];
+                const int tn = (MODE == MODE_TEXT) ? L.txt[nx.q0 + qn] : L.vis[nx.q0 + qn];
                 const __nv_bfloat16 *qr = Q + ((size_t)tn * L.h_q + nx.g * L.r + hn) * kD;
                 ptx::prefetch_l2(qr);
                 ptx::prefetch_l2(qr + 64);
@@ -526,7 +531,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         // SLC: the item's selection tiles (first key, query mask) into shared
         // memory, once every thread is done with the previous item's copy
-        if (P.mode == MODE_SLC) {
+        if (MODE == MODE_SLC) {
             group_sync(sm, gphase, ok, L);
             if (!ok) break;
             int32_t *dst = (int32_t *)(sm.base + SM_PLAN);
@@ -762,7 +767,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // CMP writes sig(g_cmp) o_cmp, SLC adds sig(g_slc) o_slc in place, SWA
         // adds sig(g_swa) o_swa and writes the bf16 output row.
         __half *part = (__half *)L.o_cmp_ws + qrow;
-        if (P.mode == MODE_CMP) {
+        if (MODE == MODE_CMP) {
             const float gc = rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3]) : 0.f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
@@ -784,12 +789,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
-        } else if (P.mode == MODE_SLC || P.mode == MODE_SWA) {
+        } else if (MODE == MODE_SLC || MODE == MODE_SWA) {
             const float g =
-                rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (P.mode == MODE_SLC ? 1 : 2)])
+                rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (MODE == MODE_SLC ? 1 : 2)])
                          : 0.f;
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            float *dbg = P.mode == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+            float *dbg = MODE == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
             __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
@@ -807,7 +812,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     if (dbg)
                         for (int z = 0; z < 8; ++z) dbg[prow + ch * 32 + k + z] = b8[z];
                     uint4 v;
-                    if (P.mode == MODE_SLC) {
+                    if (MODE == MODE_SLC) {
                         __half2 *h2 = reinterpret_cast<__half2 *>(&v);
 #pragma unroll
                         for (int z = 0; z < 4; ++z) {
@@ -865,6 +870,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
     }
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_constant__ TcParams P) {
     extern __shared__ uint8_t smem_raw[];
     const LayerParams &L = P.L;
@@ -881,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     __syncthreads();
     if (*sm.failed_flag() != 0) return;
     const Counts cn = *L.counts;
-    const Work w = make_work(P, cn);
+    const Work w = make_work<MODE>(P, cn);
     if ((int)blockIdx.x >= w.items) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -916,12 +922,12 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     const uint32_t tmem = *sm.tmem_slot();
 
     if (warp == 0) {
-        run_producer(P, w, sm, lane);
+        run_producer<MODE>(P, w, sm, lane);
     } else if (warp == 1) {
-        if (lane == 0) run_mma(P, w, sm, tmem);
+        if (lane == 0) run_mma<MODE>(P, w, sm, tmem);
         __syncwarp();
     } else {
-        run_softmax(P, w, sm, tmem);
+        run_softmax<MODE>(P, w, sm, tmem);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1190,8 +1196,11 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     st->vh_cmp = (__half *)(p + 3 * kv);
     st->plan = (int32_t *)(p + 3 * kv + kvb);
     st->part = (float *)(p + 3 * kv + kvb + up256(plan_bytes(c)));
-    cudaError_t e = cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
+                    tc_attn_kernel<MODE_TEXT>})
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) {
         delete st;
         return e;
@@ -1230,7 +1239,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     cudaError_t e;
     auto attn = [&](int mode) {
         P.mode = mode;
-        tc_attn_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(P);
+        switch (mode) {
+            case MODE_CMP: tc_attn_kernel<MODE_CMP><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            case MODE_SLC: tc_attn_kernel<MODE_SLC><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            case MODE_SWA: tc_attn_kernel<MODE_SWA><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            default: tc_attn_kernel<MODE_TEXT><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+        }
         ++*launches;
     };
     prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vhc, st->vh, st->vh_cmp);
