@@ -86,6 +86,42 @@ def algorithmic_work(wl, is_vision):
     }
 
 
+def executed_work(wl, is_vision, idx):
+    """Tensor FLOPs the attention kernels execute (every MMA of every tile,
+    masked rows and keys included): 128-row tiles against 64-key tiles, 2 *
+    128 * 64 * d flops per QK^T or P V product.  Compression: 16 queries per
+    tile (8 head slots), a statistics pass (QK^T) and an exact pass (QK^T + P V)
+    over the visible blocks; selection: 18 queries (7 heads) against the union
+    of their selected blocks (from idx [h_kv][N_v][k]); window and text: 18
+    queries against their key ranges."""
+    prod = 2.0 * 128 * 64 * wl.d
+    vis = np.nonzero(is_vision)[0]
+    txt = np.nonzero(is_vision == 0)[0]
+    nv, nb = len(vis), len(vis) // wl.block
+    r = wl.h_q // wl.h_kv
+    rpad = 1
+    while rpad < r:
+        rpad *= 2
+    qc, qt = 128 // rpad, 128 // r
+    cmp = slc = swa = text = 0.0
+    for q0 in range(0, nv, qc):
+        ql = min(nv, q0 + qc) - 1
+        t = -(-min((ql + 1) // wl.block, nb) // 64)
+        cmp += 3 * t
+    for q0 in range(0, nv, qt):
+        ql = min(nv, q0 + qt) - 1
+        lo = max(0, q0 - wl.window + 1)
+        swa += 2 * ((ql - lo + 64) // 64)
+        for g in range(wl.h_kv):
+            sel = idx[g, q0:ql + 1].ravel()
+            slc += 2 * len(np.unique(sel[sel >= 0]))
+    for x0 in range(0, len(txt), qt):
+        xl = min(len(txt), x0 + qt) - 1
+        text += 2 * ((int(txt[xl]) + 64) // 64)
+    return {"cmp": wl.h_kv * cmp * prod, "slc": slc * prod, "swa": wl.h_kv * swa * prod,
+            "text": wl.h_kv * text * prod}
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -339,6 +375,15 @@ def main():
             stage_ms[kname] = stage_ms.get(kname, 0.0) + val / reps
     layer.set_timing(False)
     torch.cuda.synchronize()
+    executed = None
+    if wl.dtype == "bf16" and wl.d == 128:
+        dbg, tens = binding.make_debug(wl.n, wl.h_q, wl.h_kv, wl.d, wl.top_k, wl.block,
+                                       dtype=td, want=("idx",))
+        layer.forward(q, k, v, isv, gate, out=out, dbg=dbg, stream=stream)
+        torch.cuda.synchronize()
+        nvis = int(x["is_vision"].sum())
+        executed = executed_work(wl, x["is_vision"], tens["idx"][:, :nvis].cpu().numpy())
+        del tens
 
     # end to end through the C ABI with host buffers (pinned)
     e2e = None
@@ -415,6 +460,12 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (no flush)"},
             "tensor_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "executed": None if executed is None else {
+                "tflop": {kk: vv / 1e12 for kk, vv in executed.items()},
+                "tflops_per_s": sum(executed.values()) / (ms * 1e-3) / 1e12,
+                "frac_of_peak": sum(executed.values()) / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "slc_frac_of_peak": (executed["slc"] / (branch_ms["slc"] * 1e-3) / 1e12 /
+                                     peaks["bf16_tflops"]) if branch_ms["slc"] else None},
             "algorithmic_gflop": {kk: vv / 1e9 for kk, vv in flop_of.items()},
             "branch_ms": branch_ms,
             "pool_hbm": {"achieved_gbs": pool_gbs, "peak_gbs": peaks["hbm_gbs"],

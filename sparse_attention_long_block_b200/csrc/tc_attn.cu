@@ -64,7 +64,7 @@ constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024;              // + alignment sla
 // barrier slots (8 bytes each) after SM_BAR; S_FULL and P_FULL per S buffer
 constexpr int B_K_FULL = 0, B_V_FULL = 2, B_K_EMPTY = 4, B_V_EMPTY = 6, B_S_FULL = 8,
               B_P_FULL = 10, B_PV_DONE = 12, B_Q_FULL = 14, B_GRP = 15, B_FINAL = 16,
-              B_COUNT = 17;
+              B_Q_EMPTY = 17, B_COUNT = 18;
 
 // TMEM columns: two S buffers (fp32, 64 each) and O (fp32, 128).  Tile x uses
 // S buffer x & 1; its P (fp16 pairs) overwrites the first 32 columns of that
@@ -79,6 +79,7 @@ struct TcParams {
     CUtensorMap tm_k, tm_v;    // K (bf16, the caller's) and V (fp16 copy): [n rows][h_kv*d]
     CUtensorMap tm_kc, tm_vc;  // compacted vision K (bf16), V (fp16), if not contiguous
     CUtensorMap tm_kb, tm_vb;  // K_cmp (bf16), V_cmp (fp16): [nb_max rows][h_kv*d]
+    CUtensorMap tm_q;          // Q (bf16) as [n][h_q][d], box {64, rows per query, queries}
     LayerParams L;
     const int32_t *plan;       // SLC: [item][1 + 2*plan_max]
     int plan_max;
@@ -105,6 +106,7 @@ struct Work {
     int items;
     int nb;
     int contiguous, vis_base;
+    int q_tma;     // Q tiles arrive by one TMA box (vision modes, contiguous vision run)
 };
 
 template <int MODE>
@@ -116,6 +118,7 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
     w.nb = cn.nb;
     w.contiguous = cn.contiguous;
     w.vis_base = cn.vis_base;
+    w.q_tma = MODE != MODE_TEXT && cn.contiguous;
     w.nsplit = 1;
     w.split_len = 0;
     if (MODE == MODE_TEXT) {
@@ -259,9 +262,24 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
         vbase = w.contiguous ? w.vis_base : 0;
     }
     const CUtensorMap *mine = is_k ? mk : mv;
+    uint32_t nq = 0;  // Q tiles loaded (lane 0, TMA path)
+    const int qrows = MODE == MODE_CMP ? w.rpad : L.r;  // MMA rows per query
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
         const Item it = make_item<MODE>(P, w, item);
         const int xc = it.g * kD;
+        if (is_k && w.q_tma && item_tiles(it) > 0) {
+            // the item's Q rows (query, head) are one box of the [n][h_q][d]
+            // tensor: queries vis_base + q0 .., heads g r .., in MMA row order;
+            // the buffer is free once the previous item's Q K^T are done
+            if (nq > 0 && !ptx::mbar_wait(sm.bar(B_Q_EMPTY), (nq - 1) & 1, abort, L.status))
+                return;
+            const uint32_t qb = sm.bar(B_Q_FULL);
+            ptx::mbar_expect_tx(qb, (uint32_t)(w.qt * qrows) * 2u * kD);
+            ptx::tma_load_3d(sm.base_u32 + SM_Q, &P.tm_q, qb, 0, it.g * L.r, w.vis_base + it.q0);
+            ptx::tma_load_3d(sm.base_u32 + SM_Q + 16384, &P.tm_q, qb, 64, it.g * L.r,
+                             w.vis_base + it.q0);
+            ++nq;
+        }
         // row coordinate of tile x of a segment (both CMP segments share keys)
         auto row_of = [&](int kind, int x) {
             const int key0 = tile_key0(P, it, item, kind, x);
@@ -353,6 +371,7 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         ptx::tc_fence_after();
         bool pending = false, pend_pv = false;
         uint32_t pend_acc = 0;
+        int uq = 0;  // Q K^T issued for this item
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
@@ -373,6 +392,8 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
                 }
                 ptx::mma_commit(sm.bar(B_S_FULL + (gt & 1)));
                 ptx::mma_commit(sm.bar(B_K_EMPTY + st));  // K is dead once Q K^T is done
+                // after the item's last Q K^T the Q buffer is free for the next item
+                if (w.q_tma && ++uq == item_tiles(it)) ptx::mma_commit(sm.bar(B_Q_EMPTY));
                 // the previous tile: its P V follows this Q K^T in the pipe, and
                 // its S buffer is free for the next Q K^T after that
                 if (pending && !finish(gt - 1, pend_pv, pend_acc)) { ok = false; break; }
@@ -491,8 +512,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             }
             continue;
         }
-        // ---- Q tile: rows gathered from their positions, 16-byte pieces
-        for (int e = rho; e < kRows * 16; e += 128) {
+        // ---- Q tile (without the TMA box): rows gathered from their
+        // positions, 16-byte pieces
+        for (int e = rho; !w.q_tma && e < kRows * 16; e += 128) {
             const int row = e >> 4, c16 = e & 15;
             const int qi = row / w.rpad, hl = row % w.rpad;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
@@ -507,8 +529,10 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             *reinterpret_cast<uint4 *>(sm.base + SM_Q + hf * 16384 + row * 128 +
                                        ((c ^ (row & 7)) << 4)) = val;
         }
-        ptx::fence_proxy_async();
-        ptx::mbar_arrive(sm.bar(B_Q_FULL));
+        if (!w.q_tma) {
+            ptx::fence_proxy_async();
+            ptx::mbar_arrive(sm.bar(B_Q_FULL));
+        }
         // L2 prefetch of this row's epilogue inputs and of its Q row in the
         // next item, so that neither waits on DRAM when it is needed
         if (rc.valid) {
@@ -890,6 +914,16 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     const Work w = make_work<MODE>(P, cn);
     if ((int)blockIdx.x >= w.items) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (w.q_tma) {
+        // MMA rows the Q box never writes (128 is not a multiple of the rows per
+        // query): zero once, so masked rows read finite values
+        const int q_rows = w.qt * (MODE == MODE_CMP ? w.rpad : L.r);
+        for (int e = q_rows * 8 + (int)threadIdx.x; e < kRows * 8; e += blockDim.x)
+            for (int hf = 0; hf < 2; ++hf)
+                *reinterpret_cast<uint4 *>(sm.base + SM_Q + hf * 16384 + e * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+        ptx::fence_proxy_async();
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(sm.bar(B_K_FULL + s), 1);
@@ -902,7 +936,8 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
             ptx::mbar_init(sm.bar(B_P_FULL + b), 4);
             ptx::mbar_init(sm.bar(B_PV_DONE + b), 1);
         }
-        ptx::mbar_init(sm.bar(B_Q_FULL), 128);
+        ptx::mbar_init(sm.bar(B_Q_FULL), w.q_tma ? 1 : 128);
+        ptx::mbar_init(sm.bar(B_Q_EMPTY), 1);
         ptx::mbar_init(sm.bar(B_GRP), 128);
         ptx::mbar_init(sm.bar(B_FINAL), 1);
         *sm.abort_flag() = 0;
@@ -1140,6 +1175,21 @@ bool make_map(CUtensorMap *m, const void *base, int h_kv, long long rows, bool f
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over Q [n][h_q][128] bf16 with boxes {64 of d, rq heads, qt tokens}
+// and the 128-byte swizzle: one box is a Q tile of qt queries x rq head rows in
+// MMA row order (row = query * rq + head).
+bool make_map_q(CUtensorMap *m, const void *q, int h_q, long long n, int rq, int qt) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || n < 1) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)h_q, (cuuint64_t)n};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)h_q * kD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rq, (cuuint32_t)qt};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
@@ -1237,8 +1287,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     };
     const int grid = 2 * st->num_sms;  // two CTAs per SM
     cudaError_t e;
-    auto attn = [&](int mode) {
+    auto attn = [&](int mode) -> cudaError_t {
         P.mode = mode;
+        if (mode != MODE_TEXT) {
+            const int rq = mode == MODE_CMP ? pow2_at_least(L.r) : L.r;
+            if (!make_map_q(&P.tm_q, L.q, c.h_q, L.n, rq, kRows / rq)) return cudaErrorInvalidValue;
+        }
         switch (mode) {
             case MODE_CMP: tc_attn_kernel<MODE_CMP><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             case MODE_SLC: tc_attn_kernel<MODE_SLC><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
@@ -1246,11 +1300,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
             default: tc_attn_kernel<MODE_TEXT><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
         }
         ++*launches;
+        return cudaSuccess;
     };
     prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vhc, st->vh, st->vh_cmp);
     ++*launches;
     begin(VNSA_STAGE_CMP);
-    attn(MODE_CMP);
+    if ((e = attn(MODE_CMP)) != cudaSuccess) return e;
     end(VNSA_STAGE_CMP);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TOPK);
@@ -1273,14 +1328,14 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     end(VNSA_STAGE_TOPK);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_SLC);
-    attn(MODE_SLC);
+    if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
     end(VNSA_STAGE_SLC);
     begin(VNSA_STAGE_SWA);
-    attn(MODE_SWA);
+    if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
     end(VNSA_STAGE_SWA);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TEXT);
-    attn(MODE_TEXT);
+    if ((e = attn(MODE_TEXT)) != cudaSuccess) return e;
     // grid-stride over (text query, head); the kernel reads N_t on the device
     text_combine_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->part, st->part_items);
     ++*launches;
