@@ -24,7 +24,9 @@ struct Counts {
     int contiguous;  // 1 if the vision tokens are one run of positions
     int vis_base;    // position of the first vision token (if contiguous)
     int nb;          // complete blocks N_v / block
-    int pad[3];
+    int pad[3];      // (decode step state)
+    int txt_contiguous;  // 1 if the text tokens are one run of positions
+    int txt_base;        // position of the first text token (if contiguous)
 };
 
 __device__ __forceinline__ float to_f(float x) { return x; }

@@ -173,6 +173,12 @@ __global__ void decode_prep_kernel(DecodeParams p) {
     } else {
         const int x = cn.n_text;
         p.txt[x] = t;
+        if (x == 0) {
+            cn.txt_base = t;
+            cn.txt_contiguous = 1;
+        } else {
+            cn.txt_contiguous = cn.txt_contiguous && (t == cn.txt_base + x);
+        }
         cn.n_text = x + 1;
         cn.pad[0] = cn.nb;
         cn.pad[1] = 0;

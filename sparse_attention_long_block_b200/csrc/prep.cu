@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restri
         cn.vis_base = nv > 0 ? vis[0] : 0;
         cn.contiguous = (nv == 0) || (vis[nv - 1] - vis[0] == nv - 1);
         cn.pad[0] = cn.pad[1] = cn.pad[2] = 0;
+        cn.txt_base = nt > 0 ? txt[0] : 0;
+        cn.txt_contiguous = (nt == 0) || (txt[nt - 1] - txt[0] == nt - 1);
         *counts = cn;
     }
 }

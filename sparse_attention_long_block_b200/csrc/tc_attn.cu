@@ -106,7 +106,8 @@ struct Work {
     int items;
     int nb;
     int contiguous, vis_base;
-    int q_tma;     // Q tiles arrive by one TMA box (vision modes, contiguous vision run)
+    int q_tma;     // Q tiles arrive by one TMA box (the item kind's tokens are one run)
+    int q_base;    // position of the first token of that run
 };
 
 template <int MODE>
@@ -118,7 +119,8 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
     w.nb = cn.nb;
     w.contiguous = cn.contiguous;
     w.vis_base = cn.vis_base;
-    w.q_tma = MODE != MODE_TEXT && cn.contiguous;
+    w.q_tma = MODE == MODE_TEXT ? cn.txt_contiguous : cn.contiguous;
+    w.q_base = MODE == MODE_TEXT ? cn.txt_base : cn.vis_base;
     w.nsplit = 1;
     w.split_len = 0;
     if (MODE == MODE_TEXT) {
@@ -275,9 +277,9 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
                 return;
             const uint32_t qb = sm.bar(B_Q_FULL);
             ptx::mbar_expect_tx(qb, (uint32_t)(w.qt * qrows) * 2u * kD);
-            ptx::tma_load_3d(sm.base_u32 + SM_Q, &P.tm_q, qb, 0, it.g * L.r, w.vis_base + it.q0);
+            ptx::tma_load_3d(sm.base_u32 + SM_Q, &P.tm_q, qb, 0, it.g * L.r, w.q_base + it.q0);
             ptx::tma_load_3d(sm.base_u32 + SM_Q + 16384, &P.tm_q, qb, 64, it.g * L.r,
-                             w.vis_base + it.q0);
+                             w.q_base + it.q0);
             ++nq;
         }
         // row coordinate of tile x of a segment (both CMP segments share keys)
@@ -1289,7 +1291,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     cudaError_t e;
     auto attn = [&](int mode) -> cudaError_t {
         P.mode = mode;
-        if (mode != MODE_TEXT) {
+        {
             const int rq = mode == MODE_CMP ? pow2_at_least(L.r) : L.r;
             if (!make_map_q(&P.tm_q, L.q, c.h_q, L.n, rq, kRows / rq)) return cudaErrorInvalidValue;
         }
