@@ -92,8 +92,8 @@ def executed_work(wl, is_vision, idx):
     128 * 64 * d flops per QK^T or P V product.  Compression: 16 queries per
     tile (8 head slots), a statistics pass (QK^T) and an exact pass (QK^T + P V)
     over the visible blocks; selection: 18 queries (7 heads) against the union
-    of their selected blocks (from idx [h_kv][N_v][k]); window and text: 18
-    queries against their key ranges."""
+    of the 64-key tiles their selected blocks reach (from idx [h_kv][N_v][k]);
+    window and text: 18 queries against their key ranges."""
     prod = 2.0 * 128 * 64 * wl.d
     vis = np.nonzero(is_vision)[0]
     txt = np.nonzero(is_vision == 0)[0]
@@ -113,8 +113,19 @@ def executed_work(wl, is_vision, idx):
         lo = max(0, q0 - wl.window + 1)
         swa += 2 * ((ql - lo + 64) // 64)
         for g in range(wl.h_kv):
-            sel = idx[g, q0:ql + 1].ravel()
-            slc += 2 * len(np.unique(sel[sel >= 0]))
+            sel = idx[g, q0:ql + 1]
+            if wl.block == 64:
+                sel = sel.ravel()
+                slc += 2 * len(np.unique(sel[sel >= 0]))
+                continue
+            # the 64-key tiles each selected block reaches, up to the query
+            ok = sel >= 0
+            a = sel.astype(np.int64) * wl.block
+            t0 = a // 64
+            t1 = np.minimum(a + wl.block - 1, np.arange(q0, ql + 1)[:, None]) // 64
+            span = int((t1 - t0)[ok].max()) if ok.any() else -1
+            parts = [(t0 + o)[ok & (t0 + o <= t1)] for o in range(span + 1)]
+            slc += 2 * (len(np.unique(np.concatenate(parts))) if parts else 0)
     for x0 in range(0, len(txt), qt):
         xl = min(len(txt), x0 + qt) - 1
         text += 2 * ((int(txt[xl]) + 64) // 64)
@@ -325,8 +336,8 @@ def main():
     isv = torch.from_numpy(x["is_vision"]).to(dev)
     gate = torch.from_numpy(x["gate"]).to(dev)
     out = torch.empty_like(q)
-    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
-                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                          top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
     stream = torch.cuda.current_stream()
 
@@ -520,8 +531,8 @@ def run_decode_bench(args, rank, world, local_rank):
     gate = torch.from_numpy(x["gate"]).to(dev)
     n = wl.n
     n0 = n - D
-    layer = binding.Layer(n_max=n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
-                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+    layer = binding.Layer(n_max=n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                          top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
     qs = [q[t].contiguous() for t in range(n0, n)]
     gs = [gate[t].contiguous() for t in range(n0, n)]

@@ -63,7 +63,13 @@ typedef struct vnsa_config {
     int n_max;        /* largest n a forward will see (sizes the workspace)     */
     int h_q, h_kv;    /* query heads, KV heads; h_q % h_kv == 0, h_q/h_kv <= 16  */
     int d;            /* head dim: 64 or 128                                    */
-    int block;        /* compression block = stride = selection block: 64       */
+    int block;        /* compression block = stride = selection block, >= 1:   */
+                      /* the vision tokens per frame (64 in the pages' setting; */
+                      /* the pages treat tokens per frame as a task knob).      */
+                      /* Every block size runs on the GPU; the tensor-core      */
+                      /* path takes bf16, d 128, 4..16 query heads per KV head  */
+                      /* and a selection of at most 1152 64-key tiles per 128-  */
+                      /* row item, other settings the SIMT kernels.             */
     int top_k;        /* blocks kept per (group, query), 1..64, >= #forced      */
     int window;       /* sliding window in vision tokens, >= 1                  */
     int force_first;  /* 1: block 0 is always selected (default 1)              */

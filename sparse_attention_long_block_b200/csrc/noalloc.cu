@@ -59,7 +59,7 @@ ScratchPlan plan_for(const vnsa_config &c, int n) {
 bool valid_config(const vnsa_config *c) {
     if (!c || c->h_q < 1 || c->h_kv < 1 || c->h_q % c->h_kv != 0) return false;
     if (c->d != 64 && c->d != 128) return false;
-    if (c->block != 64 || c->top_k < 1 || c->top_k > 64) return false;
+    if (c->block < 1 || c->top_k < 1 || c->top_k > 64) return false;
     if (c->h_q / c->h_kv > 16) return false;
     if (c->force_first < 0 || c->force_first > 1 || c->force_local < 0 || c->force_local > 1)
         return false;

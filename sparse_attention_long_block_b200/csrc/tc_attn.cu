@@ -31,6 +31,8 @@
 //         buffer that a small combine kernel reduces (or the row directly).
 #include <cuda.h>
 #include <math.h>
+
+#include <algorithm>
 #include <string.h>
 
 #include "tc_attn.h"
@@ -72,7 +74,15 @@ constexpr int B_K_FULL = 0, B_V_FULL = 2, B_K_EMPTY = 4, B_V_EMPTY = 6, B_S_FULL
 // buffer after P V of tile x (MMAs of one thread run in issue order).
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;
 
-enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3 };
+// Selection runs over 64-key tiles of vision ranks.  When the block size is a
+// multiple of 64 every tile lies inside one block and a query either takes a
+// whole tile or none of it (MODE_SLC); otherwise a tile holds parts of several
+// blocks and each row's keys are the parts of its own selected blocks
+// (MODE_SLC_UNALIGNED).
+enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3, MODE_SLC_UNALIGNED = 4 };
+__host__ __device__ constexpr bool is_slc(int m) {
+    return m == MODE_SLC || m == MODE_SLC_UNALIGNED;
+}
 enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
 
 struct TcParams {
@@ -179,7 +189,7 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
         it.seg_kind[0] = K_STATS;
         it.seg_tiles[0] = t;
         it.seg_tiles[1] = t;
-    } else if (MODE == MODE_SLC) {
+    } else if (is_slc(MODE)) {
         it.nseg = 1;
         it.seg_kind[0] = K_SLC;
         it.seg_tiles[0] = P.plan[(size_t)item * (1 + 2 * P.plan_max)];
@@ -258,7 +268,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
     if (MODE == MODE_CMP) {
         mk = &P.tm_kb;
         mv = &P.tm_vb;
-    } else if (MODE == MODE_SLC || MODE == MODE_SWA) {
+    } else if (is_slc(MODE) || MODE == MODE_SWA) {
         mk = w.contiguous ? &P.tm_k : &P.tm_kc;
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
@@ -462,6 +472,30 @@ __device__ __forceinline__ void imp_reduce_store(float (&p)[64], int lane, float
     }
 }
 
+// Valid columns of the 64-key tile at vision rank key0 for a query of vision
+// rank i whose selected blocks (block size B) are sel[0..k), ascending with -1
+// after the last: the parts of those blocks inside the tile, at or before i.
+// Tiles come in ascending order, so blocks that end before this tile are
+// skipped for good (cur).
+__device__ __forceinline__ uint64_t sel_coverage(const int32_t *sel, int &cur, int k, int B,
+                                                 int key0, int i) {
+    while (cur < k) {
+        const int j = sel[cur];
+        if (j < 0 || (j + 1) * B > key0) break;
+        ++cur;
+    }
+    uint64_t cov = 0ull;
+    for (int e = cur; e < k; ++e) {
+        const int j = sel[e];
+        if (j < 0 || j * B >= key0 + kKeys) break;
+        const int a = max(j * B - key0, 0), b = min((j + 1) * B - key0, kKeys);
+        cov |= (b >= 64 ? ~0ull : ((1ull << b) - 1ull)) & (~0ull << a);
+    }
+    const int hi = i - key0;  // causal: keys at or before the query
+    if (hi < 63) cov &= hi < 0 ? 0ull : ((2ull << hi) - 1ull);
+    return cov;
+}
+
 template <int MODE>
 __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
@@ -503,7 +537,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     pr[kD + 1] = 0.f;
                 } else {
                     // no selected / window key: this branch adds nothing
-                    float *dbg = MODE == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+                    float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
                         if (MODE == MODE_SWA)
@@ -539,7 +573,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // next item, so that neither waits on DRAM when it is needed
         if (rc.valid) {
             ptx::prefetch_l2(L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3);
-            if (MODE == MODE_SLC || MODE == MODE_SWA) {
+            if (is_slc(MODE) || MODE == MODE_SWA) {
                 const __half *part = (const __half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                 ptx::prefetch_l2(part);
                 ptx::prefetch_l2(part + 64);
@@ -555,20 +589,34 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::prefetch_l2(qr + 64);
             }
         }
-        // SLC: the item's selection tiles (first key, query mask) into shared
-        // memory, once every thread is done with the previous item's copy
-        if (MODE == MODE_SLC) {
+        // SLC: the item's selection tiles (first key, and the query mask or,
+        // for blocks not aligned to tiles, every query's selected blocks) into
+        // shared memory, once every thread is done with the previous item's copy
+        if (is_slc(MODE)) {
             group_sync(sm, gphase, ok, L);
             if (!ok) break;
             int32_t *dst = (int32_t *)(sm.base + SM_PLAN);
             const int32_t *src = P.plan + (size_t)item * (1 + 2 * P.plan_max);
             for (int x = rho; x < it.seg_tiles[0]; x += 128) {
                 dst[x] = src[1 + x] * kKeys;
-                dst[kPlanSmem + x] = src[1 + P.plan_max + x];
+                if (MODE == MODE_SLC) dst[kPlanSmem + x] = src[1 + P.plan_max + x];
+            }
+            if (MODE == MODE_SLC_UNALIGNED) {
+                for (int x = rho; x < w.qt * L.top_k; x += 128) {
+                    const int qi = x / L.top_k;
+                    dst[kPlanSmem + x] =
+                        qi < it.nq ? L.idx_src[((size_t)it.g * L.idx_rows + it.q0 + qi) * L.top_k +
+                                               x % L.top_k]
+                                   : -1;
+                }
             }
             group_sync(sm, gphase, ok, L);
             if (!ok) break;
         }
+        // MODE_SLC_UNALIGNED: this row's selected blocks (ascending, -1 after
+        // the last) and the first of them that can still reach a later tile
+        const int32_t *my_sel = plan_s + kPlanSmem + min(rc.qi, w.qt - 1) * L.top_k;
+        int sel_cur = 0;
 
         float lse2 = -INFINITY;                 // CMP: from the stats segment
         float m_run = -INFINITY, l_run = 0.f;   // running max / sum (log2 units)
@@ -582,14 +630,18 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             uint32_t nmask = 0u;
             if (kind == K_SLC && it.seg_tiles[s] > 0) {
                 nkey0 = plan_s[0];
-                nmask = (uint32_t)plan_s[kPlanSmem];
+                if (MODE == MODE_SLC) nmask = (uint32_t)plan_s[kPlanSmem];
             }
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
                 const int key0 = kind == K_SLC ? nkey0 : tile_key0(P, it, item, kind, x);
                 const uint32_t qmask = nmask;
-                // column range [lo, hi] of valid keys for this row
+                // column range [lo, hi] of valid keys for this row, or (blocks
+                // not aligned to tiles) the bit set `cov` of its valid columns
                 int lo = 1, hi = 0;
-                if (rc.valid) {
+                uint64_t cov = 0ull;
+                if (MODE == MODE_SLC_UNALIGNED) {
+                    if (rc.valid) cov = sel_coverage(my_sel, sel_cur, L.top_k, L.block, key0, rc.i);
+                } else if (rc.valid) {
                     switch (kind) {
                         case K_STATS:
                         case K_EXACT: lo = 0; hi = rc.c_vis - 1 - key0; break;
@@ -605,8 +657,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     lo = max(lo, 0);
                     hi = min(hi, kKeys - 1);
                 }
-                const bool row_in = lo <= hi;
-                const bool row_full = lo == 0 && hi == kKeys - 1;
+                const bool row_in = MODE == MODE_SLC_UNALIGNED ? cov != 0ull : lo <= hi;
+                const bool row_full =
+                    MODE == MODE_SLC_UNALIGNED ? cov == ~0ull : (lo == 0 && hi == kKeys - 1);
                 // every row of the warp either takes the whole tile or none of
                 // it (selection tiles off the diagonal, interior window and
                 // text tiles): rows are masked by their exponent bias alone
@@ -625,7 +678,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tc_fence_after();
                 if (kind == K_SLC && x + 1 < it.seg_tiles[s]) {
                     nkey0 = plan_s[x + 1];
-                    nmask = (uint32_t)plan_s[kPlanSmem + x + 1];
+                    if (MODE == MODE_SLC) nmask = (uint32_t)plan_s[kPlanSmem + x + 1];
                 }
                 float sv[64];
                 bool need = false;
@@ -656,8 +709,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
                 // mask on the raw scores (scale > 0 keeps the order)
                 if (!rowwise) {
+                    if (MODE == MODE_SLC_UNALIGNED) {
+                        const uint32_t c0 = (uint32_t)cov, c1 = (uint32_t)(cov >> 32);
 #pragma unroll
-                    for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] : -INFINITY;
+                        for (int k = 0; k < 32; ++k) {
+                            sv[k] = ((c0 >> k) & 1u) ? sv[k] : -INFINITY;
+                            sv[32 + k] = ((c1 >> k) & 1u) ? sv[32 + k] : -INFINITY;
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 64; ++k) sv[k] = (k >= lo && k <= hi) ? sv[k] : -INFINITY;
+                    }
                 }
                 float mx;  // row max of this tile, in log2 units
                 {
@@ -815,12 +877,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
-        } else if (MODE == MODE_SLC || MODE == MODE_SWA) {
+        } else if (is_slc(MODE) || MODE == MODE_SWA) {
             const float g =
-                rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (MODE == MODE_SLC ? 1 : 2)])
+                rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (is_slc(MODE) ? 1 : 2)])
                          : 0.f;
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            float *dbg = MODE == MODE_SLC ? L.dbg_o_slc : L.dbg_o_swa;
+            float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
             __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
@@ -838,7 +900,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     if (dbg)
                         for (int z = 0; z < 8; ++z) dbg[prow + ch * 32 + k + z] = b8[z];
                     uint4 v;
-                    if (MODE == MODE_SLC) {
+                    if (is_slc(MODE)) {
                         __half2 *h2 = reinterpret_cast<__half2 *>(&v);
 #pragma unroll
                         for (int z = 0; z < 4; ++z) {
@@ -1017,8 +1079,16 @@ __global__ void prepare_kernel(LayerParams p, __nv_bfloat16 *kc, __half *vhc, __
 }
 
 // ---------------------------------------------------------------------------
-// Union of the blocks selected by the queries of each SLC item, with a mask of
-// the queries that chose each block.  One warp per item.
+// Union over the queries of each SLC item of the 64-key tiles their selected
+// blocks reach (a block of B keys covers the tiles from key j*B to key
+// min(j*B + B - 1, i) of query i), with a mask of the queries that reach each
+// tile.  One warp per item.
+__device__ __forceinline__ void sel_tiles(int j, int B, int i, int &t0, int &t1) {
+    const long long a = (long long)j * B;
+    t0 = (int)(a / kKeys);
+    t1 = (int)(min(a + B - 1, (long long)i) / kKeys);
+}
+
 __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int words) {
     extern __shared__ uint32_t sh[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1039,7 +1109,11 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         for (int e = lane; e < ne; e += 32) {
             const int qi = e / p.top_k, x = e % p.top_k;
             const int j = p.idx_src[((size_t)g * p.idx_rows + q0 + qi) * p.top_k + x];
-            if (j >= 0 && (j >> 5) < words) atomicOr(&bm[j >> 5], 1u << (j & 31));
+            if (j < 0) continue;
+            int t0, t1;
+            sel_tiles(j, p.block, q0 + qi, t0, t1);
+            for (int t = t0; t <= t1 && (t >> 5) < words; ++t)
+                atomicOr(&bm[t >> 5], 1u << (t & 31));
         }
         __syncwarp();
         // exclusive prefix of popcounts over the words (lane-strided chunks)
@@ -1075,9 +1149,13 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         for (int e = lane; e < ne; e += 32) {
             const int qi = e / p.top_k, x = e % p.top_k;
             const int j = p.idx_src[((size_t)g * p.idx_rows + q0 + qi) * p.top_k + x];
-            if (j < 0 || (j >> 5) >= words) continue;
-            const int r = pre[j >> 5] + __popc(bm[j >> 5] & ((1u << (j & 31)) - 1u));
-            if (r < plan_max) atomicOr(&qm[r], 1u << qi);
+            if (j < 0) continue;
+            int t0, t1;
+            sel_tiles(j, p.block, q0 + qi, t0, t1);
+            for (int t = t0; t <= t1 && (t >> 5) < words; ++t) {
+                const int r = pre[t >> 5] + __popc(bm[t >> 5] & ((1u << (t & 31)) - 1u));
+                if (r < plan_max) atomicOr(&qm[r], 1u << qi);
+            }
         }
         __syncwarp();
         for (int x = lane; x < total && x < plan_max; x += 32) out[1 + plan_max + x] = (int)qm[x];
@@ -1209,20 +1287,38 @@ struct TcState {
     float *part;
 };
 
-bool tc_supported(const vnsa_config &c) {
+// Most 64-key selection tiles of one item: every query reaches at most top_k
+// blocks, each over at most `per_block` tiles, and there are only so many tiles.
+static int plan_tiles_max(const vnsa_config &c) {
     const int qt = kRows / (c.h_q / c.h_kv);
-    return c.dtype == VNSA_BF16 && c.d == kD && c.block == kKeys && c.h_q / c.h_kv <= 16 &&
-           qt * c.top_k <= kPlanSmem && encode_fn() != nullptr;
+    const int B = c.block;
+    int per_block;
+    if (B % kKeys == 0) per_block = B / kKeys;
+    else if (kKeys % B == 0) per_block = 1;
+    else per_block = (B + kKeys - 2) / kKeys + 1;
+    const long long bound = (long long)qt * c.top_k * per_block;
+    const long long tiles = (c.n_max + kKeys - 1) / kKeys;
+    return (int)std::min(bound, tiles);
+}
+
+// The tensor-core path: bf16, d = 128, 4 to 16 query heads per KV head (the
+// selection query masks are 32-bit: at most 32 queries per item), and an item's
+// selection plan and per-query block lists must fit the shared-memory copy.
+bool tc_supported(const vnsa_config &c) {
+    const int r = c.h_q / c.h_kv;
+    if (c.dtype != VNSA_BF16 || c.d != kD || r < 4 || r > 16) return false;
+    const int qt = kRows / r;
+    return qt * c.top_k <= kPlanSmem && plan_tiles_max(c) <= kPlanSmem && encode_fn() != nullptr;
 }
 
 static size_t plan_bytes(const vnsa_config &c) {
     const int qt = kRows / (c.h_q / c.h_kv);
     const size_t items = (size_t)c.h_kv * ((c.n_max + qt - 1) / qt);
-    return items * (1 + 2 * (size_t)qt * c.top_k) * 4;
+    return items * (1 + 2 * (size_t)plan_tiles_max(c)) * 4;
 }
 
 size_t tc_workspace_bytes(const vnsa_config &c) {
-    if (c.dtype != VNSA_BF16 || c.d != kD || c.block != kKeys) return 0;
+    if (!tc_supported(c)) return 0;
     const size_t kv = (size_t)c.n_max * c.h_kv * kD * 2;
     const size_t kvb = (size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2;
     return up256(kv) * 3 + up256(kvb) + up256(plan_bytes(c)) + kTextPartBytes;
@@ -1236,8 +1332,7 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&st->num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const int qt = kRows / (c.h_q / c.h_kv);
-    st->plan_max = qt * c.top_k;
+    st->plan_max = plan_tiles_max(c);
     st->part_items = (int)(kTextPartBytes / ((size_t)kRows * kPartStride * 4));
     char *p = (char *)ws;
     const size_t kv = up256((size_t)c.n_max * c.h_kv * kD * 2);
@@ -1250,7 +1345,7 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     st->part = (float *)(p + 3 * kv + kvb + up256(plan_bytes(c)));
     cudaError_t e = cudaSuccess;
     for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
-                    tc_attn_kernel<MODE_TEXT>})
+                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>})
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) {
@@ -1298,6 +1393,9 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         switch (mode) {
             case MODE_CMP: tc_attn_kernel<MODE_CMP><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             case MODE_SLC: tc_attn_kernel<MODE_SLC><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            case MODE_SLC_UNALIGNED:
+                tc_attn_kernel<MODE_SLC_UNALIGNED><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                break;
             case MODE_SWA: tc_attn_kernel<MODE_SWA><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             default: tc_attn_kernel<MODE_TEXT><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
         }
@@ -1316,7 +1414,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         ++*launches;
     }
     {
-        const int words = (L.nb_max + 1 + 31) / 32 + 1;
+        const int words = ((c.n_max + kKeys - 1) / kKeys + 31) / 32 + 1;
         const int wpb = 4;
         const size_t smem = (size_t)wpb * (2 * words + st->plan_max) * 4;
         if (smem > 48 * 1024) {
@@ -1330,7 +1428,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     end(VNSA_STAGE_TOPK);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_SLC);
-    if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
+    if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) return e;
     end(VNSA_STAGE_SLC);
     begin(VNSA_STAGE_SWA);
     if ((e = attn(MODE_SWA)) != cudaSuccess) return e;

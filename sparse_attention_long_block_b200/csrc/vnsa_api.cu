@@ -71,7 +71,6 @@ vnsa_status check_config(const vnsa_config *c) {
     if (c->dtype != VNSA_BF16 && c->dtype != VNSA_FP32) return VNSA_ERR_INVALID_ARG;
     if (c->n_max > kMaxTokens) return VNSA_ERR_UNSUPPORTED;
     if (c->d != 64 && c->d != 128) return VNSA_ERR_UNSUPPORTED;
-    if (c->block != 64) return VNSA_ERR_UNSUPPORTED;
     if (c->h_q / c->h_kv > 16) return VNSA_ERR_UNSUPPORTED;
     if (c->top_k > 64) return VNSA_ERR_UNSUPPORTED;
     return VNSA_OK;

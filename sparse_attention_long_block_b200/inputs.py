@@ -9,8 +9,10 @@ layer: 28 query heads, 4 KV heads, head dim 128; 64 tokens per frame; contexts
 from 8K to the 36K training length and on to 128K), with video replaced by a
 frame-mean model because no video data or trained weights are available:
 
-* For each of Q, K and V separately, every frame f (64 vision tokens) and every
-  head has a mean m_f ~ N(0, I_d); each vision token is m_f + N(0, 0.5 I_d).
+* For each of Q, K and V separately, every frame f (64 vision tokens, or
+  ``frame`` tokens: the pages call tokens per frame a task knob, and the
+  block-size workloads match the compression block to it) and every head has a
+  mean m_f ~ N(0, I_d); each vision token is m_f + N(0, 0.5 I_d).
   With ``ar1`` (the 128K workload) the K and V frame means drift:
   m_f = 0.9 m_{f-1} + sqrt(0.19) eps_f, which keeps their variance at 1.
 * A text token is its own N(0, I_d) mean plus N(0, 0.5 I_d) noise.
@@ -31,7 +33,7 @@ from dataclasses import dataclass, replace
 
 import numpy as np
 
-FRAME = 64  # vision tokens per frame (= compression block)
+FRAME = 64  # vision tokens per frame (= compression block) unless a workload sets its own
 
 
 @dataclass(frozen=True)
@@ -49,6 +51,7 @@ class Workload:
     seed: int = 0
     block: int = 64
     dense: bool = False          # Dense-NSA: every token attends densely (no vision set)
+    frame: int = FRAME           # vision tokens per frame of the frame-mean model
 
     @property
     def n(self) -> int:
@@ -77,6 +80,14 @@ WORKLOADS = {
     "dense_36k": Workload("dense_36k", 35840, 512, top_k=16, window=256, dense=True),
     "dense_128k": Workload("dense_128k", 130048, 1024, top_k=32, window=512, ar1=True,
                            dense=True),
+    # Tokens per frame as a knob (block = frame size) at the training length,
+    # each with the 1,024-token selection budget of top-16 x 64: 16 tokens per
+    # frame (top-64), 32 (top-32), 36 (6 x 6 patches, top-28) and 128 (top-8).
+    "tpf16_36k": Workload("tpf16_36k", 35840, 512, top_k=64, window=256, block=16, frame=16),
+    "tpf32_36k": Workload("tpf32_36k", 35840, 512, top_k=32, window=256, block=32, frame=32),
+    "tpf36_36k": Workload("tpf36_36k", 35856, 512, top_k=28, window=256, block=36, frame=36),
+    "tpf128_36k": Workload("tpf128_36k", 35840, 512, top_k=8, window=256, block=128,
+                           frame=128),
 }
 
 
@@ -92,8 +103,8 @@ def bf16_round(a: np.ndarray) -> np.ndarray:
     return a
 
 
-def _frame_tokens(rng, n_vision, h, d, ar1):
-    n_frames = (n_vision + FRAME - 1) // FRAME
+def _frame_tokens(rng, n_vision, h, d, ar1, frame):
+    n_frames = (n_vision + frame - 1) // frame
     means = rng.standard_normal((n_frames, h, d), dtype=np.float32)
     if ar1 and n_frames > 1:
         c = np.float32(np.sqrt(0.19))
@@ -101,7 +112,7 @@ def _frame_tokens(rng, n_vision, h, d, ar1):
             means[f] = np.float32(0.9) * means[f - 1] + c * means[f]
     noise = rng.standard_normal((n_vision, h, d), dtype=np.float32)
     noise *= np.float32(np.sqrt(0.5))
-    noise += np.repeat(means, FRAME, axis=0)[:n_vision]
+    noise += np.repeat(means, frame, axis=0)[:n_vision]
     return noise
 
 
@@ -135,7 +146,7 @@ def generate(wl: Workload, is_vision: np.ndarray | None = None) -> dict:
     tensors = {}
     for name, h in (("q", wl.h_q), ("k", wl.h_kv), ("v", wl.h_kv)):
         x = np.empty((n, h, wl.d), np.float32)
-        x[vis_pos] = _frame_tokens(rng, wl.n_vision, h, wl.d, wl.ar1 and name != "q")
+        x[vis_pos] = _frame_tokens(rng, wl.n_vision, h, wl.d, wl.ar1 and name != "q", wl.frame)
         x[txt_pos] = _text_tokens(rng, wl.n_text, h, wl.d)
         tensors[name] = x
     gate = rng.standard_normal((n, wl.h_q, 3), dtype=np.float32)

@@ -48,6 +48,14 @@ def test_workspace_bytes_valid_config():
     assert b > 4 * 8448 * (8448 // 64) * 4
 
 
+@pytest.mark.parametrize("block", [1, 16, 32, 36, 100, 128, 256])
+def test_any_block_size_is_accepted(block):
+    # tokens per frame is a knob: every block size >= 1 is a valid layer, and
+    # the importance workspace [h_kv][n_max][n_max / block] grows as it shrinks
+    b = binding.vnsa_workspace_bytes(cfg(block=block))
+    assert b >= 4 * 8448 * (8448 // block) * 4
+
+
 @pytest.mark.parametrize("bad,code", [
     (dict(h_q=28, h_kv=3), binding.VNSA_ERR_INVALID_ARG),
     (dict(top_k=1), binding.VNSA_ERR_INVALID_ARG),
@@ -58,7 +66,7 @@ def test_workspace_bytes_valid_config():
     (dict(scale=float("nan")), binding.VNSA_ERR_INVALID_ARG),
     (dict(dtype=7), binding.VNSA_ERR_INVALID_ARG),
     (dict(d=96), binding.VNSA_ERR_UNSUPPORTED),
-    (dict(block=32), binding.VNSA_ERR_UNSUPPORTED),
+    (dict(block=0), binding.VNSA_ERR_INVALID_ARG),
     (dict(top_k=65), binding.VNSA_ERR_UNSUPPORTED),
     (dict(n_max=262145), binding.VNSA_ERR_UNSUPPORTED),
     (dict(h_q=34, h_kv=2), binding.VNSA_ERR_UNSUPPORTED),

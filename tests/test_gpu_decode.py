@@ -39,8 +39,8 @@ def _run_decode(wl: Workload, x: dict, n0: int):
     v = torch.from_numpy(x["v"]).to(dev, td).contiguous()
     isv = torch.from_numpy(x["is_vision"]).to(dev)
     gate = torch.from_numpy(x["gate"]).to(dev)
-    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
-                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                          top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
     layer.forward(q[:n0].contiguous(), k[:n0].contiguous(), v[:n0].contiguous(),
                   isv[:n0].contiguous(), gate[:n0].contiguous())
@@ -122,6 +122,18 @@ def test_decode_from_short_prefill_crosses_first_blocks():
     _compare(wl, x, n0=2)
 
 
+def test_decode_block_36_straddles_tiles():
+    # block 36 (6 x 6 patches per frame): decoded vision ranks 1420..1499
+    # complete blocks 39 and 40 and open block 41
+    tail = "1" * 50 + "0" * 3 + "1" * 30
+    mask = _stream_mask(1500, 20, tail)
+    n = len(mask)
+    wl = Workload("decode_b36", int(mask.sum()), n - int(mask.sum()), top_k=8, window=100,
+                  block=36, frame=36)
+    x = generate(wl, is_vision=mask)
+    _compare(wl, x, n0=n - len(tail))
+
+
 def test_decode_long_128k_tail():
     base = WORKLOADS["long_128k"]
     # the 128K stream; the last 80 tokens (text, then vision that completes the
@@ -145,8 +157,8 @@ def test_decode_rejects_a_gap_in_the_stream():
     q, k, v = (torch.from_numpy(x[nm]).to(dev, torch.bfloat16).contiguous() for nm in ("q", "k", "v"))
     isv = torch.from_numpy(x["is_vision"]).to(dev)
     gate = torch.from_numpy(x["gate"]).to(dev)
-    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
-                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                          top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]))
     # no prefill yet
     with pytest.raises(binding.VnsaError):

@@ -26,8 +26,8 @@ def _regular(wl, x, dev):
     """o_cmp / idx / importance from vnsa_forward's debug exports."""
     import torch
     td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, top_k=wl.top_k,
-                          window=wl.window, w_k=torch.from_numpy(x["w_k"]),
+    layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
+                          top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
     dbg, t = binding.make_debug(wl.n, wl.h_q, wl.h_kv, wl.d, wl.top_k, dtype=td,
                                 want=("o_cmp", "idx", "imp"))
