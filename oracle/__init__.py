@@ -52,6 +52,12 @@ class _Cfg(ctypes.Structure):
                 ("round_cmp_bf16", ctypes.c_int)]
 
 
+class _CmpMLP(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int)] + [
+        (nm, ctypes.c_void_p) for nm in ("w1_k", "b1_k", "w2_k", "b2_k",
+                                         "w1_v", "b1_v", "w2_v", "b2_v")]
+
+
 def _load():
     global _lib
     if _lib is None:
@@ -62,6 +68,14 @@ def _load():
             ctypes.c_int] + [p] * 10
         lib.vnsa_oracle_pool_proj.restype = ctypes.c_int
         lib.vnsa_oracle_pool_proj.argtypes = [ctypes.POINTER(_Cfg)] + [p] * 7
+        lib.vnsa_oracle_forward_mlp.restype = ctypes.c_int
+        lib.vnsa_oracle_forward_mlp.argtypes = [ctypes.POINTER(_Cfg)] + [p] * 5 + [
+            ctypes.POINTER(_CmpMLP), ctypes.c_int] + [p] * 10
+        lib.vnsa_oracle_pool_mlp.restype = ctypes.c_int
+        lib.vnsa_oracle_pool_mlp.argtypes = [ctypes.POINTER(_Cfg), p, p, p,
+                                             ctypes.POINTER(_CmpMLP), p, p]
+        lib.vnsa_oracle_gate_mlp.restype = ctypes.c_int
+        lib.vnsa_oracle_gate_mlp.argtypes = [ctypes.c_int] * 4 + [p] * 5 + [ctypes.c_int, p]
         lib.vnsa_oracle_round_bf16.restype = ctypes.c_double
         lib.vnsa_oracle_round_bf16.argtypes = [ctypes.c_double]
         lib.vnsa_oracle_threads.restype = ctypes.c_int
@@ -109,25 +123,72 @@ def round_bf16(x: float) -> float:
     return float(_load().vnsa_oracle_round_bf16(float(x)))
 
 
-def pool_proj(p: OracleParams, k, v, is_vision, w_k, w_v):
-    """K_cmp, V_cmp [nb][h_kv][d] in fp64 (compression keys/values)."""
-    k, v, w_k, w_v = _f32(k), _f32(v), _f32(w_k), _f32(w_v)
+CMP_MLP_KEYS = ("w1_k", "b1_k", "w2_k", "b2_k", "w1_v", "b1_v", "w2_v", "b2_v")
+
+
+def _cmp_mlp(d: int, mlp: dict):
+    """ctypes form of a compression perceptron {"w1_k": [d][H], "b1_k": [H],
+    "w2_k": [H][d], "b2_k": [d], and the same for v} plus the arrays it points
+    to (kept alive by the caller)."""
+    arrs = {nm: _f32(mlp[nm]) for nm in CMP_MLP_KEYS}
+    hidden = arrs["b1_k"].shape[0]
+    for t in ("k", "v"):
+        if (arrs["w1_" + t].shape != (d, hidden) or arrs["b1_" + t].shape != (hidden,)
+                or arrs["w2_" + t].shape != (hidden, d) or arrs["b2_" + t].shape != (d,)):
+            raise ValueError("compression MLP weights must be [d][H], [H], [H][d], [d]")
+    s = _CmpMLP(hidden, *[arrs[nm].ctypes.data for nm in CMP_MLP_KEYS])
+    return s, arrs
+
+
+def pool_proj(p: OracleParams, k, v, is_vision, w_k=None, w_v=None, cmp_mlp=None):
+    """K_cmp, V_cmp [nb][h_kv][d] in fp64 (compression keys/values): the linear
+    map W_K, W_V, or the compression perceptron ``cmp_mlp`` (a dict of its
+    weights, see ``_cmp_mlp``)."""
+    k, v = _f32(k), _f32(v)
     isv = np.ascontiguousarray(is_vision, dtype=np.uint8)
     n = isv.shape[0]
     nb = int(isv.sum()) // p.block
     kc = np.zeros((max(nb, 0), p.h_kv, p.d), np.float64)
     vc = np.zeros_like(kc)
     cfg = _cfg(p, n)
-    rc = _load().vnsa_oracle_pool_proj(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(isv),
-                                       _ptr(w_k), _ptr(w_v), _ptr(kc), _ptr(vc))
+    if cmp_mlp is None:
+        w_k, w_v = _f32(w_k), _f32(w_v)
+        rc = _load().vnsa_oracle_pool_proj(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(isv),
+                                           _ptr(w_k), _ptr(w_v), _ptr(kc), _ptr(vc))
+    else:
+        m, keep = _cmp_mlp(p.d, cmp_mlp)
+        rc = _load().vnsa_oracle_pool_mlp(ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(isv),
+                                          ctypes.byref(m), _ptr(kc), _ptr(vc))
+        del keep
     if rc != 0:
         raise ValueError(f"oracle pool_proj rejected its arguments (code {rc})")
     return kc, vc
 
 
+def gate_mlp(x, g1, c1, g2, c2, round_hidden_bf16=False):
+    """Gate logits [n][n_out] of the layer input x [n][D] through the two-layer
+    gate perceptron (g1 [D][H], c1 [H], g2 [H][n_out], c2 [n_out]); n_out =
+    3 h_q with column 3h + c the logit of branch c of head h."""
+    x, g1, c1, g2, c2 = _f32(x), _f32(g1), _f32(c1), _f32(g2), _f32(c2)
+    n, dm = x.shape
+    hidden = c1.shape[0]
+    n_out = c2.shape[0]
+    if g1.shape != (dm, hidden) or g2.shape != (hidden, n_out):
+        raise ValueError("gate MLP weights must be [D][H] and [H][n_out]")
+    out = np.zeros((n, n_out), np.float64)
+    rc = _load().vnsa_oracle_gate_mlp(n, dm, hidden, n_out, _ptr(x), _ptr(g1), _ptr(c1),
+                                      _ptr(g2), _ptr(c2), int(bool(round_hidden_bf16)),
+                                      _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle gate_mlp rejected its arguments (code {rc})")
+    return out
+
+
 def forward(p: OracleParams, q, k, v, is_vision, gate, w_k, w_v, rows=None,
-            forced_idx=None, want=()):
-    """Layer prefill for the given global rows (all rows if None).
+            forced_idx=None, want=(), cmp_mlp=None):
+    """Layer prefill for the given global rows (all rows if None).  With
+    ``cmp_mlp`` the compression branch maps block means through that
+    perceptron instead of W_K, W_V.
 
     Returns a dict with "out" [R][h_q][d] and, for names in ``want``, any of
     "o_cmp", "o_slc", "o_swa" [R][h_q][d], "lse_cmp" [R][h_q], "idx" [R][h_kv][k],
@@ -135,7 +196,9 @@ def forward(p: OracleParams, q, k, v, is_vision, gate, w_k, w_v, rows=None,
     top-k of vision rows.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
-    gate, w_k, w_v = _f32(gate), _f32(w_k), _f32(w_v)
+    gate = _f32(gate)
+    if cmp_mlp is None:
+        w_k, w_v = _f32(w_k), _f32(w_v)
     isv = np.ascontiguousarray(is_vision, dtype=np.uint8)
     n = isv.shape[0]
     if rows is None:
@@ -164,12 +227,20 @@ def forward(p: OracleParams, q, k, v, is_vision, gate, w_k, w_v, rows=None,
             raise ValueError("forced_idx must be [rows][h_kv][top_k]")
     cfg = _cfg(p, n)
     nb_out = ctypes.c_int(0)
-    rc = _load().vnsa_oracle_forward(
-        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(isv), _ptr(gate),
-        _ptr(w_k), _ptr(w_v), nr, _ptr(rows_arr), _ptr(fidx), _ptr(res["out"]),
-        _ptr(res.get("o_cmp")), _ptr(res.get("o_slc")), _ptr(res.get("o_swa")),
-        _ptr(res.get("lse_cmp")), _ptr(res.get("idx")), _ptr(res.get("imp")),
-        ctypes.cast(ctypes.pointer(nb_out), ctypes.c_void_p))
+    tail = (nr, _ptr(rows_arr), _ptr(fidx), _ptr(res["out"]),
+            _ptr(res.get("o_cmp")), _ptr(res.get("o_slc")), _ptr(res.get("o_swa")),
+            _ptr(res.get("lse_cmp")), _ptr(res.get("idx")), _ptr(res.get("imp")),
+            ctypes.cast(ctypes.pointer(nb_out), ctypes.c_void_p))
+    if cmp_mlp is None:
+        rc = _load().vnsa_oracle_forward(
+            ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(isv), _ptr(gate),
+            _ptr(w_k), _ptr(w_v), *tail)
+    else:
+        m, keep = _cmp_mlp(p.d, cmp_mlp)
+        rc = _load().vnsa_oracle_forward_mlp(
+            ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(isv), _ptr(gate),
+            ctypes.byref(m), *tail)
+        del keep
     if rc != 0:
         raise ValueError(f"oracle forward rejected its arguments (code {rc})")
     return res

@@ -49,6 +49,19 @@
  *   R9  Every branch uses the same softmax scale (default 1/sqrt(d)).
  *   R10 A text token at global position t attends to every token u <= t,
  *       vision or text, with KV head floor(h / (H_q/H_kv)).
+ *   R11 The "learnable MLP" of the compression branch [M], when a hidden width
+ *       H_c is given instead of R3's linear map: a two-layer perceptron on the
+ *       block mean, K_cmp = SiLU(Kbar . W1 + b1) . W2 + b2 with W1 [d][H_c],
+ *       W2 [H_c][d], SiLU(z) = z / (1 + e^-z); its own weights for K and for V,
+ *       shared by the KV heads.  The hidden layer is exact; the output is
+ *       rounded as in R3.
+ *   R12 The gate [M] ("a two-layer MLP + sigmoid gate per head"): the branch
+ *       logits of token t come from the layer input x_t (h_q * d wide) through
+ *       logits = SiLU(x_t . G1 + c1) . G2 + c2, G1 [D][H], G2 [H][3 h_q]; output
+ *       column 3h + c is the logit of branch c (cmp, slc, swa) of head h, and
+ *       the sigmoid of R8 turns it into the gate.  In bf16 runs the hidden
+ *       activations are rounded to bf16 (round-to-nearest-even): they are the
+ *       operand of the second product.
  */
 #include <math.h>
 #include <stdint.h>
@@ -84,6 +97,49 @@ double vnsa_oracle_round_bf16(double x)
 }
 
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* SiLU (R11, R12): z * sigmoid(z). */
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* The compression map of one tensor (K or V), fp64: R3's linear map w [d][d]
+ * when hidden == 0, else R11's perceptron w1 [d][hidden], b1 [hidden],
+ * w2 [hidden][d], b2 [d]. */
+typedef struct {
+    int hidden;
+    const double *w, *w1, *b1, *w2, *b2;
+} cmp_map;
+
+/* Public form of R11's weights (fp32 values, as handed to the GPU). */
+typedef struct {
+    int hidden;                               /* H_c >= 1                       */
+    const float *w1_k, *b1_k, *w2_k, *b2_k;   /* [d][H_c], [H_c], [H_c][d], [d] */
+    const float *w1_v, *b1_v, *w2_v, *b2_v;
+} vnsa_oracle_cmp_mlp;
+
+/* out[d] = the compression map applied to the block mean m[d]; h: scratch of
+ * `hidden` values. */
+static void apply_cmp_map(const cmp_map *mp, int d, const double *m, double *h, double *out)
+{
+    if (mp->hidden == 0) {
+        for (int col = 0; col < d; ++col) {
+            double a = 0.0;
+            for (int e = 0; e < d; ++e) a += m[e] * mp->w[(size_t)e * d + col];
+            out[col] = a;
+        }
+        return;
+    }
+    const int H = mp->hidden;
+    for (int x = 0; x < H; ++x) {
+        double a = mp->b1[x];
+        for (int e = 0; e < d; ++e) a += m[e] * mp->w1[(size_t)e * H + x];
+        h[x] = silu(a);
+    }
+    for (int col = 0; col < d; ++col) {
+        double a = mp->b2[col];
+        for (int x = 0; x < H; ++x) a += h[x] * mp->w2[(size_t)x * d + col];
+        out[col] = a;
+    }
+}
 
 /*
  * One softmax attention of query q (d values, already fp64) over a key list.
@@ -145,14 +201,16 @@ static int check_cfg(const vnsa_oracle_cfg *c)
  * k_cmp, v_cmp: [nb][h_kv][d].  Kd, Vd: fp64 copies of K, V [n][h_kv][d].
  */
 static void pool_proj(const vnsa_oracle_cfg *c, const double *Kd, const double *Vd,
-                      const int *vis, int nb, const double *wk, const double *wv,
+                      const int *vis, int nb, const cmp_map *mk, const cmp_map *mv,
                       double *k_cmp, double *v_cmp)
 {
     const int d = c->d, hk = c->h_kv, B = c->block;
+    const int H = mk->hidden > mv->hidden ? mk->hidden : mv->hidden;
     #pragma omp parallel for schedule(static)
     for (int j = 0; j < nb; ++j) {
-        double *kbar = malloc(sizeof(double) * 2 * d);
+        double *kbar = malloc(sizeof(double) * (2 * d + (H > 0 ? H : 1)));
         double *vbar = kbar + d;
+        double *hid = vbar + d;
         for (int g = 0; g < hk; ++g) {
             for (int e = 0; e < d; ++e) { kbar[e] = 0.0; vbar[e] = 0.0; }
             for (int u = 0; u < B; ++u) {
@@ -162,19 +220,71 @@ static void pool_proj(const vnsa_oracle_cfg *c, const double *Kd, const double *
             for (int e = 0; e < d; ++e) { kbar[e] /= B; vbar[e] /= B; }
             double *ko = k_cmp + ((size_t)j * hk + g) * d;
             double *vo = v_cmp + ((size_t)j * hk + g) * d;
-            for (int col = 0; col < d; ++col) {
-                double ak = 0.0, av = 0.0;
-                for (int e = 0; e < d; ++e) {
-                    ak += kbar[e] * wk[(size_t)e * d + col];
-                    av += vbar[e] * wv[(size_t)e * d + col];
+            apply_cmp_map(mk, d, kbar, hid, ko);
+            apply_cmp_map(mv, d, vbar, hid, vo);
+            if (c->round_cmp_bf16)
+                for (int col = 0; col < d; ++col) {
+                    ko[col] = vnsa_oracle_round_bf16(ko[col]);
+                    vo[col] = vnsa_oracle_round_bf16(vo[col]);
                 }
-                if (c->round_cmp_bf16) { ak = vnsa_oracle_round_bf16(ak); av = vnsa_oracle_round_bf16(av); }
-                ko[col] = ak;
-                vo[col] = av;
-            }
         }
         free(kbar);
     }
+}
+
+/* fp64 copies of a compression map's weights (R3 from w, or R11 from the
+ * perceptron); returns 0 on allocation failure.  free_cmp_map releases them. */
+static int load_cmp_map(cmp_map *mp, int d, const float *w, int hidden, const float *w1,
+                        const float *b1, const float *w2, const float *b2)
+{
+    memset(mp, 0, sizeof(*mp));
+    mp->hidden = hidden;
+    if (hidden == 0) {
+        double *x = malloc(sizeof(double) * (size_t)d * d);
+        if (!x) return 0;
+        for (size_t e = 0; e < (size_t)d * d; ++e) x[e] = w[e];
+        mp->w = x;
+        return 1;
+    }
+    const size_t n1 = (size_t)d * hidden;
+    double *x = malloc(sizeof(double) * (2 * n1 + hidden + d));
+    if (!x) return 0;
+    for (size_t e = 0; e < n1; ++e) { x[e] = w1[e]; x[n1 + e] = w2[e]; }
+    for (int e = 0; e < hidden; ++e) x[2 * n1 + e] = b1[e];
+    for (int e = 0; e < d; ++e) x[2 * n1 + hidden + e] = b2[e];
+    mp->w1 = x;
+    mp->w2 = x + n1;
+    mp->b1 = x + 2 * n1;
+    mp->b2 = x + 2 * n1 + hidden;
+    return 1;
+}
+
+static void free_cmp_map(cmp_map *mp)
+{
+    free((void *)(mp->hidden == 0 ? mp->w : mp->w1));
+}
+
+static int load_cmp_maps(cmp_map *mk, cmp_map *mv, int d, const float *w_k, const float *w_v,
+                         const vnsa_oracle_cmp_mlp *mlp)
+{
+    int okk, okv;
+    if (mlp) {
+        okk = load_cmp_map(mk, d, NULL, mlp->hidden, mlp->w1_k, mlp->b1_k, mlp->w2_k, mlp->b2_k);
+        okv = load_cmp_map(mv, d, NULL, mlp->hidden, mlp->w1_v, mlp->b1_v, mlp->w2_v, mlp->b2_v);
+    } else {
+        okk = load_cmp_map(mk, d, w_k, 0, NULL, NULL, NULL, NULL);
+        okv = load_cmp_map(mv, d, w_v, 0, NULL, NULL, NULL, NULL);
+    }
+    if (okk && okv) return 1;
+    if (okk) free_cmp_map(mk);
+    if (okv) free_cmp_map(mv);
+    return 0;
+}
+
+static int mlp_ok(const vnsa_oracle_cmp_mlp *m)
+{
+    return m && m->hidden >= 1 && m->w1_k && m->b1_k && m->w2_k && m->b2_k && m->w1_v &&
+           m->b1_v && m->w2_v && m->b2_v;
 }
 
 /*
@@ -215,25 +325,82 @@ static int select_blocks(const double *imp, int nvis, int i, int B, int k,
     return nsel;
 }
 
+static int pool_impl(const vnsa_oracle_cfg *c, const float *k, const float *v,
+                     const uint8_t *is_vision, const float *w_k, const float *w_v,
+                     const vnsa_oracle_cmp_mlp *mlp, double *k_cmp, double *v_cmp)
+{
+    const int n = c->n, d = c->d, hk = c->h_kv;
+    int *vis = malloc(sizeof(int) * (n > 0 ? n : 1));
+    double *Kd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
+    double *Vd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
+    cmp_map mk, mv;
+    if (!vis || !Kd || !Vd || !load_cmp_maps(&mk, &mv, d, w_k, w_v, mlp)) {
+        free(vis); free(Kd); free(Vd);
+        return ORACLE_ENOMEM;
+    }
+    for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
+    int nv = partition(is_vision, n, vis);
+    pool_proj(c, Kd, Vd, vis, nv / c->block, &mk, &mv, k_cmp, v_cmp);
+    free(vis); free(Kd); free(Vd); free_cmp_map(&mk); free_cmp_map(&mv);
+    return ORACLE_OK;
+}
+
 /* K_cmp / V_cmp only (for the pooling parity checks). Outputs [nb][h_kv][d]. */
 int vnsa_oracle_pool_proj(const vnsa_oracle_cfg *c, const float *k, const float *v,
                           const uint8_t *is_vision, const float *w_k, const float *w_v,
                           double *k_cmp, double *v_cmp)
 {
-    if (!check_cfg(c)) return ORACLE_EINVAL;
-    const int n = c->n, d = c->d, hk = c->h_kv;
-    int *vis = malloc(sizeof(int) * (n > 0 ? n : 1));
-    double *Kd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
-    double *Vd = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * hk * d);
-    double *wk = malloc(sizeof(double) * (size_t)d * d);
-    double *wv = malloc(sizeof(double) * (size_t)d * d);
-    if (!vis || !Kd || !Vd || !wk || !wv) { free(vis); free(Kd); free(Vd); free(wk); free(wv); return ORACLE_ENOMEM; }
-    for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
-    for (size_t x = 0; x < (size_t)d * d; ++x) { wk[x] = w_k[x]; wv[x] = w_v[x]; }
-    int nv = partition(is_vision, n, vis);
-    pool_proj(c, Kd, Vd, vis, nv / c->block, wk, wv, k_cmp, v_cmp);
-    free(vis); free(Kd); free(Vd); free(wk); free(wv);
-    return ORACLE_OK;
+    if (!check_cfg(c) || !w_k || !w_v) return ORACLE_EINVAL;
+    return pool_impl(c, k, v, is_vision, w_k, w_v, NULL, k_cmp, v_cmp);
+}
+
+/* The same with R11's compression perceptron. */
+int vnsa_oracle_pool_mlp(const vnsa_oracle_cfg *c, const float *k, const float *v,
+                         const uint8_t *is_vision, const vnsa_oracle_cmp_mlp *mlp,
+                         double *k_cmp, double *v_cmp)
+{
+    if (!check_cfg(c) || !mlp_ok(mlp)) return ORACLE_EINVAL;
+    return pool_impl(c, k, v, is_vision, NULL, NULL, mlp, k_cmp, v_cmp);
+}
+
+/*
+ * Gate logits (R12) of n tokens: x [n][dm] (the layer input), g1 [dm][hidden],
+ * c1 [hidden], g2 [hidden][n_out], c2 [n_out] -> out [n][n_out] (n_out =
+ * 3 h_q, column 3h + c = branch c of head h).
+ */
+int vnsa_oracle_gate_mlp(int n, int dm, int hidden, int n_out, const float *x, const float *g1,
+                         const float *c1, const float *g2, const float *c2,
+                         int round_hidden_bf16, double *out)
+{
+    if (n < 0 || dm < 1 || hidden < 1 || n_out < 1 || !x || !g1 || !c1 || !g2 || !c2 || !out)
+        return ORACLE_EINVAL;
+    int fail = 0;
+    #pragma omp parallel
+    {
+        double *h = malloc(sizeof(double) * (size_t)hidden);
+        if (!h) {
+            #pragma omp atomic write
+            fail = 1;
+        }
+        #pragma omp for schedule(static)
+        for (int t = 0; t < n; ++t) {
+            if (!h) continue;
+            const float *xt = x + (size_t)t * dm;
+            for (int a = 0; a < hidden; ++a) {
+                double z = c1[a];
+                for (int e = 0; e < dm; ++e) z += (double)xt[e] * g1[(size_t)e * hidden + a];
+                h[a] = silu(z);
+                if (round_hidden_bf16) h[a] = vnsa_oracle_round_bf16(h[a]);
+            }
+            for (int o = 0; o < n_out; ++o) {
+                double z = c2[o];
+                for (int a = 0; a < hidden; ++a) z += h[a] * g2[(size_t)a * n_out + o];
+                out[(size_t)t * n_out + o] = z;
+            }
+        }
+        free(h);
+    }
+    return fail ? ORACLE_ENOMEM : ORACLE_OK;
 }
 
 /*
@@ -254,13 +421,14 @@ int vnsa_oracle_pool_proj(const vnsa_oracle_cfg *c, const float *k, const float 
  *   imp [n_rows][h_kv][nb]              block importance (0 beyond visibility)
  *   nb_out                              number of complete blocks
  */
-int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k,
+static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k,
                         const float *v, const uint8_t *is_vision, const float *gate,
-                        const float *w_k, const float *w_v, int n_rows, const int *rows,
+                        const float *w_k, const float *w_v, const vnsa_oracle_cmp_mlp *mlp,
+                        int n_rows, const int *rows,
                         const int *forced_idx, double *out, double *o_cmp, double *o_slc,
                         double *o_swa, double *lse_cmp, int *idx, double *imp, int *nb_out)
 {
-    if (!check_cfg(c) || !q || !k || !v || !is_vision || !gate || !w_k || !w_v || !out) return ORACLE_EINVAL;
+    if (!check_cfg(c) || !q || !k || !v || !is_vision || !gate || !out) return ORACLE_EINVAL;
     if (n_rows < 0 || (!rows && n_rows != c->n)) return ORACLE_EINVAL;
     const int n = c->n, d = c->d, hq = c->h_q, hk = c->h_kv, B = c->block, K = c->top_k;
     const int r = hq / hk;
@@ -270,14 +438,12 @@ int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k
     int *vpos = malloc(sizeof(int) * nn);
     double *Kd = malloc(sizeof(double) * nn * hk * d);
     double *Vd = malloc(sizeof(double) * nn * hk * d);
-    double *wk = malloc(sizeof(double) * (size_t)d * d);
-    double *wv = malloc(sizeof(double) * (size_t)d * d);
-    if (!vis || !vpos || !Kd || !Vd || !wk || !wv) {
-        free(vis); free(vpos); free(Kd); free(Vd); free(wk); free(wv);
+    cmp_map mk, mv;
+    if (!vis || !vpos || !Kd || !Vd || !load_cmp_maps(&mk, &mv, d, w_k, w_v, mlp)) {
+        free(vis); free(vpos); free(Kd); free(Vd);
         return ORACLE_ENOMEM;
     }
     for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
-    for (size_t x = 0; x < (size_t)d * d; ++x) { wk[x] = w_k[x]; wv[x] = w_v[x]; }
     const int nv = partition(is_vision, n, vis);
     for (int t = 0; t < n; ++t) vpos[t] = -1;
     for (int i = 0; i < nv; ++i) vpos[vis[i]] = i;
@@ -285,7 +451,7 @@ int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k
     if (nb_out) *nb_out = nb;
     double *k_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
     double *v_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
-    pool_proj(c, Kd, Vd, vis, nb, wk, wv, k_cmp, v_cmp);
+    pool_proj(c, Kd, Vd, vis, nb, &mk, &mv, k_cmp, v_cmp);
 
     #pragma omp parallel
     {
@@ -381,8 +547,32 @@ int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k
         free(keys); free(s); free(p); free(impg); free(taken); free(sel);
         free(qd); free(oc); free(os); free(ow);
     }
-    free(vis); free(vpos); free(Kd); free(Vd); free(wk); free(wv); free(k_cmp); free(v_cmp);
+    free(vis); free(vpos); free(Kd); free(Vd); free(k_cmp); free(v_cmp);
+    free_cmp_map(&mk); free_cmp_map(&mv);
     return ORACLE_OK;
+}
+
+int vnsa_oracle_forward(const vnsa_oracle_cfg *c, const float *q, const float *k,
+                        const float *v, const uint8_t *is_vision, const float *gate,
+                        const float *w_k, const float *w_v, int n_rows, const int *rows,
+                        const int *forced_idx, double *out, double *o_cmp, double *o_slc,
+                        double *o_swa, double *lse_cmp, int *idx, double *imp, int *nb_out)
+{
+    if (!w_k || !w_v) return ORACLE_EINVAL;
+    return forward_impl(c, q, k, v, is_vision, gate, w_k, w_v, NULL, n_rows, rows, forced_idx,
+                        out, o_cmp, o_slc, o_swa, lse_cmp, idx, imp, nb_out);
+}
+
+/* The layer prefill with R11's compression perceptron instead of R3's map. */
+int vnsa_oracle_forward_mlp(const vnsa_oracle_cfg *c, const float *q, const float *k,
+                            const float *v, const uint8_t *is_vision, const float *gate,
+                            const vnsa_oracle_cmp_mlp *mlp, int n_rows, const int *rows,
+                            const int *forced_idx, double *out, double *o_cmp, double *o_slc,
+                            double *o_swa, double *lse_cmp, int *idx, double *imp, int *nb_out)
+{
+    if (!mlp_ok(mlp)) return ORACLE_EINVAL;
+    return forward_impl(c, q, k, v, is_vision, gate, NULL, NULL, mlp, n_rows, rows, forced_idx,
+                        out, o_cmp, o_slc, o_swa, lse_cmp, idx, imp, nb_out);
 }
 
 /* Threads the OpenMP runtime will use (for the CPU-baseline report). */
