@@ -177,6 +177,47 @@ vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k,
                         int32_t *sel_out, void *stream);
 
 /*
+ * The compression branch's "learnable MLP" ("VideoNSA: Native Sparse Attention
+ * Scales Video Understanding", paper notes, section "Method": blocks are
+ * averaged into block keys/values through a learnable MLP), read as a
+ * two-layer perceptron on the block mean that replaces the linear W_K / W_V of
+ * vnsa_create:  K_cmp = SiLU(Kbar . w1_k + b1_k) . w2_k + b2_k, the same for V
+ * with its own weights, shared by the KV heads; SiLU(z) = z / (1 + e^-z).
+ *
+ * hidden: width of the hidden layer, 1..512; 0 returns to the linear maps (the
+ * weight pointers may then be NULL).  w1_* [d][hidden] and w2_* [hidden][d] in
+ * the layer dtype, b1_* [hidden] and b2_* [d] fp32; host or device pointers,
+ * copied into memory the handle owns before the call returns (it
+ * synchronises the device).  The hidden layer is computed in fp32; K_cmp,
+ * V_cmp are rounded once to the layer dtype.  Applies to later vnsa_forward and
+ * vnsa_decode calls (vnsa_select_noalloc keeps the linear maps it is given).
+ * Errors: VNSA_ERR_INVALID_ARG (hidden out of range, a NULL weight, a copy that
+ * failed), VNSA_ERR_CUDA (allocation).
+ */
+vnsa_status vnsa_set_cmp_mlp(vnsa_handle *h, int hidden, const void *w1_k, const float *b1_k,
+                             const void *w2_k, const float *b2_k, const void *w1_v,
+                             const float *b1_v, const void *w2_v, const float *b2_v);
+
+/*
+ * Gate logits from the layer input (same page and section: a two-layer MLP and
+ * a sigmoid give each head its weights for the three branches), read as
+ *   gate_logits[t] = SiLU(x_t . g1 + c1) . g2 + c2,
+ * x [n][d_model] the layer input (h_q * d wide in the pages' model), g1
+ * [d_model][hidden], g2 [hidden][3 h_q] in the layer dtype, c1 [hidden] and c2
+ * [3 h_q] fp32.  Output gate_logits [n][h_q][3] fp32: column 3h + c of token t
+ * is the logit of branch c (cmp, slc, swa) of head h, ready for vnsa_forward
+ * (which applies the sigmoid).  In bf16 the hidden activations are rounded to
+ * bf16 before the second product.  1 <= hidden <= 512; bf16 needs d_model a
+ * multiple of 8.  The tensor-core kernel runs for bf16 with d_model a multiple
+ * of 64, hidden in {64, 128, 192, 256} and 3 h_q <= 256; other settings run a
+ * SIMT kernel.  Device pointers; x, g1, g2 and gate_logits 16-byte aligned.
+ * Asynchronous on `stream`; counts toward vnsa_get_launch_count.
+ */
+vnsa_status vnsa_gate_mlp(vnsa_handle *h, int n, int d_model, int hidden, const void *x,
+                          const void *g1, const float *c1, const void *g2, const float *c2,
+                          float *gate_logits, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device status word.
  * *code receives VNSA_OK or the first device-detected error (TIMEOUT, BOUNDS).
  */

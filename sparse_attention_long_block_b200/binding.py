@@ -24,7 +24,7 @@ NUM_STAGES = 7
 EXPORTED = ("vnsa_status_string", "vnsa_stage_name", "vnsa_workspace_bytes", "vnsa_create",
             "vnsa_forward", "vnsa_forward_host", "vnsa_get_device_status", "vnsa_get_counts",
             "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy",
-            "vnsa_select_noalloc", "vnsa_decode")
+            "vnsa_select_noalloc", "vnsa_decode", "vnsa_set_cmp_mlp", "vnsa_gate_mlp")
 
 
 class vnsa_config(ctypes.Structure):
@@ -71,6 +71,8 @@ def load(path: str = LIB_PATH):
     lib.vnsa_forward.argtypes = [P, I, P, P, P, P, P, P, ctypes.POINTER(vnsa_debug), P]
     lib.vnsa_forward_host.argtypes = [P, I, P, P, P, P, P, P, P]
     lib.vnsa_decode.argtypes = [P, I, P, P, P, P, P, P, P, P]
+    lib.vnsa_set_cmp_mlp.argtypes = [P, I] + [P] * 8
+    lib.vnsa_gate_mlp.argtypes = [P, I, I, I] + [P] * 7
     lib.vnsa_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.vnsa_get_counts.argtypes = [P, P, ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.vnsa_set_timing.argtypes = [P, I]
@@ -124,6 +126,16 @@ def vnsa_forward_host(h, n, q, k, v, is_vision, gate, out, stream=0):
 def vnsa_decode(h, n, q_new, k, v, is_vision, gate_new, out_new, sel_out=None, stream=0):
     _check("vnsa_decode", load().vnsa_decode(h, n, q_new, k, v, is_vision, gate_new, out_new,
                                              sel_out, stream))
+
+
+def vnsa_set_cmp_mlp(h, hidden, w1_k, b1_k, w2_k, b2_k, w1_v, b1_v, w2_v, b2_v):
+    _check("vnsa_set_cmp_mlp", load().vnsa_set_cmp_mlp(h, hidden, w1_k, b1_k, w2_k, b2_k,
+                                                       w1_v, b1_v, w2_v, b2_v))
+
+
+def vnsa_gate_mlp(h, n, d_model, hidden, x, g1, c1, g2, c2, gate_logits, stream=0):
+    _check("vnsa_gate_mlp", load().vnsa_gate_mlp(h, n, d_model, hidden, x, g1, c1, g2, c2,
+                                                 gate_logits, stream))
 
 
 def vnsa_get_device_status(h, stream=0) -> int:
@@ -228,6 +240,45 @@ class Layer:
         vnsa_decode(self.handle, int(n), q_new.data_ptr(), k.data_ptr(), v.data_ptr(),
                     is_vision.data_ptr(), gate_new.data_ptr(), out.data_ptr(),
                     None if sel_out is None else sel_out.data_ptr(), self._stream(stream))
+        return out
+
+    CMP_MLP_KEYS = ("w1_k", "b1_k", "w2_k", "b2_k", "w1_v", "b1_v", "w2_v", "b2_v")
+
+    def set_cmp_mlp(self, mlp=None):
+        """Compression perceptron: a dict with w1_k [d][H], b1_k [H], w2_k
+        [H][d], b2_k [d] and the same for v (weights in the layer dtype, biases
+        fp32), or None for the linear W_K, W_V given at construction."""
+        import torch
+        if mlp is None:
+            vnsa_set_cmp_mlp(self.handle, 0, *([None] * 8))
+            return
+        ts = []
+        for nm in self.CMP_MLP_KEYS:
+            dt = torch.float32 if nm.startswith("b") else self.tdtype
+            ts.append(torch.as_tensor(mlp[nm]).to(device="cuda", dtype=dt).contiguous())
+        hidden = int(ts[1].shape[0])
+        vnsa_set_cmp_mlp(self.handle, hidden, *[t.data_ptr() for t in ts])
+
+    def gate_mlp(self, x, g1, c1, g2, c2, out=None, stream=None):
+        """Gate logits [n][h_q][3] fp32 of the layer input x [n][D] through the
+        gate perceptron (g1 [D][H], g2 [H][3 h_q] in the layer dtype, c1, c2
+        fp32); all contiguous CUDA tensors."""
+        import torch
+        for t in (x, g1, c1, g2, c2):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("inputs must be contiguous CUDA tensors")
+        if x.dtype != self.tdtype or g1.dtype != self.tdtype or g2.dtype != self.tdtype:
+            raise ValueError("x, g1, g2 must match the layer dtype")
+        if c1.dtype != torch.float32 or c2.dtype != torch.float32:
+            raise ValueError("c1, c2 must be float32")
+        n, dm = int(x.shape[0]), int(x.shape[1])
+        hidden = int(c1.shape[0])
+        if tuple(g1.shape) != (dm, hidden) or tuple(g2.shape) != (hidden, 3 * self.h_q):
+            raise ValueError("g1 must be [D][H] and g2 [H][3 h_q]")
+        if out is None:
+            out = torch.empty((n, self.h_q, 3), dtype=torch.float32, device=x.device)
+        vnsa_gate_mlp(self.handle, n, dm, hidden, x.data_ptr(), g1.data_ptr(), c1.data_ptr(),
+                      g2.data_ptr(), c2.data_ptr(), out.data_ptr(), self._stream(stream))
         return out
 
     def forward_host(self, q, k, v, is_vision, gate, out, stream=None):

@@ -444,7 +444,7 @@ cudaError_t launch_decode(int dtype, const DecodeParams &p, cudaStream_t s, int 
     decode_prep_kernel<<<1, 32, 0, s>>>(p);
     ++*launches;
     cudaError_t e = launch_pool_proj(dtype, p.d, p.k, p.v, p.vis, p.counts, p.w_k, p.w_v,
-                                     p.k_cmp, p.v_cmp, p.h_kv, p.block, p.nb_max, s, 1);
+                                     p.k_cmp, p.v_cmp, p.h_kv, p.block, p.nb_max, s, 1, &p.mlp);
     ++*launches;
     if (e != cudaSuccess) return e;
     if (dtype == VNSA_BF16 && p.d == 128) return launch_r<__nv_bfloat16, 128>(p, s, launches);

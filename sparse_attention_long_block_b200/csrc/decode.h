@@ -21,6 +21,7 @@ struct DecodeParams {
     uint32_t *status;
     void *k_cmp, *v_cmp;          // [nb_max][h_kv][d] block keys/values (extended)
     const void *w_k, *w_v;        // [d][d] projections
+    CmpMlp mlp;                   // compression perceptron (hidden 0: the projections)
     float *s_cmp;                 // [h_kv][r][nb_max] compression scores (log2 units)
     float *part;                  // [3][h_kv][kSplit][r][d + 2] split softmax states
     int32_t *sel;                 // [h_kv][top_k] the selection

@@ -35,11 +35,30 @@ struct LayerParams {
 cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t *vis,
                              int32_t *txt, Counts *counts, cudaStream_t s);
 
+// The compression branch's perceptron (when hidden > 0): K_cmp = SiLU(mean .
+// w1 + b1) . w2 + b2, w1 [d][hidden], w2 [hidden][d] in the layer dtype, b1, b2
+// fp32; index 0 for K, 1 for V.  hidden == 0: the linear projection W_K, W_V.
+constexpr int kCmpMlpMaxHidden = 512;
+struct CmpMlp {
+    int hidden;
+    const void *w1[2], *w2[2];
+    const float *b1[2], *b2[2];
+};
+
 // K_cmp / V_cmp: dtype 0 = bf16, 1 = fp32.
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s, int from_pad = 0);
+                             int nb_max, cudaStream_t s, int from_pad = 0,
+                             const CmpMlp *mlp = nullptr);
+
+// Gate logits [n][n_out] fp32 of the layer input x [n][dm] through the gate
+// perceptron SiLU(x . g1 + c1) . g2 + c2 (g1 [dm][hidden], g2 [hidden][n_out]
+// in the layer dtype, c1, c2 fp32); in bf16 the hidden activations are rounded
+// to bf16.  `status` receives device-detected errors.
+cudaError_t launch_gate_mlp(int dtype, int n, int dm, int hidden, int n_out, const void *x,
+                            const void *g1, const float *c1, const void *g2, const float *c2,
+                            float *out, uint32_t *status, cudaStream_t s, int *launches);
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s);
 

@@ -172,12 +172,109 @@ __global__ void __launch_bounds__(256) pool_proj_kernel(
     }
 }
 
+// The compression branch's "learnable MLP" ("VideoNSA: Native Sparse Attention
+// Scales Video Understanding", section "Method"), read as a two-layer
+// perceptron with SiLU on the block mean: the same CTA tiling and mean as
+// pool_proj_kernel, then hidden = SiLU(mean . w1 + b1) in fp32 shared memory and
+// K_cmp = hidden . w2 + b2, rounded once to the storage type.
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) pool_mlp_kernel(
+    const T *__restrict__ k, const T *__restrict__ v, const int32_t *__restrict__ vis,
+    const Counts *__restrict__ counts, CmpMlp mlp, T *__restrict__ k_cmp,
+    T *__restrict__ v_cmp, int h_kv, int block, int from_pad) {
+    constexpr int JB = 16;
+    constexpr int PER = D / 32;
+    constexpr int NPART = 256 / D;
+    constexpr int JBP = JB / NPART;
+    __shared__ float mean[JB][D];
+    __shared__ float hid[JB][kCmpMlpMaxHidden];
+    const int nb = counts->nb;
+    const int j0 = (from_pad ? counts->pad[0] : 0) + blockIdx.x * JB;
+    if (j0 >= nb) return;
+    const int g = blockIdx.y;
+    const int z = blockIdx.z;
+    const T *src = z ? v : k;
+    const T *W1 = (const T *)mlp.w1[z];
+    const T *W2 = (const T *)mlp.w2[z];
+    const float *B1 = mlp.b1[z];
+    const float *B2 = mlp.b2[z];
+    const int H = mlp.hidden;
+    T *dst = z ? v_cmp : k_cmp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float inv = 1.0f / (float)block;
+    for (int jb = warp; jb < JB; jb += 8) {
+        const int j = j0 + jb;
+        float acc[PER];
+#pragma unroll
+        for (int c = 0; c < PER; ++c) acc[c] = 0.f;
+        if (j < nb) {
+            const int32_t *rows = vis + (size_t)j * block;
+#pragma unroll 8
+            for (int u = 0; u < block; ++u) {
+                const T *p = src + ((size_t)rows[u] * h_kv + g) * D + lane * PER;
+                float x[PER];
+                load_row_part<T, PER>(p, x);
+#pragma unroll
+                for (int c = 0; c < PER; ++c) acc[c] += x[c];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < PER; ++c) mean[jb][lane * PER + c] = acc[c] * inv;
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < H; x += 256) {
+        float a[JB];
+        const float b = B1[x];
+#pragma unroll
+        for (int jb = 0; jb < JB; ++jb) a[jb] = b;
+        for (int e = 0; e < D; ++e) {
+            const float w = to_f(W1[(size_t)e * H + x]);
+#pragma unroll
+            for (int jb = 0; jb < JB; ++jb) a[jb] = fmaf(mean[jb][e], w, a[jb]);
+        }
+#pragma unroll
+        for (int jb = 0; jb < JB; ++jb) hid[jb][x] = silu_f(a[jb]);
+    }
+    __syncthreads();
+    const int col = threadIdx.x % D, part = threadIdx.x / D;
+    float o[JBP];
+    const float b2 = B2[col];
+#pragma unroll
+    for (int x = 0; x < JBP; ++x) o[x] = b2;
+    for (int e = 0; e < H; ++e) {
+        const float w = to_f(W2[(size_t)e * D + col]);
+#pragma unroll
+        for (int x = 0; x < JBP; ++x) o[x] = fmaf(hid[part * JBP + x][e], w, o[x]);
+    }
+#pragma unroll
+    for (int x = 0; x < JBP; ++x) {
+        const int j = j0 + part * JBP + x;
+        if (j < nb) dst[((size_t)j * h_kv + g) * D + col] = from_f<T>(o[x]);
+    }
+}
+
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s, int from_pad) {
+                             int nb_max, cudaStream_t s, int from_pad, const CmpMlp *mlp) {
     if (nb_max <= 0) return cudaSuccess;
     dim3 grid(from_pad ? 1 : (nb_max + 15) / 16, h_kv, 2);
+    if (mlp && mlp->hidden > 0) {
+        if (mlp->hidden > kCmpMlpMaxHidden) return cudaErrorInvalidValue;
+#define VNSA_POOL_MLP(T, D)                                                              \
+    pool_mlp_kernel<T, D><<<grid, 256, 0, s>>>((const T *)k, (const T *)v, vis, counts,  \
+                                               *mlp, (T *)k_cmp, (T *)v_cmp, h_kv, block, \
+                                               from_pad)
+        if (dtype == VNSA_BF16 && d == 128) VNSA_POOL_MLP(__nv_bfloat16, 128);
+        else if (dtype == VNSA_BF16 && d == 64) VNSA_POOL_MLP(__nv_bfloat16, 64);
+        else if (dtype == VNSA_FP32 && d == 128) VNSA_POOL_MLP(float, 128);
+        else if (dtype == VNSA_FP32 && d == 64) VNSA_POOL_MLP(float, 64);
+        else return cudaErrorInvalidValue;
+#undef VNSA_POOL_MLP
+        return cudaGetLastError();
+    }
 #define VNSA_POOL(T, D)                                                                  \
     pool_proj_kernel<T, D><<<grid, 256, 0, s>>>(                                         \
         (const T *)k, (const T *)v, vis, counts, (const T *)w_k, (const T *)w_v,         \

@@ -1274,6 +1274,19 @@ size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
+bool tma_map_2d_bf16(CUtensorMap *m, const void *base, long long inner, long long rows,
+                     int box_inner, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || inner < 1 || rows < 1) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct TcState {
     vnsa_config cfg;
     int num_sms;

@@ -2,6 +2,8 @@
 // layer prefill, behind the C ABI of vnsa_api.cu.
 #pragma once
 
+#include <cuda.h>
+
 #include "kernels.h"
 
 namespace vnsa {
@@ -24,5 +26,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &p, cudaStream_t s, cudaEv
                        int *ran, int *launches, bool forced);
 
 void tc_destroy(TcState *st);
+
+// 2-D TMA map over a row-major bf16 matrix [rows][inner] (row stride inner * 2
+// bytes, a multiple of 16) with boxes of box_inner x box_rows elements and the
+// 128-byte swizzle (box_inner * 2 must be 128).  False if the driver entry
+// point is missing or the encoding fails.
+bool tma_map_2d_bf16(CUtensorMap *m, const void *base, long long inner, long long rows,
+                     int box_inner, int box_rows);
 
 }  // namespace vnsa

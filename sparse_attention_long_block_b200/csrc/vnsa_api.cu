@@ -97,6 +97,8 @@ struct vnsa_handle {
     cudaEvent_t ev[2 * VNSA_NUM_STAGES];
     int ran[VNSA_NUM_STAGES];
     int launches;
+    CmpMlp mlp;     // compression perceptron (hidden 0: the linear W_K, W_V)
+    char *mlp_mem;  // its weights (owned)
 };
 
 extern "C" {
@@ -262,7 +264,7 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     begin(VNSA_STAGE_POOL);
     VNSA_RUN(launch_pool_proj(dt, c.d, k, v, p.vis, h->counts, h->ws + h->L.w_k,
                               h->ws + h->L.w_v, (void *)p.k_cmp, (void *)p.v_cmp, c.h_kv,
-                              c.block, h->nb_max, s));
+                              c.block, h->nb_max, s, 0, &h->mlp));
     end(VNSA_STAGE_POOL);
     if (use_tc) {
         // counts its own launches
@@ -339,6 +341,7 @@ vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k,
     p.v_cmp = h->ws + h->L.v_cmp;
     p.w_k = h->ws + h->L.w_k;
     p.w_v = h->ws + h->L.w_v;
+    p.mlp = h->mlp;
     char *dec = h->ws + h->L.dec;
     p.s_cmp = (float *)dec;
     p.part = (float *)(dec + (size_t)c.h_kv * h->r * (h->nb_max > 0 ? h->nb_max : 1) * 4);
@@ -458,6 +461,91 @@ vnsa_status vnsa_get_launch_count(vnsa_handle *h, int *launches) {
     return VNSA_OK;
 }
 
+vnsa_status vnsa_set_cmp_mlp(vnsa_handle *h, int hidden, const void *w1_k, const float *b1_k,
+                             const void *w2_k, const float *b2_k, const void *w1_v,
+                             const float *b1_v, const void *w2_v, const float *b2_v) {
+    if (!h || hidden < 0 || hidden > kCmpMlpMaxHidden) return VNSA_ERR_INVALID_ARG;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return VNSA_ERR_CUDA;
+    vnsa_status rc = VNSA_OK;
+    if (hidden == 0) {
+        // back to the linear projections given at create
+        cudaDeviceSynchronize();
+        if (h->mlp_mem) cudaFree(h->mlp_mem);
+        h->mlp_mem = nullptr;
+        memset(&h->mlp, 0, sizeof(h->mlp));
+    } else if (!w1_k || !b1_k || !w2_k || !b2_k || !w1_v || !b1_v || !w2_v || !b2_v) {
+        rc = VNSA_ERR_INVALID_ARG;
+    } else {
+        const size_t d = (size_t)h->cfg.d, H = (size_t)hidden;
+        const size_t wb = d * H * h->esize;  // each of w1, w2
+        const size_t sizes[4] = {wb, H * 4, wb, d * 4};
+        size_t total = 0;
+        for (int t = 0; t < 2; ++t)
+            for (int x = 0; x < 4; ++x) total += (sizes[x] + 255) / 256 * 256;
+        char *mem = nullptr;
+        if (cudaMalloc(&mem, total) != cudaSuccess) {
+            cudaGetLastError();
+            rc = VNSA_ERR_CUDA;
+        } else {
+            const void *src[2][4] = {{w1_k, b1_k, w2_k, b2_k}, {w1_v, b1_v, w2_v, b2_v}};
+            void *dst[2][4];
+            size_t off = 0;
+            bool ok = true;
+            for (int t = 0; t < 2; ++t)
+                for (int x = 0; x < 4; ++x) {
+                    dst[t][x] = mem + off;
+                    off += (sizes[x] + 255) / 256 * 256;
+                    ok = ok && cudaMemcpy(dst[t][x], src[t][x], sizes[x], cudaMemcpyDefault) ==
+                                   cudaSuccess;
+                }
+            if (!ok) {
+                cudaGetLastError();
+                cudaFree(mem);
+                rc = VNSA_ERR_INVALID_ARG;
+            } else {
+                cudaDeviceSynchronize();
+                if (h->mlp_mem) cudaFree(h->mlp_mem);
+                h->mlp_mem = mem;
+                h->mlp.hidden = hidden;
+                for (int t = 0; t < 2; ++t) {
+                    h->mlp.w1[t] = dst[t][0];
+                    h->mlp.b1[t] = (const float *)dst[t][1];
+                    h->mlp.w2[t] = dst[t][2];
+                    h->mlp.b2[t] = (const float *)dst[t][3];
+                }
+            }
+        }
+    }
+    if (cur != h->device && cur >= 0) cudaSetDevice(cur);
+    return rc;
+}
+
+vnsa_status vnsa_gate_mlp(vnsa_handle *h, int n, int d_model, int hidden, const void *x,
+                          const void *g1, const float *c1, const void *g2, const float *c2,
+                          float *gate_logits, void *stream) {
+    if (!h || !x || !g1 || !c1 || !g2 || !c2 || !gate_logits) return VNSA_ERR_INVALID_ARG;
+    if (n < 1 || d_model < 1 || hidden < 1 || hidden > kCmpMlpMaxHidden)
+        return VNSA_ERR_INVALID_ARG;
+    if (h->cfg.dtype == VNSA_BF16 && d_model % 8 != 0) return VNSA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(g1) || !aligned16(g2) || !aligned16(gate_logits))
+        return VNSA_ERR_INVALID_ARG;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return VNSA_ERR_CUDA;
+    h->launches = 0;
+    cudaError_t e = launch_gate_mlp((int)h->cfg.dtype, n, d_model, hidden, 3 * h->cfg.h_q, x, g1,
+                                    c1, g2, c2, gate_logits, h->status, (cudaStream_t)stream,
+                                    &h->launches);
+    if (cur != h->device && cur >= 0) cudaSetDevice(cur);
+    if (e != cudaSuccess) {
+        fprintf(stderr, "vnsa_gate_mlp: %s\n", cudaGetErrorString(e));
+        return VNSA_ERR_CUDA;
+    }
+    return VNSA_OK;
+}
+
 vnsa_status vnsa_destroy(vnsa_handle *h) {
     if (!h) return VNSA_ERR_INVALID_ARG;
     cudaDeviceSynchronize();
@@ -465,6 +553,7 @@ vnsa_status vnsa_destroy(vnsa_handle *h) {
     for (int e = 0; e < 2 * VNSA_NUM_STAGES; ++e)
         if (h->ev[e]) cudaEventDestroy(h->ev[e]);
     if (h->stage) cudaFree(h->stage);
+    if (h->mlp_mem) cudaFree(h->mlp_mem);
     if (h->ws) cudaFree(h->ws);
     cudaGetLastError();
     delete h;

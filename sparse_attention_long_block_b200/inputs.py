@@ -165,6 +165,42 @@ def generate(wl: Workload, is_vision: np.ndarray | None = None) -> dict:
                 gate=gate, w_k=w_k, w_v=w_v)
 
 
+def cmp_mlp_weights(wl: Workload, hidden: int, seed: int = 100) -> dict:
+    """Random weights of the compression perceptron (hidden width `hidden`):
+    w1_k, w1_v [d][H] ~ N(0, 1/d), w2_k, w2_v [H][d] ~ N(0, 1/H) (rounded to
+    bf16 for bf16 workloads), biases b1 ~ N(0, 0.01), b2 ~ N(0, 0.01) in fp32."""
+    rng = np.random.default_rng(seed)
+    d = wl.d
+    out = {}
+    for t in ("k", "v"):
+        w1 = rng.standard_normal((d, hidden), dtype=np.float32) * np.float32(1 / np.sqrt(d))
+        b1 = rng.standard_normal(hidden, dtype=np.float32) * np.float32(0.1)
+        w2 = rng.standard_normal((hidden, d), dtype=np.float32) * np.float32(1 / np.sqrt(hidden))
+        b2 = rng.standard_normal(d, dtype=np.float32) * np.float32(0.1)
+        if wl.dtype == "bf16":
+            w1, w2 = bf16_round(w1), bf16_round(w2)
+        out.update({"w1_" + t: w1, "b1_" + t: b1, "w2_" + t: w2, "b2_" + t: b2})
+    return out
+
+
+def gate_mlp_inputs(wl: Workload, d_model: int, hidden: int, n: int | None = None,
+                    seed: int = 200) -> dict:
+    """Layer input and gate-perceptron weights: x [n][d_model] ~ N(0, 1) (a
+    normalised hidden state), g1 [d_model][H] ~ N(0, 1/d_model), c1 [H] ~
+    N(0, 0.01), g2 [H][3 h_q] ~ N(0, 1/H), c2 [3 h_q] ~ N(0, 1); x, g1, g2
+    rounded to bf16 for bf16 workloads."""
+    rng = np.random.default_rng(seed)
+    n = wl.n if n is None else n
+    x = rng.standard_normal((n, d_model), dtype=np.float32)
+    g1 = rng.standard_normal((d_model, hidden), dtype=np.float32) * np.float32(1 / np.sqrt(d_model))
+    c1 = rng.standard_normal(hidden, dtype=np.float32) * np.float32(0.1)
+    g2 = rng.standard_normal((hidden, 3 * wl.h_q), dtype=np.float32) * np.float32(1 / np.sqrt(hidden))
+    c2 = rng.standard_normal(3 * wl.h_q, dtype=np.float32)
+    if wl.dtype == "bf16":
+        x, g1, g2 = bf16_round(x), bf16_round(g1), bf16_round(g2)
+    return dict(x=x, g1=g1, c1=c1, g2=g2, c2=c2)
+
+
 def interleaved_mask(n_vision: int, n_text: int, seed: int = 1,
                      text_runs: int = 4) -> np.ndarray:
     """A vision/text mask with the text split into runs placed between vision

@@ -48,10 +48,11 @@ def stratified_rows(is_vision: np.ndarray, block: int = 64, every: int = 97,
     return np.array(sorted(rows), dtype=np.int32)
 
 
-def run_gpu(wl: Workload, x: dict, want=(), forced_idx=None, ranks=None):
+def run_gpu(wl: Workload, x: dict, want=(), forced_idx=None, ranks=None, cmp_mlp=None):
     """Run the CUDA layer through the C ABI; returns numpy results.  With
     `ranks`, the per-vision-rank exports (idx, imp) are cut to those ranks on
-    the device before the copy to the host."""
+    the device before the copy to the host; with `cmp_mlp` (weights dict) the
+    compression branch uses that perceptron."""
     import torch
     from sparse_attention_long_block_b200 import binding
     td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -64,6 +65,8 @@ def run_gpu(wl: Workload, x: dict, want=(), forced_idx=None, ranks=None):
     layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
                           top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+    if cmp_mlp is not None:
+        layer.set_cmp_mlp({nm: torch.from_numpy(a) for nm, a in cmp_mlp.items()})
     fidx = None
     if forced_idx is not None:
         fidx = torch.from_numpy(np.ascontiguousarray(forced_idx, np.int32)).to(dev)
@@ -120,9 +123,11 @@ def check_selection(gpu_idx_rows, ora_idx, ora_imp, top_k, force_first=True,
     return sorted(set(swapped))
 
 
-def compare_layer(wl: Workload, x: dict, rows=None, want_branches=True, check_imp=True):
+def compare_layer(wl: Workload, x: dict, rows=None, want_branches=True, check_imp=True,
+                  cmp_mlp=None):
     """Full comparison of the CUDA layer with the oracle on `rows` (all if
-    None).  Returns a dict of error statistics."""
+    None), optionally with a compression perceptron.  Returns a dict of error
+    statistics."""
     p = oracle_params(wl)
     want = ("idx", "imp") + (("o_cmp", "o_slc", "o_swa") if want_branches else ())
     isv = x["is_vision"]
@@ -134,12 +139,13 @@ def compare_layer(wl: Workload, x: dict, rows=None, want_branches=True, check_im
     ranks = rank_of[rows]
     is_v = ranks >= 0
     vr = ranks[is_v]
-    g = run_gpu(wl, x, want=want + (("lse_cmp",) if want_branches else ()), ranks=vr)
+    g = run_gpu(wl, x, want=want + (("lse_cmp",) if want_branches else ()), ranks=vr,
+                cmp_mlp=cmp_mlp)
     assert g["status"] == 0, f"device status {g['status']}"
     nv_gpu, nt_gpu = g["counts"]
     assert nv_gpu == int(isv.sum()) and nt_gpu == len(isv) - int(isv.sum())
     o = oracle.forward(p, x["q"], x["k"], x["v"], isv, x["gate"], x["w_k"], x["w_v"],
-                       rows=rows, want=want + ("lse_cmp",))
+                       rows=rows, want=want + ("lse_cmp",), cmp_mlp=cmp_mlp)
     tol = TOL[wl.dtype]
     stats = {}
     # selection sets (g["idx"], g["imp"] are already cut to the ranks vr)
@@ -162,7 +168,7 @@ def compare_layer(wl: Workload, x: dict, rows=None, want_branches=True, check_im
         sub = np.nonzero(is_v)[0][swapped_local]
         fidx = np.transpose(g["idx"][:, swapped_local, :], (1, 0, 2))
         o2 = oracle.forward(p, x["q"], x["k"], x["v"], isv, x["gate"], x["w_k"], x["w_v"],
-                            rows=rows[sub], forced_idx=fidx, want=("o_slc",))
+                            rows=rows[sub], forced_idx=fidx, want=("o_slc",), cmp_mlp=cmp_mlp)
         ref_out[sub] = o2["out"]
         if "o_slc" in o:
             o["o_slc"][sub] = o2["o_slc"]
@@ -188,10 +194,11 @@ def compare_layer(wl: Workload, x: dict, rows=None, want_branches=True, check_im
     return stats
 
 
-def compare_pool(wl: Workload, x: dict):
+def compare_pool(wl: Workload, x: dict, cmp_mlp=None):
     p = oracle_params(wl)
-    kc, vc = oracle.pool_proj(p, x["k"], x["v"], x["is_vision"], x["w_k"], x["w_v"])
-    g = run_gpu(wl, x, want=("k_cmp", "v_cmp"))
+    kc, vc = oracle.pool_proj(p, x["k"], x["v"], x["is_vision"], x["w_k"], x["w_v"],
+                              cmp_mlp=cmp_mlp)
+    g = run_gpu(wl, x, want=("k_cmp", "v_cmp"), cmp_mlp=cmp_mlp)
     nb = kc.shape[0]
     out = {}
     vis = np.nonzero(x["is_vision"])[0][: nb * wl.block]
@@ -205,7 +212,22 @@ def compare_pool(wl: Workload, x: dict):
             # can exceed that ulp of the (small) exact value; the bf16 rounding of
             # the fp32 result then adds one more ulp.
             mabs = np.abs(src[vis].astype(np.float64)).reshape(nb, wl.block, wl.h_kv, wl.d).mean(1)
-            acc = (wl.block + wl.d) * 2.0 ** -24 * (mabs @ np.abs(w.astype(np.float64)))
+            if cmp_mlp is None:
+                acc = (wl.block + wl.d) * 2.0 ** -24 * (mabs @ np.abs(w.astype(np.float64)))
+            else:
+                # perceptron: |SiLU(z)| <= |z| and |SiLU'| <= 1.1 bound the hidden
+                # layer by A1 = mean|x|.|W1| + |b1| and its fp32 error (sum, product,
+                # exp) by (1.1 (B + d) 2^-24 + 2^-22) A1; the second product adds
+                # (H + 1) 2^-24 (A1.|W2| + |b2|)
+                t = name[0]
+                w1 = np.abs(cmp_mlp["w1_" + t].astype(np.float64))
+                w2 = np.abs(cmp_mlp["w2_" + t].astype(np.float64))
+                b1 = np.abs(cmp_mlp["b1_" + t].astype(np.float64))
+                b2 = np.abs(cmp_mlp["b2_" + t].astype(np.float64))
+                hid = w1.shape[1]
+                a1 = mabs @ w1 + b1
+                e_h = (1.1 * (wl.block + wl.d) * 2.0 ** -24 + 2.0 ** -22) * a1
+                acc = e_h @ w2 + (hid + 1) * 2.0 ** -24 * (a1 @ w2 + b2)
             ulp = np.maximum(np.abs(ref), 1e-30) * 2.0 ** -7 + acc * (1 + 2.0 ** -7)
             bad = np.abs(got - ref) > ulp
             out[name + "_ulp_flips"] = int((got != ref).sum())

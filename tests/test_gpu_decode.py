@@ -29,7 +29,7 @@ def _stream_mask(n_vision, n_text_head, tail):
     return np.array(mask, np.uint8)
 
 
-def _run_decode(wl: Workload, x: dict, n0: int):
+def _run_decode(wl: Workload, x: dict, n0: int, cmp_mlp=None):
     import torch
     from sparse_attention_long_block_b200 import binding
     td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -42,6 +42,8 @@ def _run_decode(wl: Workload, x: dict, n0: int):
     layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
                           top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+    if cmp_mlp is not None:
+        layer.set_cmp_mlp({nm: torch.from_numpy(a) for nm, a in cmp_mlp.items()})
     layer.forward(q[:n0].contiguous(), k[:n0].contiguous(), v[:n0].contiguous(),
                   isv[:n0].contiguous(), gate[:n0].contiguous())
     outs, sels = [], []
@@ -59,15 +61,15 @@ def _run_decode(wl: Workload, x: dict, n0: int):
     return out, sel, status, (nv, nt)
 
 
-def _compare(wl: Workload, x: dict, n0: int):
-    out, sel, status, counts = _run_decode(wl, x, n0)
+def _compare(wl: Workload, x: dict, n0: int, cmp_mlp=None):
+    out, sel, status, counts = _run_decode(wl, x, n0, cmp_mlp)
     assert status == 0
     isv = x["is_vision"]
     assert counts == (int(isv.sum()), wl.n - int(isv.sum()))
     rows = np.arange(n0, wl.n, dtype=np.int32)
     p = oracle_params(wl)
     o = oracle.forward(p, x["q"], x["k"], x["v"], isv, x["gate"], x["w_k"], x["w_v"],
-                       rows=rows, want=("idx", "imp"))
+                       rows=rows, want=("idx", "imp"), cmp_mlp=cmp_mlp)
     ref = o["out"].copy()
     is_v = isv[rows] != 0
     if is_v.any():
@@ -81,7 +83,7 @@ def _compare(wl: Workload, x: dict, n0: int):
             sub = np.nonzero(is_v)[0][swapped]
             fidx = sel[sub]
             o2 = oracle.forward(p, x["q"], x["k"], x["v"], isv, x["gate"], x["w_k"], x["w_v"],
-                                rows=rows[sub], forced_idx=fidx)
+                                rows=rows[sub], forced_idx=fidx, cmp_mlp=cmp_mlp)
             ref[sub] = o2["out"]
     # a text step exports no selection
     assert (sel[~is_v] == -1).all()
