@@ -26,7 +26,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_attention_long_block_b200.inputs import WORKLOADS, generate  # noqa: E402
+from sparse_attention_long_block_b200.inputs import (WORKLOADS, cmp_mlp_weights,  # noqa: E402
+                                                     gate_mlp_inputs, generate)
 
 METRIC = "layer_prefill_tokens_per_s"
 UNIT = "tokens/s"
@@ -301,6 +302,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=96)
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    ap.add_argument("--mlp", action="store_true",
+                    help="each step also computes the gate logits from the layer input "
+                         "through the gate perceptron, and compression uses its perceptron")
+    ap.add_argument("--gate-hidden", type=int, default=256)
+    ap.add_argument("--cmp-hidden", type=int, default=128)
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -340,8 +346,24 @@ def main():
                           top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
                           w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
     stream = torch.cuda.current_stream()
+    gm = None
+    if args.mlp:
+        # the perceptrons: gate logits from the layer input x [n][h_q d] each
+        # step (into the gate buffer the layer reads), compression through its
+        # perceptron
+        gi = gate_mlp_inputs(wl, wl.h_q * wl.d, args.gate_hidden, seed=200 + rank)
+        gm = {kk: torch.from_numpy(vv).to(dev, td if kk in ("x", "g1", "g2") else torch.float32)
+              for kk, vv in gi.items()}
+        del gi
+        layer.set_cmp_mlp({kk: torch.from_numpy(vv)
+                           for kk, vv in cmp_mlp_weights(wl, args.cmp_hidden).items()})
+
+    def gate_step():
+        layer.gate_mlp(gm["x"], gm["g1"], gm["c1"], gm["g2"], gm["c2"], out=gate, stream=stream)
 
     def step():
+        if gm is not None:
+            gate_step()
         layer.forward(q, k, v, isv, gate, out=out, stream=stream)
 
     def barrier():
@@ -354,6 +376,10 @@ def main():
     if layer.device_status() != 0:
         raise SystemExit("device status error during warm-up")
     launches_per_step = layer.launches()
+    if gm is not None:
+        gate_step()
+        torch.cuda.synchronize()
+        launches_per_step += layer.launches()
 
     sampler = ClockSampler(smi_index(local_rank)) if rank == 0 else None
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -396,9 +422,33 @@ def main():
         executed = executed_work(wl, x["is_vision"], tens["idx"][:, :nvis].cpu().numpy())
         del tens
 
+    # the gate perceptron alone (same stream, after warm-up), for its roofline
+    gate_mlp = None
+    if gm is not None:
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(args.steps):
+            gate_step()
+        gb.record(stream)
+        gb.synchronize()
+        g_ms = ga.elapsed_time(gb) / max(args.steps, 1)
+        dm, hid, n_out = wl.h_q * wl.d, args.gate_hidden, 3 * wl.h_q
+        es = 2 if wl.dtype == "bf16" else 4
+        g_bytes = wl.n * dm * es + (dm * hid + hid * n_out) * es + wl.n * n_out * 4
+        g_flops = 2.0 * wl.n * (dm * hid + hid * n_out)
+        pk = load_peaks()
+        gate_mlp = {"ms": g_ms, "d_model": dm, "hidden": hid, "bytes": g_bytes,
+                    "flops": g_flops,
+                    "hbm_gbs": g_bytes / (g_ms * 1e-3) / 1e9,
+                    "hbm_frac": g_bytes / (g_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                    "tflops": g_flops / (g_ms * 1e-3) / 1e12,
+                    "tensor_frac": g_flops / (g_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                    "bound": ("hbm" if g_bytes / pk["hbm_gbs"] / 1e9 >
+                              g_flops / pk["bf16_tflops"] / 1e12 else "tensor")}
+
     # end to end through the C ABI with host buffers (pinned)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and gm is None:
         hq = torch.from_numpy(x["q"]).to(td).pin_memory()
         hk = torch.from_numpy(x["k"]).to(td).pin_memory()
         hv = torch.from_numpy(x["v"]).to(td).pin_memory()
@@ -469,7 +519,11 @@ def main():
                        "block": wl.block, "top_k": wl.top_k, "window": wl.window,
                        "attention": "dense (all tokens text)" if wl.dense else "hybrid",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (no flush)"},
+                       "l2": "inputs larger than L2 (no flush)",
+                       "perceptrons": None if gm is None else {
+                           "gate": f"x [{wl.n}][{wl.h_q * wl.d}] -> {args.gate_hidden} -> "
+                                   f"{3 * wl.h_q} logits, every step",
+                           "compression_hidden": args.cmp_hidden}},
             "tensor_peak_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "executed": None if executed is None else {
                 "tflop": {kk: vv / 1e12 for kk, vv in executed.items()},
@@ -482,6 +536,7 @@ def main():
             "pool_hbm": {"achieved_gbs": pool_gbs, "peak_gbs": peaks["hbm_gbs"],
                          "frac": pool_gbs / peaks["hbm_gbs"]},
             "roofline": roofline,
+            "gate_mlp": gate_mlp,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
