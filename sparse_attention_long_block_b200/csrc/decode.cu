@@ -15,9 +15,9 @@
 //   1. decode_prep:   appends the token to its list (one thread);
 //   2. pool:          K_cmp / V_cmp of the block the token completes, if any;
 //   3. decode_cmp:    compression scores and split partial softmax states;
-//   4. decode_select: the compression output, the group importance and top-k;
+//   4. decode_select: the group importance and top-k;
 //   5. decode_attn:   selection + window (vision) or dense (text) partials;
-//   6. decode_combine: the partials, the gates and the output row.
+//   6. decode_combine: the three branches' partials, the gates and the output row.
 // Every kernel spreads its keys over kSplit CTAs per KV group (split-K); the
 // query's group heads are processed together so every K/V row is read once.
 #include <math.h>
@@ -29,7 +29,8 @@ namespace vnsa {
 
 namespace {
 
-constexpr int kWarps = 4;  // warps per CTA of the split kernels
+constexpr int kWarps = 8;  // warps per CTA of the split kernels
+constexpr int kBatch = 4;  // keys a warp loads before it computes (loads in flight)
 
 // Row pieces: lane owns elements [lane * PER, lane * PER + PER) of a d-row.
 template <typename T, int PER>
@@ -94,16 +95,55 @@ struct Acc {
 #pragma unroll
         for (int e = 0; e < PER; ++e) o[e] = 0.f;
     }
-    __device__ void add(float s, const float (&v)[PER]) {
-        const float mn = fmaxf(m, s);
-        const float corr = exp2f(m - mn);  // 0 when m = -inf
-        const float p = exp2f(s - mn);
-        l = l * corr + p;
+    // U keys at once (scores s, log2 units; -inf for a key to skip): one
+    // rescale of the state per batch
+    template <int U>
+    __device__ void add_batch(const float (&s)[U], const float (&v)[U][PER]) {
+        float mx = m;
 #pragma unroll
-        for (int e = 0; e < PER; ++e) o[e] = o[e] * corr + p * v[e];
-        m = mn;
+        for (int u = 0; u < U; ++u) mx = fmaxf(mx, s[u]);
+        if (mx == -INFINITY) return;  // no key so far and none in this batch
+        const float corr = exp2f(m - mx);  // 0 when m = -inf
+        l *= corr;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] *= corr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float pu = exp2f(s[u] - mx);  // 0 for a skipped key
+            l += pu;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[e] = fmaf(pu, v[u][e], o[e]);
+        }
+        m = mx;
     }
 };
+
+// Scores (log2 units) of R heads against U keys: the U x R warp reductions are
+// independent, so their shuffles overlap.
+template <int PER, int R, int U>
+__device__ __forceinline__ void batch_scores(const float (&q)[R][PER], const float (&kx)[U][PER],
+                                             int r, float scale_log2, float (&s)[U][R]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int hh = 0; hh < R; ++hh) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) a = fmaf(q[hh][e], kx[u][e], a);
+            s[u][hh] = a;
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int hh = 0; hh < R; ++hh)
+                if (hh < r) s[u][hh] += __shfl_xor_sync(0xffffffffu, s[u][hh], o);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int hh = 0; hh < R; ++hh) s[u][hh] *= scale_log2;
+}
 
 // Combine the kWarps per-warp states of R heads through shared memory and
 // write one partial [R][D + 2] (O, m, l) per CTA.
@@ -212,29 +252,37 @@ __global__ void __launch_bounds__(kWarps * 32) decode_cmp_kernel(DecodeParams p)
         if (hh < r) load_piece<T, PER>(Q + (size_t)(g * r + hh) * D + lane * PER, q[hh]);
     }
     const int lo = (int)((long long)c * b / kSplit), hi = (int)((long long)c * (b + 1) / kSplit);
-    for (int j = lo + warp; j < hi; j += kWarps) {
-        float kx[PER], vx[PER];
-        load_piece<T, PER>(KC + ((size_t)j * p.h_kv + g) * D + lane * PER, kx);
-        load_piece<T, PER>(VC + ((size_t)j * p.h_kv + g) * D + lane * PER, vx);
+    for (int j0 = lo + warp * kBatch; j0 < hi; j0 += kWarps * kBatch) {
+        float kx[kBatch][PER], vx[kBatch][PER];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = min(j0 + u, hi - 1);  // in range; keys past hi are skipped
+            load_piece<T, PER>(KC + ((size_t)j * p.h_kv + g) * D + lane * PER, kx[u]);
+            load_piece<T, PER>(VC + ((size_t)j * p.h_kv + g) * D + lane * PER, vx[u]);
+        }
+        float sc[kBatch][R];
+        batch_scores<PER, R, kBatch>(q, kx, r, p.scale_log2, sc);
 #pragma unroll
         for (int hh = 0; hh < R; ++hh) {
             if (hh >= r) break;
-            float s = 0.f;
+            float su[kBatch];
 #pragma unroll
-            for (int e = 0; e < PER; ++e) s = fmaf(q[hh][e], kx[e], s);
-            s = warp_sum(s) * p.scale_log2;
-            if (lane == 0) p.s_cmp[((size_t)g * r + hh) * p.nb_max + j] = s;
-            acc[hh].add(s, vx);
+            for (int u = 0; u < kBatch; ++u) {
+                const bool in = j0 + u < hi;
+                su[u] = in ? sc[u][hh] : -INFINITY;
+                if (in && lane == u) p.s_cmp[((size_t)g * r + hh) * p.nb_max + j0 + u] = sc[u][hh];
+            }
+            acc[hh].add_batch<kBatch>(su, vx);
         }
     }
     combine_warps<PER, R>(acc, r, sm, part_of(p, 0, g, b));
 }
 
 // ---------------------------------------------------------------------------
-// Per group: the compression output (ungated), the group importance of every
-// visible block, and the top-k selection.
+// Per group: the group importance of every visible block and the top-k
+// selection.
 template <int D>
-__global__ void __launch_bounds__(256) decode_select_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(1024) decode_select_kernel(DecodeParams p) {
     extern __shared__ float sm[];  // lse [16], split weights [16][kSplit], importance
     __shared__ uint64_t buf[128];
     const Counts cn = *p.counts;
@@ -245,19 +293,15 @@ __global__ void __launch_bounds__(256) decode_select_kernel(DecodeParams p) {
     float *lse = sm;
     float *fw = sm + 16;                    // [16][kSplit]
     float *imp = fw + 16 * kSplit + 4;      // 16-byte aligned: 16 + 16 * 37 + 4 floats
-    // compression partials -> o_cmp (normalised) and the log2-sum-exp per head
+    // the log2-sum-exp of every head from the compression partials
     const float *part0 = part_of(p, 0, g, 0);
     split_weights(part0, r, D, fw, lse);
     __syncthreads();
-    for (int x = threadIdx.x; x < r * D; x += blockDim.x) {
-        const int hh = x / D, e = x % D;
-        float O = 0.f;
-        for (int b = 0; b < kSplit; ++b) O += part0[((size_t)b * r + hh) * (D + 2) + e] * fw[hh * kSplit + b];
-        p.o_cmp[(size_t)(g * r + hh) * D + e] = O;
-    }
     // importance: the exact compression probabilities summed over the heads
+    // (the head loads of a block are issued together)
     for (int j = threadIdx.x; j < c; j += blockDim.x) {
         float s = 0.f;
+#pragma unroll 8
         for (int hh = 0; hh < r; ++hh)
             s += exp2f(p.s_cmp[((size_t)g * r + hh) * p.nb_max + j] - lse[hh]);
         imp[j] = s;
@@ -294,18 +338,28 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
     for (int hh = 0; hh < R; ++hh)
         if (hh < r) load_piece<T, PER>(Q + (size_t)(g * r + hh) * D + lane * PER, q[hh]);
     auto vis_pos = [&](int u) { return cn.contiguous ? cn.vis_base + u : p.vis[u]; };
-    // one key at position t into the R accumulators
-    auto attend = [&](Acc<PER>(&acc)[R], int t) {
-        float kx[PER], vx[PER];
-        load_piece<T, PER>(K + ((size_t)t * p.h_kv + g) * D + lane * PER, kx);
-        load_piece<T, PER>(V + ((size_t)t * p.h_kv + g) * D + lane * PER, vx);
+    // kBatch keys at positions t[u] (-1: skip) into the R accumulators; all
+    // loads are issued before any score is computed
+    auto attend = [&](Acc<PER>(&acc)[R], const int (&t)[kBatch]) {
+        float kx[kBatch][PER], vx[kBatch][PER];
+        int any = 0;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            any |= t[u] >= 0;
+            const size_t row = ((size_t)max(t[u], 0) * p.h_kv + g) * D + lane * PER;
+            load_piece<T, PER>(K + row, kx[u]);
+            load_piece<T, PER>(V + row, vx[u]);
+        }
+        if (!any) return;
+        float sc[kBatch][R];
+        batch_scores<PER, R, kBatch>(q, kx, r, p.scale_log2, sc);
 #pragma unroll
         for (int hh = 0; hh < R; ++hh) {
             if (hh >= r) break;
-            float s = 0.f;
+            float su[kBatch];
 #pragma unroll
-            for (int e = 0; e < PER; ++e) s = fmaf(q[hh][e], kx[e], s);
-            acc[hh].add(warp_sum(s) * p.scale_log2, vx);
+            for (int u = 0; u < kBatch; ++u) su[u] = t[u] >= 0 ? sc[u][hh] : -INFINITY;
+            acc[hh].add_batch<kBatch>(su, vx);
         }
     };
     Acc<PER> acc[R];
@@ -318,11 +372,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
             for (int hh = 0; hh < R; ++hh) acc[hh].init();
             const int nk = p.top_k * p.block;
             const int lo = (int)((long long)nk * b / kSplit), hi = (int)((long long)nk * (b + 1) / kSplit);
-            for (int x = lo + warp; x < hi; x += kWarps) {
-                const int blk = sel[x / p.block];
-                const int u = blk * p.block + x % p.block;
-                if (blk < 0 || u > i) continue;
-                attend(acc, vis_pos(u));
+            for (int x0 = lo + warp * kBatch; x0 < hi; x0 += kWarps * kBatch) {
+                int t[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int x = x0 + u;
+                    t[u] = -1;
+                    if (x < hi) {
+                        const int blk = sel[x / p.block];
+                        const int rank = blk * p.block + x % p.block;
+                        if (blk >= 0 && rank <= i) t[u] = vis_pos(rank);
+                    }
+                }
+                attend(acc, t);
             }
             __syncthreads();
             combine_warps<PER, R>(acc, r, sm, part_of(p, 1, g, b));
@@ -334,7 +396,12 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
             for (int hh = 0; hh < R; ++hh) acc[hh].init();
             const int u0 = max(0, i - p.window + 1), nk = i - u0 + 1;
             const int lo = (int)((long long)nk * b / kSplit), hi = (int)((long long)nk * (b + 1) / kSplit);
-            for (int x = lo + warp; x < hi; x += kWarps) attend(acc, vis_pos(u0 + x));
+            for (int x0 = lo + warp * kBatch; x0 < hi; x0 += kWarps * kBatch) {
+                int t[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) t[u] = x0 + u < hi ? vis_pos(u0 + x0 + u) : -1;
+                attend(acc, t);
+            }
             combine_warps<PER, R>(acc, r, sm, part_of(p, 2, g, b));
         }
     } else {
@@ -343,23 +410,31 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
         for (int hh = 0; hh < R; ++hh) acc[hh].init();
         const int nk = p.n;
         const int lo = (int)((long long)nk * b / kSplit), hi = (int)((long long)nk * (b + 1) / kSplit);
-        for (int x = lo + warp; x < hi; x += kWarps) attend(acc, x);
+        for (int x0 = lo + warp * kBatch; x0 < hi; x0 += kWarps * kBatch) {
+            int t[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) t[u] = x0 + u < hi ? x0 + u : -1;
+            attend(acc, t);
+        }
         combine_warps<PER, R>(acc, r, sm, part_of(p, 2, g, b));
     }
 }
 
 // ---------------------------------------------------------------------------
-// One CTA per query head: the branch partials, the gates, the output row.
+// One CTA per query head: the branch partials (compression, selection,
+// window or text), the gates, the output row.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
-    __shared__ float fw[2][kSplit];
+    __shared__ float fw[3][kSplit];
     const Counts cn = *p.counts;
     const bool vision = cn.pad[1] != 0;
     const int h = blockIdx.x, g = h / p.r, hh = h % p.r, e = threadIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // split weights of this head for branch 1 (selection) and 2 (window/text)
-    if (warp < 2) {
-        const float *part = part_of(p, 1 + warp, g, 0);
+    // split weights of this head for branch br (0 compression, 1 selection,
+    // 2 window / text), one warp per branch (D = 64: two warps take three)
+    for (int br = warp; br < 3; br += D / 32) {
+        if (!vision && br != 2) continue;
+        const float *part = part_of(p, br, g, 0);
         float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 #pragma unroll
         for (int z = 0; z < 2; ++z) {
@@ -379,20 +454,25 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
 #pragma unroll
         for (int z = 0; z < 2; ++z) {
             const int b = lane + 32 * z;
-            if (b < kSplit) fw[warp][b] = (L > 0.f && l[z] > 0.f) ? exp2f(m[z] - M) / L : 0.f;
+            if (b < kSplit) fw[br][b] = (L > 0.f && l[z] > 0.f) ? exp2f(m[z] - M) / L : 0.f;
         }
     }
     __syncthreads();
+    // every split's element is loaded before the sum (kSplit loads in flight)
     auto branch = [&](int br) {
         const float *part = part_of(p, br, g, 0);
+        float x[kSplit];
+#pragma unroll
+        for (int b = 0; b < kSplit; ++b) x[b] = part[((size_t)b * p.r + hh) * (D + 2) + e];
         float O = 0.f;
-        for (int b = 0; b < kSplit; ++b) O += part[((size_t)b * p.r + hh) * (D + 2) + e] * fw[br - 1][b];
+#pragma unroll
+        for (int b = 0; b < kSplit; ++b) O = fmaf(x[b], fw[br][b], O);
         return O;
     };
     float o;
     if (vision) {
         const float *gl = p.gate + (size_t)h * 3;
-        o = sigmoidf_(gl[0]) * p.o_cmp[(size_t)h * D + e] + sigmoidf_(gl[1]) * branch(1) +
+        o = sigmoidf_(gl[0]) * branch(0) + sigmoidf_(gl[1]) * branch(1) +
             sigmoidf_(gl[2]) * branch(2);
     } else {
         o = branch(2);
@@ -416,7 +496,7 @@ cudaError_t launch_typed(const DecodeParams &p, cudaStream_t s, int *launches) {
     if (e != cudaSuccess) return e;
     const dim3 split(kSplit, p.h_kv);
     decode_cmp_kernel<T, D, R><<<split, kWarps * 32, part_smem, s>>>(p);
-    decode_select_kernel<D><<<p.h_kv, 256, sel_smem, s>>>(p);
+    decode_select_kernel<D><<<p.h_kv, 1024, sel_smem, s>>>(p);
     decode_attn_kernel<T, D, R><<<split, kWarps * 32, part_smem, s>>>(p);
     decode_combine_kernel<T, D><<<p.h_q, D, 0, s>>>(p);
     *launches += 4;

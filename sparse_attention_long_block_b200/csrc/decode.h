@@ -25,7 +25,6 @@ struct DecodeParams {
     float *s_cmp;                 // [h_kv][r][nb_max] compression scores (log2 units)
     float *part;                  // [3][h_kv][kSplit][r][d + 2] split softmax states
     int32_t *sel;                 // [h_kv][top_k] the selection
-    float *o_cmp;                 // [h_q][d] ungated compression output
     int32_t *sel_out;             // optional export [h_kv][top_k]
 };
 

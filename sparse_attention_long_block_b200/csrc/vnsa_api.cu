@@ -25,7 +25,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
     size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, idx, o_cmp, tc, dec,
-        dec_sel, dec_ocmp;
+        dec_sel;
     size_t total;
     size_t imp_stride;
 };
@@ -53,7 +53,6 @@ Layout make_layout(const vnsa_config &c) {
     L.tc = take(tc_workspace_bytes(c));
     L.dec = take(decode_workspace_bytes(c.h_kv, c.h_q / c.h_kv, c.d, (int)nb));
     L.dec_sel = take((size_t)c.h_kv * c.top_k * 4);
-    L.dec_ocmp = take((size_t)c.h_q * c.d * 4);
     L.total = off;
     return L;
 }
@@ -346,7 +345,6 @@ vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k,
     p.s_cmp = (float *)dec;
     p.part = (float *)(dec + (size_t)c.h_kv * h->r * (h->nb_max > 0 ? h->nb_max : 1) * 4);
     p.sel = (int32_t *)(h->ws + h->L.dec_sel);
-    p.o_cmp = (float *)(h->ws + h->L.dec_ocmp);
     p.sel_out = sel_out;
     h->launches = 0;
     for (int x = 0; x < VNSA_NUM_STAGES; ++x) h->ran[x] = 0;
