@@ -636,16 +636,20 @@ def run_decode_bench(args, rank, world, local_rank):
     layer.close()
 
 
+# the sources that define the tensor-core attention kernel and its launches
+ATTN_KERNEL_SOURCES = ("tc_attn.cu", "tc_attn.h", "tc_ptx.cuh", "common.cuh", "kernels.h")
+
+
 def layer_build_id():
-    """Identity of the kernel sources (hash of csrc) for stored traffic records:
-    a record taken on other kernels is not reported."""
+    """Identity of the attention kernel's sources (a hash of the files that
+    define it) for stored traffic records: a record taken on another build of
+    that kernel is not reported."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_long_block_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in ATTN_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
