@@ -1084,6 +1084,10 @@ __global__ void prepare_kernel(LayerParams p, __nv_bfloat16 *kc, __half *vhc, __
 // min(j*B + B - 1, i) of query i), with a mask of the queries that reach each
 // tile.  One warp per item.
 __device__ __forceinline__ void sel_tiles(int j, int B, int i, int &t0, int &t1) {
+    if (B == kKeys) {  // one tile per block
+        t0 = t1 = j;
+        return;
+    }
     const long long a = (long long)j * B;
     t0 = (int)(a / kKeys);
     t1 = (int)(min(a + B - 1, (long long)i) / kKeys);

@@ -15,121 +15,121 @@ namespace vnsa {
 //
 // Importance values are non-negative floats, so their bit patterns order like
 // the values; a block's sort key is (bits << 32) | ~index, so that the larger
-// key is the block the rule prefers (keys are unique).  Pass 1 (float4 loads
-// of the importance row) keeps each lane's two largest candidate bit
-// patterns; the m-th largest of those 64 values cannot exceed the m-th
-// largest candidate, so only candidates at or above it can be selected.
-// Pass 2 re-reads the row (now in cache) and collects those survivors; if at
-// most 128 survive they are sorted (bitonic, in shared memory) and the first
-// m taken, otherwise m rounds of a warp argmax over keys below the previous
-// pick select them exactly.  Shared memory is 1 KB per warp.
-__device__ __forceinline__ void warp_sort_desc(uint64_t *v, int n, int lane) {
-    // bitonic sort of n (power of two, <= 256) keys in shared memory, descending
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = lane; t < n / 2; t += 32) {
-                const int lo = 2 * t - (t & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = ((lo & size) == 0);
-                const uint64_t a = v[lo], b = v[hi];
-                if ((a < b) == desc) {
-                    v[lo] = b;
-                    v[hi] = a;
-                }
-            }
-            __syncwarp();
-        }
-    }
-}
-
-constexpr int kTopkBuf = 128;  // survivors sorted in shared memory, per warp
+// key is the block the rule prefers (keys are unique).
+//   1. Each lane keeps the T largest candidate bit patterns of blocks lane,
+//      lane + 32, ... (neighbouring blocks, whose importances tend to be alike,
+//      fall to different lanes); T = 2 for m <= 32, else 4.  t0 = the m-th
+//      largest of those 32 T values, found bit by bit with warp ballots, cannot
+//      exceed the m-th largest candidate, so only candidates at or above it can
+//      be selected; with T = 4 it stays close to it even for m near 64.
+//   2. A second pass over the row (now in cache) collects those survivors in
+//      block order into shared memory (ballot compaction).
+//   3. Each survivor's rank is the number of survivors with a larger key; the
+//      m of rank < m are the selection.  (More than 128 survivors: m rounds of
+//      a warp argmax over the keys below the previous pick.)
+//   4. The output position of a selected block is the number of selected
+//      blocks with a lower index plus the forced blocks below it.
+// No sorting network: shared memory is touched once per survivor and once per
+// rank comparison (broadcast reads).  Shared memory is 1 KB per warp.
+constexpr int kTopkBuf = 128;  // survivors per warp in shared memory
 
 // The selection of one (group, query) row by one warp.  row: the query's
-// importance over its c visible blocks (16-byte aligned; global memory when
-// kGlobal, else shared memory); own: the query's own block; buf: 128 keys of
-// warp scratch in shared memory; out: top_k entries, ascending, -1 padded.
+// importance over its c visible blocks (global memory when kGlobal, else
+// shared memory); own: the query's own block; buf: 128 keys of warp scratch in
+// shared memory; out: top_k entries, ascending, -1 padded.
 template <bool kGlobal>
-__device__ __forceinline__ void topk_select_row(const float *row, int c, int own, int top_k, int force_first,
-                                int force_local, uint64_t *buf, int lane, int32_t *out,
-                                uint32_t *status) {
+__device__ __forceinline__ void topk_select_row(const float *row, int c, int own, int top_k,
+                                                int force_first, int force_local, uint64_t *buf,
+                                                int lane, int32_t *out, uint32_t *status) {
     const bool f0 = force_first && c > 0;
     const bool fo = force_local && own < c && !(f0 && own == 0);
     const int nforced =
         (force_first ? 1 : 0) + ((force_local && !(force_first && own == 0)) ? 1 : 0);
     const int m = top_k - nforced;
     const int ncand = c - (f0 ? 1 : 0) - (fo ? 1 : 0);
-    const float4 *row4 = reinterpret_cast<const float4 *>(row);
-    const int c4 = (c + 3) / 4;
-    auto load4 = [&](int q) { return kGlobal ? __ldg(row4 + q) : row4[q]; };
+    const unsigned lt = (1u << lane) - 1u;  // lanes below this one
+    auto load = [&](int j) { return kGlobal ? __ldg(row + j) : row[j]; };
     auto is_cand = [&](int j) { return j < c && !(f0 && j == 0) && !(fo && j == own); };
+    auto bits_of = [&](float v) { return __float_as_uint(fmaxf(v, 0.f)); };
     auto key_of = [&](float v, int j) {
-        return ((uint64_t)__float_as_uint(fmaxf(v, 0.f)) << 32) | (uint32_t)(~(uint32_t)j);
+        return ((uint64_t)bits_of(v) << 32) | (uint32_t)(~(uint32_t)j);
     };
-    int sel = 0;  // selected non-forced blocks, their keys in buf[0, sel)
+    int nsel = 0;  // selected non-forced blocks, their keys in buf[0, nsel)
     if (m > 0 && ncand > m) {
-        uint32_t t1 = 0, t2 = 0;  // the lane's two largest candidate bit patterns
-#pragma unroll 4
-        for (int q = lane; q < c4; q += 32) {
-            const float4 v4 = load4(q);
-            const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                if (!is_cand(4 * q + e)) continue;
-                const uint32_t kj = __float_as_uint(fmaxf(vv[e], 0.f));
-                if (kj > t1) { t2 = t1; t1 = kj; }
-                else if (kj > t2) { t2 = kj; }
+        // 1. the lane's T largest candidate bit patterns, descending
+        uint32_t t[4] = {0u, 0u, 0u, 0u};
+        if (m <= 32) {
+#pragma unroll 8
+            for (int j = lane; j < c; j += 32) {
+                if (!is_cand(j)) continue;
+                const uint32_t kj = bits_of(load(j));
+                if (kj > t[0]) { t[1] = t[0]; t[0] = kj; }
+                else if (kj > t[1]) { t[1] = kj; }
+            }
+        } else {
+#pragma unroll 8
+            for (int j = lane; j < c; j += 32) {
+                if (!is_cand(j)) continue;
+                const uint32_t kj = bits_of(load(j));
+                if (kj <= t[3]) continue;
+                if (kj > t[0]) { t[3] = t[2]; t[2] = t[1]; t[1] = t[0]; t[0] = kj; }
+                else if (kj > t[1]) { t[3] = t[2]; t[2] = t[1]; t[1] = kj; }
+                else if (kj > t[2]) { t[3] = t[2]; t[2] = kj; }
+                else { t[3] = kj; }
             }
         }
-        // lower bound t0 of the m-th largest candidate value
-        buf[lane] = t1;
-        buf[lane + 32] = t2;
-        __syncwarp();
-        warp_sort_desc(buf, 64, lane);
-        const uint32_t t0 = (uint32_t)buf[min(m, 64) - 1];
-        __syncwarp();
-        // survivors: candidates with bits >= t0
-        int cnt = 0;
-#pragma unroll 2
-        for (int base = 0; base < c4; base += 32) {
-            const int q = base + lane;
-            float vv[4] = {0.f, 0.f, 0.f, 0.f};
-            if (q < c4) {
-                const float4 v4 = load4(q);
-                vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
-            }
+        // t0: the largest x with at least m of the values >= x (zeros of unused
+        // slots and of lanes with fewer candidates only lower it)
+        uint32_t t0 = 0;
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t x = t0 | (1u << bit);
+            int n = 0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 4 * q + e;
-                const bool sv = q < c4 && is_cand(j) && __float_as_uint(fmaxf(vv[e], 0.f)) >= t0;
-                const unsigned bal = __ballot_sync(0xffffffffu, sv);
-                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-                if (sv && pos < kTopkBuf) buf[pos] = key_of(vv[e], j);
-                cnt += __popc(bal);
-            }
+            for (int s = 0; s < 4; ++s) n += __popc(__ballot_sync(0xffffffffu, t[s] >= x));
+            if (n >= m) t0 = x;
+        }
+        // 2. survivors in block order
+        int cnt = 0;
+#pragma unroll 4
+        for (int base = 0; base < c; base += 32) {
+            const int j = base + lane;
+            const float v = j < c ? load(j) : 0.f;
+            const bool sv = is_cand(j) && bits_of(v) >= t0;
+            const unsigned bal = __ballot_sync(0xffffffffu, sv);
+            const int pos = cnt + __popc(bal & lt);
+            if (sv && pos < kTopkBuf) buf[pos] = key_of(v, j);
+            cnt += __popc(bal);
         }
         __syncwarp();
         if (cnt <= kTopkBuf) {
-            int n2 = 32;
-            while (n2 < cnt) n2 <<= 1;
-            for (int x = cnt + lane; x < n2; x += 32) buf[x] = 0ull;  // smallest keys
+            // 3. rank of each survivor among the survivors; rank < m is selected,
+            // and buf[rank] then holds the selection in descending key order
+            uint64_t k4[kTopkBuf / 32];
+            int r4[kTopkBuf / 32];
+#pragma unroll
+            for (int s = 0; s < kTopkBuf / 32; ++s) {
+                k4[s] = lane + 32 * s < cnt ? buf[lane + 32 * s] : 0ull;
+                r4[s] = 0;
+            }
+            for (int y = 0; y < cnt; ++y) {
+                const uint64_t ky = buf[y];
+#pragma unroll
+                for (int s = 0; s < kTopkBuf / 32; ++s) r4[s] += ky > k4[s] ? 1 : 0;
+            }
             __syncwarp();
-            warp_sort_desc(buf, n2, lane);
+#pragma unroll
+            for (int s = 0; s < kTopkBuf / 32; ++s)
+                if (lane + 32 * s < cnt && r4[s] < m) buf[r4[s]] = k4[s];
         } else {
             // exact fallback: m rounds of a warp argmax over the keys below the
             // previous pick
             uint64_t last = ~0ull;
             for (int round = 0; round < m; ++round) {
                 uint64_t best = 0;
-                for (int q = lane; q < c4; q += 32) {
-                    const float4 v4 = load4(q);
-                    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * q + e;
-                        if (!is_cand(j)) continue;
-                        const uint64_t kk = key_of(vv[e], j);
-                        if (kk < last && kk > best) best = kk;
-                    }
+                for (int j = lane; j < c; j += 32) {
+                    if (!is_cand(j)) continue;
+                    const uint64_t kk = key_of(load(j), j);
+                    if (kk < last && kk > best) best = kk;
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
@@ -142,7 +142,7 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
                 __syncwarp();
             }
         }
-        sel = m;
+        nsel = m;
     } else if (m > 0) {
         // every non-forced visible block is selected
         int cnt = 0;
@@ -150,40 +150,44 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
             const int j = base + lane;
             const bool t = is_cand(j);
             const unsigned bal = __ballot_sync(0xffffffffu, t);
-            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            const int pos = cnt + __popc(bal & lt);
             if (t && pos < kTopkBuf) buf[pos] = (uint32_t)(~(uint32_t)j);
             cnt += __popc(bal);
         }
-        sel = min(cnt, kTopkBuf);
+        nsel = min(cnt, kTopkBuf);
     }
     __syncwarp();
-    // ascending output: the picks and the visible forced blocks sorted by
-    // index (keys ~j, descending), then the own block when it is forced but
-    // not yet complete (it is above every visible one)
-    for (int x = lane; x < sel; x += 32) buf[x] = (uint32_t)buf[x];
-    __syncwarp();
-    int total = sel;
+    // 4. ascending output: block 0 (forced, visible) first; a selected block j
+    // goes after the selected blocks below it and after the forced own block if
+    // that is below j; the forced own block after the selected blocks below it
+    int below_own = 0;
+    for (int base = 0; base < nsel; base += 32) {
+        const int x = base + lane;
+        int jx = 0, before = 0;
+        if (x < nsel) {
+            jx = (int)(~(uint32_t)buf[x]);
+            for (int y = 0; y < nsel; ++y) before += (int)(~(uint32_t)buf[y]) < jx ? 1 : 0;
+        }
+        below_own += __popc(__ballot_sync(0xffffffffu, x < nsel && fo && jx < own));
+        const int pos = (f0 ? 1 : 0) + before + ((fo && jx > own) ? 1 : 0);
+        if (x < nsel && pos < top_k) out[pos] = jx;
+    }
     if (lane == 0) {
-        if (f0) buf[total] = (uint32_t)(~0u);
-        if (fo) buf[total + (f0 ? 1 : 0)] = (uint32_t)(~(uint32_t)own);
+        if (f0) out[0] = 0;
+        if (fo) {
+            const int pos = (f0 ? 1 : 0) + below_own;
+            if (pos < top_k) out[pos] = own;
+        }
     }
-    total += (f0 ? 1 : 0) + (fo ? 1 : 0);
-    int n2 = 32;
-    while (n2 < total) n2 <<= 1;
-    __syncwarp();
-    for (int x = total + lane; x < n2; x += 32) buf[x] = 0ull;
-    __syncwarp();
-    warp_sort_desc(buf, n2, lane);
-    for (int x = lane; x < total && x < top_k; x += 32) out[x] = (int)(~(uint32_t)buf[x]);
-    int cnt = total;
+    int total = nsel + (f0 ? 1 : 0) + (fo ? 1 : 0);
     const bool extra = (force_local && own >= c) || (force_first && c == 0);
     if (extra) {
-        if (lane == 0 && cnt < top_k) out[cnt] = own;
-        ++cnt;
+        if (lane == 0 && total < top_k) out[total] = own;
+        ++total;
     }
-    for (int x = cnt + lane; x < top_k; x += 32) out[x] = -1;
-    if (cnt > top_k && lane == 0) report(status, VNSA_ERR_BOUNDS);
+    for (int x = total + lane; x < top_k; x += 32) out[x] = -1;
+    if (total > top_k && lane == 0) report(status, VNSA_ERR_BOUNDS);
+    __syncwarp();
 }
-
 
 }  // namespace vnsa
