@@ -96,3 +96,14 @@ def test_forward_rejects_null_handle_and_bad_n():
     assert rc == binding.VNSA_ERR_INVALID_ARG
     rc = lib.vnsa_destroy(None)
     assert rc == binding.VNSA_ERR_INVALID_ARG
+
+
+def test_perceptron_entry_points_reject_null_handle():
+    lib = binding.load()
+    p = ctypes.c_void_p(4096)
+    rc = lib.vnsa_set_cmp_mlp(None, 16, p, p, p, p, p, p, p, p)
+    assert rc == binding.VNSA_ERR_INVALID_ARG
+    rc = lib.vnsa_gate_mlp(None, 8, 64, 16, p, p, p, p, p, p, None)
+    assert rc == binding.VNSA_ERR_INVALID_ARG
+    rc = lib.vnsa_decode(None, 2, p, p, p, p, p, p, None, None)
+    assert rc == binding.VNSA_ERR_INVALID_ARG
