@@ -134,7 +134,10 @@ vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v
  * cudaStream_t; NULL = the legacy default stream).  Pointers must be device
  * pointers, 16-byte aligned, in the layouts above.  `dbg` may be NULL.
  * Returns after enqueueing; errors found by the kernels are reported by
- * vnsa_get_device_status.
+ * vnsa_get_device_status.  The call neither allocates nor synchronises, so it
+ * may be captured into a CUDA graph on `stream`; a replay recomputes the layer
+ * from the captured buffers' current contents (same n and pointers; the
+ * handle's workspace is reused, so replays on one handle must not overlap).
  */
 vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k,
                          const void *v, const uint8_t *is_vision,
