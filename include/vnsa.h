@@ -155,6 +155,39 @@ vnsa_status vnsa_forward_host(vnsa_handle *h, int n, const void *q, const void *
                               const float *gate_logits, void *out, void *stream);
 
 /*
+ * Streamed layer prefills from HOST buffers, for a caller that feeds one layer
+ * call after another from host memory: the copies of neighbouring calls
+ * overlap the attention of the call between them.  (Not a step of the method:
+ * the pages run the layer on data already on the device.)
+ *
+ * vnsa_forward_host_async enqueues one call and returns without waiting.  Its
+ * inputs are copied on a copy stream the handle owns into one of two device
+ * staging slots (call t uses slot t % 2; allocated on the first call, held
+ * until vnsa_destroy), the layer runs on `stream` as vnsa_forward, and `out`
+ * is copied back on a second handle-owned copy stream.  Events order the
+ * three: call t's input copies wait for the attention of call t - 2, its
+ * attention for its input copies and for call t - 2's output copy, its output
+ * copy for its attention.  While call t computes, the inputs of call t + 1 and
+ * the output of call t - 1 cross the bus.  *ticket receives the call's number
+ * (0, 1, 2, ... per handle).  The host buffers (same layouts as vnsa_forward)
+ * must stay valid and unchanged until vnsa_host_wait(ticket) returns; only
+ * page-locked buffers let the copies run asynchronously.  Calls on one handle
+ * must come from one host thread and use one `stream`.  Argument errors return
+ * before anything is enqueued; device-detected errors go to the status word.
+ *
+ * vnsa_host_wait blocks the host until call `ticket`'s output is in host
+ * memory (VNSA_ERR_INVALID_ARG for a ticket not issued yet).  vnsa_host_join
+ * makes `stream` wait, without blocking the host, until every call submitted
+ * so far has its output on the host (e.g. before recording a timing event).
+ */
+vnsa_status vnsa_forward_host_async(vnsa_handle *h, int n, const void *q, const void *k,
+                                    const void *v, const uint8_t *is_vision,
+                                    const float *gate_logits, void *out, void *stream,
+                                    unsigned long long *ticket);
+vnsa_status vnsa_host_wait(vnsa_handle *h, unsigned long long ticket);
+vnsa_status vnsa_host_join(vnsa_handle *h, void *stream);
+
+/*
  * One decode step ("VideoNSA: Native Sparse Attention Scales Video
  * Understanding", paper notes, section "Method", applied to a single new
  * token): the attention output of token n-1, appended to the token stream that

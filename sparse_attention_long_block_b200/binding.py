@@ -24,7 +24,8 @@ NUM_STAGES = 7
 EXPORTED = ("vnsa_status_string", "vnsa_stage_name", "vnsa_workspace_bytes", "vnsa_create",
             "vnsa_forward", "vnsa_forward_host", "vnsa_get_device_status", "vnsa_get_counts",
             "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy",
-            "vnsa_select_noalloc", "vnsa_decode", "vnsa_set_cmp_mlp", "vnsa_gate_mlp")
+            "vnsa_select_noalloc", "vnsa_decode", "vnsa_set_cmp_mlp", "vnsa_gate_mlp",
+            "vnsa_forward_host_async", "vnsa_host_wait", "vnsa_host_join")
 
 
 class vnsa_config(ctypes.Structure):
@@ -70,6 +71,10 @@ def load(path: str = LIB_PATH):
     lib.vnsa_create.argtypes = [ctypes.POINTER(vnsa_config), P, P, ctypes.POINTER(P)]
     lib.vnsa_forward.argtypes = [P, I, P, P, P, P, P, P, ctypes.POINTER(vnsa_debug), P]
     lib.vnsa_forward_host.argtypes = [P, I, P, P, P, P, P, P, P]
+    lib.vnsa_forward_host_async.argtypes = [P, I, P, P, P, P, P, P, P,
+                                            ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.vnsa_host_wait.argtypes = [P, ctypes.c_ulonglong]
+    lib.vnsa_host_join.argtypes = [P, P]
     lib.vnsa_decode.argtypes = [P, I, P, P, P, P, P, P, P, P]
     lib.vnsa_set_cmp_mlp.argtypes = [P, I] + [P] * 8
     lib.vnsa_gate_mlp.argtypes = [P, I, I, I] + [P] * 7
@@ -121,6 +126,21 @@ def vnsa_forward(h, n, q, k, v, is_vision, gate, out, dbg=None, stream=0):
 
 def vnsa_forward_host(h, n, q, k, v, is_vision, gate, out, stream=0):
     _check("vnsa_forward_host", load().vnsa_forward_host(h, n, q, k, v, is_vision, gate, out, stream))
+
+
+def vnsa_forward_host_async(h, n, q, k, v, is_vision, gate, out, stream=0) -> int:
+    t = ctypes.c_ulonglong(0)
+    _check("vnsa_forward_host_async", load().vnsa_forward_host_async(
+        h, n, q, k, v, is_vision, gate, out, stream, ctypes.byref(t)))
+    return int(t.value)
+
+
+def vnsa_host_wait(h, ticket):
+    _check("vnsa_host_wait", load().vnsa_host_wait(h, int(ticket)))
+
+
+def vnsa_host_join(h, stream=0):
+    _check("vnsa_host_join", load().vnsa_host_join(h, stream))
 
 
 def vnsa_decode(h, n, q_new, k, v, is_vision, gate_new, out_new, sel_out=None, stream=0):
@@ -288,6 +308,23 @@ class Layer:
                           is_vision.data_ptr(), gate.data_ptr(), out.data_ptr(),
                           self._stream(stream))
         return out
+
+    def forward_host_async(self, q, k, v, is_vision, gate, out, stream=None) -> int:
+        """Enqueue one layer call on host (pinned) tensors; returns its ticket.
+        The tensors must stay untouched until wait_host(ticket) returns."""
+        n = int(q.shape[0])
+        for t in (q, k, v, is_vision, gate, out):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("host tensors must be contiguous CPU tensors")
+        return vnsa_forward_host_async(self.handle, n, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       is_vision.data_ptr(), gate.data_ptr(), out.data_ptr(),
+                                       self._stream(stream))
+
+    def wait_host(self, ticket):
+        vnsa_host_wait(self.handle, ticket)
+
+    def join_host(self, stream=None):
+        vnsa_host_join(self.handle, self._stream(stream))
 
     def device_status(self, stream=None) -> int:
         return vnsa_get_device_status(self.handle, self._stream(stream))

@@ -77,6 +77,36 @@ vnsa_status check_config(const vnsa_config *c) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Streamed host calls (vnsa_forward_host_async): two device staging slots,
+// one copy stream per direction, and per slot the events that order them.
+// Call t uses slot t & 1.  Its input copies wait until the attention of call
+// t - 2 (the slot's previous user) has run; its attention waits for its input
+// copies and for the output copy of call t - 2; its output copy waits for its
+// attention.  So while call t computes, the inputs of call t + 1 and the output
+// of call t - 1 cross the bus.
+struct HostPipe {
+    char *mem;
+    size_t slot_bytes;
+    cudaStream_t h2d, d2h;
+    cudaEvent_t in_done[2], comp_done[2], out_done[2];
+    unsigned long long next;  // tickets issued so far
+};
+
+void host_pipe_free(HostPipe *p) {
+    if (!p) return;
+    if (p->h2d) cudaStreamSynchronize(p->h2d);
+    if (p->d2h) cudaStreamSynchronize(p->d2h);
+    for (int s = 0; s < 2; ++s) {
+        if (p->in_done[s]) cudaEventDestroy(p->in_done[s]);
+        if (p->comp_done[s]) cudaEventDestroy(p->comp_done[s]);
+        if (p->out_done[s]) cudaEventDestroy(p->out_done[s]);
+    }
+    if (p->h2d) cudaStreamDestroy(p->h2d);
+    if (p->d2h) cudaStreamDestroy(p->d2h);
+    if (p->mem) cudaFree(p->mem);
+    delete p;
+}
+
 }  // namespace
 
 struct vnsa_handle {
@@ -98,6 +128,7 @@ struct vnsa_handle {
     int launches;
     CmpMlp mlp;     // compression perceptron (hidden 0: the linear W_K, W_V)
     char *mlp_mem;  // its weights (owned)
+    HostPipe *pipe; // streamed host calls (created on first use)
 };
 
 extern "C" {
@@ -406,6 +437,106 @@ vnsa_status vnsa_forward_host(vnsa_handle *h, int n, const void *q, const void *
     return VNSA_OK;
 }
 
+vnsa_status vnsa_forward_host_async(vnsa_handle *h, int n, const void *q, const void *k,
+                                    const void *v, const uint8_t *is_vision,
+                                    const float *gate_logits, void *out, void *stream,
+                                    unsigned long long *ticket) {
+    if (!h || !q || !k || !v || !is_vision || !gate_logits || !out || !ticket)
+        return VNSA_ERR_INVALID_ARG;
+    if (n < 1 || n > h->cfg.n_max) return VNSA_ERR_INVALID_ARG;
+    const vnsa_config &c = h->cfg;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return VNSA_ERR_CUDA;
+    const size_t nm = (size_t)c.n_max;
+    const size_t bq = align_up(nm * c.h_q * c.d * h->esize);
+    const size_t bk = align_up(nm * c.h_kv * c.d * h->esize);
+    const size_t bg = align_up(nm * c.h_q * 3 * 4);
+    const size_t bi = align_up(nm);
+    if (!h->pipe) {
+        HostPipe *p = new (std::nothrow) HostPipe();
+        if (!p) return VNSA_ERR_CUDA;
+        p->slot_bytes = 2 * bq + 2 * bk + bg + bi;
+        bool ok = cudaMalloc(&p->mem, 2 * p->slot_bytes) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&p->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&p->d2h, cudaStreamNonBlocking) == cudaSuccess;
+        for (int s = 0; ok && s < 2; ++s)
+            ok = cudaEventCreateWithFlags(&p->in_done[s], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&p->comp_done[s], cudaEventDisableTiming) ==
+                     cudaSuccess &&
+                 cudaEventCreateWithFlags(&p->out_done[s], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            cudaGetLastError();
+            host_pipe_free(p);
+            return VNSA_ERR_CUDA;
+        }
+        h->pipe = p;
+    }
+    HostPipe *p = h->pipe;
+    const unsigned long long t = p->next;
+    const int slot = (int)(t & 1ull);
+    char *dq = p->mem + slot * p->slot_bytes, *dk = dq + bq, *dv = dk + bk, *dg = dv + bk,
+         *di = dg + bg, *dout = di + bi;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t nq = (size_t)n * c.h_q * c.d * h->esize;
+    const size_t nk = (size_t)n * c.h_kv * c.d * h->esize;
+    // inputs of this slot: free once the attention of call t - 2 has run
+    bool ok = (t < 2 || cudaStreamWaitEvent(p->h2d, p->comp_done[slot], 0) == cudaSuccess) &&
+              cudaMemcpyAsync(dq, q, nq, cudaMemcpyHostToDevice, p->h2d) == cudaSuccess &&
+              cudaMemcpyAsync(dk, k, nk, cudaMemcpyHostToDevice, p->h2d) == cudaSuccess &&
+              cudaMemcpyAsync(dv, v, nk, cudaMemcpyHostToDevice, p->h2d) == cudaSuccess &&
+              cudaMemcpyAsync(dg, gate_logits, (size_t)n * c.h_q * 3 * 4,
+                              cudaMemcpyHostToDevice, p->h2d) == cudaSuccess &&
+              cudaMemcpyAsync(di, is_vision, (size_t)n, cudaMemcpyHostToDevice, p->h2d) ==
+                  cudaSuccess &&
+              cudaEventRecord(p->in_done[slot], p->h2d) == cudaSuccess &&
+              cudaStreamWaitEvent(s, p->in_done[slot], 0) == cudaSuccess &&
+              // output of this slot: free once call t - 2's copy to the host ran
+              (t < 2 || cudaStreamWaitEvent(s, p->out_done[slot], 0) == cudaSuccess);
+    if (!ok) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    vnsa_status st = vnsa_forward(h, n, dq, dk, dv, (const uint8_t *)di, (const float *)dg,
+                                  dout, nullptr, stream);
+    if (st != VNSA_OK) return st;
+    ok = cudaEventRecord(p->comp_done[slot], s) == cudaSuccess &&
+         cudaStreamWaitEvent(p->d2h, p->comp_done[slot], 0) == cudaSuccess &&
+         cudaMemcpyAsync(out, dout, nq, cudaMemcpyDeviceToHost, p->d2h) == cudaSuccess &&
+         cudaEventRecord(p->out_done[slot], p->d2h) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    p->next = t + 1;
+    *ticket = t;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_host_wait(vnsa_handle *h, unsigned long long ticket) {
+    if (!h || !h->pipe || ticket >= h->pipe->next) return VNSA_ERR_INVALID_ARG;
+    // the slot's event was last recorded for `ticket` or a later call on the
+    // same slot; copies to the host run in submission order on one stream
+    if (cudaEventSynchronize(h->pipe->out_done[ticket & 1ull]) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_host_join(vnsa_handle *h, void *stream) {
+    if (!h) return VNSA_ERR_INVALID_ARG;
+    HostPipe *p = h->pipe;
+    if (!p || p->next == 0) return VNSA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the last call's copy to the host follows every earlier one on its stream
+    if (cudaStreamWaitEvent(s, p->out_done[(p->next - 1) & 1ull], 0) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    return VNSA_OK;
+}
+
 vnsa_status vnsa_get_device_status(vnsa_handle *h, void *stream, uint32_t *code) {
     if (!h || !code) return VNSA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -551,6 +682,7 @@ vnsa_status vnsa_destroy(vnsa_handle *h) {
     for (int e = 0; e < 2 * VNSA_NUM_STAGES; ++e)
         if (h->ev[e]) cudaEventDestroy(h->ev[e]);
     if (h->stage) cudaFree(h->stage);
+    host_pipe_free(h->pipe);
     if (h->mlp_mem) cudaFree(h->mlp_mem);
     if (h->ws) cudaFree(h->ws);
     cudaGetLastError();
