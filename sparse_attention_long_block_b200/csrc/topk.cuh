@@ -19,14 +19,18 @@ namespace vnsa {
 //   1. Each lane keeps the T largest candidate bit patterns of blocks lane,
 //      lane + 32, ... (neighbouring blocks, whose importances tend to be alike,
 //      fall to different lanes); T = 2 for m <= 32, else 4.  t0 = the m-th
-//      largest of those 32 T values, found bit by bit with warp ballots, cannot
-//      exceed the m-th largest candidate, so only candidates at or above it can
-//      be selected; with T = 4 it stays close to it even for m near 64.
+//      largest of those 32 T values (m rounds of a warp max, each round taking
+//      one copy of the maximum out of its lane's list) cannot exceed the m-th
+//      largest candidate, so only candidates at or above it can be selected;
+//      with T = 4 it stays close to it even for m near 64.
 //   2. A second pass over the row (now in cache) collects those survivors in
 //      block order into shared memory (ballot compaction).
 //   3. Each survivor's rank is the number of survivors with a larger key; the
-//      m of rank < m are the selection.  (More than 128 survivors: m rounds of
-//      a warp argmax over the keys below the previous pick.)
+//      m of rank < m are the selection.  Survivors are in block order, so a
+//      ballot prefix over "selected" gives each selected block its output
+//      position (plus the forced blocks below it).  (More than 128 survivors:
+//      m rounds of a warp argmax over the keys below the previous pick, then
+//      4.)
 //   4. The output position of a selected block is the number of selected
 //      blocks with a lower index plus the forced blocks below it.
 // No sorting network: shared memory is touched once per survivor and once per
@@ -55,6 +59,8 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
         return ((uint64_t)bits_of(v) << 32) | (uint32_t)(~(uint32_t)j);
     };
     int nsel = 0;  // selected non-forced blocks, their keys in buf[0, nsel)
+    bool direct = false;   // positions already written by the survivor ranks
+    int below_direct = 0;  // and the count of selected blocks below `own`
     if (m > 0 && ncand > m) {
         // 1. the lane's T largest candidate bit patterns, descending
         uint32_t t[4] = {0u, 0u, 0u, 0u};
@@ -78,15 +84,23 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
                 else { t[3] = kj; }
             }
         }
-        // t0: the largest x with at least m of the values >= x (zeros of unused
-        // slots and of lanes with fewer candidates only lower it)
+        // t0: the m-th largest of the 32 T values, counted with multiplicity
+        // (zeros of unused slots and of lanes with fewer candidates only lower
+        // it): round r takes the warp maximum and removes one copy of it, the
+        // head of the lowest lane that holds it
         uint32_t t0 = 0;
-        for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t x = t0 | (1u << bit);
-            int n = 0;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) n += __popc(__ballot_sync(0xffffffffu, t[s] >= x));
-            if (n >= m) t0 = x;
+        if (m <= 32) {
+            for (int r = 0; r < m; ++r) {
+                t0 = __reduce_max_sync(0xffffffffu, t[0]);
+                const unsigned who = __ballot_sync(0xffffffffu, t[0] == t0);
+                if (lane == __ffs(who) - 1) { t[0] = t[1]; t[1] = 0u; }
+            }
+        } else {
+            for (int r = 0; r < m; ++r) {
+                t0 = __reduce_max_sync(0xffffffffu, t[0]);
+                const unsigned who = __ballot_sync(0xffffffffu, t[0] == t0);
+                if (lane == __ffs(who) - 1) { t[0] = t[1]; t[1] = t[2]; t[2] = t[3]; t[3] = 0u; }
+            }
         }
         // 2. survivors in block order
         int cnt = 0;
@@ -102,8 +116,8 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
         }
         __syncwarp();
         if (cnt <= kTopkBuf) {
-            // 3. rank of each survivor among the survivors; rank < m is selected,
-            // and buf[rank] then holds the selection in descending key order
+            // 3. rank of each survivor among the survivors (only the words that
+            // hold survivors are compared); rank < m is selected
             uint64_t k4[kTopkBuf / 32];
             int r4[kTopkBuf / 32];
 #pragma unroll
@@ -111,15 +125,38 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
                 k4[s] = lane + 32 * s < cnt ? buf[lane + 32 * s] : 0ull;
                 r4[s] = 0;
             }
-            for (int y = 0; y < cnt; ++y) {
-                const uint64_t ky = buf[y];
+            if (cnt <= 32) {
+                for (int y = 0; y < cnt; ++y) r4[0] += buf[y] > k4[0] ? 1 : 0;
+            } else if (cnt <= 64) {
+                for (int y = 0; y < cnt; ++y) {
+                    const uint64_t ky = buf[y];
+                    r4[0] += ky > k4[0] ? 1 : 0;
+                    r4[1] += ky > k4[1] ? 1 : 0;
+                }
+            } else {
+                for (int y = 0; y < cnt; ++y) {
+                    const uint64_t ky = buf[y];
 #pragma unroll
-                for (int s = 0; s < kTopkBuf / 32; ++s) r4[s] += ky > k4[s] ? 1 : 0;
+                    for (int s = 0; s < kTopkBuf / 32; ++s) r4[s] += ky > k4[s] ? 1 : 0;
+                }
             }
-            __syncwarp();
+            // output positions: survivors are in block order, so the selected
+            // ones below a block are counted by a ballot prefix
+            int base = 0;
 #pragma unroll
-            for (int s = 0; s < kTopkBuf / 32; ++s)
-                if (lane + 32 * s < cnt && r4[s] < m) buf[r4[s]] = k4[s];
+            for (int s = 0; s < kTopkBuf / 32; ++s) {
+                if (32 * s >= cnt) break;
+                const bool sel = lane + 32 * s < cnt && r4[s] < m;
+                const unsigned bal = __ballot_sync(0xffffffffu, sel);
+                const int jx = (int)(~(uint32_t)k4[s]);
+                if (sel) {
+                    const int pos = (f0 ? 1 : 0) + base + __popc(bal & lt) + ((fo && jx > own) ? 1 : 0);
+                    if (pos < top_k) out[pos] = jx;
+                }
+                below_direct += __popc(__ballot_sync(0xffffffffu, sel && fo && jx < own));
+                base += __popc(bal);
+            }
+            direct = true;
         } else {
             // exact fallback: m rounds of a warp argmax over the keys below the
             // previous pick
@@ -160,8 +197,8 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
     // 4. ascending output: block 0 (forced, visible) first; a selected block j
     // goes after the selected blocks below it and after the forced own block if
     // that is below j; the forced own block after the selected blocks below it
-    int below_own = 0;
-    for (int base = 0; base < nsel; base += 32) {
+    int below_own = direct ? below_direct : 0;
+    for (int base = 0; !direct && base < nsel; base += 32) {
         const int x = base + lane;
         int jx = 0, before = 0;
         if (x < nsel) {
