@@ -107,3 +107,13 @@ def test_perceptron_entry_points_reject_null_handle():
     assert rc == binding.VNSA_ERR_INVALID_ARG
     rc = lib.vnsa_decode(None, 2, p, p, p, p, p, p, None, None)
     assert rc == binding.VNSA_ERR_INVALID_ARG
+
+
+def test_streamed_host_calls_reject_null_handle_and_unissued_tickets():
+    lib = binding.load()
+    p = ctypes.c_void_p(4096)
+    t = ctypes.c_ulonglong(7)
+    rc = lib.vnsa_forward_host_async(None, 10, p, p, p, p, p, p, None, ctypes.byref(t))
+    assert rc == binding.VNSA_ERR_INVALID_ARG and t.value == 7
+    assert lib.vnsa_host_wait(None, 0) == binding.VNSA_ERR_INVALID_ARG
+    assert lib.vnsa_host_join(None, None) == binding.VNSA_ERR_INVALID_ARG
