@@ -94,6 +94,8 @@ def executed_work(wl, is_vision, idx):
     tile (8 head slots), a statistics pass (QK^T) and an exact pass (QK^T + P V)
     over the visible blocks; selection: 18 queries (7 heads) against the union
     of the 64-key tiles their selected blocks reach (from idx [h_kv][N_v][k]);
+    with block 64 the tiles that only one of the 18 queries reaches run
+    tile-major instead, up to 18 such (query, tile) pairs per 128-row tile;
     window and text: 18 queries against their key ranges."""
     prod = 2.0 * 128 * 64 * wl.d
     vis = np.nonzero(is_vision)[0]
@@ -109,6 +111,7 @@ def executed_work(wl, is_vision, idx):
         ql = min(nv, q0 + qc) - 1
         t = -(-min((ql + 1) // wl.block, nb) // 64)
         cmp += 3 * t
+    single = np.zeros((wl.h_kv, (nv + 63) // 64 + 1), np.int64)  # pairs per (group, tile)
     for q0 in range(0, nv, qt):
         ql = min(nv, q0 + qt) - 1
         lo = max(0, q0 - wl.window + 1)
@@ -117,7 +120,14 @@ def executed_work(wl, is_vision, idx):
             sel = idx[g, q0:ql + 1]
             if wl.block == 64:
                 sel = sel.ravel()
-                slc += 2 * len(np.unique(sel[sel >= 0]))
+                u, cnt = np.unique(sel[sel >= 0], return_counts=True)
+                ones = u[cnt == 1]
+                keep = len(u) - len(ones)
+                if len(ones) and keep:
+                    slc += 2 * keep
+                    single[g, ones] += 1
+                else:
+                    slc += 2 * len(u)
                 continue
             # the 64-key tiles each selected block reaches, up to the query
             ok = sel >= 0
@@ -127,6 +137,7 @@ def executed_work(wl, is_vision, idx):
             span = int((t1 - t0)[ok].max()) if ok.any() else -1
             parts = [(t0 + o)[ok & (t0 + o <= t1)] for o in range(span + 1)]
             slc += 2 * (len(np.unique(np.concatenate(parts))) if parts else 0)
+    slc += 2 * float((-(-single // qt)).sum())
     for x0 in range(0, len(txt), qt):
         xl = min(len(txt), x0 + qt) - 1
         text += 2 * ((int(txt[xl]) + 64) // 64)

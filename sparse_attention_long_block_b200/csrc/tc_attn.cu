@@ -79,11 +79,12 @@ constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;
 // whole tile or none of it (MODE_SLC); otherwise a tile holds parts of several
 // blocks and each row's keys are the parts of its own selected blocks
 // (MODE_SLC_UNALIGNED).
-enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3, MODE_SLC_UNALIGNED = 4 };
+enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3, MODE_SLC_UNALIGNED = 4,
+            MODE_SGL = 5 };
 __host__ __device__ constexpr bool is_slc(int m) {
     return m == MODE_SLC || m == MODE_SLC_UNALIGNED;
 }
-enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
+enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4, K_SGL = 5 };
 
 struct TcParams {
     CUtensorMap tm_k, tm_v;    // K (bf16, the caller's) and V (fp16 copy): [n rows][h_kv*d]
@@ -96,6 +97,20 @@ struct TcParams {
     float *part;               // TEXT partials: [item][128][kPartStride]
     int part_items;
     int mode;
+    // Selection tiles that a single query of an item reaches (block 64 only):
+    // the union kernel takes them out of the item's plan and records each
+    // (query, tile) pair; MODE_SGL attends them tile-major, up to 18 pairs of
+    // one tile per item, and the merge kernel folds them into the selection
+    // output.
+    int sgl_on;                // 1: the selection branch runs split this way
+    int sgl_nbt;               // 64-key tiles per group (bucket stride)
+    const int32_t *sgl_meta;   // [0] pairs, [1] items, then hist, off [h_kv*nbt], choff [+1]
+    const int4 *sgl_sorted;    // pairs grouped by bucket: (pair id, vision rank, position, 0)
+    const int4 *sgl_items;     // per item: (bucket, first entry of sgl_sorted, pairs, 0)
+    __half *sgl_o;             // [pair][r][d] normalised output of the pair's tile
+    float *sgl_lse;            // [pair][r] its log-sum-exp (log2 units)
+    __half *slc_u;             // [n_max][h_q][d] normalised output of the union tiles
+    float *slc_lse;            // [n_max][h_q] their log-sum-exp (log2 units)
 };
 
 __host__ __device__ __forceinline__ int pow2_at_least(int r) {
@@ -144,6 +159,11 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
         const int per = (span + w.nsplit - 1) / w.nsplit;
         w.split_len = (per + kKeys - 1) / kKeys * kKeys;
         w.items = tiles * w.nsplit;
+    } else if (MODE == MODE_SGL) {
+        w.n_q = cn.n_vision;
+        w.n_tiles_q = 0;
+        w.q_tma = 0;  // Q rows are gathered: the item's queries are scattered
+        w.items = P.sgl_meta[1];
     } else {
         w.n_q = cn.n_vision;
         w.n_tiles_q = (w.n_q + w.qt - 1) / w.qt;
@@ -165,6 +185,21 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     const LayerParams &L = P.L;
     Item it;
     int tile;
+    if (MODE == MODE_SGL) {
+        const int4 e = P.sgl_items[item];  // bucket b = (group, tile)
+        const int lo = e.x;
+        it.g = lo / P.sgl_nbt;
+        it.split = 0;
+        it.q0 = e.y;  // first entry in sgl_sorted
+        it.nq = e.z;
+        it.nseg = 1;
+        it.seg_kind[0] = K_SGL;
+        it.seg_tiles[0] = 1;
+        it.seg_kind[1] = K_EXACT;
+        it.seg_tiles[1] = 0;
+        it.key_lo = (lo % P.sgl_nbt) * kKeys;
+        return it;
+    }
     if (MODE == MODE_TEXT) {
         const int per_split = L.h_kv * w.n_tiles_q;
         it.split = item / per_split;
@@ -243,6 +278,7 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
     switch (kind) {
         case K_SLC: return P.plan[(size_t)item * (1 + 2 * P.plan_max) + 1 + x] * kKeys;
         case K_SWA:
+        case K_SGL:
         case K_TEXT: return it.key_lo + x * kKeys;
         default: return x * kKeys;
     }
@@ -268,7 +304,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
     if (MODE == MODE_CMP) {
         mk = &P.tm_kb;
         mv = &P.tm_vb;
-    } else if (is_slc(MODE) || MODE == MODE_SWA) {
+    } else if (is_slc(MODE) || MODE == MODE_SWA || MODE == MODE_SGL) {
         mk = w.contiguous ? &P.tm_k : &P.tm_kc;
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
@@ -295,7 +331,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
         // row coordinate of tile x of a segment (both CMP segments share keys)
         auto row_of = [&](int kind, int x) {
             const int key0 = tile_key0(P, it, item, kind, x);
-            return (kind == K_SLC || kind == K_SWA) ? vbase + key0 : key0;
+            return (kind == K_SLC || kind == K_SWA || kind == K_SGL) ? vbase + key0 : key0;
         };
         if (is_k) {
             const int pf0 = min(kPrefetch, it.seg_tiles[0]);
@@ -429,6 +465,7 @@ struct RowCtx {
     int i;      // vision rank (CMP/SLC/SWA) or text rank (TEXT)
     int t;      // position of the query token
     int c_vis;  // visible compressed blocks
+    int sid;    // MODE_SGL: the row's (query, tile) pair
 };
 
 __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool &ok,
@@ -517,8 +554,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         rc.h = it.g * L.r + min(rc.hl, L.r - 1);
         rc.valid = rc.qi < it.nq && rc.hl < L.r;
         rc.i = it.q0 + min(rc.qi, max(it.nq - 1, 0));
-        if (MODE == MODE_TEXT) rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
-        else rc.t = it.nq > 0 ? L.vis[rc.i] : 0;
+        rc.sid = 0;
+        if (MODE == MODE_SGL) {
+            const int4 e = P.sgl_sorted[rc.i];  // it.q0 indexes the pair list here
+            rc.sid = e.x;
+            rc.i = e.y;
+            rc.t = e.z;
+        } else if (MODE == MODE_TEXT) {
+            rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
+        } else {
+            rc.t = it.nq > 0 ? L.vis[rc.i] : 0;
+        }
         rc.c_vis = min((rc.i + 1) / L.block, w.nb);
         if (item_tiles(it) == 0) {
             // nothing attended: empty branch outputs
@@ -535,6 +581,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
+                } else if (MODE == MODE_SLC && P.sgl_on) {
+                    // no union tile: the merge takes the single-query tiles alone
+                    for (int e = 0; e < kD; e += 8)
+                        *reinterpret_cast<uint4 *>(P.slc_u + ((size_t)rc.i * L.h_q + rc.h) * kD +
+                                                   e) = make_uint4(0u, 0u, 0u, 0u);
+                    P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
                 } else {
                     // no selected / window key: this branch adds nothing
                     float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
@@ -549,8 +601,20 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             continue;
         }
         // ---- Q tile (without the TMA box): rows gathered from their
-        // positions, 16-byte pieces
-        for (int e = rho; !w.q_tma && e < kRows * 16; e += 128) {
+        // positions, 16-byte pieces.  MODE_SGL: each thread gathers its own
+        // row (its query is known only through the pair list).
+        if (MODE == MODE_SGL) {
+            const __nv_bfloat16 *src = Q + ((size_t)rc.t * L.h_q + rc.h) * kD;
+#pragma unroll
+            for (int c16 = 0; c16 < 16; ++c16) {
+                const uint4 val = rc.valid ? __ldg(reinterpret_cast<const uint4 *>(src + c16 * 8))
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                const int hf = c16 >> 3, c = c16 & 7;
+                *reinterpret_cast<uint4 *>(sm.base + SM_Q + hf * 16384 + rho * 128 +
+                                           ((c ^ (rho & 7)) << 4)) = val;
+            }
+        }
+        for (int e = rho; MODE != MODE_SGL && !w.q_tma && e < kRows * 16; e += 128) {
             const int row = e >> 4, c16 = e & 15;
             const int qi = row / w.rpad, hl = row % w.rpad;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
@@ -579,7 +643,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::prefetch_l2(part + 64);
             }
         }
-        if (item + (int)gridDim.x < w.items) {
+        if (MODE == MODE_SGL && item + (int)gridDim.x < w.items) {
+            const Item nx = make_item<MODE>(P, w, item + gridDim.x);
+            const int qn = rho / w.rpad, hn = rho % w.rpad;
+            if (qn < nx.nq && hn < L.r) {
+                const int tn = P.sgl_sorted[nx.q0 + qn].z;
+                const __nv_bfloat16 *qr = Q + ((size_t)tn * L.h_q + nx.g * L.r + hn) * kD;
+                ptx::prefetch_l2(qr);
+                ptx::prefetch_l2(qr + 64);
+            }
+        }
+        if (MODE != MODE_SGL && item + (int)gridDim.x < w.items) {
             const Item nx = make_item<MODE>(P, w, item + gridDim.x);
             const int qn = rho / w.rpad, hn = rho % w.rpad;
             if (qn < nx.nq && hn < L.r) {
@@ -652,6 +726,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                             }
                             break;
                         case K_SWA: lo = rc.i - L.window + 1 - key0; hi = rc.i - key0; break;
+                        case K_SGL: lo = 0; hi = rc.i - key0; break;
                         default: lo = 0; hi = rc.t - key0; break;
                     }
                     lo = max(lo, 0);
@@ -877,6 +952,33 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
+        } else if (MODE == MODE_SGL || (MODE == MODE_SLC && P.sgl_on)) {
+            // normalised output (fp16) and log-sum-exp of this row's tiles, for
+            // the merge: one (query, tile) pair (MODE_SGL) or the union tiles
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __half *orow = MODE == MODE_SGL ? P.sgl_o + ((size_t)rc.sid * L.r + rc.hl) * kD
+                                            : P.slc_u + qrow;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                float o[32];
+                ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
+                ptx::tmem_wait_ld();
+                if (!rc.valid) continue;
+#pragma unroll
+                for (int k = 0; k < 32; k += 8) {
+                    uint4 v;
+                    __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+#pragma unroll
+                    for (int z = 0; z < 4; ++z)
+                        h2[z] = __floats2half2_rn(o[k + 2 * z] * inv, o[k + 2 * z + 1] * inv);
+                    *reinterpret_cast<uint4 *>(orow + ch * 32 + k) = v;
+                }
+            }
+            if (rc.valid) {
+                const float lse = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+                if (MODE == MODE_SGL) P.sgl_lse[(size_t)rc.sid * L.r + rc.hl] = lse;
+                else P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = lse;
+            }
         } else if (is_slc(MODE) || MODE == MODE_SWA) {
             const float g =
                 rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (is_slc(MODE) ? 1 : 2)])
@@ -1093,13 +1195,25 @@ __device__ __forceinline__ void sel_tiles(int j, int B, int i, int &t0, int &t1)
     t1 = (int)(min(a + B - 1, (long long)i) / kKeys);
 }
 
-__global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int words) {
+// Where single-query tiles go (SglArgs.on): pair records, the per-bucket
+// counts, and each query's list of its pairs.
+struct SglArgs {
+    int on, nbt, cap;
+    int32_t *meta;  // [0] pairs, [1] items, [2, 2 + h_kv*nbt) pairs per bucket
+    int4 *rec;      // [cap] (bucket, vision rank, rank in bucket, position); bucket -1: unused
+    int32_t *of;    // [h_kv][n_max][top_k] pair ids of each query
+    int32_t *n;     // [h_kv][n_max] how many
+};
+
+__global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int words, SglArgs sg) {
     extern __shared__ uint32_t sh[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wpb = blockDim.x >> 5;
-    uint32_t *bm = sh + (size_t)warp * (2 * words + plan_max);
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t *bm = sh + (size_t)warp * (2 * words + plan_max + 32);
     uint32_t *pre = bm + words;
     uint32_t *qm = pre + words;
+    uint32_t *qcnt = qm + plan_max;  // per query of the item: its single-query tiles
     const Counts cn = *p.counts;
     const int qt = kRows / p.r;
     const int n_tiles = (cn.n_vision + qt - 1) / qt;
@@ -1162,12 +1276,260 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
             }
         }
         __syncwarp();
-        for (int x = lane; x < total && x < plan_max; x += 32) out[1 + plan_max + x] = (int)qm[x];
+        int tot = min(total, plan_max);
+        if (sg.on) {
+            // Tiles that exactly one query reaches leave the plan for the
+            // tile-major pass (MODE_SGL), as long as one tile stays and the
+            // pair records have room; their ids are taken in one block per item.
+            qcnt[lane] = 0u;
+            int nsing = 0;
+            for (int x = lane; x < tot; x += 32) nsing += __popc(qm[x]) == 1 ? 1 : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) nsing += __shfl_xor_sync(0xffffffffu, nsing, o);
+            int base = -1;
+            if (lane == 0 && nsing > 0 && nsing < tot) base = atomicAdd(&sg.meta[0], nsing);
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (base >= 0 && base + nsing > sg.cap) {
+                // no room: the item keeps its tiles; ids below the capacity that
+                // it took are marked unused for the scatter
+                for (int x = base + lane; x < sg.cap; x += 32) sg.rec[x] = make_int4(-1, 0, 0, 0);
+                base = -1;
+            }
+            __syncwarp();
+            if (base >= 0) {
+                int kept = 0, si = 0;
+                for (int xb = 0; xb < tot; xb += 32) {
+                    const int x = xb + lane;
+                    const uint32_t m = x < tot ? qm[x] : 0u;
+                    const int tl = x < tot ? out[1 + x] : 0;
+                    const bool single = x < tot && __popc(m) == 1;
+                    const bool keep = x < tot && !single;
+                    // every lane holds its entry before any entry is moved down
+                    const unsigned bk = __ballot_sync(0xffffffffu, keep);
+                    const unsigned bs = __ballot_sync(0xffffffffu, single);
+                    if (keep) {
+                        const int pos = kept + __popc(bk & lt);
+                        out[1 + pos] = tl;
+                        qm[pos] = m;
+                    }
+                    if (single) {
+                        const int sid = base + si + __popc(bs & lt);
+                        const int qi = __ffs(m) - 1;
+                        const int i = q0 + qi;
+                        const int bucket = g * sg.nbt + tl;
+                        const int lp = atomicAdd(&sg.meta[2 + bucket], 1);
+                        sg.rec[sid] = make_int4(bucket, i, lp, p.vis[i]);
+                        const int slot = (int)atomicAdd(&qcnt[qi], 1u);
+                        sg.of[((size_t)g * p.n_max + i) * p.top_k + slot] = sid;
+                    }
+                    kept += __popc(bk);
+                    si += __popc(bs);
+                    __syncwarp();
+                }
+                tot = kept;
+            }
+            __syncwarp();
+            for (int qi = lane; qi < nq; qi += 32)
+                sg.n[(size_t)g * p.n_max + q0 + qi] = (int)qcnt[qi];
+        }
+        for (int x = lane; x < tot; x += 32) out[1 + plan_max + x] = (int)qm[x];
         if (lane == 0) {
-            out[0] = min(total, plan_max);
+            out[0] = tot;
             if (total > plan_max) report(p.status, VNSA_ERR_BOUNDS);
         }
         __syncwarp();
+    }
+}
+
+// Offsets of the single-query pairs grouped by bucket (group, tile) and of the
+// MODE_SGL items (chunks of qt pairs of one bucket): exclusive prefix sums
+// over the bucket counts, one block.
+__global__ void __launch_bounds__(1024) sgl_scan_kernel(int32_t *meta, int nbk, int qt) {
+    __shared__ int wsum[2][32];
+    const int32_t *hist = meta + 2;
+    int32_t *off = meta + 2 + nbk, *choff = meta + 2 + 2 * nbk;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (nbk + blockDim.x - 1) / blockDim.x;
+    const int b0 = min(nbk, tid * per), b1 = min(nbk, b0 + per);
+    int a = 0, c = 0;
+    for (int b = b0; b < b1; ++b) {
+        a += hist[b];
+        c += (hist[b] + qt - 1) / qt;
+    }
+    int ia = a, ic = c;  // inclusive scans within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int va = __shfl_up_sync(0xffffffffu, ia, o), vc = __shfl_up_sync(0xffffffffu, ic, o);
+        if (lane >= o) {
+            ia += va;
+            ic += vc;
+        }
+    }
+    if (lane == 31) {
+        wsum[0][warp] = ia;
+        wsum[1][warp] = ic;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int xa = lane < (int)(blockDim.x >> 5) ? wsum[0][lane] : 0;
+        int xc = lane < (int)(blockDim.x >> 5) ? wsum[1][lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int va = __shfl_up_sync(0xffffffffu, xa, o), vc = __shfl_up_sync(0xffffffffu, xc, o);
+            if (lane >= o) {
+                xa += va;
+                xc += vc;
+            }
+        }
+        wsum[0][lane] = xa;  // inclusive over warps
+        wsum[1][lane] = xc;
+    }
+    __syncthreads();
+    int ra = ia - a + (warp > 0 ? wsum[0][warp - 1] : 0);
+    int rc = ic - c + (warp > 0 ? wsum[1][warp - 1] : 0);
+    for (int b = b0; b < b1; ++b) {
+        off[b] = ra;
+        choff[b] = rc;
+        ra += hist[b];
+        rc += (hist[b] + qt - 1) / qt;
+    }
+    if (tid == (int)blockDim.x - 1) {
+        choff[nbk] = rc;
+        meta[1] = rc;
+    }
+}
+
+// Pairs in bucket order: pair `sid` goes to off[bucket] + its rank in the
+// bucket, as (sid, vision rank, position, 0); and the MODE_SGL item table:
+// chunk c of bucket b is item choff[b] + c, (b, off[b] + c qt, pairs, 0).
+__global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *sorted,
+                                   int4 *items, int nbk, int cap, int qt) {
+    const int n = min(meta[0], cap);
+    const int32_t *hist = meta + 2, *off = meta + 2 + nbk, *choff = meta + 2 + 2 * nbk;
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x, step = gridDim.x * blockDim.x;
+    for (int sid = tid; sid < n; sid += step) {
+        const int4 e = rec[sid];
+        if (e.x >= 0) sorted[off[e.x] + e.z] = make_int4(sid, e.y, e.w, 0);
+    }
+    for (int b = tid; b < nbk; b += step) {
+        const int cnt = hist[b];
+        for (int c = 0; c * qt < cnt; ++c)
+            items[choff[b] + c] = make_int4(b, off[b] + c * qt, min(qt, cnt - c * qt), 0);
+    }
+}
+
+// The selection output of each (vision query, head): the union tiles' softmax
+// (slc_u, slc_lse) and the query's single-query tiles (sgl_o, sgl_lse), each
+// normalised with its own log-sum-exp, combined by their weights
+// 2^(lse - max) / sum; then partial += sigmoid(g_slc) * o_slc (fp16) and the
+// optional export.  One warp per (group, query).  Lane s holds single-query
+// tile s of the query (its id and its per-head lse and weight; 32 at a time),
+// lane hl < r the union's scalars of head hl; half2 element k of a lane
+// belongs to head k / 2.  KMAX = half2 elements per lane = 2 r at most.
+struct SglMergeArgs {
+    const int32_t *of, *n;
+    const __half *sgl_o, *slc_u;
+    const float *sgl_lse, *slc_lse;
+};
+
+template <int KMAX>
+__global__ void __launch_bounds__(256) sgl_merge_kernel(LayerParams p, SglMergeArgs a) {
+    constexpr int RMAX = KMAX / 2;
+    const Counts cn = *p.counts;
+    const int lane = threadIdx.x & 31;
+    const int r = p.r;
+    const long long rows = (long long)p.h_kv * cn.n_vision;
+    for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < rows;
+         wid += ((long long)gridDim.x * blockDim.x) >> 5) {
+        const int g = (int)(wid / cn.n_vision), i = (int)(wid % cn.n_vision);
+        const int h0 = g * r;
+        const int t = p.vis[i];
+        const int ns = a.n[(size_t)g * p.n_max + i];
+        const int32_t *sids = a.of + ((size_t)g * p.n_max + i) * p.top_k;
+        const float lu = lane < r ? a.slc_lse[(size_t)i * p.h_q + h0 + lane] : -INFINITY;
+        const float gl = lane < r ? sigmoidf_(p.gate[((size_t)t * p.h_q + h0 + lane) * 3 + 1]) : 0.f;
+        // per-head maximum and sum over the union and every single-query tile
+        float mx[RMAX], sm[RMAX];
+#pragma unroll
+        for (int hl = 0; hl < RMAX; ++hl) mx[hl] = __shfl_sync(0xffffffffu, lu, hl);
+        for (int s0 = 0; s0 < ns; s0 += 32) {
+            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
+#pragma unroll
+            for (int hl = 0; hl < RMAX; ++hl) {
+                float v = (sid >= 0 && hl < r) ? a.sgl_lse[(size_t)sid * r + hl] : -INFINITY;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                mx[hl] = fmaxf(mx[hl], v);
+            }
+        }
+#pragma unroll
+        for (int hl = 0; hl < RMAX; ++hl) {
+            const float u = __shfl_sync(0xffffffffu, lu, hl);
+            sm[hl] = mx[hl] == -INFINITY ? 0.f : exp2f(u - mx[hl]);
+        }
+        for (int s0 = 0; s0 < ns; s0 += 32) {
+            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
+#pragma unroll
+            for (int hl = 0; hl < RMAX; ++hl) {
+                float v = (sid >= 0 && hl < r && mx[hl] != -INFINITY)
+                              ? exp2f(a.sgl_lse[(size_t)sid * r + hl] - mx[hl])
+                              : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                sm[hl] += v;
+            }
+        }
+        // union part, then the single-query tiles 32 at a time
+        float2 acc[KMAX];
+        {
+            const __half2 *u = reinterpret_cast<const __half2 *>(a.slc_u + ((size_t)i * p.h_q + h0) * kD);
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                const int hl = k >> 1;
+                const float lh = __shfl_sync(0xffffffffu, lu, hl);
+                const float wk = sm[hl] > 0.f ? exp2f(lh - mx[hl]) / sm[hl] : 0.f;
+                const float2 f = k < 2 * r ? __half22float2(u[lane + 32 * k]) : make_float2(0.f, 0.f);
+                acc[k] = make_float2(wk * f.x, wk * f.y);
+            }
+        }
+        for (int s0 = 0; s0 < ns; s0 += 32) {
+            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
+            float wl[RMAX];  // this lane's tile: weight per head
+#pragma unroll
+            for (int hl = 0; hl < RMAX; ++hl)
+                wl[hl] = (sid >= 0 && hl < r && sm[hl] > 0.f)
+                             ? exp2f(a.sgl_lse[(size_t)sid * r + hl] - mx[hl]) / sm[hl]
+                             : 0.f;
+            const int nc = min(32, ns - s0);
+            for (int c = 0; c < nc; ++c) {
+                const int sc = __shfl_sync(0xffffffffu, sid, c);
+                const __half2 *o = reinterpret_cast<const __half2 *>(a.sgl_o + (size_t)sc * r * kD);
+#pragma unroll
+                for (int k = 0; k < KMAX; ++k) {
+                    const float wk = __shfl_sync(0xffffffffu, wl[k >> 1], c);
+                    if (k < 2 * r) {
+                        const float2 f = __half22float2(o[lane + 32 * k]);
+                        acc[k].x += wk * f.x;
+                        acc[k].y += wk * f.y;
+                    }
+                }
+            }
+        }
+        __half2 *part = reinterpret_cast<__half2 *>((__half *)p.o_cmp_ws + ((size_t)i * p.h_q + h0) * kD);
+        float *dbg = p.dbg_o_slc ? p.dbg_o_slc + ((size_t)t * p.h_q + h0) * kD : nullptr;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            const float gk = __shfl_sync(0xffffffffu, gl, k >> 1);
+            if (k < 2 * r) {
+                const int e = lane + 32 * k;
+                const float2 f = __half22float2(part[e]);
+                part[e] = __floats2half2_rn(f.x + gk * acc[k].x, f.y + gk * acc[k].y);
+                if (dbg) {
+                    dbg[2 * e] = acc[k].x;
+                    dbg[2 * e + 1] = acc[k].y;
+                }
+            }
+        }
     }
 }
 
@@ -1302,7 +1664,45 @@ struct TcState {
     __half *vh_cmp;     // V_cmp in fp16
     int32_t *plan;
     float *part;
+    // single-query selection tiles (block 64): see TcParams
+    int sgl_on, sgl_nbt, sgl_cap;
+    int32_t *sgl_meta, *sgl_of, *sgl_n;
+    int4 *sgl_rec, *sgl_sorted, *sgl_items;
+    __half *sgl_o, *slc_u;
+    float *sgl_lse, *slc_lse;
 };
+
+// Single-query pairs the workspace holds, per query and group on average;
+// beyond it items keep their single-query tiles in the union.
+constexpr int kSglPerQuery = 6;
+
+struct SglSizes {
+    int on, nbt, nbk, cap;
+    size_t meta, rec, sorted, items, of, n, o, lse, u, ulse, total;
+};
+
+static SglSizes sgl_sizes(const vnsa_config &c) {
+    SglSizes z;
+    memset(&z, 0, sizeof(z));
+    z.on = c.block == kKeys;
+    if (!z.on) return z;
+    const int r = c.h_q / c.h_kv;
+    z.nbt = (c.n_max + kKeys - 1) / kKeys;
+    z.nbk = c.h_kv * z.nbt;
+    z.cap = (int)std::min<long long>((long long)c.h_kv * c.n_max * kSglPerQuery, 1ll << 30);
+    z.meta = up256((size_t)(2 + 3 * z.nbk + 1) * 4);
+    z.rec = up256((size_t)z.cap * 16);
+    z.sorted = up256((size_t)z.cap * 16);
+    z.items = up256(((size_t)z.cap / (kRows / r) + z.nbk + 1) * 16);
+    z.of = up256((size_t)c.h_kv * c.n_max * c.top_k * 4);
+    z.n = up256((size_t)c.h_kv * c.n_max * 4);
+    z.o = up256((size_t)z.cap * r * kD * 2);
+    z.lse = up256((size_t)z.cap * r * 4);
+    z.u = up256((size_t)c.n_max * c.h_q * kD * 2);
+    z.ulse = up256((size_t)c.n_max * c.h_q * 4);
+    z.total = z.meta + z.rec + z.sorted + z.items + z.of + z.n + z.o + z.lse + z.u + z.ulse;
+    return z;
+}
 
 // Most 64-key selection tiles of one item: every query reaches at most top_k
 // blocks, each over at most `per_block` tiles, and there are only so many tiles.
@@ -1338,7 +1738,8 @@ size_t tc_workspace_bytes(const vnsa_config &c) {
     if (!tc_supported(c)) return 0;
     const size_t kv = (size_t)c.n_max * c.h_kv * kD * 2;
     const size_t kvb = (size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2;
-    return up256(kv) * 3 + up256(kvb) + up256(plan_bytes(c)) + kTextPartBytes;
+    return up256(kv) * 3 + up256(kvb) + up256(plan_bytes(c)) + kTextPartBytes +
+           sgl_sizes(c).total;
 }
 
 cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
@@ -1360,9 +1761,27 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     st->vh_cmp = (__half *)(p + 3 * kv);
     st->plan = (int32_t *)(p + 3 * kv + kvb);
     st->part = (float *)(p + 3 * kv + kvb + up256(plan_bytes(c)));
+    {
+        const SglSizes z = sgl_sizes(c);
+        st->sgl_on = z.on;
+        st->sgl_nbt = z.nbt;
+        st->sgl_cap = z.cap;
+        char *q = p + 3 * kv + kvb + up256(plan_bytes(c)) + kTextPartBytes;
+        st->sgl_meta = (int32_t *)q;
+        st->sgl_rec = (int4 *)(q += z.meta);
+        st->sgl_sorted = (int4 *)(q += z.rec);
+        st->sgl_items = (int4 *)(q += z.sorted);
+        st->sgl_of = (int32_t *)(q += z.items);
+        st->sgl_n = (int32_t *)(q += z.of);
+        st->sgl_o = (__half *)(q += z.n);
+        st->sgl_lse = (float *)(q += z.o);
+        st->slc_u = (__half *)(q += z.lse);
+        st->slc_lse = (float *)(q += z.u);
+    }
     cudaError_t e = cudaSuccess;
     for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
-                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>})
+                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>,
+                    tc_attn_kernel<MODE_SGL>})
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) {
@@ -1384,6 +1803,16 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     P.plan_max = st->plan_max;
     P.part = st->part;
     P.part_items = st->part_items;
+    const bool sgl = st->sgl_on && c.block == kKeys;
+    P.sgl_on = 0;  // set for the selection launch below
+    P.sgl_nbt = st->sgl_nbt;
+    P.sgl_meta = st->sgl_meta;
+    P.sgl_sorted = st->sgl_sorted;
+    P.sgl_items = st->sgl_items;
+    P.sgl_o = st->sgl_o;
+    P.sgl_lse = st->sgl_lse;
+    P.slc_u = st->slc_u;
+    P.slc_lse = st->slc_lse;
     const int nb_rows = c.n_max / c.block > 0 ? c.n_max / c.block : 1;
     if (!make_map(&P.tm_k, L.k, c.h_kv, L.n, false) ||
         !make_map(&P.tm_v, st->vh, c.h_kv, L.n, true) ||
@@ -1414,6 +1843,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
                 tc_attn_kernel<MODE_SLC_UNALIGNED><<<grid, kThreads, SMEM_BYTES, s>>>(P);
                 break;
             case MODE_SWA: tc_attn_kernel<MODE_SWA><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            case MODE_SGL: tc_attn_kernel<MODE_SGL><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             default: tc_attn_kernel<MODE_TEXT><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
         }
         ++*launches;
@@ -1433,19 +1863,59 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     {
         const int words = ((c.n_max + kKeys - 1) / kKeys + 31) / 32 + 1;
         const int wpb = 4;
-        const size_t smem = (size_t)wpb * (2 * words + st->plan_max) * 4;
+        const size_t smem = (size_t)wpb * (2 * words + st->plan_max + 32) * 4;
         if (smem > 48 * 1024) {
             e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem);
             if (e != cudaSuccess) return e;
         }
-        union_kernel<<<st->num_sms * 8, wpb * 32, smem, s>>>(L, st->plan, st->plan_max, words);
+        SglArgs sa;
+        memset(&sa, 0, sizeof(sa));
+        if (sgl) {
+            // pair count and per-bucket counts start at zero
+            e = cudaMemsetAsync(st->sgl_meta, 0, (size_t)(2 + c.h_kv * st->sgl_nbt) * 4, s);
+            if (e != cudaSuccess) return e;
+            sa.on = 1;
+            sa.nbt = st->sgl_nbt;
+            sa.cap = st->sgl_cap;
+            sa.meta = st->sgl_meta;
+            sa.rec = st->sgl_rec;
+            sa.of = st->sgl_of;
+            sa.n = st->sgl_n;
+        }
+        union_kernel<<<st->num_sms * 8, wpb * 32, smem, s>>>(L, st->plan, st->plan_max, words, sa);
         ++*launches;
+        if (sgl) {
+            const int nbk = c.h_kv * st->sgl_nbt;
+            sgl_scan_kernel<<<1, 1024, 0, s>>>(st->sgl_meta, nbk, kRows / L.r);
+            sgl_scatter_kernel<<<st->num_sms * 4, 256, 0, s>>>(st->sgl_meta, st->sgl_rec,
+                                                               st->sgl_sorted, st->sgl_items, nbk,
+                                                               st->sgl_cap, kRows / L.r);
+            *launches += 2;
+        }
     }
     end(VNSA_STAGE_TOPK);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_SLC);
-    if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) return e;
+    if (sgl) {
+        // single-query tiles tile-major, then the union tiles, then the merge
+        if ((e = attn(MODE_SGL)) != cudaSuccess) return e;
+        P.sgl_on = 1;
+        if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
+        P.sgl_on = 0;
+        SglMergeArgs ma;
+        ma.of = st->sgl_of;
+        ma.n = st->sgl_n;
+        ma.sgl_o = st->sgl_o;
+        ma.slc_u = st->slc_u;
+        ma.sgl_lse = st->sgl_lse;
+        ma.slc_lse = st->slc_lse;
+        if (L.r <= 8) sgl_merge_kernel<16><<<st->num_sms * 8, 256, 0, s>>>(L, ma);
+        else sgl_merge_kernel<32><<<st->num_sms * 8, 256, 0, s>>>(L, ma);
+        ++*launches;
+    } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
+        return e;
+    }
     end(VNSA_STAGE_SLC);
     begin(VNSA_STAGE_SWA);
     if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
