@@ -7,7 +7,7 @@
 // selection and a sliding window mixed by per-head sigmoid gates; text tokens
 // attend densely (GQA).
 //
-// One persistent kernel serves four modes; two CTAs share each SM so that one
+// One persistent kernel serves the modes below; two CTAs share each SM so that one
 // CTA's softmax overlaps the other's tensor-core work.  A CTA (6 warps) walks
 // work items; an item is an M tile of 128 MMA rows, row = (query, head of one
 // GQA group): consecutive queries times the group's heads, so every K/V tile
@@ -24,8 +24,13 @@
 //         (the block importance, a warp reduce-scatter: rows are 16 queries x
 //         8 head slots) and O = P V, already normalised.
 //   SLC   the union of the blocks the item's queries selected; a row masks the
-//         blocks its query did not select.  Epilogue: partial = sig(g_cmp) o_cmp
-//         + sig(g_slc) o_slc, kept in fp32 in the workspace.
+//         blocks its query did not select.  Epilogue: the fp16 gated partial
+//         (sig(g_cmp) o_cmp so far) gains sig(g_slc) o_slc.  With block 64 the
+//         tiles only one of the item's queries reaches are left to SGL, and the
+//         epilogue writes the normalised output and log-sum-exp for the merge.
+//   SGL   one 64-key tile per item; rows = up to 18 (query, tile) pairs of that
+//         tile x the group's heads, Q rows gathered per row; per pair the
+//         normalised output and log-sum-exp.
 //   SWA   the window keys; epilogue: out = partial + sig(g_swa) o_swa (bf16).
 //   TEXT  items = (text query tile, key split); partial O, max and sum to a
 //         buffer that a small combine kernel reduces (or the row directly).
