@@ -38,7 +38,9 @@ def _worker(rank, world, port, out):
 def test_replicas_are_distinct_and_time_is_max_over_ranks():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    # the manager process is spawned too: this process may already run
+    # threads (the oracle's OpenMP pool), and forking it could deadlock
+    manager = mp.get_context("spawn").Manager()
     out = manager.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     seeds = {out[r][0] for r in range(world)}
