@@ -64,7 +64,9 @@ def load_peaks():
 
 def algorithmic_work(wl, is_vision):
     """Algorithmic FLOPs per branch (4 d H_q per attended (query, key) pair)
-    and the bytes of the HBM-bound pooling step, from the mask and config."""
+    and the bytes of the HBM-bound steps (pooling; top-k: the fp32 importance
+    of every visible block read once, the selection written), from the mask and
+    config."""
     vis = np.nonzero(is_vision)[0]
     txt = np.nonzero(is_vision == 0)[0]
     nv = len(vis)
@@ -84,6 +86,7 @@ def algorithmic_work(wl, is_vision):
         "swa": f * float(swa_tokens.sum()),
         "text": f * float((txt.astype(np.int64) + 1).sum()),
         "pool_bytes": float(2 * nb * B * wl.h_kv * wl.d * es + 2 * nb * wl.h_kv * wl.d * es),
+        "topk_bytes": float(4 * wl.h_kv * int(c.sum()) + 4 * wl.h_kv * nv * wl.top_k),
     }
 
 
@@ -536,6 +539,7 @@ def main():
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_source": peaks["source"] + " burst bf16"}
     pool_gbs = work["pool_bytes"] / (branch_ms["pool"] * 1e-3) / 1e9 if branch_ms["pool"] else 0
+    topk_gbs = work["topk_bytes"] / (branch_ms["topk"] * 1e-3) / 1e9 if branch_ms["topk"] else 0
     value = world * wl.n / (ms / 1e3)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -570,6 +574,9 @@ def main():
             "branch_ms": branch_ms,
             "pool_hbm": {"achieved_gbs": pool_gbs, "peak_gbs": peaks["hbm_gbs"],
                          "frac": pool_gbs / peaks["hbm_gbs"]},
+            "topk_hbm": {"achieved_gbs": topk_gbs, "peak_gbs": peaks["hbm_gbs"],
+                         "frac": topk_gbs / peaks["hbm_gbs"], "bytes": work["topk_bytes"],
+                         "stage": "top-k and the selection-union launches"},
             "roofline": roofline,
             "gate_mlp": gate_mlp,
             "cpu_baseline": cpu,

@@ -51,6 +51,10 @@ def test_algorithmic_pairs_match_enumeration(wl, mask):
     f = 4.0 * wl.d * wl.h_q
     for name in ("cmp", "slc", "swa", "text"):
         assert got[name] == f * want[name], name
+    # top-k reads one fp32 importance per visible (group, query, block) and
+    # writes top_k int32 per (group, query)
+    nv = int(x["is_vision"].sum())
+    assert got["topk_bytes"] == 4.0 * wl.h_kv * want["cmp"] + 4.0 * wl.h_kv * nv * wl.top_k
 
 
 def test_selection_executed_work_splits_single_query_tiles():
