@@ -28,9 +28,9 @@
 //         (sig(g_cmp) o_cmp so far) gains sig(g_slc) o_slc.  With block 64 the
 //         tiles only one of the item's queries reaches are left to SGL, and the
 //         epilogue writes the normalised output and log-sum-exp for the merge.
-//   SGL   one 64-key tile per item; rows = up to 18 (query, tile) pairs of that
-//         tile x the group's heads, Q rows gathered per row; per pair the
-//         normalised output and log-sum-exp.
+//   SGL   one 64-key tile per item; rows = up to 128 / r (query, tile) pairs
+//         of that tile x the group's r heads, Q rows gathered per row; per
+//         pair the normalised output and log-sum-exp.
 //   SWA   the window keys; epilogue: out = partial + sig(g_swa) o_swa (bf16).
 //   TEXT  items = (text query tile, key split); partial O, max and sum to a
 //         buffer that a small combine kernel reduces (or the row directly).
@@ -104,9 +104,9 @@ struct TcParams {
     int mode;
     // Selection tiles that a single query of an item reaches (block 64 only):
     // the union kernel takes them out of the item's plan and records each
-    // (query, tile) pair; MODE_SGL attends them tile-major, up to 18 pairs of
-    // one tile per item, and the merge kernel folds them into the selection
-    // output.
+    // (query, tile) pair; MODE_SGL attends them tile-major, up to 128 / r pairs
+    // of one tile per item (18 for 7 heads per group), and the merge kernel
+    // folds them into the selection output.
     int sgl_on;                // 1: the selection branch runs split this way
     int sgl_nbt;               // 64-key tiles per group (bucket stride)
     const int32_t *sgl_meta;   // [0] pairs, [1] items, then hist, off [h_kv*nbt], choff [+1]
