@@ -272,6 +272,30 @@ vnsa_status vnsa_get_counts(vnsa_handle *h, void *stream, int *n_vision, int *n_
 vnsa_status vnsa_set_timing(vnsa_handle *h, int enable);
 vnsa_status vnsa_get_timing(vnsa_handle *h, float *ms);
 
+/*
+ * Limit of the kernels' bounded waits, in nanoseconds of device time, for the
+ * later calls on this handle; 0 restores the default (400 ms).  A wait that
+ * runs out makes its thread block stop its work, wait (within its own bound)
+ * for the copies and tensor-core operations it has in flight, free its tensor
+ * memory and exit; the status word then reads VNSA_ERR_TIMEOUT and the layer's
+ * output of that call is undefined.  Later kernels of the call skip their work
+ * once the status word is set.  A very small limit makes a forward time out on
+ * purpose, which is how failure detection is tested.  (A library knob, not a
+ * step of the method.)
+ */
+vnsa_status vnsa_set_wait_limit(vnsa_handle *h, unsigned long long ns);
+
+/* Which kernels a handle's layer runs on. */
+typedef enum vnsa_path {
+    VNSA_PATH_SIMT = 0,     /* CUDA-core kernels (fp32, d 64, 1..3 query heads per
+                               KV head, or a selection plan beyond the shared-
+                               memory copy); far slower at scale                */
+    VNSA_PATH_TCGEN05 = 1   /* tensor-core (tcgen05 + TMA) attention kernels    */
+} vnsa_path;
+
+/* *path receives the kernel family vnsa_forward uses for this handle. */
+vnsa_status vnsa_get_path(const vnsa_handle *h, int *path);
+
 /* Kernel launches the last forward enqueued (for launch accounting). */
 vnsa_status vnsa_get_launch_count(vnsa_handle *h, int *launches);
 
@@ -298,16 +322,34 @@ vnsa_status vnsa_destroy(vnsa_handle *h);
  * memory that the library declares statically; each GPU that loads the library
  * holds it until the process exits.  A call whose intermediates do not fit
  * returns VNSA_ERR_UNSUPPORTED before launching anything (for 28/4 heads, d 128
- * this allows about 5,000 tokens).  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current; make
- * that first call before any stream capture.  All calls on a device share the
- * one array and it keeps the previous call's contents, so calls that overlap
- * on the GPU (different streams, or concurrent host threads) race and must be
- * serialised by the caller.  Asynchronous on `stream` (a cudaStream_t).
+ * this allows about 5,000 tokens).  cfg is checked exactly as vnsa_create
+ * checks it, with n in place of n_max (same limits, same codes).  The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current and keeps it for the process; the address belongs
+ * to the device's primary context, the one the CUDA runtime uses, so callers
+ * that run under a context of their own (a driver-API cuCtxCreate) cannot use
+ * this entry point.  Make that first call before any stream capture.  All calls
+ * on a device share the one array and it keeps the previous call's contents, so
+ * calls that overlap on the GPU (different streams, or concurrent host threads)
+ * race and must be serialised by the caller.  Asynchronous on `stream` (a
+ * cudaStream_t).  Errors the kernels detect (an index out of range) go to a
+ * status word inside the array, cleared when a call starts: read it with
+ * vnsa_select_noalloc_status after the call and before the next one.
  */
 vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const void *q, const void *k,
                                 const void *v, const uint8_t *is_vision, const void *w_k,
                                 const void *w_v, float *o_cmp, int32_t *idx, void *stream);
+
+/*
+ * Device status of the last vnsa_select_noalloc call on the current device:
+ * synchronises `stream` (the call's stream), then reads and clears the status
+ * word the call's kernels write.  *code receives VNSA_OK or the first
+ * device-detected error (e.g. VNSA_ERR_BOUNDS).  Allocates nothing.  Errors:
+ * VNSA_ERR_INVALID_ARG (code NULL), VNSA_ERR_NO_DEVICE, VNSA_ERR_CUDA.  (No
+ * counterpart in the paper: a library-only entry point, like the call it
+ * reports on.)
+ */
+vnsa_status vnsa_select_noalloc_status(void *stream, uint32_t *code);
 
 #ifdef __cplusplus
 }

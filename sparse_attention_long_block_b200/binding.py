@@ -19,13 +19,15 @@ LIB_PATH = os.path.join(HERE, "libvnsa.so")
 VNSA_OK, VNSA_ERR_INVALID_ARG, VNSA_ERR_UNSUPPORTED, VNSA_ERR_CUDA = 0, 1, 2, 3
 VNSA_ERR_TIMEOUT, VNSA_ERR_BOUNDS, VNSA_ERR_NO_DEVICE = 4, 5, 6
 VNSA_BF16, VNSA_FP32 = 0, 1
+VNSA_PATH_SIMT, VNSA_PATH_TCGEN05 = 0, 1
 NUM_STAGES = 7
 
 EXPORTED = ("vnsa_status_string", "vnsa_stage_name", "vnsa_workspace_bytes", "vnsa_create",
             "vnsa_forward", "vnsa_forward_host", "vnsa_get_device_status", "vnsa_get_counts",
             "vnsa_set_timing", "vnsa_get_timing", "vnsa_get_launch_count", "vnsa_destroy",
             "vnsa_select_noalloc", "vnsa_decode", "vnsa_set_cmp_mlp", "vnsa_gate_mlp",
-            "vnsa_forward_host_async", "vnsa_host_wait", "vnsa_host_join")
+            "vnsa_forward_host_async", "vnsa_host_wait", "vnsa_host_join",
+            "vnsa_select_noalloc_status", "vnsa_set_wait_limit", "vnsa_get_path")
 
 
 class vnsa_config(ctypes.Structure):
@@ -85,6 +87,9 @@ def load(path: str = LIB_PATH):
     lib.vnsa_get_launch_count.argtypes = [P, ctypes.POINTER(I)]
     lib.vnsa_destroy.argtypes = [P]
     lib.vnsa_select_noalloc.argtypes = [ctypes.POINTER(vnsa_config), I, P, P, P, P, P, P, P, P, P]
+    lib.vnsa_select_noalloc_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.vnsa_set_wait_limit.argtypes = [P, ctypes.c_ulonglong]
+    lib.vnsa_get_path.argtypes = [P, ctypes.POINTER(I)]
     for name in EXPORTED:
         if name not in ("vnsa_status_string", "vnsa_stage_name"):
             getattr(lib, name).restype = I
@@ -195,6 +200,25 @@ def vnsa_select_noalloc(cfg: vnsa_config, n, q, k, v, is_vision, w_k, w_v, o_cmp
     """Selection chain with no device allocation (static library scratch)."""
     _check("vnsa_select_noalloc", load().vnsa_select_noalloc(
         ctypes.byref(cfg), n, q, k, v, is_vision, w_k, w_v, o_cmp, idx, stream))
+
+
+def vnsa_set_wait_limit(h, ns: int):
+    _check("vnsa_set_wait_limit", load().vnsa_set_wait_limit(h, int(ns)))
+
+
+def vnsa_get_path(h) -> int:
+    out = ctypes.c_int(-1)
+    _check("vnsa_get_path", load().vnsa_get_path(h, ctypes.byref(out)))
+    return int(out.value)
+
+
+def vnsa_select_noalloc_status(stream=0) -> int:
+    """Synchronise `stream`, then read and clear the device status word of the
+    last vnsa_select_noalloc call on the current device."""
+    code = ctypes.c_uint32(0)
+    _check("vnsa_select_noalloc_status",
+           load().vnsa_select_noalloc_status(stream, ctypes.byref(code)))
+    return int(code.value)
 
 
 # --- torch-facing convenience -------------------------------------------------
@@ -340,6 +364,14 @@ class Layer:
 
     def launches(self) -> int:
         return vnsa_get_launch_count(self.handle)
+
+    def set_wait_limit(self, ns: int):
+        """Limit of the kernels' bounded waits in ns (0: the default)."""
+        vnsa_set_wait_limit(self.handle, ns)
+
+    def path(self) -> str:
+        """"tcgen05" or "simt": the kernel family this layer runs on."""
+        return "tcgen05" if vnsa_get_path(self.handle) == VNSA_PATH_TCGEN05 else "simt"
 
     def close(self):
         if getattr(self, "handle", None):

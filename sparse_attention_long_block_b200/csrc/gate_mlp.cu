@@ -137,9 +137,7 @@ __global__ void __launch_bounds__(kGmThreads, 1) gate_mlp_tc_kernel(const __grid
             // no load may still be landing in shared memory when the CTA ends
             for (uint32_t back = 1; back <= (uint32_t)kGmStages && back <= it; ++back) {
                 const uint32_t u = it - back;
-                if (!ptx::mbar_wait(bar(GB_FULL + u % kGmStages), (u / kGmStages) & 1, abort,
-                                    P.status))
-                    break;
+                if (!ptx::mbar_drain(bar(GB_FULL + u % kGmStages), (u / kGmStages) & 1)) break;
             }
         }
     } else if (warp == 1) {
@@ -184,7 +182,7 @@ __global__ void __launch_bounds__(kGmThreads, 1) gate_mlp_tc_kernel(const __grid
             }
             // every MMA this thread issued has completed once this barrier flips
             ptx::mma_commit(bar(GB_FINAL));
-            ptx::mbar_wait(bar(GB_FINAL), 0, abort, P.status, 200000000ull);
+            ptx::mbar_drain(bar(GB_FINAL), 0);
         }
         __syncwarp();
     } else {

@@ -30,6 +30,7 @@ struct LayerParams {
     size_t idx_rows;                  // rows per group of idx_src
     float *o_cmp_ws;                  // [n_max][h_q][d] fp32 ungated compression output
     float *dbg_o_cmp, *dbg_o_slc, *dbg_o_swa;  // optional [n][h_q][d] exports
+    unsigned long long wait_ns;       // limit of the kernels' bounded waits (0: default)
 };
 
 cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t *vis,

@@ -15,10 +15,19 @@
 // library holds kScratchBytes of it until the process exits.  Host code cannot
 // use the symbol as a device address (the host-side name is only a stand-in),
 // so the first call on each device looks the address up with
-// cudaGetSymbolAddress while that device is current and caches it.
+// cudaGetSymbolAddress while that device is current and caches it (one atomic
+// slot per device ordinal; the address belongs to the device's primary
+// context, which is the context the CUDA runtime uses).
+//
+// The first 256 bytes of the array hold the device status word of the last
+// call (read and cleared by vnsa_select_noalloc_status); the intermediates of
+// a call follow it.
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
+#include "config.h"
 #include "kernels.h"
 
 namespace {
@@ -28,12 +37,17 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 
-void *g_scratch_addr[kMaxDevices];  // per-device address, looked up on first use
+// per-device address of g_select_scratch, looked up on first use; racing
+// first calls store the same value
+std::atomic<void *> g_scratch_addr[kMaxDevices];
+
+constexpr size_t kStatusOffset = 0;     // the status word of the last call
+constexpr size_t kScratchHeader = 256;  // intermediates start after it
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct ScratchPlan {
-    size_t vis, txt, counts, status, k_cmp, v_cmp, lse, imp, total;
+    size_t vis, txt, counts, k_cmp, v_cmp, lse, imp, total;
     size_t imp_stride;
 };
 
@@ -42,12 +56,11 @@ ScratchPlan plan_for(const vnsa_config &c, int n) {
     const size_t nb = (size_t)(n / c.block);
     ScratchPlan s;
     s.imp_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
-    size_t off = 0;
+    size_t off = kScratchHeader;
     auto take = [&](size_t b) { size_t o = off; off += up256(b > 0 ? b : 1); return o; };
     s.vis = take((size_t)n * 4);
     s.txt = take((size_t)n * 4);
     s.counts = take(sizeof(vnsa::Counts));
-    s.status = take(16);
     s.k_cmp = take(nb * c.h_kv * c.d * es);
     s.v_cmp = take(nb * c.h_kv * c.d * es);
     s.lse = take((size_t)n * c.h_q * 4);
@@ -56,16 +69,26 @@ ScratchPlan plan_for(const vnsa_config &c, int n) {
     return s;
 }
 
-bool valid_config(const vnsa_config *c) {
-    if (!c || c->h_q < 1 || c->h_kv < 1 || c->h_q % c->h_kv != 0) return false;
-    if (c->d != 64 && c->d != 128) return false;
-    if (c->block < 1 || c->top_k < 1 || c->top_k > 64) return false;
-    if (c->h_q / c->h_kv > 16) return false;
-    if (c->force_first < 0 || c->force_first > 1 || c->force_local < 0 || c->force_local > 1)
-        return false;
-    if (c->top_k < c->force_first + c->force_local) return false;
-    if (!(c->scale >= 0.f) || isinf(c->scale)) return false;
-    return c->dtype == VNSA_BF16 || c->dtype == VNSA_FP32;
+// The device address of the scratch array on the current device (looked up
+// once per device), or nullptr with *st set on failure.
+char *scratch_base(vnsa_status *st) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        *st = VNSA_ERR_NO_DEVICE;
+        return nullptr;
+    }
+    void *ptr = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
+        if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            *st = VNSA_ERR_CUDA;
+            return nullptr;
+        }
+        g_scratch_addr[dev].store(ptr, std::memory_order_release);
+    }
+    *st = VNSA_OK;
+    return (char *)ptr;
 }
 
 }  // namespace
@@ -76,28 +99,17 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
                                            const void *w_v, float *o_cmp, int32_t *idx,
                                            void *stream) {
     using namespace vnsa;
-    if (!valid_config(cfg) || n < 1 || !q || !k || !v || !is_vision || !w_k || !w_v || !o_cmp ||
-        !idx)
-        return VNSA_ERR_INVALID_ARG;
+    const vnsa_status cst = check_config(cfg, n);
+    if (cst != VNSA_OK) return cst;
+    if (!q || !k || !v || !is_vision || !w_k || !w_v || !o_cmp || !idx) return VNSA_ERR_INVALID_ARG;
     const uintptr_t al = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)w_k |
                          (uintptr_t)w_v | (uintptr_t)o_cmp | (uintptr_t)idx;
     if (al & 15u) return VNSA_ERR_INVALID_ARG;
     const ScratchPlan s = plan_for(*cfg, n);
     if (s.total > kScratchBytes) return VNSA_ERR_UNSUPPORTED;  // too large for the scratch
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        cudaGetLastError();
-        return VNSA_ERR_NO_DEVICE;
-    }
-    if (!g_scratch_addr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess || !ptr) {
-            cudaGetLastError();
-            return VNSA_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = ptr;
-    }
-    char *base = (char *)g_scratch_addr[dev];
+    vnsa_status bst;
+    char *base = scratch_base(&bst);
+    if (!base) return bst;
     cudaStream_t st = (cudaStream_t)stream;
     const vnsa_config &c = *cfg;
     const int dt = (int)c.dtype;
@@ -125,7 +137,7 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
     p.vis = (const int32_t *)(base + s.vis);
     p.txt = (const int32_t *)(base + s.txt);
     p.counts = (const Counts *)(base + s.counts);
-    p.status = (uint32_t *)(base + s.status);
+    p.status = (uint32_t *)(base + kStatusOffset);
     p.k_cmp = base + s.k_cmp;
     p.v_cmp = base + s.v_cmp;
     p.lse = (float *)(base + s.lse);
@@ -138,7 +150,7 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
 
     // The array keeps the previous call's contents; only the status word must
     // start at zero (the kernels overwrite everything else they later read).
-    cudaError_t e = cudaMemsetAsync(base + s.status, 0, 16, st);
+    cudaError_t e = cudaMemsetAsync(base + kStatusOffset, 0, 16, st);
     if (e == cudaSuccess)
         e = launch_partition(is_vision, n, c.block, (int32_t *)p.vis, (int32_t *)p.txt,
                              (Counts *)p.counts, st);
@@ -151,5 +163,24 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
         cudaGetLastError();
         return VNSA_ERR_CUDA;
     }
+    return VNSA_OK;
+}
+
+extern "C" vnsa_status vnsa_select_noalloc_status(void *stream, uint32_t *code) {
+    if (!code) return VNSA_ERR_INVALID_ARG;
+    *code = 0;
+    vnsa_status bst;
+    char *base = scratch_base(&bst);
+    if (!base) return bst;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpy(&word, base + kStatusOffset, sizeof(word), cudaMemcpyDeviceToHost) !=
+            cudaSuccess ||
+        cudaMemset(base + kStatusOffset, 0, sizeof(word)) != cudaSuccess) {
+        cudaGetLastError();
+        return VNSA_ERR_CUDA;
+    }
+    *code = word;
     return VNSA_OK;
 }

@@ -324,8 +324,8 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
             // the item's Q rows (query, head) are one box of the [n][h_q][d]
             // tensor: queries vis_base + q0 .., heads g r .., in MMA row order;
             // the buffer is free once the previous item's Q K^T are done
-            if (nq > 0 && !ptx::mbar_wait(sm.bar(B_Q_EMPTY), (nq - 1) & 1, abort, L.status))
-                return;
+            if (nq > 0 && !ptx::mbar_wait(sm.bar(B_Q_EMPTY), (nq - 1) & 1, abort, L.status, L.wait_ns))
+                goto drain;
             const uint32_t qb = sm.bar(B_Q_FULL);
             ptx::mbar_expect_tx(qb, (uint32_t)(w.qt * qrows) * 2u * kD);
             ptx::tma_load_3d(sm.base_u32 + SM_Q, &P.tm_q, qb, 0, it.g * L.r, w.q_base + it.q0);
@@ -358,8 +358,8 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
                 const uint32_t st = t % kStages;
                 if (t >= (uint32_t)kStages &&
                     !ptx::mbar_wait(sm.bar(ring_empty + st), ((t / kStages) - 1) & 1, abort,
-                                    L.status))
-                    return;
+                                    L.status, L.wait_ns))
+                    goto drain;
                 const uint32_t dst = ring_base + st * K_BYTES;
                 ptx::mbar_expect_tx(sm.bar(ring_full + st), K_BYTES);
                 ptx::tma_load_2d(dst, mine, sm.bar(ring_full + st), xc, y);
@@ -374,12 +374,14 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
             }
         }
     }
-    // no load may still be landing in shared memory when the CTA ends
+    // no load may still be landing in shared memory when the CTA ends (also
+    // after an abort: these waits do not give up on the abort flag)
+drain:
     for (uint32_t back = 1; back <= (uint32_t)kStages && back <= t; ++back) {
         const uint32_t u = t - back;
-        if (!ptx::mbar_wait(sm.bar(ring_full + u % kStages), (u / kStages) & 1, abort, L.status))
-            return;
+        if (!ptx::mbar_drain(sm.bar(ring_full + u % kStages), (u / kStages) & 1)) return;
     }
+    if (is_k && nq > 0) ptx::mbar_drain(sm.bar(B_Q_FULL), (nq - 1) & 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -398,11 +400,11 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
     // Tile `pg` (global count) is finished once its softmax is done with the S
     // buffer: wait for that, then issue its P V if the tile has one.
     auto finish = [&](uint32_t pg, bool has_pv, uint32_t acc) -> bool {
-        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (pg & 1)), (pg >> 1) & 1, abort, L.status))
+        if (!ptx::mbar_wait(sm.bar(B_P_FULL + (pg & 1)), (pg >> 1) & 1, abort, L.status, L.wait_ns))
             return false;
         if (!has_pv) return true;
         const uint32_t sv = npv % kStages;
-        if (!ptx::mbar_wait(sm.bar(B_V_FULL + sv), (npv / kStages) & 1, abort, L.status))
+        if (!ptx::mbar_wait(sm.bar(B_V_FULL + sv), (npv / kStages) & 1, abort, L.status, L.wait_ns))
             return false;
         ptx::tc_fence_after();
         const uint32_t vb = sm.base_u32 + SM_KV + kStages * K_BYTES + sv * K_BYTES;
@@ -419,7 +421,7 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
         const Item it = make_item<MODE>(P, w, item);
         if (item_tiles(it) == 0) continue;
-        if (!ptx::mbar_wait(sm.bar(B_Q_FULL), nitems & 1, abort, L.status)) { ok = false; break; }
+        if (!ptx::mbar_wait(sm.bar(B_Q_FULL), nitems & 1, abort, L.status, L.wait_ns)) { ok = false; break; }
         ++nitems;
         ptx::tc_fence_after();
         bool pending = false, pend_pv = false;
@@ -429,7 +431,7 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
             const int kind = it.seg_kind[s];
             for (int x = 0; x < it.seg_tiles[s]; ++x, ++gt) {
                 const uint32_t st = gt % kStages;
-                if (!ptx::mbar_wait(sm.bar(B_K_FULL + st), (gt / kStages) & 1, abort, L.status)) {
+                if (!ptx::mbar_wait(sm.bar(B_K_FULL + st), (gt / kStages) & 1, abort, L.status, L.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -457,9 +459,10 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         }
         if (ok && pending && !finish(gt - 1, pend_pv, pend_acc)) ok = false;
     }
-    // every MMA this thread issued has completed once this barrier flips
+    // every MMA this thread issued has completed once this barrier flips (also
+    // after an abort, before the CTA frees its TMEM)
     ptx::mma_commit(sm.bar(B_FINAL));
-    ptx::mbar_wait(sm.bar(B_FINAL), 0, abort, L.status, 200000000ull);
+    ptx::mbar_drain(sm.bar(B_FINAL), 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -476,7 +479,7 @@ struct RowCtx {
 __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool &ok,
                                            const LayerParams &L) {
     ptx::mbar_arrive(sm.bar(B_GRP));
-    bool r = ptx::mbar_wait(sm.bar(B_GRP), phase & 1, sm.abort_flag(), L.status);
+    bool r = ptx::mbar_wait(sm.bar(B_GRP), phase & 1, sm.abort_flag(), L.status, L.wait_ns);
     ++phase;
     ok = __all_sync(0xffffffffu, r && ok);
 }
@@ -752,7 +755,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 const bool kill = rowwise && !row_in;
                 const uint32_t sbuf = gt & 1;
                 const uint32_t s_col = tmem + lane_base + TM_S + sbuf * 64;
-                bool r = ptx::mbar_wait(sm.bar(B_S_FULL + sbuf), (gt >> 1) & 1, abort, L.status);
+                bool r = ptx::mbar_wait(sm.bar(B_S_FULL + sbuf), (gt >> 1) & 1, abort, L.status, L.wait_ns);
                 ok = __all_sync(0xffffffffu, r && ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -868,7 +871,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     // O may only be rescaled once every earlier P V has landed
                     if (npv > 0) {
                         bool r2 = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)),
-                                                 ((npv - 1) >> 1) & 1, abort, L.status);
+                                                 ((npv - 1) >> 1) & 1, abort, L.status, L.wait_ns);
                         ok = __all_sync(0xffffffffu, r2 && ok);
                         if (!ok) break;
                     }
@@ -924,7 +927,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // ---- epilogue: wait for the item's last P V (#npv-1)
         {
             bool r = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)), ((npv - 1) >> 1) & 1,
-                                    abort, L.status);
+                                    abort, L.status, L.wait_ns);
             ok = __all_sync(0xffffffffu, r && ok);
             if (!ok) break;
             ptx::tc_fence_after();
@@ -1233,6 +1236,12 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
             const int qi = e / p.top_k, x = e % p.top_k;
             const int j = p.idx_src[((size_t)g * p.idx_rows + q0 + qi) * p.top_k + x];
             if (j < 0) continue;
+            if (j > (q0 + qi) / p.block) {
+                // a block after the query's own (a caller selection out of
+                // range): reported and left out
+                report(p.status, VNSA_ERR_BOUNDS);
+                continue;
+            }
             int t0, t1;
             sel_tiles(j, p.block, q0 + qi, t0, t1);
             for (int t = t0; t <= t1 && (t >> 5) < words; ++t)
@@ -1272,7 +1281,7 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         for (int e = lane; e < ne; e += 32) {
             const int qi = e / p.top_k, x = e % p.top_k;
             const int j = p.idx_src[((size_t)g * p.idx_rows + q0 + qi) * p.top_k + x];
-            if (j < 0) continue;
+            if (j < 0 || j > (q0 + qi) / p.block) continue;
             int t0, t1;
             sel_tiles(j, p.block, q0 + qi, t0, t1);
             for (int t = t0; t <= t1 && (t >> 5) < words; ++t) {

@@ -47,12 +47,14 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of the given parity.  Gives up after `limit_ns`
-// of device time or as soon as another CTA or thread has reported an error
-// (the shared abort flag or the global status word), recording a timeout.
-// Returns false if it gave up.
+// of device time (0: the default, 400 ms) or as soon as another CTA or thread
+// has reported an error (the shared abort flag or the global status word),
+// recording a timeout.  Returns false if it gave up.
+constexpr uint64_t kDefaultWaitNs = 400000000ull;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint32_t *status, uint64_t limit_ns = 400000000ull) {
+                                          uint32_t *status, uint64_t limit_ns = 0) {
     if (mbar_try(bar, parity)) return true;
+    if (limit_ns == 0) limit_ns = kDefaultWaitNs;
     const uint64_t t0 = globaltimer();
     uint32_t spins = 0;
     while (true) {
@@ -66,6 +68,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                 return false;
             }
         }
+    }
+}
+
+// Wait for a phase of an operation this CTA started itself (a TMA load, an MMA
+// commit) before the CTA exits or frees TMEM.  Such operations complete on
+// their own, so unlike mbar_wait this ignores the abort flag and the status
+// word; it is still bounded (limit_ns) and returns false if it gave up.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity,
+                                           uint64_t limit_ns = 1000000000ull) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    uint32_t spins = 0;
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (((++spins) & 63u) == 0 && globaltimer() - t0 > limit_ns) return false;
     }
 }
 

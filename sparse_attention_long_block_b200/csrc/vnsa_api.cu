@@ -10,6 +10,7 @@
 
 #include <new>
 
+#include "config.h"
 #include "decode.h"
 #include "kernels.h"
 #include "tc_attn.h"
@@ -18,7 +19,6 @@ using namespace vnsa;
 
 namespace {
 
-constexpr int kMaxTokens = 262144;
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -55,24 +55,6 @@ Layout make_layout(const vnsa_config &c) {
     L.dec_sel = take((size_t)c.h_kv * c.top_k * 4);
     L.total = off;
     return L;
-}
-
-vnsa_status check_config(const vnsa_config *c) {
-    if (!c) return VNSA_ERR_INVALID_ARG;
-    if (c->n_max < 1 || c->h_q < 1 || c->h_kv < 1 || c->d < 1) return VNSA_ERR_INVALID_ARG;
-    if (c->h_q % c->h_kv != 0) return VNSA_ERR_INVALID_ARG;
-    if (c->top_k < 1 || c->window < 1 || c->block < 1) return VNSA_ERR_INVALID_ARG;
-    if ((c->force_first != 0 && c->force_first != 1) ||
-        (c->force_local != 0 && c->force_local != 1))
-        return VNSA_ERR_INVALID_ARG;
-    if (c->top_k < c->force_first + c->force_local) return VNSA_ERR_INVALID_ARG;
-    if (!(c->scale >= 0.f) || isinf(c->scale)) return VNSA_ERR_INVALID_ARG;
-    if (c->dtype != VNSA_BF16 && c->dtype != VNSA_FP32) return VNSA_ERR_INVALID_ARG;
-    if (c->n_max > kMaxTokens) return VNSA_ERR_UNSUPPORTED;
-    if (c->d != 64 && c->d != 128) return VNSA_ERR_UNSUPPORTED;
-    if (c->h_q / c->h_kv > 16) return VNSA_ERR_UNSUPPORTED;
-    if (c->top_k > 64) return VNSA_ERR_UNSUPPORTED;
-    return VNSA_OK;
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -129,6 +111,7 @@ struct vnsa_handle {
     CmpMlp mlp;     // compression perceptron (hidden 0: the linear W_K, W_V)
     char *mlp_mem;  // its weights (owned)
     HostPipe *pipe; // streamed host calls (created on first use)
+    unsigned long long wait_ns;  // limit of the kernels' bounded waits (0: default)
 };
 
 extern "C" {
@@ -155,7 +138,7 @@ const char *vnsa_stage_name(int stage) {
 
 vnsa_status vnsa_workspace_bytes(const vnsa_config *cfg, size_t *bytes) {
     if (!bytes) return VNSA_ERR_INVALID_ARG;
-    vnsa_status st = check_config(cfg);
+    vnsa_status st = check_config(cfg, cfg ? cfg->n_max : 0);
     if (st != VNSA_OK) return st;
     *bytes = make_layout(*cfg).total;
     return VNSA_OK;
@@ -165,7 +148,7 @@ vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v
                         vnsa_handle **out) {
     if (!out) return VNSA_ERR_INVALID_ARG;
     *out = nullptr;
-    vnsa_status st = check_config(cfg);
+    vnsa_status st = check_config(cfg, cfg ? cfg->n_max : 0);
     if (st != VNSA_OK) return st;
     if (!w_k || !w_v || !aligned16(w_k) || !aligned16(w_v)) return VNSA_ERR_INVALID_ARG;
     int ndev = 0;
@@ -256,6 +239,7 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     p.idx_src = p.idx;
     p.idx_rows = (size_t)c.n_max;
     p.o_cmp_ws = (float *)(h->ws + h->L.o_cmp);
+    p.wait_ns = h->wait_ns;
     const bool forced = dbg && dbg->forced_idx;
     if (forced) {
         p.idx_src = dbg->forced_idx;
@@ -581,6 +565,18 @@ vnsa_status vnsa_get_timing(vnsa_handle *h, float *ms) {
             return VNSA_ERR_CUDA;
         }
     }
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_set_wait_limit(vnsa_handle *h, unsigned long long ns) {
+    if (!h) return VNSA_ERR_INVALID_ARG;
+    h->wait_ns = ns;
+    return VNSA_OK;
+}
+
+vnsa_status vnsa_get_path(const vnsa_handle *h, int *path) {
+    if (!h || !path) return VNSA_ERR_INVALID_ARG;
+    *path = tc_supported(h->cfg) ? VNSA_PATH_TCGEN05 : VNSA_PATH_SIMT;
     return VNSA_OK;
 }
 

@@ -87,26 +87,71 @@ def run_gpu(wl: Workload, x: dict, want=(), forced_idx=None, ranks=None, cmp_mlp
     return res
 
 
+def expected_candidates(i, block, force_first=True, force_local=True):
+    """The blocks a vision query of rank i may select, and the forced ones
+    ("VideoNSA: Native Sparse Attention Scales Video Understanding", paper
+    notes, section "Method", read as: the complete blocks at or before i,
+    plus block 0 and the query's own block, which are always kept)."""
+    forced = set()
+    if force_first:
+        forced.add(0)
+    if force_local:
+        forced.add(i // block)
+    visible = set(range((i + 1) // block))
+    return visible | forced, forced
+
+
+def check_selection_row(row, i, top_k, block, force_first=True, force_local=True,
+                        expect_count=None):
+    """Structure of one exported selection row [top_k] of the vision query of
+    rank i: the selected blocks strictly ascending (so duplicate-free), then -1
+    padding only; exactly min(top_k, #candidates) entries (or `expect_count`);
+    every entry a candidate; every forced block present.  Raises on a
+    violation; returns the selected blocks as a list."""
+    row = [int(j) for j in row]
+    cands, forced = expected_candidates(i, block, force_first, force_local)
+    n_valid = 0
+    while n_valid < len(row) and row[n_valid] >= 0:
+        n_valid += 1
+    sel = row[:n_valid]
+    if any(j != -1 for j in row[n_valid:]):
+        raise AssertionError(f"rank {i}: entries after the first -1 are not all -1: {row}")
+    if any(b <= a for a, b in zip(sel, sel[1:])):
+        raise AssertionError(f"rank {i}: selection not strictly ascending: {row}")
+    want = min(top_k, len(cands)) if expect_count is None else expect_count
+    if n_valid != want:
+        raise AssertionError(f"rank {i}: {n_valid} blocks selected, expected {want}: {row}")
+    bad = [j for j in sel if j not in cands]
+    if bad:
+        raise AssertionError(f"rank {i}: blocks {bad} are not visible to the query: {row}")
+    missing = sorted(forced - set(sel))
+    if missing:
+        raise AssertionError(f"rank {i}: forced blocks {missing} missing: {row}")
+    return sel
+
+
 def check_selection(gpu_idx_rows, ora_idx, ora_imp, top_k, force_first=True,
                     force_local=True, block=64, ranks=None):
-    """gpu_idx_rows, ora_idx: [R][G][k]; ora_imp [R][G][nb].  Returns the row
-    indices (into R) whose set differs within the tie band; raises on a
-    difference outside it."""
+    """gpu_idx_rows, ora_idx: [R][G][k]; ora_imp [R][G][nb]; ranks [R] the
+    vision ranks of the rows (required).  Every GPU row must be a well-formed
+    selection (check_selection_row) with as many blocks as the oracle's row.
+    Returns the row indices (into R) whose block set differs from the
+    oracle's within the tie band; raises on a difference outside it."""
+    if ranks is None:
+        raise ValueError("check_selection needs the vision ranks of the rows")
     swapped = []
     R, G, _ = ora_idx.shape
     for r in range(R):
+        i = int(ranks[r])
+        _, forced = expected_candidates(i, block, force_first, force_local)
         for g in range(G):
-            a = set(int(j) for j in gpu_idx_rows[r, g] if j >= 0)
-            b = set(int(j) for j in ora_idx[r, g] if j >= 0)
+            b_list = check_selection_row(ora_idx[r, g], i, top_k, block, force_first,
+                                         force_local)
+            a_list = check_selection_row(gpu_idx_rows[r, g], i, top_k, block, force_first,
+                                         force_local, expect_count=len(b_list))
+            a, b = set(a_list), set(b_list)
             if a == b:
                 continue
-            i = int(ranks[r]) if ranks is not None else None
-            forced = set()
-            if i is not None:
-                if force_first:
-                    forced.add(0)
-                if force_local:
-                    forced.add(i // block)
             chosen = [j for j in b if j not in forced]
             if not chosen:
                 raise AssertionError(f"row {r} group {g}: sets differ {sorted(a ^ b)} "

@@ -117,3 +117,24 @@ def test_streamed_host_calls_reject_null_handle_and_unissued_tickets():
     assert rc == binding.VNSA_ERR_INVALID_ARG and t.value == 7
     assert lib.vnsa_host_wait(None, 0) == binding.VNSA_ERR_INVALID_ARG
     assert lib.vnsa_host_join(None, None) == binding.VNSA_ERR_INVALID_ARG
+
+
+def test_new_knobs_reject_null_handle_and_noalloc_rejects_bad_config_on_host():
+    lib = binding.load()
+    assert lib.vnsa_set_wait_limit(None, 5) == binding.VNSA_ERR_INVALID_ARG
+    out = ctypes.c_int(-1)
+    assert lib.vnsa_get_path(None, ctypes.byref(out)) == binding.VNSA_ERR_INVALID_ARG
+    assert lib.vnsa_select_noalloc_status(None, None) == binding.VNSA_ERR_INVALID_ARG
+    # the allocation-free selection checks its config exactly as vnsa_create
+    # does (n standing in for n_max), before touching a device
+    p = ctypes.c_void_p(4096)
+    for bad, code in ((dict(d=96), binding.VNSA_ERR_UNSUPPORTED),
+                      (dict(top_k=65), binding.VNSA_ERR_UNSUPPORTED),
+                      (dict(window=0), binding.VNSA_ERR_INVALID_ARG),
+                      (dict(h_q=28, h_kv=3), binding.VNSA_ERR_INVALID_ARG)):
+        c = cfg(**bad)
+        rc = lib.vnsa_select_noalloc(ctypes.byref(c), 64, p, p, p, p, p, p, p, p, None)
+        assert rc == code, bad
+    c = cfg()
+    rc = lib.vnsa_select_noalloc(ctypes.byref(c), 262145, p, p, p, p, p, p, p, p, None)
+    assert rc == binding.VNSA_ERR_UNSUPPORTED
