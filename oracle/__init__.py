@@ -49,7 +49,7 @@ class _Cfg(ctypes.Structure):
                 ("d", ctypes.c_int), ("block", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("window", ctypes.c_int), ("force_first", ctypes.c_int),
                 ("force_local", ctypes.c_int), ("scale", ctypes.c_double),
-                ("round_cmp_bf16", ctypes.c_int)]
+                ("round_cmp_bf16", ctypes.c_int), ("stride", ctypes.c_int)]
 
 
 class _CmpMLP(ctypes.Structure):
@@ -96,13 +96,14 @@ class OracleParams:
     force_local: bool = True
     scale: float | None = None      # None -> 1/sqrt(d)
     round_cmp_bf16: bool = False
+    stride: int | None = None       # compression stride (R13); None -> block
 
 
 def _cfg(p: OracleParams, n: int) -> _Cfg:
     scale = p.scale if p.scale is not None else 1.0 / np.sqrt(p.d)
     return _Cfg(n, p.h_q, p.h_kv, p.d, p.block, p.top_k, p.window,
                 int(p.force_first), int(p.force_local), float(scale),
-                int(p.round_cmp_bf16))
+                int(p.round_cmp_bf16), int(p.stride or 0))
 
 
 def _f32(a):
@@ -141,13 +142,16 @@ def _cmp_mlp(d: int, mlp: dict):
 
 
 def pool_proj(p: OracleParams, k, v, is_vision, w_k=None, w_v=None, cmp_mlp=None):
-    """K_cmp, V_cmp [nb][h_kv][d] in fp64 (compression keys/values): the linear
-    map W_K, W_V, or the compression perceptron ``cmp_mlp`` (a dict of its
-    weights, see ``_cmp_mlp``)."""
+    """K_cmp, V_cmp [nc][h_kv][d] in fp64 (compression keys/values of the nc
+    compression blocks, overlapping when the stride is below the block): the
+    linear map W_K, W_V, or the compression perceptron ``cmp_mlp`` (a dict of
+    its weights, see ``_cmp_mlp``)."""
     k, v = _f32(k), _f32(v)
     isv = np.ascontiguousarray(is_vision, dtype=np.uint8)
     n = isv.shape[0]
-    nb = int(isv.sum()) // p.block
+    nv = int(isv.sum())
+    stride = p.stride or p.block
+    nb = (nv - p.block) // stride + 1 if nv >= p.block else 0
     kc = np.zeros((max(nb, 0), p.h_kv, p.d), np.float64)
     vc = np.zeros_like(kc)
     cfg = _cfg(p, n)

@@ -8,7 +8,8 @@ implementation of the same definitions:
   * "VideoNSA: Native Sparse Attention Scales Video Understanding" (paper
     notes), section "Method": vision/text split, the three branches, the
     per-head sigmoid gate, dense GQA for text, outputs at original positions;
-  * the readings R1-R10 stated at the top of ``vnsa_oracle.c``.
+  * the readings R1-R10 and R13 (overlapping compression blocks) stated at
+    the top of ``vnsa_oracle.c``.
 
 The top-k step is not sorted here: every subset of the candidate blocks of the
 right size is enumerated and the unique subset whose members all beat all
@@ -73,11 +74,12 @@ def _topm(imp_by_block, candidates, m):
 
 def layer(q, k, v, is_vision, gate, w_k, w_v, *, h_q, h_kv, d, block, top_k,
           window, force_first=True, force_local=True, scale=None,
-          round_cmp_bf16=False):
+          round_cmp_bf16=False, stride=None):
     """All rows of the layer.  Array-likes are nested lists / numpy arrays:
     q [n][h_q][d], k, v [n][h_kv][d], gate [n][h_q][3], w_k, w_v [d][d].
-    Returns dict(out=[n][h_q][d], idx={(t, g): sorted list}, imp={(t,g):{j:val}},
-    o_cmp / o_slc / o_swa = {(t, h): vec})."""
+    ``stride``: compression stride (None: the block size).
+    Returns dict(out=[n][h_q][d], idx={(t, g): sorted list}, imp={(t,g):{j:val}}
+    (selection-block importance), o_cmp / o_slc / o_swa = {(t, h): vec})."""
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     n = len(is_vision)
@@ -91,11 +93,19 @@ def layer(q, k, v, is_vision, gate, w_k, w_v, *, h_q, h_kv, d, block, top_k,
     pos_of_rank = {i: t for t, i in vision_rank.items()}
     nv = len(vision_rank)
     nb = nv // block
+    stride = block if stride is None else stride
+    # Compression blocks: the vision ranks each one averages (they overlap
+    # when the stride is below the block size).
+    cmp_members = {}
+    c = 0
+    while c * stride + block <= nv:
+        cmp_members[c] = [c * stride + u for u in range(block)]
+        c += 1
     # Compression keys/values per (block, kv head): mean over the block's
     # tokens, then the row vector times W.
     kcmp, vcmp = {}, {}
-    for j in range(nb):
-        members = [pos_of_rank[j * block + u] for u in range(block)]
+    for j, ranks in cmp_members.items():
+        members = [pos_of_rank[u] for u in ranks]
         for g in range(h_kv):
             kbar = [sum(float(k[t][g][e]) for t in members) / block for e in range(d)]
             vbar = [sum(float(v[t][g][e]) for t in members) / block for e in range(d)]
@@ -119,16 +129,24 @@ def layer(q, k, v, is_vision, gate, w_k, w_v, *, h_q, h_kv, d, block, top_k,
             continue
         i = vision_rank[t]
         visible = [j for j in range(nb) if (j + 1) * block - 1 <= i]
+        cmp_visible = [cb for cb, ranks in cmp_members.items() if max(ranks) <= i]
         for g in range(h_kv):
             heads = [g * r + x for x in range(r)]
-            imp = {j: 0.0 for j in visible}
+            imp_cmp = {cb: 0.0 for cb in cmp_visible}
             per_head_cmp = {}
             for h in heads:
-                kv = {j: (kcmp[(j, g)], vcmp[(j, g)]) for j in visible}
+                kv = {cb: (kcmp[(cb, g)], vcmp[(cb, g)]) for cb in cmp_visible}
                 o, probs = _softmax_attend([float(x) for x in q[t][h]], kv, scale)
                 per_head_cmp[h] = o
-                for j, pr in probs.items():
-                    imp[j] += pr
+                for cb, pr in probs.items():
+                    imp_cmp[cb] += pr
+            # each compression block's mass goes to the selection blocks its
+            # tokens fall in, one token's share (1 / block) at a time
+            imp = {j: 0.0 for j in visible}
+            for cb, mass in imp_cmp.items():
+                for u in cmp_members[cb]:
+                    if u // block in imp:
+                        imp[u // block] += mass / block
             res["imp"][(t, g)] = imp
             forced = set()
             if force_first:

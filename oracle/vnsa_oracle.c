@@ -62,6 +62,17 @@
  *       the sigmoid of R8 turns it into the gate.  In bf16 runs the hidden
  *       activations are rounded to bf16 (round-to-nearest-even): they are the
  *       operand of the second product.
+ *   R13 Compression blocks may overlap (a compression stride s below the
+ *       block size B, the native sparse attention design the pages build on):
+ *       compression block c averages the B vision tokens [c s, c s + B), for
+ *       c = 0 .. nc-1 with nc = floor((N_v - B) / s) + 1, and is visible to
+ *       query i iff its last token c s + B - 1 is at or before i (R2 is the
+ *       case s = B).  Selection blocks stay the non-overlapping blocks of B
+ *       tokens.  The importance of selection block j is the group's
+ *       compression probability mass distributed over the selection blocks in
+ *       proportion to the tokens of each compression block that lie in them:
+ *       imp[j] = sum_c |[c s, c s + B) ^ [j B, j B + B)| / B * p_c.  With s = B
+ *       this is p_j, R4 unchanged.  Candidates and forced blocks follow R5.
  */
 #include <math.h>
 #include <stdint.h>
@@ -82,6 +93,7 @@ typedef struct {
     int force_local;    /* always keep the query's own block             */
     double scale;       /* softmax scale                                 */
     int round_cmp_bf16; /* round K_cmp / V_cmp to bf16 (R3)              */
+    int stride;         /* compression stride, 1..block (0: = block, R13) */
 } vnsa_oracle_cfg;
 
 enum { ORACLE_OK = 0, ORACLE_EINVAL = 1, ORACLE_ENOMEM = 2 };
@@ -183,11 +195,21 @@ static int partition(const uint8_t *is_vision, int n, int *vis)
     return nv;
 }
 
+/* Compression stride (R13): 0 means the block size. */
+static int cmp_stride(const vnsa_oracle_cfg *c) { return c->stride > 0 ? c->stride : c->block; }
+
+/* Number of compression blocks over nv vision tokens (R13). */
+static int cmp_blocks(const vnsa_oracle_cfg *c, int nv)
+{
+    return nv >= c->block ? (nv - c->block) / cmp_stride(c) + 1 : 0;
+}
+
 static int check_cfg(const vnsa_oracle_cfg *c)
 {
     if (!c || c->n < 0 || c->h_q <= 0 || c->h_kv <= 0 || c->d <= 0) return 0;
     if (c->h_q % c->h_kv != 0) return 0;
     if (c->block <= 0 || c->window <= 0 || c->top_k <= 0) return 0;
+    if (c->stride < 0 || c->stride > c->block) return 0;
     int forced = (c->force_first ? 1 : 0) + (c->force_local ? 1 : 0);
     if (c->top_k < forced) return 0;
     return 1;
@@ -196,15 +218,16 @@ static int check_cfg(const vnsa_oracle_cfg *c)
 /*
  * Compression keys/values [M], [A]: each block of B consecutive vision tokens
  * is averaged, and the mean is mapped to one block key / block value:
- *   Kbar_j = (1/B) sum_{u<B} K[vis[jB+u]],   K_cmp_j = Kbar_j . W_K   (R3),
- * per KV head, for the nb = floor(N_v/B) complete blocks.  Same for V.
- * k_cmp, v_cmp: [nb][h_kv][d].  Kd, Vd: fp64 copies of K, V [n][h_kv][d].
+ *   Kbar_j = (1/B) sum_{u<B} K[vis[j s + u]],   K_cmp_j = Kbar_j . W_K   (R3),
+ * per KV head, for the nb compression blocks (stride s = B unless R13).  Same
+ * for V.  k_cmp, v_cmp: [nb][h_kv][d].  Kd, Vd: fp64 copies of K, V
+ * [n][h_kv][d].
  */
 static void pool_proj(const vnsa_oracle_cfg *c, const double *Kd, const double *Vd,
                       const int *vis, int nb, const cmp_map *mk, const cmp_map *mv,
                       double *k_cmp, double *v_cmp)
 {
-    const int d = c->d, hk = c->h_kv, B = c->block;
+    const int d = c->d, hk = c->h_kv, B = c->block, S = cmp_stride(c);
     const int H = mk->hidden > mv->hidden ? mk->hidden : mv->hidden;
     #pragma omp parallel for schedule(static)
     for (int j = 0; j < nb; ++j) {
@@ -214,7 +237,7 @@ static void pool_proj(const vnsa_oracle_cfg *c, const double *Kd, const double *
         for (int g = 0; g < hk; ++g) {
             for (int e = 0; e < d; ++e) { kbar[e] = 0.0; vbar[e] = 0.0; }
             for (int u = 0; u < B; ++u) {
-                size_t row = ((size_t)vis[j * B + u] * hk + g) * d;
+                size_t row = ((size_t)vis[j * S + u] * hk + g) * d;
                 for (int e = 0; e < d; ++e) { kbar[e] += Kd[row + e]; vbar[e] += Vd[row + e]; }
             }
             for (int e = 0; e < d; ++e) { kbar[e] /= B; vbar[e] /= B; }
@@ -340,12 +363,13 @@ static int pool_impl(const vnsa_oracle_cfg *c, const float *k, const float *v,
     }
     for (size_t x = 0; x < (size_t)n * hk * d; ++x) { Kd[x] = k[x]; Vd[x] = v[x]; }
     int nv = partition(is_vision, n, vis);
-    pool_proj(c, Kd, Vd, vis, nv / c->block, &mk, &mv, k_cmp, v_cmp);
+    pool_proj(c, Kd, Vd, vis, cmp_blocks(c, nv), &mk, &mv, k_cmp, v_cmp);
     free(vis); free(Kd); free(Vd); free_cmp_map(&mk); free_cmp_map(&mv);
     return ORACLE_OK;
 }
 
-/* K_cmp / V_cmp only (for the pooling parity checks). Outputs [nb][h_kv][d]. */
+/* K_cmp / V_cmp only (for the pooling parity checks). Outputs [nc][h_kv][d],
+ * nc compression blocks (R13). */
 int vnsa_oracle_pool_proj(const vnsa_oracle_cfg *c, const float *k, const float *v,
                           const uint8_t *is_vision, const float *w_k, const float *w_v,
                           double *k_cmp, double *v_cmp)
@@ -418,8 +442,9 @@ int vnsa_oracle_gate_mlp(int n, int dm, int hidden, int n_out, const float *x, c
  *   o_cmp, o_slc, o_swa [n_rows][h_q][d] ungated branch outputs (vision rows)
  *   lse_cmp [n_rows][h_q]               compression log-sum-exp (-inf if empty)
  *   idx [n_rows][h_kv][top_k]           selected blocks (-1 for text rows)
- *   imp [n_rows][h_kv][nb]              block importance (0 beyond visibility)
- *   nb_out                              number of complete blocks
+ *   imp [n_rows][h_kv][nb]              selection-block importance (R4, R13; 0
+ *                                       beyond visibility)
+ *   nb_out                              number of complete selection blocks
  */
 static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k,
                         const float *v, const uint8_t *is_vision, const float *gate,
@@ -447,11 +472,13 @@ static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k
     const int nv = partition(is_vision, n, vis);
     for (int t = 0; t < n; ++t) vpos[t] = -1;
     for (int i = 0; i < nv; ++i) vpos[vis[i]] = i;
-    const int nb = nv / B;
+    const int nb = nv / B;            /* selection blocks */
+    const int S = cmp_stride(c);
+    const int nc = cmp_blocks(c, nv); /* compression blocks (nc = nb when S = B) */
     if (nb_out) *nb_out = nb;
-    double *k_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
-    double *v_cmp = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1) * hk * d);
-    pool_proj(c, Kd, Vd, vis, nb, &mk, &mv, k_cmp, v_cmp);
+    double *k_cmp = malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1) * hk * d);
+    double *v_cmp = malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1) * hk * d);
+    pool_proj(c, Kd, Vd, vis, nc, &mk, &mv, k_cmp, v_cmp);
 
     #pragma omp parallel
     {
@@ -460,6 +487,7 @@ static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k
         double *s = malloc(sizeof(double) * nn);
         double *p = malloc(sizeof(double) * nn);
         double *impg = malloc(sizeof(double) * (size_t)(nb > 0 ? nb : 1));
+        double *impc = malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
         char *taken = malloc((size_t)(nb > 0 ? nb : 1));
         int *sel = malloc(sizeof(int) * (size_t)K);
         double *qd = malloc(sizeof(double) * d);
@@ -489,22 +517,36 @@ static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k
                 if (imp) for (int x = 0; x < hk * nb; ++x) imp[(size_t)rr * hk * nb + x] = 0.0;
                 continue;
             }
-            /* R2: visible compressed blocks of vision query i. */
+            /* R2 / R13: visible compression blocks of vision query i (last
+             * token at or before i), and the complete selection blocks at or
+             * before i (the top-k candidates). */
+            int ncv = i >= B - 1 ? (i - B + 1) / S + 1 : 0;
+            if (ncv > nc) ncv = nc;
             int nvis = (i + 1) / B;
             if (nvis > nb) nvis = nb;
             for (int g = 0; g < hk; ++g) {
                 /* Compression branch and importance (R4). */
                 for (int j = 0; j < nb; ++j) impg[j] = 0.0;
-                for (int j = 0; j < nvis; ++j) keys[j] = j;
+                for (int x = 0; x < ncv; ++x) { impc[x] = 0.0; keys[x] = x; }
                 for (int hl = 0; hl < r; ++hl) {
                     const int h = g * r + hl;
                     for (int e = 0; e < d; ++e) qd[e] = q[((size_t)t * hq + h) * d + e];
                     double lse = attend(qd, k_cmp + (size_t)g * d, v_cmp + (size_t)g * d,
-                                        (size_t)hk * d, keys, nvis, d, c->scale, oc, p, s);
-                    for (int j = 0; j < nvis; ++j) impg[j] += p[j];
+                                        (size_t)hk * d, keys, ncv, d, c->scale, oc, p, s);
+                    for (int x = 0; x < ncv; ++x) impc[x] += p[x];
                     if (lse_cmp) lse_cmp[(size_t)rr * hq + h] = lse;
                     memcpy(orow + (size_t)h * d, oc, sizeof(double) * d); /* park o_cmp */
                     if (o_cmp) memcpy(o_cmp + ((size_t)rr * hq + h) * d, oc, sizeof(double) * d);
+                }
+                /* R13: each compression block's mass to the selection blocks
+                 * its tokens lie in, in proportion (the identity when S = B). */
+                for (int x = 0; x < ncv; ++x) {
+                    const int a0 = x * S, a1 = x * S + B; /* tokens [a0, a1) */
+                    for (int j = a0 / B; j <= (a1 - 1) / B && j < nb; ++j) {
+                        const int lo2 = a0 > j * B ? a0 : j * B;
+                        const int hi2 = a1 < (j + 1) * B ? a1 : (j + 1) * B;
+                        impg[j] += (double)(hi2 - lo2) / B * impc[x];
+                    }
                 }
                 if (imp) memcpy(imp + ((size_t)rr * hk + g) * nb, impg, sizeof(double) * nb);
                 /* Selection of blocks (R5), or the caller's forced indices. */
@@ -544,7 +586,7 @@ static int forward_impl(const vnsa_oracle_cfg *c, const float *q, const float *k
                 }
             }
         }
-        free(keys); free(s); free(p); free(impg); free(taken); free(sel);
+        free(keys); free(s); free(p); free(impg); free(impc); free(taken); free(sel);
         free(qd); free(oc); free(os); free(ow);
     }
     free(vis); free(vpos); free(Kd); free(Vd); free(k_cmp); free(v_cmp);
