@@ -63,9 +63,9 @@ typedef struct vnsa_config {
     int n_max;        /* largest n a forward will see (sizes the workspace)     */
     int h_q, h_kv;    /* query heads, KV heads; h_q % h_kv == 0, h_q/h_kv <= 16  */
     int d;            /* head dim: 64 or 128                                    */
-    int block;        /* compression block = stride = selection block, >= 1:   */
-                      /* the vision tokens per frame (64 in the pages' setting; */
-                      /* the pages treat tokens per frame as a task knob).      */
+    int block;        /* compression block = selection block, >= 1: the vision */
+                      /* tokens per frame (64 in the pages' setting; the pages  */
+                      /* treat tokens per frame as a task knob).                */
                       /* Every block size runs on the GPU; the tensor-core      */
                       /* path takes bf16, d 128, 4..16 query heads per KV head  */
                       /* and a selection of at most 1152 64-key tiles per 128-  */
@@ -76,6 +76,15 @@ typedef struct vnsa_config {
     int force_local;  /* 1: the query's own block is always selected (def. 1)   */
     float scale;      /* softmax scale; 0 -> 1/sqrt(d)                          */
     vnsa_dtype dtype; /* storage type of q, k, v, w, out                        */
+    int cmp_stride;   /* compression stride, 1..block; 0 -> block.  Below the   */
+                      /* block size the compression blocks overlap (the native  */
+                      /* sparse attention design the pages build on): block c   */
+                      /* averages vision tokens [c*s, c*s + block) and is       */
+                      /* visible to query i once its last token is <= i; the    */
+                      /* importance of selection block j is the compression     */
+                      /* mass spread over the selection blocks by the tokens    */
+                      /* each compression block puts in them.  vnsa_decode      */
+                      /* takes cmp_stride = block only.                         */
 } vnsa_config;
 
 typedef struct vnsa_handle vnsa_handle;
@@ -92,11 +101,13 @@ typedef struct vnsa_debug {
     float *o_swa;            /* [n][h_q][d] ungated window output, by position       */
     float *lse_cmp;          /* [n][h_q] compression log-sum-exp (natural log), rank */
     int32_t *idx;            /* [h_kv][n][top_k] selected blocks, ascending, -1 pad  */
-    float *imp;              /* [h_kv][n][imp_stride] importance; only the visible
-                                blocks j < (i+1)/block of row i are written          */
+    float *imp;              /* [h_kv][n][imp_stride] selection-block importance;
+                                only the visible blocks j < (i+1)/block of row i
+                                are written                                          */
     int imp_stride;          /* row stride of imp in floats (>= n / block)           */
-    void *k_cmp;             /* [nb][h_kv][d] dtype block keys                       */
-    void *v_cmp;             /* [nb][h_kv][d] dtype block values                     */
+    void *k_cmp;             /* [nc][h_kv][d] dtype block keys (nc compression
+                                blocks: nb when cmp_stride = block)                  */
+    void *v_cmp;             /* [nc][h_kv][d] dtype block values                     */
     const int32_t *forced_idx; /* input [h_kv][n][top_k]: used instead of the top-k  */
 } vnsa_debug;
 
@@ -206,7 +217,8 @@ vnsa_status vnsa_host_join(vnsa_handle *h, void *stream);
  * token).  The handle's workspace keeps the stream's vision/text lists and the
  * block keys/values; the step extends them (pooling the block the token
  * completes, if any).  n <= n_max.  Asynchronous on `stream`; device-detected
- * errors go to the status word.
+ * errors go to the status word.  A handle whose cmp_stride is below its block
+ * returns VNSA_ERR_UNSUPPORTED.
  */
 vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k, const void *v,
                         const uint8_t *is_vision, const float *gate_new, void *out_new,

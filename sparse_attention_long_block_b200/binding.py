@@ -35,7 +35,7 @@ class vnsa_config(ctypes.Structure):
                 ("d", ctypes.c_int), ("block", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("window", ctypes.c_int), ("force_first", ctypes.c_int),
                 ("force_local", ctypes.c_int), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("cmp_stride", ctypes.c_int)]
 
 
 class vnsa_debug(ctypes.Structure):
@@ -226,7 +226,7 @@ class Layer:
     """One configured layer (a vnsa handle) fed with torch CUDA tensors."""
 
     def __init__(self, *, n_max, h_q, h_kv, d, top_k, window, w_k, w_v, block=64,
-                 force_first=True, force_local=True, scale=0.0, dtype="bf16"):
+                 force_first=True, force_local=True, scale=0.0, dtype="bf16", stride=0):
         import torch
         if not torch.cuda.is_available():
             raise RuntimeError("vnsa needs a CUDA device; there is no CPU path")
@@ -234,7 +234,8 @@ class Layer:
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         self.cfg = vnsa_config(int(n_max), int(h_q), int(h_kv), int(d), int(block), int(top_k),
                                int(window), int(bool(force_first)), int(bool(force_local)),
-                               float(scale), VNSA_BF16 if dtype == "bf16" else VNSA_FP32)
+                               float(scale), VNSA_BF16 if dtype == "bf16" else VNSA_FP32,
+                               int(stride))
         self.h_q, self.h_kv, self.d, self.top_k, self.block = h_q, h_kv, d, top_k, block
         w_k = self._dev(w_k)
         w_v = self._dev(w_v)
@@ -385,11 +386,13 @@ class Layer:
             pass
 
 
-def make_debug(n, h_q, h_kv, d, top_k, block=64, dtype=None, want=(), forced_idx=None):
+def make_debug(n, h_q, h_kv, d, top_k, block=64, dtype=None, want=(), forced_idx=None,
+               stride=0):
     """Allocate the requested debug exports as torch CUDA tensors.
 
     Returns (vnsa_debug struct, dict of tensors).  ``forced_idx``
-    [h_kv][n][top_k] int32 CUDA tensor overrides the top-k."""
+    [h_kv][n][top_k] int32 CUDA tensor overrides the top-k.  ``stride``: the
+    compression stride (0: the block), which sets the rows of k_cmp / v_cmp."""
     import torch
     dev = "cuda"
     t = {}
@@ -409,9 +412,11 @@ def make_debug(n, h_q, h_kv, d, top_k, block=64, dtype=None, want=(), forced_idx
         t["imp"] = torch.zeros((h_kv, n, stride), dtype=torch.float32, device=dev)
         dbg.imp = t["imp"].data_ptr()
         dbg.imp_stride = stride
+    s = stride or block
+    n_cmp = (n - block) // s + 1 if n >= block else 0
     for name in ("k_cmp", "v_cmp"):
         if name in want:
-            t[name] = torch.zeros((max(1, n // block), h_kv, d), dtype=dtype, device=dev)
+            t[name] = torch.zeros((max(1, n_cmp), h_kv, d), dtype=dtype, device=dev)
             setattr(dbg, name, t[name].data_ptr())
     if forced_idx is not None:
         t["forced_idx"] = forced_idx

@@ -27,7 +27,16 @@ struct Counts {
     int pad[3];      // (decode step state)
     int txt_contiguous;  // 1 if the text tokens are one run of positions
     int txt_base;        // position of the first text token (if contiguous)
+    int nc;              // compression blocks (N_v - block) / stride + 1 (= nb at stride block)
 };
+
+// Compression blocks visible to vision query i: those whose last token
+// c*S + B - 1 is at or before i, at most nc.  With S = B this is (i + 1) / B.
+__host__ __device__ __forceinline__ int cmp_visible(int i, int B, int S, int nc) {
+    if (i < B - 1) return 0;
+    const int c = (i - B + 1) / S + 1;
+    return c < nc ? c : nc;
+}
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }

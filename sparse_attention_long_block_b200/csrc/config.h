@@ -11,6 +11,14 @@ namespace vnsa {
 
 constexpr int kMaxTokens = 262144;  // tokens per call (n_max, or n without a handle)
 
+// The compression stride of a config (0 stands for the block size).
+inline int cmp_stride_of(const vnsa_config &c) { return c.cmp_stride > 0 ? c.cmp_stride : c.block; }
+
+// Compression blocks over n vision tokens: [c*s, c*s + block) for c < this.
+inline int cmp_blocks(int n, int block, int stride) {
+    return n >= block ? (n - block) / stride + 1 : 0;
+}
+
 // Argument errors (VNSA_ERR_INVALID_ARG) first, then layers that are valid
 // but not implemented (VNSA_ERR_UNSUPPORTED).  `n` is the token count the
 // workspace is sized for: cfg->n_max for a handle, the call's n otherwise.
@@ -23,6 +31,7 @@ inline vnsa_status check_config(const vnsa_config *c, int n) {
         (c->force_local != 0 && c->force_local != 1))
         return VNSA_ERR_INVALID_ARG;
     if (c->top_k < c->force_first + c->force_local) return VNSA_ERR_INVALID_ARG;
+    if (c->cmp_stride < 0 || c->cmp_stride > c->block) return VNSA_ERR_INVALID_ARG;
     if (!(c->scale >= 0.f) || isinf(c->scale)) return VNSA_ERR_INVALID_ARG;
     if (c->dtype != VNSA_BF16 && c->dtype != VNSA_FP32) return VNSA_ERR_INVALID_ARG;
     if (n > kMaxTokens) return VNSA_ERR_UNSUPPORTED;

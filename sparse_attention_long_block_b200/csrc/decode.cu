@@ -207,6 +207,7 @@ __global__ void decode_prep_kernel(DecodeParams p) {
         }
         cn.n_vision = i + 1;
         cn.nb = cn.n_vision / p.block;
+        cn.nc = cn.nb;  // decode runs with the compression stride equal to the block
         cn.pad[0] = (cn.n_vision % p.block == 0) ? cn.nb - 1 : cn.nb;  // block to pool
         cn.pad[1] = 1;
         cn.pad[2] = i;
@@ -524,7 +525,8 @@ cudaError_t launch_decode(int dtype, const DecodeParams &p, cudaStream_t s, int 
     decode_prep_kernel<<<1, 32, 0, s>>>(p);
     ++*launches;
     cudaError_t e = launch_pool_proj(dtype, p.d, p.k, p.v, p.vis, p.counts, p.w_k, p.w_v,
-                                     p.k_cmp, p.v_cmp, p.h_kv, p.block, p.nb_max, s, 1, &p.mlp);
+                                     p.k_cmp, p.v_cmp, p.h_kv, p.block, p.block, p.nb_max, s,
+                                     1, &p.mlp);
     ++*launches;
     if (e != cudaSuccess) return e;
     if (dtype == VNSA_BF16 && p.d == 128) return launch_r<__nv_bfloat16, 128>(p, s, launches);

@@ -12,7 +12,8 @@ namespace vnsa {
 // Everything one forward needs, passed by value to the kernels.
 struct LayerParams {
     int n, n_max, h_q, h_kv, d, r, block, top_k, window, force_first, force_local;
-    int nb_max;
+    int stride;                       // compression stride (block: no overlap)
+    int nb_max;                       // capacity in compression blocks (K_cmp, imp rows)
     float scale_log2;                 // softmax scale * log2(e)
     const void *q, *k, *v;            // [n][h][d] dtype
     const uint8_t *is_vision;         // [n]
@@ -23,8 +24,10 @@ struct LayerParams {
     uint32_t *status;
     const void *k_cmp, *v_cmp;        // [nb][h_kv][d] dtype
     float *lse;                       // [n_max][h_q] natural-log LSE of compression
-    float *imp;                       // [h_kv][n_max][imp_stride]
+    float *imp;                       // [h_kv][n_max][imp_stride] compression-block importance
     size_t imp_stride;
+    float *imp_sel;                   // [h_kv][n_max][imp_sel_stride] selection-block
+    size_t imp_sel_stride;            // importance (top-k input); = imp at stride block
     int32_t *idx;                     // [h_kv][n_max][top_k] (workspace)
     const int32_t *idx_src;           // selection read by the selection branch
     size_t idx_rows;                  // rows per group of idx_src
@@ -33,8 +36,8 @@ struct LayerParams {
     unsigned long long wait_ns;       // limit of the kernels' bounded waits (0: default)
 };
 
-cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t *vis,
-                             int32_t *txt, Counts *counts, cudaStream_t s);
+cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int stride,
+                             int32_t *vis, int32_t *txt, Counts *counts, cudaStream_t s);
 
 // The compression branch's perceptron (when hidden > 0): K_cmp = SiLU(mean .
 // w1 + b1) . w2 + b2, w1 [d][hidden], w2 [hidden][d] in the layer dtype, b1, b2
@@ -50,7 +53,7 @@ struct CmpMlp {
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s, int from_pad = 0,
+                             int stride, int nb_max, cudaStream_t s, int from_pad = 0,
                              const CmpMlp *mlp = nullptr);
 
 // Gate logits [n][n_out] fp32 of the layer input x [n][dm] through the gate
@@ -62,6 +65,10 @@ cudaError_t launch_gate_mlp(int dtype, int n, int dm, int hidden, int n_out, con
                             float *out, uint32_t *status, cudaStream_t s, int *launches);
 
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s);
+
+// Selection-block importance (imp_sel) from the compression-block importance
+// (imp) when the compression blocks overlap (stride < block).
+cudaError_t launch_imp_remap(const LayerParams &p, cudaStream_t s);
 
 // Copies of workspace tensors into the optional debug buffers of vnsa_debug.
 cudaError_t launch_export(const LayerParams &p, int esize, float *lse_out, int32_t *idx_out,

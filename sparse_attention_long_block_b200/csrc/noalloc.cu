@@ -47,24 +47,28 @@ constexpr size_t kScratchHeader = 256;  // intermediates start after it
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct ScratchPlan {
-    size_t vis, txt, counts, k_cmp, v_cmp, lse, imp, total;
-    size_t imp_stride;
+    size_t vis, txt, counts, k_cmp, v_cmp, lse, imp, imp_sel, total;
+    size_t imp_stride, imp_sel_stride;
 };
 
 ScratchPlan plan_for(const vnsa_config &c, int n) {
     const size_t es = c.dtype == VNSA_BF16 ? 2 : 4;
-    const size_t nb = (size_t)(n / c.block);
+    const size_t nb = (size_t)(n / c.block);  // selection blocks
+    const int stride = vnsa::cmp_stride_of(c);
+    const size_t nc = (size_t)vnsa::cmp_blocks(n, c.block, stride);  // compression blocks
     ScratchPlan s;
-    s.imp_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
+    s.imp_stride = nc > 0 ? (nc + 3) / 4 * 4 : 4;
+    s.imp_sel_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
     size_t off = kScratchHeader;
     auto take = [&](size_t b) { size_t o = off; off += up256(b > 0 ? b : 1); return o; };
     s.vis = take((size_t)n * 4);
     s.txt = take((size_t)n * 4);
     s.counts = take(sizeof(vnsa::Counts));
-    s.k_cmp = take(nb * c.h_kv * c.d * es);
-    s.v_cmp = take(nb * c.h_kv * c.d * es);
+    s.k_cmp = take(nc * c.h_kv * c.d * es);
+    s.v_cmp = take(nc * c.h_kv * c.d * es);
     s.lse = take((size_t)n * c.h_q * 4);
     s.imp = take((size_t)c.h_kv * n * s.imp_stride * 4);
+    s.imp_sel = stride != c.block ? take((size_t)c.h_kv * n * s.imp_sel_stride * 4) : s.imp;
     s.total = off;
     return s;
 }
@@ -124,11 +128,12 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
     p.d = c.d;
     p.r = c.h_q / c.h_kv;
     p.block = c.block;
+    p.stride = cmp_stride_of(c);
     p.top_k = c.top_k;
     p.window = c.window;
     p.force_first = c.force_first;
     p.force_local = c.force_local;
-    p.nb_max = n / c.block;
+    p.nb_max = cmp_blocks(n, c.block, p.stride);
     p.scale_log2 = scale * kLog2e;
     p.q = q;
     p.k = k;
@@ -143,6 +148,8 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
     p.lse = (float *)(base + s.lse);
     p.imp = (float *)(base + s.imp);
     p.imp_stride = s.imp_stride;
+    p.imp_sel = (float *)(base + s.imp_sel);
+    p.imp_sel_stride = s.imp_sel == s.imp ? s.imp_stride : s.imp_sel_stride;
     p.idx = idx;  // caller's output [h_kv][n][top_k]
     p.idx_src = idx;
     p.idx_rows = (size_t)n;
@@ -152,12 +159,13 @@ extern "C" vnsa_status vnsa_select_noalloc(const vnsa_config *cfg, int n, const 
     // start at zero (the kernels overwrite everything else they later read).
     cudaError_t e = cudaMemsetAsync(base + kStatusOffset, 0, 16, st);
     if (e == cudaSuccess)
-        e = launch_partition(is_vision, n, c.block, (int32_t *)p.vis, (int32_t *)p.txt,
+        e = launch_partition(is_vision, n, c.block, p.stride, (int32_t *)p.vis, (int32_t *)p.txt,
                              (Counts *)p.counts, st);
     if (e == cudaSuccess)
         e = launch_pool_proj(dt, c.d, k, v, p.vis, p.counts, w_k, w_v, (void *)p.k_cmp,
-                             (void *)p.v_cmp, c.h_kv, c.block, p.nb_max, st);
+                             (void *)p.v_cmp, c.h_kv, c.block, p.stride, p.nb_max, st);
     if (e == cudaSuccess) e = launch_cmp_simt(dt, p, st);
+    if (e == cudaSuccess && p.stride != p.block) e = launch_imp_remap(p, st);
     if (e == cudaSuccess) e = launch_topk(p, st);
     if (e != cudaSuccess) {
         cudaGetLastError();

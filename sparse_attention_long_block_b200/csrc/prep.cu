@@ -18,7 +18,7 @@ namespace vnsa {
 // vis[i] = position of the i-th vision token, txt[x] = position of the x-th
 // text token.
 __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restrict__ isv,
-                                                         int n, int block,
+                                                         int n, int block, int stride,
                                                          int32_t *__restrict__ vis,
                                                          int32_t *__restrict__ txt,
                                                          Counts *counts) {
@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restri
         cn.n_vision = nv;
         cn.n_text = nt;
         cn.nb = nv / block;
+        cn.nc = nv >= block ? (nv - block) / stride + 1 : 0;
         cn.vis_base = nv > 0 ? vis[0] : 0;
         cn.contiguous = (nv == 0) || (vis[nv - 1] - vis[0] == nv - 1);
         cn.pad[0] = cn.pad[1] = cn.pad[2] = 0;
@@ -85,16 +86,18 @@ __global__ void __launch_bounds__(1024) partition_kernel(const uint8_t *__restri
     }
 }
 
-cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int32_t *vis,
-                             int32_t *txt, Counts *counts, cudaStream_t s) {
-    partition_kernel<<<1, 1024, 0, s>>>(is_vision, n, block, vis, txt, counts);
+cudaError_t launch_partition(const uint8_t *is_vision, int n, int block, int stride,
+                             int32_t *vis, int32_t *txt, Counts *counts, cudaStream_t s) {
+    partition_kernel<<<1, 1024, 0, s>>>(is_vision, n, block, stride, vis, txt, counts);
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Pool + projection.  CTA (tile of JB blocks, KV head g, K or V): mean of each
-// block's `block` vision rows in fp32, then mean . W (d x d) and one rounding
-// to the storage type.  Rows are read with vector loads, one row per warp step.
+// Pool + projection.  CTA (tile of JB compression blocks, KV head g, K or V):
+// mean of each block's `block` vision rows in fp32 (block j starts at vision
+// rank j * stride: the blocks overlap when stride < block), then mean . W
+// (d x d) and one rounding to the storage type.  Rows are read with vector
+// loads, one row per warp step.
 template <typename T, int PER>
 __device__ __forceinline__ void load_row_part(const T *p, float (&x)[PER]) {
     if constexpr (sizeof(T) == 2 && PER == 4) {
@@ -118,13 +121,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_proj_kernel(
     const T *__restrict__ k, const T *__restrict__ v, const int32_t *__restrict__ vis,
     const Counts *__restrict__ counts, const T *__restrict__ w_k, const T *__restrict__ w_v,
-    T *__restrict__ k_cmp, T *__restrict__ v_cmp, int h_kv, int block, int from_pad) {
+    T *__restrict__ k_cmp, T *__restrict__ v_cmp, int h_kv, int block, int stride,
+    int from_pad) {
     constexpr int JB = 16;             // blocks per CTA
     constexpr int PER = D / 32;        // elements per lane in a row
     constexpr int NPART = 256 / D;     // threads per output column
     constexpr int JBP = JB / NPART;    // blocks per thread in the projection
     __shared__ float mean[JB][D];
-    const int nb = counts->nb;
+    const int nb = counts->nc;
     // from_pad: only the blocks from counts->pad[0] on (the block a decode
     // step completed, or none)
     const int j0 = (from_pad ? counts->pad[0] : 0) + blockIdx.x * JB;
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(256) pool_proj_kernel(
 #pragma unroll
         for (int c = 0; c < PER; ++c) acc[c] = 0.f;
         if (j < nb) {
-            const int32_t *rows = vis + (size_t)j * block;
+            const int32_t *rows = vis + (size_t)j * stride;
 #pragma unroll 8
             for (int u = 0; u < block; ++u) {
                 const T *p = src + ((size_t)rows[u] * h_kv + g) * D + lane * PER;
@@ -183,14 +187,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) pool_mlp_kernel(
     const T *__restrict__ k, const T *__restrict__ v, const int32_t *__restrict__ vis,
     const Counts *__restrict__ counts, CmpMlp mlp, T *__restrict__ k_cmp,
-    T *__restrict__ v_cmp, int h_kv, int block, int from_pad) {
+    T *__restrict__ v_cmp, int h_kv, int block, int stride, int from_pad) {
     constexpr int JB = 16;
     constexpr int PER = D / 32;
     constexpr int NPART = 256 / D;
     constexpr int JBP = JB / NPART;
     __shared__ float mean[JB][D];
     __shared__ float hid[JB][kCmpMlpMaxHidden];
-    const int nb = counts->nb;
+    const int nb = counts->nc;
     const int j0 = (from_pad ? counts->pad[0] : 0) + blockIdx.x * JB;
     if (j0 >= nb) return;
     const int g = blockIdx.y;
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(256) pool_mlp_kernel(
 #pragma unroll
         for (int c = 0; c < PER; ++c) acc[c] = 0.f;
         if (j < nb) {
-            const int32_t *rows = vis + (size_t)j * block;
+            const int32_t *rows = vis + (size_t)j * stride;
 #pragma unroll 8
             for (int u = 0; u < block; ++u) {
                 const T *p = src + ((size_t)rows[u] * h_kv + g) * D + lane * PER;
@@ -258,7 +262,8 @@ __global__ void __launch_bounds__(256) pool_mlp_kernel(
 cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
                              const int32_t *vis, const Counts *counts, const void *w_k,
                              const void *w_v, void *k_cmp, void *v_cmp, int h_kv, int block,
-                             int nb_max, cudaStream_t s, int from_pad, const CmpMlp *mlp) {
+                             int stride, int nb_max, cudaStream_t s, int from_pad,
+                             const CmpMlp *mlp) {
     if (nb_max <= 0) return cudaSuccess;
     dim3 grid(from_pad ? 1 : (nb_max + 15) / 16, h_kv, 2);
     if (mlp && mlp->hidden > 0) {
@@ -266,7 +271,7 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 #define VNSA_POOL_MLP(T, D)                                                              \
     pool_mlp_kernel<T, D><<<grid, 256, 0, s>>>((const T *)k, (const T *)v, vis, counts,  \
                                                *mlp, (T *)k_cmp, (T *)v_cmp, h_kv, block, \
-                                               from_pad)
+                                               stride, from_pad)
         if (dtype == VNSA_BF16 && d == 128) VNSA_POOL_MLP(__nv_bfloat16, 128);
         else if (dtype == VNSA_BF16 && d == 64) VNSA_POOL_MLP(__nv_bfloat16, 64);
         else if (dtype == VNSA_FP32 && d == 128) VNSA_POOL_MLP(float, 128);
@@ -278,7 +283,7 @@ cudaError_t launch_pool_proj(int dtype, int d, const void *k, const void *v,
 #define VNSA_POOL(T, D)                                                                  \
     pool_proj_kernel<T, D><<<grid, 256, 0, s>>>(                                         \
         (const T *)k, (const T *)v, vis, counts, (const T *)w_k, (const T *)w_v,         \
-        (T *)k_cmp, (T *)v_cmp, h_kv, block, from_pad)
+        (T *)k_cmp, (T *)v_cmp, h_kv, block, stride, from_pad)
     if (dtype == VNSA_BF16 && d == 128) VNSA_POOL(__nv_bfloat16, 128);
     else if (dtype == VNSA_BF16 && d == 64) VNSA_POOL(__nv_bfloat16, 64);
     else if (dtype == VNSA_FP32 && d == 128) VNSA_POOL(float, 128);
@@ -299,7 +304,8 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
     if (i >= cn.n_vision) return;
     int c = (i + 1) / p.block;
     if (c > cn.nb) c = cn.nb;
-    topk_select_row<true>(p.imp + ((size_t)g * p.n_max + i) * p.imp_stride, c, i / p.block,
+    topk_select_row<true>(p.imp_sel + ((size_t)g * p.n_max + i) * p.imp_sel_stride, c,
+                          i / p.block,
                           p.top_k, p.force_first, p.force_local, sh_buf[warp], lane,
                           p.idx + ((size_t)g * p.n_max + i) * p.top_k, p.status);
 }
@@ -307,6 +313,47 @@ __global__ void __launch_bounds__(256) topk_kernel(LayerParams p) {
 cudaError_t launch_topk(const LayerParams &p, cudaStream_t s) {
     dim3 grid((p.n_max + 7) / 8, p.h_kv);
     topk_kernel<<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+// Overlapping compression blocks (stride S < block B; "VideoNSA: Native Sparse
+// Attention Scales Video Understanding", paper notes, section "Method", and the
+// native sparse attention design it builds on): the importance of selection
+// block j is the group's compression probability mass spread over the
+// selection blocks by the tokens each compression block puts in them,
+//   imp_sel[j] = sum_c |[c S, c S + B) ^ [j B, j B + B)| / B * imp[c],
+// over the compression blocks c visible to the query (last token <= i); only
+// the selection blocks j < (i + 1) / B (the top-k candidates) are written.
+// One warp per (group, vision query), lanes over j.
+__global__ void __launch_bounds__(256) imp_remap_kernel(LayerParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 8 + warp;
+    const int g = blockIdx.y;
+    const Counts cn = *p.counts;
+    if (i >= cn.n_vision) return;
+    const int B = p.block, S = p.stride;
+    const int ncv = cmp_visible(i, B, S, cn.nc);
+    const int nsel = min((i + 1) / B, cn.nb);
+    const float *src = p.imp + ((size_t)g * p.n_max + i) * p.imp_stride;
+    float *dst = p.imp_sel + ((size_t)g * p.n_max + i) * p.imp_sel_stride;
+    const float inv_b = 1.f / (float)B;
+    for (int j = lane; j < nsel; j += 32) {
+        const int a = j * B, b = a + B;             // tokens of selection block j
+        int c0 = a - B + 1 > 0 ? (a - B + 1 + S - 1) / S : 0;  // first c with c S + B > a
+        int c1 = (b - 1) / S;                       // last c with c S < b
+        if (c1 > ncv - 1) c1 = ncv - 1;
+        float acc = 0.f;
+        for (int c = c0; c <= c1; ++c) {
+            const int lo = max(c * S, a), hi = min(c * S + B, b);
+            acc = fmaf((float)(hi - lo) * inv_b, src[c], acc);
+        }
+        dst[j] = acc;
+    }
+}
+
+cudaError_t launch_imp_remap(const LayerParams &p, cudaStream_t s) {
+    dim3 grid((p.n_max + 7) / 8, p.h_kv);
+    imp_remap_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -340,10 +387,10 @@ __global__ void export_kernel(LayerParams p, int esize, float *lse_out, int32_t 
             const size_t g = gi / nv, i = gi % nv;
             if ((int)j < (int)((i + 1) / p.block))
                 imp_out[(g * p.n + i) * imp_stride_out + j] =
-                    p.imp[(g * p.n_max + i) * p.imp_stride + j];
+                    p.imp_sel[(g * p.n_max + i) * p.imp_sel_stride + j];
         }
     }
-    const size_t words = nb * p.h_kv * p.d * esize / 4;
+    const size_t words = (size_t)cn.nc * p.h_kv * p.d * esize / 4;
     if (kc_out)
         for (size_t x = tid; x < words; x += step) kc_out[x] = ((const uint32_t *)p.k_cmp)[x];
     if (vc_out)

@@ -84,7 +84,8 @@ __device__ __forceinline__ void load_query(float *qs, const T *qrow, float mul, 
 // Compression attention over the block keys/values, with exact probabilities
 // (two passes: log-sum-exp, then p = exp(s - lse)) so that the importance of
 // block j for group g, sum over the group's heads of p_h[j], can be summed.
-// Block j is visible to vision query i iff (j+1)*B - 1 <= i.
+// Block j is visible to vision query i iff its last token j*S + B - 1 <= i
+// (S = B unless the compression blocks overlap).
 template <typename T, int D>
 __global__ void cmp_simt_kernel(LayerParams p) {
     extern __shared__ float smem[];
@@ -96,8 +97,7 @@ __global__ void cmp_simt_kernel(LayerParams p) {
     const int t = p.vis[i];
     float *imp_s = smem;                              // [nb_max]
     float *qs = smem + p.nb_max + warp * D;           // [r][D]
-    int c = (i + 1) / p.block;
-    if (c > cn.nb) c = cn.nb;
+    const int c = cmp_visible(i, p.block, p.stride, cn.nc);
     load_query<T, D>(qs, (const T *)p.q + ((size_t)t * p.h_q + h) * D, p.scale_log2, lane);
     __syncthreads();
     const size_t stride = (size_t)p.h_kv * D;

@@ -18,20 +18,23 @@
 //              O += P V (M 128, N 128, K 64, fp16, P read from TMEM);
 //   warps 2-5  one thread per row: S row from TMEM, mask, softmax, P (fp16)
 //              into the same TMEM buffer, lazy O rescaling, epilogue.
+// P V takes fp16 operands: P keeps 11 significant bits (bf16 would keep 8,
+// which costs up to ~6e-3 of output error).  V and V_cmp enter as fp16 copies
+// divided by a power of two chosen per call from their largest magnitude, so
+// no bf16 value overflows fp16; the epilogues multiply that power back.
 // Modes:
 //   CMP   keys = compressed blocks.  Segment 1: each row's log-sum-exp.
 //         Segment 2: exact probabilities, their sum over the group's heads
 //         (the block importance, a warp reduce-scatter: rows are 16 queries x
 //         8 head slots) and O = P V, already normalised.
 //   SLC   the union of the blocks the item's queries selected; a row masks the
-//         blocks its query did not select.  Epilogue: the fp16 gated partial
+//         blocks its query did not select.  Epilogue: the fp32 gated partial
 //         (sig(g_cmp) o_cmp so far) gains sig(g_slc) o_slc.  With block 64 the
-//         tiles only one of the item's queries reaches are left to SGL, and the
-//         epilogue writes the normalised output and log-sum-exp for the merge.
-//   SGL   one 64-key tile per item; rows = up to 128 / r (query, tile) pairs
-//         of that tile x the group's r heads, Q rows gathered per row; per
-//         pair the normalised output and log-sum-exp.
-//   SWA   the window keys; epilogue: out = partial + sig(g_swa) o_swa (bf16).
+//         tiles only one of the item's queries reaches are attended by the
+//         tile-major pass (sgl_attn.cu) beforehand; the epilogue merges their
+//         normalised outputs with the union's softmax by log-sum-exp weights.
+//   SWA   the window keys; epilogue: out = partial + sig(g_swa) o_swa, the one
+//         rounding of the vision row (to bf16).
 //   TEXT  items = (text query tile, key split); partial O, max and sum to a
 //         buffer that a small combine kernel reduces (or the row directly).
 #include <cuda.h>
@@ -40,6 +43,8 @@
 #include <algorithm>
 #include <string.h>
 
+#include "config.h"
+#include "sgl_attn.h"
 #include "tc_attn.h"
 #include "tc_ptx.cuh"
 
@@ -84,17 +89,17 @@ constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;
 // whole tile or none of it (MODE_SLC); otherwise a tile holds parts of several
 // blocks and each row's keys are the parts of its own selected blocks
 // (MODE_SLC_UNALIGNED).
-enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3, MODE_SLC_UNALIGNED = 4,
-            MODE_SGL = 5 };
+enum Mode { MODE_CMP = 0, MODE_SLC = 1, MODE_SWA = 2, MODE_TEXT = 3, MODE_SLC_UNALIGNED = 4 };
 __host__ __device__ constexpr bool is_slc(int m) {
     return m == MODE_SLC || m == MODE_SLC_UNALIGNED;
 }
-enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4, K_SGL = 5 };
+enum Kind { K_STATS = 0, K_EXACT = 1, K_SLC = 2, K_SWA = 3, K_TEXT = 4 };
 
 struct TcParams {
-    CUtensorMap tm_k, tm_v;    // K (bf16, the caller's) and V (fp16 copy): [n rows][h_kv*d]
-    CUtensorMap tm_kc, tm_vc;  // compacted vision K (bf16), V (fp16), if not contiguous
-    CUtensorMap tm_kb, tm_vb;  // K_cmp (bf16), V_cmp (fp16): [nb_max rows][h_kv*d]
+    CUtensorMap tm_k, tm_v;    // K (bf16, the caller's) and V (scaled fp16 copy): [n rows][h_kv*d]
+    CUtensorMap tm_kc, tm_vc;  // compacted vision K (bf16), V (scaled fp16), if not contiguous
+    CUtensorMap tm_kb, tm_vb;  // K_cmp (bf16), V_cmp (scaled fp16): [nb_max rows][h_kv*d]
+    const float *v_scale;      // [0]: the power of two V was divided by, [1]: V_cmp's
     CUtensorMap tm_q;          // Q (bf16) as [n][h_q][d], box {64, rows per query, queries}
     LayerParams L;
     const int32_t *plan;       // SLC: [item][1 + 2*plan_max]
@@ -104,18 +109,14 @@ struct TcParams {
     int mode;
     // Selection tiles that a single query of an item reaches (block 64 only):
     // the union kernel takes them out of the item's plan and records each
-    // (query, tile) pair; MODE_SGL attends them tile-major, up to 128 / r pairs
-    // of one tile per item (18 for 7 heads per group), and the merge kernel
-    // folds them into the selection output.
+    // (query, tile) pair; the tile-major pass (sgl_attn.cu) attends them, and
+    // the selection epilogue merges each query's pairs into its output.
     int sgl_on;                // 1: the selection branch runs split this way
-    int sgl_nbt;               // 64-key tiles per group (bucket stride)
-    const int32_t *sgl_meta;   // [0] pairs, [1] items, then hist, off [h_kv*nbt], choff [+1]
-    const int4 *sgl_sorted;    // pairs grouped by bucket: (pair id, vision rank, position, 0)
-    const int4 *sgl_items;     // per item: (bucket, first entry of sgl_sorted, pairs, 0)
-    __half *sgl_o;             // [pair][r][d] normalised output of the pair's tile
-    float *sgl_lse;            // [pair][r] its log-sum-exp (log2 units)
-    __half *slc_u;             // [n_max][h_q][d] normalised output of the union tiles
-    float *slc_lse;            // [n_max][h_q] their log-sum-exp (log2 units)
+    const int32_t *sgl_of;     // [h_kv][n_max][top_k] pair ids of each query
+    const int32_t *sgl_n;      // [h_kv][n_max] how many
+    const __half *sgl_o;       // [pair][r][d] normalised output / its scale (fp16)
+    const float *sgl_lse;      // [pair][r] log-sum-exp of the pair's keys (log2 units)
+    const float *sgl_scale;    // [pair][r] the power of two the stored row was divided by
 };
 
 __host__ __device__ __forceinline__ int pow2_at_least(int r) {
@@ -146,7 +147,7 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
     const LayerParams &L = P.L;
     w.rpad = MODE == MODE_CMP ? pow2_at_least(L.r) : L.r;
     w.qt = kRows / w.rpad;
-    w.nb = cn.nb;
+    w.nb = MODE == MODE_CMP ? cn.nc : cn.nb;  // compression blocks for CMP
     w.contiguous = cn.contiguous;
     w.vis_base = cn.vis_base;
     w.q_tma = MODE == MODE_TEXT ? cn.txt_contiguous : cn.contiguous;
@@ -164,11 +165,6 @@ __device__ __forceinline__ Work make_work(const TcParams &P, const Counts &cn) {
         const int per = (span + w.nsplit - 1) / w.nsplit;
         w.split_len = (per + kKeys - 1) / kKeys * kKeys;
         w.items = tiles * w.nsplit;
-    } else if (MODE == MODE_SGL) {
-        w.n_q = cn.n_vision;
-        w.n_tiles_q = 0;
-        w.q_tma = 0;  // Q rows are gathered: the item's queries are scattered
-        w.items = P.sgl_meta[1];
     } else {
         w.n_q = cn.n_vision;
         w.n_tiles_q = (w.n_q + w.qt - 1) / w.qt;
@@ -190,21 +186,6 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     const LayerParams &L = P.L;
     Item it;
     int tile;
-    if (MODE == MODE_SGL) {
-        const int4 e = P.sgl_items[item];  // bucket b = (group, tile)
-        const int lo = e.x;
-        it.g = lo / P.sgl_nbt;
-        it.split = 0;
-        it.q0 = e.y;  // first entry in sgl_sorted
-        it.nq = e.z;
-        it.nseg = 1;
-        it.seg_kind[0] = K_SGL;
-        it.seg_tiles[0] = 1;
-        it.seg_kind[1] = K_EXACT;
-        it.seg_tiles[1] = 0;
-        it.key_lo = (lo % P.sgl_nbt) * kKeys;
-        return it;
-    }
     if (MODE == MODE_TEXT) {
         const int per_split = L.h_kv * w.n_tiles_q;
         it.split = item / per_split;
@@ -223,7 +204,7 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     it.seg_tiles[1] = 0;
     it.seg_kind[1] = K_EXACT;
     if (MODE == MODE_CMP) {
-        const int c_last = min((ql + 1) / L.block, w.nb);
+        const int c_last = cmp_visible(ql, L.block, L.stride, w.nb);
         const int t = (c_last + kKeys - 1) / kKeys;
         it.nseg = 2;
         it.seg_kind[0] = K_STATS;
@@ -283,7 +264,6 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
     switch (kind) {
         case K_SLC: return P.plan[(size_t)item * (1 + 2 * P.plan_max) + 1 + x] * kKeys;
         case K_SWA:
-        case K_SGL:
         case K_TEXT: return it.key_lo + x * kKeys;
         default: return x * kKeys;
     }
@@ -309,7 +289,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
     if (MODE == MODE_CMP) {
         mk = &P.tm_kb;
         mv = &P.tm_vb;
-    } else if (is_slc(MODE) || MODE == MODE_SWA || MODE == MODE_SGL) {
+    } else if (is_slc(MODE) || MODE == MODE_SWA) {
         mk = w.contiguous ? &P.tm_k : &P.tm_kc;
         mv = w.contiguous ? &P.tm_v : &P.tm_vc;
         vbase = w.contiguous ? w.vis_base : 0;
@@ -336,7 +316,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
         // row coordinate of tile x of a segment (both CMP segments share keys)
         auto row_of = [&](int kind, int x) {
             const int key0 = tile_key0(P, it, item, kind, x);
-            return (kind == K_SLC || kind == K_SWA || kind == K_SGL) ? vbase + key0 : key0;
+            return (kind == K_SLC || kind == K_SWA) ? vbase + key0 : key0;
         };
         if (is_k) {
             const int pf0 = min(kPrefetch, it.seg_tiles[0]);
@@ -473,7 +453,6 @@ struct RowCtx {
     int i;      // vision rank (CMP/SLC/SWA) or text rank (TEXT)
     int t;      // position of the query token
     int c_vis;  // visible compressed blocks
-    int sid;    // MODE_SGL: the row's (query, tile) pair
 };
 
 __device__ __forceinline__ void group_sync(const Smem &sm, uint32_t &phase, bool &ok,
@@ -562,26 +541,20 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         rc.h = it.g * L.r + min(rc.hl, L.r - 1);
         rc.valid = rc.qi < it.nq && rc.hl < L.r;
         rc.i = it.q0 + min(rc.qi, max(it.nq - 1, 0));
-        rc.sid = 0;
-        if (MODE == MODE_SGL) {
-            const int4 e = P.sgl_sorted[rc.i];  // it.q0 indexes the pair list here
-            rc.sid = e.x;
-            rc.i = e.y;
-            rc.t = e.z;
-        } else if (MODE == MODE_TEXT) {
+        if (MODE == MODE_TEXT) {
             rc.t = it.nq > 0 ? L.txt[rc.i] : 0;
         } else {
             rc.t = it.nq > 0 ? L.vis[rc.i] : 0;
         }
-        rc.c_vis = min((rc.i + 1) / L.block, w.nb);
+        rc.c_vis = cmp_visible(rc.i, L.block, L.stride, w.nb);
         if (item_tiles(it) == 0) {
             // nothing attended: empty branch outputs
             if (rc.valid) {
-                __half *part = (__half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+                float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                 const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
                 if (MODE == MODE_CMP) {
-                    for (int e = 0; e < kD; e += 8)
-                        *reinterpret_cast<uint4 *>(part + e) = make_uint4(0u, 0u, 0u, 0u);
+                    for (int e = 0; e < kD; e += 4)
+                        *reinterpret_cast<float4 *>(part + e) = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (L.dbg_o_cmp)
                         for (int e = 0; e < kD; ++e) L.dbg_o_cmp[prow + e] = 0.f;
                     L.lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
@@ -589,40 +562,23 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
-                } else if (MODE == MODE_SLC && P.sgl_on) {
-                    // no union tile: the merge takes the single-query tiles alone
-                    for (int e = 0; e < kD; e += 8)
-                        *reinterpret_cast<uint4 *>(P.slc_u + ((size_t)rc.i * L.h_q + rc.h) * kD +
-                                                   e) = make_uint4(0u, 0u, 0u, 0u);
-                    P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
                 } else {
-                    // no selected / window key: this branch adds nothing
+                    // no selected / window key (and, for the selection, no
+                    // single-query pair: the union keeps at least one tile of an
+                    // item that has any): this branch adds nothing
                     float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
                         if (MODE == MODE_SWA)
-                            ((__nv_bfloat16 *)L.out)[prow + e] =
-                                __float2bfloat16_rn(__half2float(part[e]));
+                            ((__nv_bfloat16 *)L.out)[prow + e] = __float2bfloat16_rn(part[e]);
                     }
                 }
             }
             continue;
         }
         // ---- Q tile (without the TMA box): rows gathered from their
-        // positions, 16-byte pieces.  MODE_SGL: each thread gathers its own
-        // row (its query is known only through the pair list).
-        if (MODE == MODE_SGL) {
-            const __nv_bfloat16 *src = Q + ((size_t)rc.t * L.h_q + rc.h) * kD;
-#pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
-                const uint4 val = rc.valid ? __ldg(reinterpret_cast<const uint4 *>(src + c16 * 8))
-                                           : make_uint4(0u, 0u, 0u, 0u);
-                const int hf = c16 >> 3, c = c16 & 7;
-                *reinterpret_cast<uint4 *>(sm.base + SM_Q + hf * 16384 + rho * 128 +
-                                           ((c ^ (rho & 7)) << 4)) = val;
-            }
-        }
-        for (int e = rho; MODE != MODE_SGL && !w.q_tma && e < kRows * 16; e += 128) {
+        // positions, 16-byte pieces
+        for (int e = rho; !w.q_tma && e < kRows * 16; e += 128) {
             const int row = e >> 4, c16 = e & 15;
             const int qi = row / w.rpad, hl = row % w.rpad;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
@@ -646,22 +602,22 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         if (rc.valid) {
             ptx::prefetch_l2(L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3);
             if (is_slc(MODE) || MODE == MODE_SWA) {
-                const __half *part = (const __half *)L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
-                ptx::prefetch_l2(part);
-                ptx::prefetch_l2(part + 64);
+                const float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
+#pragma unroll
+                for (int z = 0; z < kD; z += 32) ptx::prefetch_l2(part + z);
+            }
+            if (MODE == MODE_SLC && P.sgl_on) {
+                // the query's single-query pair outputs, read by the merge
+                const size_t qg = (size_t)it.g * L.n_max + rc.i;
+                const int ns = P.sgl_n[qg];
+                for (int z = 0; z < ns; ++z) {
+                    const __half *po = P.sgl_o + ((size_t)P.sgl_of[qg * L.top_k + z] * L.r + rc.hl) * kD;
+                    ptx::prefetch_l2(po);
+                    ptx::prefetch_l2(po + 64);
+                }
             }
         }
-        if (MODE == MODE_SGL && item + (int)gridDim.x < w.items) {
-            const Item nx = make_item<MODE>(P, w, item + gridDim.x);
-            const int qn = rho / w.rpad, hn = rho % w.rpad;
-            if (qn < nx.nq && hn < L.r) {
-                const int tn = P.sgl_sorted[nx.q0 + qn].z;
-                const __nv_bfloat16 *qr = Q + ((size_t)tn * L.h_q + nx.g * L.r + hn) * kD;
-                ptx::prefetch_l2(qr);
-                ptx::prefetch_l2(qr + 64);
-            }
-        }
-        if (MODE != MODE_SGL && item + (int)gridDim.x < w.items) {
+        if (item + (int)gridDim.x < w.items) {
             const Item nx = make_item<MODE>(P, w, item + gridDim.x);
             const int qn = rho / w.rpad, hn = rho % w.rpad;
             if (qn < nx.nq && hn < L.r) {
@@ -734,7 +690,6 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                             }
                             break;
                         case K_SWA: lo = rc.i - L.window + 1 - key0; hi = rc.i - key0; break;
-                        case K_SGL: lo = 0; hi = rc.i - key0; break;
                         default: lo = 0; hi = rc.t - key0; break;
                     }
                     lo = max(lo, 0);
@@ -905,7 +860,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     // block importance: the sum of the probabilities over the
                     // query's head slots (P is already handed to the MMA)
                     const int iq = it.q0 + rc.qi;
-                    const int cq = min((iq + 1) / L.block, w.nb);
+                    const int cq = cmp_visible(iq, L.block, L.stride, w.nb);
                     float *irow = rc.qi < it.nq
                                       ? L.imp + ((size_t)it.g * L.n_max + iq) * L.imp_stride + key0
                                       : nullptr;
@@ -934,10 +889,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         const size_t qrow = ((size_t)rc.i * L.h_q + rc.h) * kD;   // by vision rank
         const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;   // by position
-        // The gated vision partial lives in the workspace as fp16 [N_v][h_q][d]:
+        // The gated vision partial lives in the workspace as fp32 [N_v][h_q][d]:
         // CMP writes sig(g_cmp) o_cmp, SLC adds sig(g_slc) o_slc in place, SWA
-        // adds sig(g_swa) o_swa and writes the bf16 output row.
-        __half *part = (__half *)L.o_cmp_ws + qrow;
+        // adds sig(g_swa) o_swa and rounds the sum once, to the bf16 output row.
+        float *part = L.o_cmp_ws + qrow;
+        // O was accumulated against V (or V_cmp) divided by this power of two
+        const float vsc = P.v_scale[MODE == MODE_CMP ? 1 : 0];
         if (MODE == MODE_CMP) {
             const float gc = rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3]) : 0.f;
 #pragma unroll
@@ -947,25 +904,33 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (rc.valid) {
 #pragma unroll
-                    for (int k = 0; k < 32; k += 8) {
-                        uint4 v;
-                        __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+                    for (int k = 0; k < 32; ++k) o[k] *= vsc;
 #pragma unroll
-                        for (int z = 0; z < 4; ++z)
-                            h2[z] = __floats2half2_rn(gc * o[k + 2 * z], gc * o[k + 2 * z + 1]);
-                        __stcs(reinterpret_cast<uint4 *>(part + ch * 32 + k), v);
-                    }
+                    for (int k = 0; k < 32; k += 4)
+                        __stcg(reinterpret_cast<float4 *>(part + ch * 32 + k),
+                               make_float4(gc * o[k], gc * o[k + 1], gc * o[k + 2], gc * o[k + 3]));
                     if (L.dbg_o_cmp)
                         for (int k = 0; k < 32; ++k) L.dbg_o_cmp[prow + ch * 32 + k] = o[k];
                 }
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
-        } else if (MODE == MODE_SGL || (MODE == MODE_SLC && P.sgl_on)) {
-            // normalised output (fp16) and log-sum-exp of this row's tiles, for
-            // the merge: one (query, tile) pair (MODE_SGL) or the union tiles
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __half *orow = MODE == MODE_SGL ? P.sgl_o + ((size_t)rc.sid * L.r + rc.hl) * kD
-                                            : P.slc_u + qrow;
+        } else if (MODE == MODE_SLC && P.sgl_on) {
+            // The selection softmax of this row is split into the union's
+            // tiles (O, m_run, l_run here) and the query's single-query pairs
+            // (normalised outputs and log-sum-exps from the tile-major pass):
+            // each part is weighted by 2^(lse_part - M) / sum over the parts.
+            const float g = rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + 1]) : 0.f;
+            const float lse_u = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+            const size_t qg = (size_t)it.g * L.n_max + rc.i;
+            const int ns = rc.valid ? P.sgl_n[qg] : 0;
+            const int32_t *sids = P.sgl_of + qg * L.top_k;
+            float M = lse_u;
+            for (int z = 0; z < ns; ++z) M = fmaxf(M, P.sgl_lse[(size_t)sids[z] * L.r + rc.hl]);
+            const float wu = lse_u == -INFINITY ? 0.f : ptx::ex2(lse_u - M);
+            float W = wu;
+            for (int z = 0; z < ns; ++z) W += ptx::ex2(P.sgl_lse[(size_t)sids[z] * L.r + rc.hl] - M);
+            const float inv = W > 0.f ? 1.f / W : 0.f;
+            const float cu = l_run > 0.f ? wu * inv * vsc / l_run : 0.f;  // factor on the raw O
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
@@ -973,25 +938,43 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
 #pragma unroll
-                for (int k = 0; k < 32; k += 8) {
-                    uint4 v;
-                    __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+                for (int k = 0; k < 32; ++k) o[k] *= cu;
+#pragma unroll 2
+                for (int z = 0; z < ns; ++z) {
+                    const size_t pr = (size_t)sids[z] * L.r + rc.hl;
+                    const float wp = ptx::ex2(P.sgl_lse[pr] - M) * inv * P.sgl_scale[pr];
+                    const uint4 *src = reinterpret_cast<const uint4 *>(P.sgl_o + pr * kD + ch * 32);
+                    uint4 u[4];
 #pragma unroll
-                    for (int z = 0; z < 4; ++z)
-                        h2[z] = __floats2half2_rn(o[k + 2 * z] * inv, o[k + 2 * z + 1] * inv);
-                    *reinterpret_cast<uint4 *>(orow + ch * 32 + k) = v;
+                    for (int c = 0; c < 4; ++c) u[c] = __ldcs(src + c);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const __half2 *h2 = reinterpret_cast<const __half2 *>(&u[c]);
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) {
+                            const float2 f = __half22float2(h2[y]);
+                            o[8 * c + 2 * y] += wp * f.x;
+                            o[8 * c + 2 * y + 1] += wp * f.y;
+                        }
+                    }
                 }
-            }
-            if (rc.valid) {
-                const float lse = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
-                if (MODE == MODE_SGL) P.sgl_lse[(size_t)rc.sid * L.r + rc.hl] = lse;
-                else P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = lse;
+                if (L.dbg_o_slc)
+                    for (int k = 0; k < 32; ++k) L.dbg_o_slc[prow + ch * 32 + k] = o[k];
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    float4 pv = __ldcg(reinterpret_cast<const float4 *>(part + ch * 32 + k));
+                    pv.x += g * o[k];
+                    pv.y += g * o[k + 1];
+                    pv.z += g * o[k + 2];
+                    pv.w += g * o[k + 3];
+                    __stcg(reinterpret_cast<float4 *>(part + ch * 32 + k), pv);
+                }
             }
         } else if (is_slc(MODE) || MODE == MODE_SWA) {
             const float g =
                 rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (is_slc(MODE) ? 1 : 2)])
                          : 0.f;
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const float inv = l_run > 0.f ? vsc / l_run : 0.f;
             float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
             __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
@@ -1002,37 +985,33 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 if (!rc.valid) continue;
 #pragma unroll
                 for (int k = 0; k < 32; k += 8) {
-                    uint4 pv4 = __ldcs(reinterpret_cast<const uint4 *>(part + ch * 32 + k));
-                    const __half2 *ph = reinterpret_cast<const __half2 *>(&pv4);
+                    const float4 p0 = __ldcg(reinterpret_cast<const float4 *>(part + ch * 32 + k));
+                    const float4 p1 = __ldcg(reinterpret_cast<const float4 *>(part + ch * 32 + k + 4));
                     float b8[8];
 #pragma unroll
                     for (int z = 0; z < 8; ++z) b8[z] = l_run > 0.f ? o[k + z] * inv : 0.f;
                     if (dbg)
                         for (int z = 0; z < 8; ++z) dbg[prow + ch * 32 + k + z] = b8[z];
-                    uint4 v;
+                    const float f8[8] = {p0.x + g * b8[0], p0.y + g * b8[1], p0.z + g * b8[2],
+                                         p0.w + g * b8[3], p1.x + g * b8[4], p1.y + g * b8[5],
+                                         p1.z + g * b8[6], p1.w + g * b8[7]};
                     if (is_slc(MODE)) {
-                        __half2 *h2 = reinterpret_cast<__half2 *>(&v);
-#pragma unroll
-                        for (int z = 0; z < 4; ++z) {
-                            const float2 f = __half22float2(ph[z]);
-                            h2[z] = __floats2half2_rn(f.x + g * b8[2 * z], f.y + g * b8[2 * z + 1]);
-                        }
-                        __stcs(reinterpret_cast<uint4 *>(part + ch * 32 + k), v);
+                        __stcg(reinterpret_cast<float4 *>(part + ch * 32 + k),
+                               make_float4(f8[0], f8[1], f8[2], f8[3]));
+                        __stcg(reinterpret_cast<float4 *>(part + ch * 32 + k + 4),
+                               make_float4(f8[4], f8[5], f8[6], f8[7]));
                     } else {
+                        uint4 v;
                         __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(&v);
 #pragma unroll
-                        for (int z = 0; z < 4; ++z) {
-                            const float2 f = __half22float2(ph[z]);
-                            b2[z] = __floats2bfloat162_rn(f.x + g * b8[2 * z],
-                                                          f.y + g * b8[2 * z + 1]);
-                        }
+                        for (int z = 0; z < 4; ++z) b2[z] = __floats2bfloat162_rn(f8[2 * z], f8[2 * z + 1]);
                         __stcs(reinterpret_cast<uint4 *>(orow + ch * 32 + k), v);
                     }
                 }
             }
         } else if (w.nsplit == 1) {
             // one key split: the item holds the whole softmax, write the row
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const float inv = l_run > 0.f ? vsc / l_run : 0.f;
             __nv_bfloat16 *orow = (__nv_bfloat16 *)L.out + prow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
@@ -1057,7 +1036,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (rc.valid) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) pr[ch * 32 + k] = o[k];
+                    for (int k = 0; k < 32; ++k) pr[ch * 32 + k] = o[k] * vsc;
                 }
             }
             if (rc.valid) {
@@ -1145,47 +1124,91 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Operand preparation for the tensor-core kernels:
-//  * fp16 copies of V (all positions) and of V_cmp for the P V products.  A
-//    bf16 value converts to fp16 exactly when its magnitude lies in the fp16
-//    normal range; a value beyond the fp16 range is reported as a bounds error.
-//  * vision K (bf16) and V (fp16) in vision order when the vision tokens are
-//    not one contiguous run of positions (the TMA tiles need consecutive rows).
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u, bool &overflow) {
+// Operands of the P V products.  P is fp16 (11 significant bits), so V and
+// V_cmp enter as fp16 copies; to keep every bf16 value inside the fp16 range,
+// each is divided by a power of two 2^e chosen per call so that its largest
+// magnitude lands in [2^14, 2^15) (e may be negative: small values then keep
+// fp16's full precision too).  Division by a power of two is exact; the
+// epilogues multiply O by 2^e.  Inf / NaN inputs keep e = 0.
+//
+// vmax_kernel: the largest |V| over the n tokens and |V_cmp| over the blocks
+// (atomicMax on the bit patterns of non-negative floats, which order like the
+// values); *vmax must start at zero.
+__global__ void vmax_kernel(LayerParams p, unsigned *vmax) {
+    const Counts cn = *p.counts;
+    const size_t row_vec = (size_t)p.h_kv * kD / 8;  // 16-byte pieces per row
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t step = (size_t)gridDim.x * blockDim.x;
+    float m[2] = {0.f, 0.f};
+    const uint4 *src[2] = {reinterpret_cast<const uint4 *>(p.v),
+                           reinterpret_cast<const uint4 *>(p.v_cmp)};
+    const size_t cnt[2] = {(size_t)p.n * row_vec, (size_t)cn.nc * row_vec};
+#pragma unroll
+    for (int w = 0; w < 2; ++w)
+        for (size_t e = tid; e < cnt[w]; e += step) {
+            const uint4 u = __ldg(src[w] + e);
+            const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(b[i]);
+                m[w] = fmaxf(m[w], fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const float r = warp_max(m[w]);
+        if ((threadIdx.x & 31) == 0 && r > 0.f) atomicMax(vmax + w, __float_as_uint(r));
+    }
+}
+
+// 2^-e for the largest magnitude m (see above), and 2^e into *scale_out.
+__device__ __forceinline__ float v_prescale(unsigned mbits, float *scale_out) {
+    const float m = __uint_as_float(mbits);
+    int e = 0;
+    if (m > 0.f && m <= 3.0e38f) e = (int)((mbits >> 23) & 255u) - 127 - 14;
+    if (e < -100) e = -100;
+    if (scale_out) *scale_out = ldexpf(1.f, e);
+    return ldexpf(1.f, -e);
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u, float mul) {
     const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
     uint4 r;
     __half2 *h = reinterpret_cast<__half2 *>(&r);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(b[i]);
-        h[i] = __floats2half2_rn(f.x, f.y);
-        if (fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f) overflow = true;
+        h[i] = __floats2half2_rn(f.x * mul, f.y * mul);
     }
     return r;
 }
 
-__global__ void prepare_kernel(LayerParams p, __nv_bfloat16 *kc, __half *vhc, __half *vh,
-                               __half *vh_cmp) {
+// The scaled fp16 copies of V (all positions) and V_cmp, and the vision K
+// (bf16) and V (scaled fp16) in vision order when the vision tokens are not
+// one contiguous run of positions (the TMA tiles need consecutive rows).
+__global__ void prepare_kernel(LayerParams p, const unsigned *vmax, float *v_scale,
+                               __nv_bfloat16 *kc, __half *vhc, __half *vh, __half *vh_cmp) {
     const Counts cn = *p.counts;
+    const bool first = blockIdx.x == 0 && threadIdx.x == 0;
+    const float mv = v_prescale(vmax[0], first ? v_scale : nullptr);
+    const float mc = v_prescale(vmax[1], first ? v_scale + 1 : nullptr);
     const size_t row_vec = (size_t)p.h_kv * kD / 8;  // 16-byte pieces per row
     const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t step = (size_t)gridDim.x * blockDim.x;
-    bool overflow = false;
     const uint4 *v = reinterpret_cast<const uint4 *>(p.v);
     for (size_t e = tid; e < (size_t)p.n * row_vec; e += step)
-        reinterpret_cast<uint4 *>(vh)[e] = bf16x8_to_f16x8(__ldg(v + e), overflow);
+        reinterpret_cast<uint4 *>(vh)[e] = bf16x8_to_f16x8(__ldg(v + e), mv);
     const uint4 *vb = reinterpret_cast<const uint4 *>(p.v_cmp);
-    for (size_t e = tid; e < (size_t)cn.nb * row_vec; e += step)
-        reinterpret_cast<uint4 *>(vh_cmp)[e] = bf16x8_to_f16x8(vb[e], overflow);
+    for (size_t e = tid; e < (size_t)cn.nc * row_vec; e += step)
+        reinterpret_cast<uint4 *>(vh_cmp)[e] = bf16x8_to_f16x8(vb[e], mc);
     if (!cn.contiguous) {
         for (size_t e = tid; e < (size_t)cn.n_vision * row_vec; e += step) {
             const size_t u = e / row_vec, c = e % row_vec;
             const size_t src = (size_t)p.vis[u] * row_vec + c;
             reinterpret_cast<uint4 *>(kc)[e] = __ldg(reinterpret_cast<const uint4 *>(p.k) + src);
-            reinterpret_cast<uint4 *>(vhc)[e] = bf16x8_to_f16x8(__ldg(v + src), overflow);
+            reinterpret_cast<uint4 *>(vhc)[e] = bf16x8_to_f16x8(__ldg(v + src), mv);
         }
     }
-    if (overflow) report(p.status, VNSA_ERR_BOUNDS);
 }
 
 // ---------------------------------------------------------------------------
@@ -1293,7 +1316,7 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         int tot = min(total, plan_max);
         if (sg.on) {
             // Tiles that exactly one query reaches leave the plan for the
-            // tile-major pass (MODE_SGL), as long as one tile stays and the
+            // tile-major pass (sgl_attn.cu), as long as one tile stays and the
             // pair records have room; their ids are taken in one block per item.
             qcnt[lane] = 0u;
             int nsing = 0;
@@ -1356,7 +1379,7 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
 }
 
 // Offsets of the single-query pairs grouped by bucket (group, tile) and of the
-// MODE_SGL items (chunks of qt pairs of one bucket): exclusive prefix sums
+// tile-major pass's chunks (qt pairs of one bucket): exclusive prefix sums
 // over the bucket counts, one block.
 __global__ void __launch_bounds__(1024) sgl_scan_kernel(int32_t *meta, int nbk, int qt) {
     __shared__ int wsum[2][32];
@@ -1414,7 +1437,7 @@ __global__ void __launch_bounds__(1024) sgl_scan_kernel(int32_t *meta, int nbk, 
 }
 
 // Pairs in bucket order: pair `sid` goes to off[bucket] + its rank in the
-// bucket, as (sid, vision rank, position, 0); and the MODE_SGL item table:
+// bucket, as (sid, vision rank, position, 0); and the tile-major pass's chunk table:
 // chunk c of bucket b is item choff[b] + c, (b, off[b] + c qt, pairs, 0).
 __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *sorted,
                                    int4 *items, int nbk, int cap, int qt) {
@@ -1429,121 +1452,6 @@ __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *s
         const int cnt = hist[b];
         for (int c = 0; c * qt < cnt; ++c)
             items[choff[b] + c] = make_int4(b, off[b] + c * qt, min(qt, cnt - c * qt), 0);
-    }
-}
-
-// The selection output of each (vision query, head): the union tiles' softmax
-// (slc_u, slc_lse) and the query's single-query tiles (sgl_o, sgl_lse), each
-// normalised with its own log-sum-exp, combined by their weights
-// 2^(lse - max) / sum; then partial += sigmoid(g_slc) * o_slc (fp16) and the
-// optional export.  One warp per (group, query).  Lane s holds single-query
-// tile s of the query (its id and its per-head lse and weight; 32 at a time),
-// lane hl < r the union's scalars of head hl; half2 element k of a lane
-// belongs to head k / 2.  KMAX = half2 elements per lane = 2 r at most.
-struct SglMergeArgs {
-    const int32_t *of, *n;
-    const __half *sgl_o, *slc_u;
-    const float *sgl_lse, *slc_lse;
-};
-
-template <int KMAX>
-__global__ void __launch_bounds__(256) sgl_merge_kernel(LayerParams p, SglMergeArgs a) {
-    constexpr int RMAX = KMAX / 2;
-    const Counts cn = *p.counts;
-    const int lane = threadIdx.x & 31;
-    const int r = p.r;
-    const long long rows = (long long)p.h_kv * cn.n_vision;
-    for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < rows;
-         wid += ((long long)gridDim.x * blockDim.x) >> 5) {
-        const int g = (int)(wid / cn.n_vision), i = (int)(wid % cn.n_vision);
-        const int h0 = g * r;
-        const int t = p.vis[i];
-        const int ns = a.n[(size_t)g * p.n_max + i];
-        const int32_t *sids = a.of + ((size_t)g * p.n_max + i) * p.top_k;
-        const float lu = lane < r ? a.slc_lse[(size_t)i * p.h_q + h0 + lane] : -INFINITY;
-        const float gl = lane < r ? sigmoidf_(p.gate[((size_t)t * p.h_q + h0 + lane) * 3 + 1]) : 0.f;
-        // per-head maximum and sum over the union and every single-query tile
-        float mx[RMAX], sm[RMAX];
-#pragma unroll
-        for (int hl = 0; hl < RMAX; ++hl) mx[hl] = __shfl_sync(0xffffffffu, lu, hl);
-        for (int s0 = 0; s0 < ns; s0 += 32) {
-            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
-#pragma unroll
-            for (int hl = 0; hl < RMAX; ++hl) {
-                float v = (sid >= 0 && hl < r) ? a.sgl_lse[(size_t)sid * r + hl] : -INFINITY;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                mx[hl] = fmaxf(mx[hl], v);
-            }
-        }
-#pragma unroll
-        for (int hl = 0; hl < RMAX; ++hl) {
-            const float u = __shfl_sync(0xffffffffu, lu, hl);
-            sm[hl] = mx[hl] == -INFINITY ? 0.f : exp2f(u - mx[hl]);
-        }
-        for (int s0 = 0; s0 < ns; s0 += 32) {
-            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
-#pragma unroll
-            for (int hl = 0; hl < RMAX; ++hl) {
-                float v = (sid >= 0 && hl < r && mx[hl] != -INFINITY)
-                              ? exp2f(a.sgl_lse[(size_t)sid * r + hl] - mx[hl])
-                              : 0.f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                sm[hl] += v;
-            }
-        }
-        // union part, then the single-query tiles 32 at a time
-        float2 acc[KMAX];
-        {
-            const __half2 *u = reinterpret_cast<const __half2 *>(a.slc_u + ((size_t)i * p.h_q + h0) * kD);
-#pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                const int hl = k >> 1;
-                const float lh = __shfl_sync(0xffffffffu, lu, hl);
-                const float wk = sm[hl] > 0.f ? exp2f(lh - mx[hl]) / sm[hl] : 0.f;
-                const float2 f = k < 2 * r ? __half22float2(u[lane + 32 * k]) : make_float2(0.f, 0.f);
-                acc[k] = make_float2(wk * f.x, wk * f.y);
-            }
-        }
-        for (int s0 = 0; s0 < ns; s0 += 32) {
-            const int sid = s0 + lane < ns ? sids[s0 + lane] : -1;
-            float wl[RMAX];  // this lane's tile: weight per head
-#pragma unroll
-            for (int hl = 0; hl < RMAX; ++hl)
-                wl[hl] = (sid >= 0 && hl < r && sm[hl] > 0.f)
-                             ? exp2f(a.sgl_lse[(size_t)sid * r + hl] - mx[hl]) / sm[hl]
-                             : 0.f;
-            const int nc = min(32, ns - s0);
-            for (int c = 0; c < nc; ++c) {
-                const int sc = __shfl_sync(0xffffffffu, sid, c);
-                const __half2 *o = reinterpret_cast<const __half2 *>(a.sgl_o + (size_t)sc * r * kD);
-#pragma unroll
-                for (int k = 0; k < KMAX; ++k) {
-                    const float wk = __shfl_sync(0xffffffffu, wl[k >> 1], c);
-                    if (k < 2 * r) {
-                        const float2 f = __half22float2(o[lane + 32 * k]);
-                        acc[k].x += wk * f.x;
-                        acc[k].y += wk * f.y;
-                    }
-                }
-            }
-        }
-        __half2 *part = reinterpret_cast<__half2 *>((__half *)p.o_cmp_ws + ((size_t)i * p.h_q + h0) * kD);
-        float *dbg = p.dbg_o_slc ? p.dbg_o_slc + ((size_t)t * p.h_q + h0) * kD : nullptr;
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            const float gk = __shfl_sync(0xffffffffu, gl, k >> 1);
-            if (k < 2 * r) {
-                const int e = lane + 32 * k;
-                const float2 f = __half22float2(part[e]);
-                part[e] = __floats2half2_rn(f.x + gk * acc[k].x, f.y + gk * acc[k].y);
-                if (dbg) {
-                    dbg[2 * e] = acc[k].x;
-                    dbg[2 * e + 1] = acc[k].y;
-                }
-            }
-        }
     }
 }
 
@@ -1673,17 +1581,19 @@ struct TcState {
     int plan_max;
     int part_items;
     __nv_bfloat16 *kc;  // vision K in vision order (non-contiguous vision only)
-    __half *vhc;        // vision V (fp16) in vision order (non-contiguous vision only)
-    __half *vh;         // V in fp16, all positions
-    __half *vh_cmp;     // V_cmp in fp16
+    __half *vhc;        // vision V (scaled fp16) in vision order (non-contiguous vision only)
+    __half *vh;         // V as scaled fp16, all positions
+    __half *vh_cmp;     // V_cmp as scaled fp16
+    unsigned *vmax;     // [2] largest |V|, |V_cmp| of the call (float bits)
+    float *v_scale;     // [2] their powers of two
     int32_t *plan;
     float *part;
-    // single-query selection tiles (block 64): see TcParams
+    // single-query selection tiles (block 64): see TcParams and sgl_attn.h
     int sgl_on, sgl_nbt, sgl_cap;
     int32_t *sgl_meta, *sgl_of, *sgl_n;
     int4 *sgl_rec, *sgl_sorted, *sgl_items;
-    __half *sgl_o, *slc_u;
-    float *sgl_lse, *slc_lse;
+    __half *sgl_o;
+    float *sgl_lse, *sgl_scale;
 };
 
 // Single-query pairs the workspace holds, per query and group on average;
@@ -1692,7 +1602,7 @@ constexpr int kSglPerQuery = 6;
 
 struct SglSizes {
     int on, nbt, nbk, cap;
-    size_t meta, rec, sorted, items, of, n, o, lse, u, ulse, total;
+    size_t meta, rec, sorted, items, of, n, o, lse, scale, total;
 };
 
 static SglSizes sgl_sizes(const vnsa_config &c) {
@@ -1712,9 +1622,8 @@ static SglSizes sgl_sizes(const vnsa_config &c) {
     z.n = up256((size_t)c.h_kv * c.n_max * 4);
     z.o = up256((size_t)z.cap * r * kD * 2);
     z.lse = up256((size_t)z.cap * r * 4);
-    z.u = up256((size_t)c.n_max * c.h_q * kD * 2);
-    z.ulse = up256((size_t)c.n_max * c.h_q * 4);
-    z.total = z.meta + z.rec + z.sorted + z.items + z.of + z.n + z.o + z.lse + z.u + z.ulse;
+    z.scale = up256((size_t)z.cap * r * 4);
+    z.total = z.meta + z.rec + z.sorted + z.items + z.of + z.n + z.o + z.lse + z.scale;
     return z;
 }
 
@@ -1751,8 +1660,8 @@ static size_t plan_bytes(const vnsa_config &c) {
 size_t tc_workspace_bytes(const vnsa_config &c) {
     if (!tc_supported(c)) return 0;
     const size_t kv = (size_t)c.n_max * c.h_kv * kD * 2;
-    const size_t kvb = (size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2;
-    return up256(kv) * 3 + up256(kvb) + up256(plan_bytes(c)) + kTextPartBytes +
+    const size_t kvb = (size_t)(cmp_blocks(c.n_max, c.block, cmp_stride_of(c)) + 1) * c.h_kv * kD * 2;
+    return up256(kv) * 3 + up256(kvb) + 256 + up256(plan_bytes(c)) + kTextPartBytes +
            sgl_sizes(c).total;
 }
 
@@ -1768,11 +1677,15 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
     st->part_items = (int)(kTextPartBytes / ((size_t)kRows * kPartStride * 4));
     char *p = (char *)ws;
     const size_t kv = up256((size_t)c.n_max * c.h_kv * kD * 2);
-    const size_t kvb = up256((size_t)(c.n_max / c.block + 1) * c.h_kv * kD * 2);
+    const size_t kvb =
+        up256((size_t)(cmp_blocks(c.n_max, c.block, cmp_stride_of(c)) + 1) * c.h_kv * kD * 2);
     st->kc = (__nv_bfloat16 *)p;
     st->vhc = (__half *)(p + kv);
     st->vh = (__half *)(p + 2 * kv);
     st->vh_cmp = (__half *)(p + 3 * kv);
+    st->vmax = (unsigned *)(p + 3 * kv + kvb);
+    st->v_scale = (float *)(p + 3 * kv + kvb + 16);
+    p += 256;  // vmax and v_scale
     st->plan = (int32_t *)(p + 3 * kv + kvb);
     st->part = (float *)(p + 3 * kv + kvb + up256(plan_bytes(c)));
     {
@@ -1789,15 +1702,14 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
         st->sgl_n = (int32_t *)(q += z.of);
         st->sgl_o = (__half *)(q += z.n);
         st->sgl_lse = (float *)(q += z.o);
-        st->slc_u = (__half *)(q += z.lse);
-        st->slc_lse = (float *)(q += z.u);
+        st->sgl_scale = (float *)(q += z.lse);
     }
     cudaError_t e = cudaSuccess;
     for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
-                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>,
-                    tc_attn_kernel<MODE_SGL>})
+                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>})
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e == cudaSuccess) e = sgl_prepare();
     if (e != cudaSuccess) {
         delete st;
         return e;
@@ -1819,15 +1731,12 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     P.part_items = st->part_items;
     const bool sgl = st->sgl_on && c.block == kKeys;
     P.sgl_on = 0;  // set for the selection launch below
-    P.sgl_nbt = st->sgl_nbt;
-    P.sgl_meta = st->sgl_meta;
-    P.sgl_sorted = st->sgl_sorted;
-    P.sgl_items = st->sgl_items;
+    P.sgl_of = st->sgl_of;
+    P.sgl_n = st->sgl_n;
     P.sgl_o = st->sgl_o;
     P.sgl_lse = st->sgl_lse;
-    P.slc_u = st->slc_u;
-    P.slc_lse = st->slc_lse;
-    const int nb_rows = c.n_max / c.block > 0 ? c.n_max / c.block : 1;
+    P.sgl_scale = st->sgl_scale;
+    const int nb_rows = L.nb_max > 0 ? L.nb_max : 1;  // compression blocks
     if (!make_map(&P.tm_k, L.k, c.h_kv, L.n, false) ||
         !make_map(&P.tm_v, st->vh, c.h_kv, L.n, true) ||
         !make_map(&P.tm_kc, st->kc, c.h_kv, c.n_max, false) ||
@@ -1835,6 +1744,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         !make_map(&P.tm_kb, L.k_cmp, c.h_kv, nb_rows, false) ||
         !make_map(&P.tm_vb, st->vh_cmp, c.h_kv, nb_rows, true))
         return cudaErrorInvalidValue;
+    P.v_scale = st->v_scale;
     auto begin = [&](int stg) {
         if (ev) cudaEventRecord(ev[2 * stg], s);
         ran[stg] = 1;
@@ -1857,19 +1767,27 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
                 tc_attn_kernel<MODE_SLC_UNALIGNED><<<grid, kThreads, SMEM_BYTES, s>>>(P);
                 break;
             case MODE_SWA: tc_attn_kernel<MODE_SWA><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
-            case MODE_SGL: tc_attn_kernel<MODE_SGL><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             default: tc_attn_kernel<MODE_TEXT><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
         }
         ++*launches;
         return cudaSuccess;
     };
-    prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->kc, st->vhc, st->vh, st->vh_cmp);
-    ++*launches;
+    cudaError_t e0 = cudaMemsetAsync(st->vmax, 0, 2 * sizeof(unsigned), s);
+    if (e0 != cudaSuccess) return e0;
+    vmax_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->vmax);
+    prepare_kernel<<<st->num_sms * 4, 256, 0, s>>>(L, st->vmax, st->v_scale, st->kc, st->vhc,
+                                                   st->vh, st->vh_cmp);
+    *launches += 2;
     begin(VNSA_STAGE_CMP);
     if ((e = attn(MODE_CMP)) != cudaSuccess) return e;
     end(VNSA_STAGE_CMP);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TOPK);
+    if (L.stride != L.block) {
+        // overlapping compression blocks: their importance onto the selection blocks
+        if ((e = launch_imp_remap(L, s)) != cudaSuccess) return e;
+        ++*launches;
+    }
     if (!forced) {
         if ((e = launch_topk(L, s)) != cudaSuccess) return e;
         ++*launches;
@@ -1912,21 +1830,34 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_SLC);
     if (sgl) {
-        // single-query tiles tile-major, then the union tiles, then the merge
-        if ((e = attn(MODE_SGL)) != cudaSuccess) return e;
+        // single-query tiles tile-major, then the union tiles, whose epilogue
+        // merges each query's pairs into its selection output
+        SglParams sp;
+        memset(&sp, 0, sizeof(sp));
+        sp.tm_k = P.tm_k;
+        sp.tm_v = P.tm_v;
+        sp.tm_kc = P.tm_kc;
+        sp.tm_vc = P.tm_vc;
+        sp.v_scale = st->v_scale;
+        sp.counts = L.counts;
+        sp.q = (const __nv_bfloat16 *)L.q;
+        sp.h_q = c.h_q;
+        sp.r = L.r;
+        sp.nbt = st->sgl_nbt;
+        sp.scale_log2 = L.scale_log2;
+        sp.n_items = st->sgl_meta + 1;
+        sp.sorted = st->sgl_sorted;
+        sp.items = st->sgl_items;
+        sp.o = st->sgl_o;
+        sp.lse = st->sgl_lse;
+        sp.oscale = st->sgl_scale;
+        sp.status = L.status;
+        sp.wait_ns = L.wait_ns;
+        if ((e = launch_sgl_attn(sp, st->num_sms, s)) != cudaSuccess) return e;
+        ++*launches;
         P.sgl_on = 1;
         if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
         P.sgl_on = 0;
-        SglMergeArgs ma;
-        ma.of = st->sgl_of;
-        ma.n = st->sgl_n;
-        ma.sgl_o = st->sgl_o;
-        ma.slc_u = st->slc_u;
-        ma.sgl_lse = st->sgl_lse;
-        ma.slc_lse = st->slc_lse;
-        if (L.r <= 8) sgl_merge_kernel<16><<<st->num_sms * 8, 256, 0, s>>>(L, ma);
-        else sgl_merge_kernel<32><<<st->num_sms * 8, 256, 0, s>>>(L, ma);
-        ++*launches;
     } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
         return e;
     }

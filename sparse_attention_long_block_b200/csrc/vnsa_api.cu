@@ -24,18 +24,21 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-    size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, idx, o_cmp, tc, dec,
-        dec_sel;
+    size_t vis, txt, counts, status, w_k, w_v, k_cmp, v_cmp, lse, imp, imp_sel, idx, o_cmp, tc,
+        dec, dec_sel;
     size_t total;
-    size_t imp_stride;
+    size_t imp_stride, imp_sel_stride;
 };
 
 Layout make_layout(const vnsa_config &c) {
     const size_t es = c.dtype == VNSA_BF16 ? 2 : 4;
     const size_t n = (size_t)c.n_max;
-    const size_t nb = (size_t)(c.n_max / c.block);
+    const size_t nb = (size_t)(c.n_max / c.block);  // selection blocks
+    const int stride = cmp_stride_of(c);
+    const size_t nc = (size_t)cmp_blocks(c.n_max, c.block, stride);  // compression blocks
     Layout L;
-    L.imp_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
+    L.imp_stride = nc > 0 ? (nc + 3) / 4 * 4 : 4;
+    L.imp_sel_stride = nb > 0 ? (nb + 3) / 4 * 4 : 4;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes > 0 ? bytes : 1); return o; };
     L.vis = take(n * 4);
@@ -44,10 +47,13 @@ Layout make_layout(const vnsa_config &c) {
     L.status = take(16);
     L.w_k = take((size_t)c.d * c.d * es);
     L.w_v = take((size_t)c.d * c.d * es);
-    L.k_cmp = take(nb * c.h_kv * c.d * es);
-    L.v_cmp = take(nb * c.h_kv * c.d * es);
+    L.k_cmp = take(nc * c.h_kv * c.d * es);
+    L.v_cmp = take(nc * c.h_kv * c.d * es);
     L.lse = take(n * c.h_q * 4);
     L.imp = take((size_t)c.h_kv * n * L.imp_stride * 4);
+    // the selection-block importance has a buffer of its own only when the
+    // compression blocks overlap
+    L.imp_sel = stride != c.block ? take((size_t)c.h_kv * n * L.imp_sel_stride * 4) : L.imp;
     L.idx = take((size_t)c.h_kv * n * c.top_k * 4);
     L.o_cmp = take(n * c.h_q * c.d * 4);
     L.tc = take(tc_workspace_bytes(c));
@@ -163,7 +169,7 @@ vnsa_status vnsa_create(const vnsa_config *cfg, const void *w_k, const void *w_v
     cudaGetDevice(&h->device);
     h->r = cfg->h_q / cfg->h_kv;
     h->stream_n = -1;
-    h->nb_max = cfg->n_max / cfg->block;
+    h->nb_max = cmp_blocks(cfg->n_max, cfg->block, cmp_stride_of(*cfg));
     h->esize = cfg->dtype == VNSA_BF16 ? 2 : 4;
     h->L = make_layout(h->cfg);
     if (cudaMalloc(&h->ws, h->L.total) != cudaSuccess) {
@@ -214,6 +220,7 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     p.d = c.d;
     p.r = h->r;
     p.block = c.block;
+    p.stride = cmp_stride_of(c);
     p.top_k = c.top_k;
     p.window = c.window;
     p.force_first = c.force_first;
@@ -235,6 +242,8 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     p.lse = (float *)(h->ws + h->L.lse);
     p.imp = (float *)(h->ws + h->L.imp);
     p.imp_stride = h->L.imp_stride;
+    p.imp_sel = (float *)(h->ws + h->L.imp_sel);
+    p.imp_sel_stride = h->L.imp_sel == h->L.imp ? h->L.imp_stride : h->L.imp_sel_stride;
     p.idx = (int32_t *)(h->ws + h->L.idx);
     p.idx_src = p.idx;
     p.idx_rows = (size_t)c.n_max;
@@ -272,13 +281,13 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
     } while (0)
 
     begin(VNSA_STAGE_PARTITION);
-    VNSA_RUN(launch_partition(is_vision, n, c.block, (int32_t *)p.vis, (int32_t *)p.txt,
-                              h->counts, s));
+    VNSA_RUN(launch_partition(is_vision, n, c.block, p.stride, (int32_t *)p.vis,
+                              (int32_t *)p.txt, h->counts, s));
     end(VNSA_STAGE_PARTITION);
     begin(VNSA_STAGE_POOL);
     VNSA_RUN(launch_pool_proj(dt, c.d, k, v, p.vis, h->counts, h->ws + h->L.w_k,
                               h->ws + h->L.w_v, (void *)p.k_cmp, (void *)p.v_cmp, c.h_kv,
-                              c.block, h->nb_max, s, 0, &h->mlp));
+                              c.block, p.stride, h->nb_max, s, 0, &h->mlp));
     end(VNSA_STAGE_POOL);
     if (use_tc) {
         // counts its own launches
@@ -288,11 +297,10 @@ vnsa_status vnsa_forward(vnsa_handle *h, int n, const void *q, const void *k, co
         begin(VNSA_STAGE_CMP);
         VNSA_RUN(launch_cmp_simt(dt, p, s));
         end(VNSA_STAGE_CMP);
-        if (!forced) {
-            begin(VNSA_STAGE_TOPK);
-            VNSA_RUN(launch_topk(p, s));
-            end(VNSA_STAGE_TOPK);
-        }
+        begin(VNSA_STAGE_TOPK);
+        if (p.stride != p.block) VNSA_RUN(launch_imp_remap(p, s));
+        if (!forced) VNSA_RUN(launch_topk(p, s));
+        end(VNSA_STAGE_TOPK);
         begin(VNSA_STAGE_SWA);
         VNSA_RUN(launch_vision_simt(dt, p, s));
         end(VNSA_STAGE_SWA);
@@ -320,6 +328,7 @@ vnsa_status vnsa_decode(vnsa_handle *h, int n, const void *q_new, const void *k,
     if (!h || !q_new || !k || !v || !is_vision || !gate_new || !out_new)
         return VNSA_ERR_INVALID_ARG;
     if (n < 2 || n > h->cfg.n_max || h->stream_n != (long long)n - 1) return VNSA_ERR_INVALID_ARG;
+    if (cmp_stride_of(h->cfg) != h->cfg.block) return VNSA_ERR_UNSUPPORTED;
     if (!aligned16(q_new) || !aligned16(k) || !aligned16(v) || !aligned16(out_new) ||
         !aligned16(gate_new) || (sel_out && !aligned16(sel_out)))
         return VNSA_ERR_INVALID_ARG;

@@ -50,6 +50,7 @@ class Workload:
     ar1: bool = False            # AR(1) drift of K/V frame means
     seed: int = 0
     block: int = 64
+    stride: int = 0              # compression stride (0: the block; below it blocks overlap)
     dense: bool = False          # Dense-NSA: every token attends densely (no vision set)
     frame: int = FRAME           # vision tokens per frame of the frame-mean model
 

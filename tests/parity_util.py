@@ -20,7 +20,7 @@ TIE_REL = 1e-3
 def oracle_params(wl: Workload) -> oracle.OracleParams:
     return oracle.OracleParams(h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
                                top_k=wl.top_k, window=wl.window,
-                               round_cmp_bf16=(wl.dtype == "bf16"))
+                               round_cmp_bf16=(wl.dtype == "bf16"), stride=wl.stride or None)
 
 
 def stratified_rows(is_vision: np.ndarray, block: int = 64, every: int = 97,
@@ -64,14 +64,14 @@ def run_gpu(wl: Workload, x: dict, want=(), forced_idx=None, ranks=None, cmp_mlp
     gate = torch.from_numpy(x["gate"]).to(dev)
     layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
                           top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
-                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype, stride=wl.stride)
     if cmp_mlp is not None:
         layer.set_cmp_mlp({nm: torch.from_numpy(a) for nm, a in cmp_mlp.items()})
     fidx = None
     if forced_idx is not None:
         fidx = torch.from_numpy(np.ascontiguousarray(forced_idx, np.int32)).to(dev)
     dbg, tens = binding.make_debug(wl.n, wl.h_q, wl.h_kv, wl.d, wl.top_k, wl.block, dtype=td,
-                                   want=want, forced_idx=fidx)
+                                   want=want, forced_idx=fidx, stride=wl.stride)
     out = layer.forward(q, k, v, isv, gate, dbg=dbg if (want or fidx is not None) else None)
     torch.cuda.synchronize()
     status = layer.device_status()
@@ -244,9 +244,12 @@ def compare_pool(wl: Workload, x: dict, cmp_mlp=None):
     kc, vc = oracle.pool_proj(p, x["k"], x["v"], x["is_vision"], x["w_k"], x["w_v"],
                               cmp_mlp=cmp_mlp)
     g = run_gpu(wl, x, want=("k_cmp", "v_cmp"), cmp_mlp=cmp_mlp)
-    nb = kc.shape[0]
+    nb = kc.shape[0]  # compression blocks (they overlap when the stride is below the block)
     out = {}
-    vis = np.nonzero(x["is_vision"])[0][: nb * wl.block]
+    stride = wl.stride or wl.block
+    allv = np.nonzero(x["is_vision"])[0]
+    vis = np.concatenate([allv[c * stride: c * stride + wl.block] for c in range(nb)]) \
+        if nb else allv[:0]
     for name, ref, src, w in (("k_cmp", kc, x["k"], x["w_k"]), ("v_cmp", vc, x["v"], x["w_v"])):
         got = g[name][:nb].astype(np.float64)
         if wl.dtype == "bf16":

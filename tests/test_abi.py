@@ -138,3 +138,19 @@ def test_new_knobs_reject_null_handle_and_noalloc_rejects_bad_config_on_host():
     c = cfg()
     rc = lib.vnsa_select_noalloc(ctypes.byref(c), 262145, p, p, p, p, p, p, p, p, None)
     assert rc == binding.VNSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("stride,code", [(-1, binding.VNSA_ERR_INVALID_ARG),
+                                         (65, binding.VNSA_ERR_INVALID_ARG)])
+def test_compression_stride_beyond_the_block_is_rejected(stride, code):
+    with pytest.raises(binding.VnsaError) as e:
+        binding.vnsa_workspace_bytes(cfg(cmp_stride=stride))
+    assert e.value.code == code
+
+
+def test_overlapping_compression_blocks_grow_the_workspace():
+    # stride 16 under block 64: four times the compression blocks, plus a
+    # selection-importance buffer of its own
+    plain = binding.vnsa_workspace_bytes(cfg())
+    assert binding.vnsa_workspace_bytes(cfg(cmp_stride=64)) == plain
+    assert binding.vnsa_workspace_bytes(cfg(cmp_stride=16)) > plain + 3 * 4 * 8448 * 132 * 4
