@@ -99,7 +99,8 @@ def executed_work(wl, is_vision, idx):
     of the 64-key tiles their selected blocks reach (from idx [h_kv][N_v][k]);
     with block 64 the tiles that only one of the 18 queries reaches run
     tile-major instead, up to 18 such (query, tile) pairs per 128-row tile;
-    window and text: 18 queries against their key ranges."""
+    window and text: 18 queries against their key ranges.  (Up to 8 of a
+    query's single tiles, in tile order, leave the union.)"""
     prod = 2.0 * 128 * 64 * wl.d
     vis = np.nonzero(is_vision)[0]
     txt = np.nonzero(is_vision == 0)[0]
@@ -122,13 +123,18 @@ def executed_work(wl, is_vision, idx):
         for g in range(wl.h_kv):
             sel = idx[g, q0:ql + 1]
             if wl.block == 64:
-                sel = sel.ravel()
-                u, cnt = np.unique(sel[sel >= 0], return_counts=True)
-                ones = u[cnt == 1]
-                keep = len(u) - len(ones)
-                if len(ones) and keep:
+                flat = sel.ravel()
+                u, cnt = np.unique(flat[flat >= 0], return_counts=True)
+                ones = set(u[cnt == 1].tolist())
+                # up to 8 single tiles per query (in tile order) leave the union
+                pairs = []
+                for row in sel:
+                    mine = sorted(j for j in row if j >= 0 and j in ones)
+                    pairs += mine[:8]
+                keep = len(u) - len(pairs)
+                if pairs and keep:
                     slc += 2 * keep
-                    single[g, ones] += 1
+                    single[g, pairs] += 1
                 else:
                     slc += 2 * len(u)
                 continue

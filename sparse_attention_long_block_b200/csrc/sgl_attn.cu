@@ -14,9 +14,10 @@
 // Per chunk: S = Q K^T (M 128, N 64, K 128, bf16), the softmax of each row over
 // the tile's keys at or before its query, P (fp16) back into TMEM, O = P V
 // against the scaled fp16 copy of V (the scale is multiplied back here).
-// Each pair row's output is written normalised, divided by a power of two that
-// brings its largest magnitude into [2^14, 2^15) (fp16 keeps 11 significant bits
-// and cannot overflow), with its log-sum-exp; the union pass merges them.
+// Each pair row's output is written normalised in fp16, in the units of the
+// scaled V copy (a convex combination of values below 2^15, so it cannot
+// overflow), with its log-sum-exp and the power of two that restores its
+// units; the union pass merges them.
 //
 //   warp 0     lane 0: TMA loads of each new tile's K and V (one stage)
 //   warp 1     lane 0: the MMAs
@@ -172,33 +173,37 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
     const int slot = rho / r, hl = rho % r;
     const float sc = P.scale_log2;
 
-    // Q row of chunk x (global index) into buffer `buf`, 16-byte pieces in the
-    // 128-byte swizzled K-major layout of the MMA's A operand; rows without a
-    // pair are zero-filled.  One cp.async group per call (empty past the range).
-    auto gather = [&](int x, int buf) {
-        if (x < hi) {
-            const int4 it = P.items[x];
-            const bool valid = slot < it.z;
-            const __nv_bfloat16 *src = P.q;
-            if (valid) {
-                const int t = P.sorted[it.y + slot].z;
-                const int h = (it.x / P.nbt) * r + hl;
-                src = P.q + ((size_t)t * P.h_q + h) * kD;
-            }
-            const uint32_t qb = sm.u32 + SM_Q + (uint32_t)buf * Q_BYTES;
+    const int qt = kRows / r;  // pairs per chunk
+    // This row's entry in chunk x (global index): (pair id, vision rank,
+    // position, bucket), pair id -1 for no pair; one independent load, made
+    // two chunks before its use (the entries rotate through e_a, e_b, e_c).
+    auto entry = [&](int x) -> int4 {
+        return (x < hi && slot < qt) ? P.sorted[(size_t)x * qt + slot] : make_int4(-1, 0, 0, 0);
+    };
+    auto q_src = [&](const int4 &e) -> const __nv_bfloat16 * {
+        if (e.x < 0) return nullptr;
+        const int h = (e.w / P.nbt) * r + hl;
+        return P.q + ((size_t)e.z * P.h_q + h) * kD;
+    };
+    // The row into Q buffer `buf`, 16-byte pieces in the 128-byte swizzled
+    // K-major layout of the MMA's A operand; a row without a pair is
+    // zero-filled.  One cp.async group per call.
+    auto gather = [&](const __nv_bfloat16 *src, int buf) {
+        const uint32_t qb = sm.u32 + SM_Q + (uint32_t)buf * Q_BYTES;
+        const bool valid = src != nullptr;
 #pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
-                const int hf = c16 >> 3, c = c16 & 7;
-                const uint32_t dst = qb + (uint32_t)hf * 16384u + (uint32_t)rho * 128u +
-                                     (uint32_t)((c ^ (rho & 7)) << 4);
-                ptx::cp_async16(dst, valid ? (const void *)(src + c16 * 8) : (const void *)src,
-                                valid ? 16u : 0u);
-            }
+        for (int c16 = 0; c16 < 16; ++c16) {
+            const int hf = c16 >> 3, c = c16 & 7;
+            const uint32_t dst = qb + (uint32_t)hf * 16384u + (uint32_t)rho * 128u +
+                                 (uint32_t)((c ^ (rho & 7)) << 4);
+            ptx::cp_async16(dst, valid ? (const void *)(src + c16 * 8) : (const void *)P.q,
+                            valid ? 16u : 0u);
         }
         ptx::cp_async_commit();
     };
-    gather(lo, 0);
-    gather(lo + 1, 1);
+    int4 e_a = entry(lo), e_b = entry(lo + 1), e_c = entry(lo + 2);
+    gather(q_src(e_a), 0);
+    gather(q_src(e_b), 1);
     ptx::cp_async_wait<1>();
     ptx::fence_proxy_async();
     if (hi > lo) ptx::mbar_arrive(sm.bar(B_Q_FULL));
@@ -206,15 +211,12 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
     bool ok = true;
     for (int x = lo; ok && x < hi; ++x) {
         const int j = x - lo;
-        const int4 it = P.items[x];
-        const int tile = it.x % P.nbt;
-        const bool valid = slot < it.z;
-        int sid = 0, i = 0;
-        if (valid) {
-            const int4 e = P.sorted[it.y + slot];
-            sid = e.x;
-            i = e.y;
-        }
+        const int4 e = e_a;  // this chunk's entry
+        e_a = e_b;           // chunk x + 1
+        e_b = e_c;           // chunk x + 2: gathered below
+        e_c = entry(x + 3);
+        const bool valid = e.x >= 0;
+        const int sid = e.x, i = e.y, tile = e.w % P.nbt;
         const int hi_key = valid ? min(i - tile * kKeys, kKeys - 1) : -1;
         const bool none = __all_sync(0xffffffffu, hi_key < 0);
         const uint32_t s_col = tmem + lane_base + TM_S + (uint32_t)(j & 1) * 64u;
@@ -227,7 +229,7 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
         ptx::tc_fence_after();
         // Q K^T of this chunk is done, so its buffer takes chunk x + 2; the
         // next chunk's rows (gathered one chunk ago) are handed to the MMA
-        gather(x + 2, j & 1);
+        gather(q_src(e_b), j & 1);
         ptx::cp_async_wait<1>();
         ptx::fence_proxy_async();
         if (x + 1 < hi) ptx::mbar_arrive(sm.bar(B_Q_FULL + ((j + 1) & 1)));
@@ -291,24 +293,8 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
             if (!ok) break;
         }
         ptx::tc_fence_after();
-        // epilogue: largest magnitude of the row, then the scaled fp16 row
-        float amax = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-            float o[32];
-            ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(o[k]));
-        }
-        const float inv_l = l_run > 0.f ? *P.v_scale / l_run : 0.f;
-        const float onorm = amax * inv_l;  // largest |normalised output|
-        float osc = 1.f;
-        if (onorm >= 0x1p-100f && onorm <= 3.0e38f) {
-            const int e = (int)((__float_as_uint(onorm) >> 23) & 255u) - 127;  // floor(log2)
-            osc = ldexpf(1.f, e - 14);
-        }
-        const float mul = inv_l / osc;
+        // epilogue: the normalised row in the scaled V's units (fp16)
+        const float mul = l_run > 0.f ? 1.f / l_run : 0.f;
         __half *orow = P.o + ((size_t)sid * r + hl) * kD;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -326,10 +312,8 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
                 *reinterpret_cast<uint4 *>(orow + ch * 32 + k) = v;
             }
         }
-        if (hi_key >= 0) {
+        if (hi_key >= 0)
             P.lse[(size_t)sid * r + hl] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
-            P.oscale[(size_t)sid * r + hl] = osc;
-        }
     }
     // no copy may still be landing in shared memory when the CTA ends
     ptx::cp_async_wait<0>();

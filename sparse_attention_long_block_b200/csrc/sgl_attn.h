@@ -12,22 +12,22 @@
 namespace vnsa {
 
 struct SglParams {
-    CUtensorMap tm_k, tm_v;    // K (bf16) and V (fp16 copy divided by *v_scale) as
-                               // [n][h_kv * 128], 64 x 64 boxes
+    CUtensorMap tm_k, tm_v;    // K (bf16) and V (fp16 copy divided by a power of two)
+                               // as [n][h_kv * 128], 64 x 64 boxes
     CUtensorMap tm_kc, tm_vc;  // the same in vision order (used when the vision tokens
                                // are not one contiguous run)
-    const float *v_scale;      // the power of two V was divided by
     const Counts *counts;      // vision count, contiguity and first vision position
     const __nv_bfloat16 *q;  // [n][h_q][128]
     int h_q, r;              // query heads; heads per KV group (rows per pair)
     int nbt;                 // 64-key tiles per group: bucket b = group * nbt + tile
     float scale_log2;        // softmax scale * log2(e)
     const int32_t *n_items;  // number of chunks (device)
-    const int4 *sorted;      // pairs in bucket order: (pair id, vision rank, position, 0)
-    const int4 *items;       // chunk c: (bucket, first entry of sorted, pairs, 0)
-    __half *o;               // [pair][r][128] normalised output / scale (fp16)
-    float *lse;              // [pair][r] log-sum-exp of the pair's keys (log2 units)
-    float *oscale;           // [pair][r] the power of two the stored row was divided by
+    const int4 *sorted;      // entry (chunk x, slot s) at x * (128 / r) + s: (pair id,
+                             // vision rank, position, bucket); pair id -1: no pair
+    const int4 *items;       // chunk c: (bucket, first entry, pairs, 0)
+    __half *o;               // [pair id][r][128] normalised output in the units of the
+                             // scaled V copy (fp16)
+    float *lse;              // [pair id][r] log-sum-exp of the pair's keys (log2 units)
     uint32_t *status;        // device status word
     unsigned long long wait_ns;
 };

@@ -61,6 +61,7 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 constexpr int kTextSplitKeys = 8192;
 constexpr size_t kTextPartBytes = 256ull << 20;
 constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
+constexpr int kSglSlots = 8;         // single-query pairs per (group, query) at most
 
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
 constexpr uint32_t SM_KV = 32768;                             // K ring, then V ring
@@ -112,11 +113,8 @@ struct TcParams {
     // (query, tile) pair; the tile-major pass (sgl_attn.cu) attends them, and
     // the selection epilogue merges each query's pairs into its output.
     int sgl_on;                // 1: the selection branch runs split this way
-    const int32_t *sgl_of;     // [h_kv][n_max][top_k] pair ids of each query
-    const int32_t *sgl_n;      // [h_kv][n_max] how many
-    const __half *sgl_o;       // [pair][r][d] normalised output / its scale (fp16)
-    const float *sgl_lse;      // [pair][r] log-sum-exp of the pair's keys (log2 units)
-    const float *sgl_scale;    // [pair][r] the power of two the stored row was divided by
+    __half *slc_u;             // [n_max][h_q][d] the union tiles' normalised output
+    float *slc_lse;            // [n_max][h_q] their log-sum-exp (log2 units)
 };
 
 __host__ __device__ __forceinline__ int pow2_at_least(int r) {
@@ -562,10 +560,15 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     float *pr = P.part + ((size_t)item * kRows + rho) * kPartStride;
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
+                } else if (MODE == MODE_SLC && P.sgl_on) {
+                    // no union tile (nor single-query pair: the union keeps at
+                    // least one tile of an item that has any)
+                    for (int e = 0; e < kD; e += 8)
+                        *reinterpret_cast<uint4 *>(P.slc_u + ((size_t)rc.i * L.h_q + rc.h) * kD +
+                                                   e) = make_uint4(0u, 0u, 0u, 0u);
+                    P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = -INFINITY;
                 } else {
-                    // no selected / window key (and, for the selection, no
-                    // single-query pair: the union keeps at least one tile of an
-                    // item that has any): this branch adds nothing
+                    // no selected / window key: this branch adds nothing
                     float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
@@ -605,16 +608,6 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 const float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
 #pragma unroll
                 for (int z = 0; z < kD; z += 32) ptx::prefetch_l2(part + z);
-            }
-            if (MODE == MODE_SLC && P.sgl_on) {
-                // the query's single-query pair outputs, read by the merge
-                const size_t qg = (size_t)it.g * L.n_max + rc.i;
-                const int ns = P.sgl_n[qg];
-                for (int z = 0; z < ns; ++z) {
-                    const __half *po = P.sgl_o + ((size_t)P.sgl_of[qg * L.top_k + z] * L.r + rc.hl) * kD;
-                    ptx::prefetch_l2(po);
-                    ptx::prefetch_l2(po + 64);
-                }
             }
         }
         if (item + (int)gridDim.x < w.items) {
@@ -915,22 +908,13 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             }
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
         } else if (MODE == MODE_SLC && P.sgl_on) {
-            // The selection softmax of this row is split into the union's
-            // tiles (O, m_run, l_run here) and the query's single-query pairs
-            // (normalised outputs and log-sum-exps from the tile-major pass):
-            // each part is weighted by 2^(lse_part - M) / sum over the parts.
-            const float g = rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + 1]) : 0.f;
-            const float lse_u = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
-            const size_t qg = (size_t)it.g * L.n_max + rc.i;
-            const int ns = rc.valid ? P.sgl_n[qg] : 0;
-            const int32_t *sids = P.sgl_of + qg * L.top_k;
-            float M = lse_u;
-            for (int z = 0; z < ns; ++z) M = fmaxf(M, P.sgl_lse[(size_t)sids[z] * L.r + rc.hl]);
-            const float wu = lse_u == -INFINITY ? 0.f : ptx::ex2(lse_u - M);
-            float W = wu;
-            for (int z = 0; z < ns; ++z) W += ptx::ex2(P.sgl_lse[(size_t)sids[z] * L.r + rc.hl] - M);
-            const float inv = W > 0.f ? 1.f / W : 0.f;
-            const float cu = l_run > 0.f ? wu * inv * vsc / l_run : 0.f;  // factor on the raw O
+            // The selection softmax of this row is split into the union's tiles
+            // and the query's single-query pairs (the tile-major pass); the
+            // merge kernel combines them.  Here: the union part, normalised, in
+            // the units of the scaled V copy (fp16: a convex combination of
+            // values below 2^15), and its log-sum-exp (log2 units).
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __half *orow = P.slc_u + qrow;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
@@ -938,38 +922,17 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] *= cu;
-#pragma unroll 2
-                for (int z = 0; z < ns; ++z) {
-                    const size_t pr = (size_t)sids[z] * L.r + rc.hl;
-                    const float wp = ptx::ex2(P.sgl_lse[pr] - M) * inv * P.sgl_scale[pr];
-                    const uint4 *src = reinterpret_cast<const uint4 *>(P.sgl_o + pr * kD + ch * 32);
-                    uint4 u[4];
+                for (int k = 0; k < 32; k += 8) {
+                    uint4 v;
+                    __half2 *h2 = reinterpret_cast<__half2 *>(&v);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) u[c] = __ldcs(src + c);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const __half2 *h2 = reinterpret_cast<const __half2 *>(&u[c]);
-#pragma unroll
-                        for (int y = 0; y < 4; ++y) {
-                            const float2 f = __half22float2(h2[y]);
-                            o[8 * c + 2 * y] += wp * f.x;
-                            o[8 * c + 2 * y + 1] += wp * f.y;
-                        }
-                    }
-                }
-                if (L.dbg_o_slc)
-                    for (int k = 0; k < 32; ++k) L.dbg_o_slc[prow + ch * 32 + k] = o[k];
-#pragma unroll
-                for (int k = 0; k < 32; k += 4) {
-                    float4 pv = __ldcg(reinterpret_cast<const float4 *>(part + ch * 32 + k));
-                    pv.x += g * o[k];
-                    pv.y += g * o[k + 1];
-                    pv.z += g * o[k + 2];
-                    pv.w += g * o[k + 3];
-                    __stcg(reinterpret_cast<float4 *>(part + ch * 32 + k), pv);
+                    for (int z = 0; z < 4; ++z)
+                        h2[z] = __floats2half2_rn(o[k + 2 * z] * inv, o[k + 2 * z + 1] * inv);
+                    __stcg(reinterpret_cast<uint4 *>(orow + ch * 32 + k), v);
                 }
             }
+            if (rc.valid)
+                P.slc_lse[(size_t)rc.i * L.h_q + rc.h] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
         } else if (is_slc(MODE) || MODE == MODE_SWA) {
             const float g =
                 rc.valid ? sigmoidf_(L.gate[((size_t)rc.t * L.h_q + rc.h) * 3 + (is_slc(MODE) ? 1 : 2)])
@@ -1231,9 +1194,8 @@ __device__ __forceinline__ void sel_tiles(int j, int B, int i, int &t0, int &t1)
 struct SglArgs {
     int on, nbt, cap;
     int32_t *meta;  // [0] pairs, [1] items, [2, 2 + h_kv*nbt) pairs per bucket
-    int4 *rec;      // [cap] (bucket, vision rank, rank in bucket, position); bucket -1: unused
-    int32_t *of;    // [h_kv][n_max][top_k] pair ids of each query
-    int32_t *n;     // [h_kv][n_max] how many
+    int4 *rec;      // [cap] (bucket, pair id, rank in bucket, position)
+    int32_t *n;     // [h_kv][n_max] pairs (slots used) of each query
 };
 
 __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int words, SglArgs sg) {
@@ -1241,10 +1203,11 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wpb = blockDim.x >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    uint32_t *bm = sh + (size_t)warp * (2 * words + plan_max + 32);
+    uint32_t *bm = sh + (size_t)warp * (2 * words + 2 * plan_max + 32);
     uint32_t *pre = bm + words;
     uint32_t *qm = pre + words;
     uint32_t *qcnt = qm + plan_max;  // per query of the item: its single-query tiles
+    int *sslot = (int *)(qcnt + 32); // per tile: its pair slot, -1 if it stays
     const Counts cn = *p.counts;
     const int qt = kRows / p.r;
     const int n_tiles = (cn.n_vision + qt - 1) / qt;
@@ -1315,59 +1278,79 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         __syncwarp();
         int tot = min(total, plan_max);
         if (sg.on) {
-            // Tiles that exactly one query reaches leave the plan for the
-            // tile-major pass (sgl_attn.cu), as long as one tile stays and the
-            // pair records have room; their ids are taken in one block per item.
+            // Tiles that exactly one query of the item reaches leave the plan for
+            // the tile-major pass (sgl_attn.cu): up to kSglSlots of them per query,
+            // in tile order (the rest stay), and only while at least one tile
+            // stays.  The pair (vision query i of group g, slot s) has the id
+            // (g n_max + i) kSglSlots + s, so the selection epilogue finds a
+            // query's pairs without a lookup.
             qcnt[lane] = 0u;
-            int nsing = 0;
-            for (int x = lane; x < tot; x += 32) nsing += __popc(qm[x]) == 1 ? 1 : 0;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) nsing += __shfl_xor_sync(0xffffffffu, nsing, o);
-            int base = -1;
-            if (lane == 0 && nsing > 0 && nsing < tot) base = atomicAdd(&sg.meta[0], nsing);
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (base >= 0 && base + nsing > sg.cap) {
-                // no room: the item keeps its tiles; ids below the capacity that
-                // it took are marked unused for the scatter
-                for (int x = base + lane; x < sg.cap; x += 32) sg.rec[x] = make_int4(-1, 0, 0, 0);
-                base = -1;
+            __syncwarp();
+            int npair = 0;
+            for (int xb = 0; xb < tot; xb += 32) {
+                const int x = xb + lane;
+                const uint32_t m = x < tot ? qm[x] : 0u;
+                const bool single = x < tot && __popc(m) == 1;
+                const int key = single ? __ffs(m) - 1 : 32 + lane;  // others: unique keys
+                const unsigned grp = __match_any_sync(0xffffffffu, key);
+                const int slot = single ? (int)qcnt[key] + __popc(grp & lt) : -1;
+                __syncwarp();
+                if (single && (grp & lt) == 0) qcnt[key] += (uint32_t)__popc(grp);
+                __syncwarp();
+                const bool pair = single && slot < kSglSlots;
+                if (x < tot) sslot[x] = pair ? slot : -1;
+                npair += __popc(__ballot_sync(0xffffffffu, pair));
             }
             __syncwarp();
-            if (base >= 0) {
+            if (npair >= tot) {  // every tile would leave: the item keeps them all
+                for (int x = lane; x < tot; x += 32) sslot[x] = -1;
+                npair = 0;
+            }
+            int base = 0;
+            if (npair > 0) {
+                if (lane == 0) base = atomicAdd(&sg.meta[0], npair);
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (base + npair > sg.cap) {  // cannot happen: cap holds every slot
+                    if (lane == 0) report(p.status, VNSA_ERR_BOUNDS);
+                    for (int x = lane; x < tot; x += 32) sslot[x] = -1;
+                    npair = 0;
+                }
+            }
+            __syncwarp();
+            if (npair > 0) {
                 int kept = 0, si = 0;
                 for (int xb = 0; xb < tot; xb += 32) {
                     const int x = xb + lane;
                     const uint32_t m = x < tot ? qm[x] : 0u;
                     const int tl = x < tot ? out[1 + x] : 0;
-                    const bool single = x < tot && __popc(m) == 1;
-                    const bool keep = x < tot && !single;
+                    const int sl = x < tot ? sslot[x] : -1;
+                    const bool pair = sl >= 0;
+                    const bool keep = x < tot && !pair;
                     // every lane holds its entry before any entry is moved down
                     const unsigned bk = __ballot_sync(0xffffffffu, keep);
-                    const unsigned bs = __ballot_sync(0xffffffffu, single);
+                    const unsigned bp = __ballot_sync(0xffffffffu, pair);
                     if (keep) {
                         const int pos = kept + __popc(bk & lt);
                         out[1 + pos] = tl;
                         qm[pos] = m;
                     }
-                    if (single) {
-                        const int sid = base + si + __popc(bs & lt);
-                        const int qi = __ffs(m) - 1;
-                        const int i = q0 + qi;
+                    if (pair) {
+                        const int i = q0 + __ffs(m) - 1;
+                        const int id = (g * p.n_max + i) * kSglSlots + sl;
                         const int bucket = g * sg.nbt + tl;
                         const int lp = atomicAdd(&sg.meta[2 + bucket], 1);
-                        sg.rec[sid] = make_int4(bucket, i, lp, p.vis[i]);
-                        const int slot = (int)atomicAdd(&qcnt[qi], 1u);
-                        sg.of[((size_t)g * p.n_max + i) * p.top_k + slot] = sid;
+                        sg.rec[base + si + __popc(bp & lt)] = make_int4(bucket, id, lp, p.vis[i]);
                     }
                     kept += __popc(bk);
-                    si += __popc(bs);
+                    si += __popc(bp);
                     __syncwarp();
                 }
                 tot = kept;
             }
             __syncwarp();
             for (int qi = lane; qi < nq; qi += 32)
-                sg.n[(size_t)g * p.n_max + q0 + qi] = (int)qcnt[qi];
+                sg.n[(size_t)g * p.n_max + q0 + qi] =
+                    npair > 0 ? min((int)qcnt[qi], kSglSlots) : 0;
         }
         for (int x = lane; x < tot; x += 32) out[1 + plan_max + x] = (int)qm[x];
         if (lane == 0) {
@@ -1436,22 +1419,148 @@ __global__ void __launch_bounds__(1024) sgl_scan_kernel(int32_t *meta, int nbk, 
     }
 }
 
-// Pairs in bucket order: pair `sid` goes to off[bucket] + its rank in the
-// bucket, as (sid, vision rank, position, 0); and the tile-major pass's chunk table:
-// chunk c of bucket b is item choff[b] + c, (b, off[b] + c qt, pairs, 0).
+// The tile-major pass's chunk table and entries.  Chunk c of bucket b is item
+// choff[b] + c = (b, first entry, pairs, 0); entries are laid out qt per chunk,
+// entry (chunk x, slot s) at x qt + s = (pair id, vision rank, position,
+// bucket), and the slots of a bucket's last chunk past its pairs hold
+// (-1, 0, 0, bucket).  So a row of the tile-major pass finds its entry in one
+// independent load.
 __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *sorted,
-                                   int4 *items, int nbk, int cap, int qt) {
+                                   int4 *items, int nbk, int cap, int qt, int n_max) {
     const int n = min(meta[0], cap);
-    const int32_t *hist = meta + 2, *off = meta + 2 + nbk, *choff = meta + 2 + 2 * nbk;
+    const int32_t *hist = meta + 2, *choff = meta + 2 + 2 * nbk;
     const int tid = blockIdx.x * blockDim.x + threadIdx.x, step = gridDim.x * blockDim.x;
-    for (int sid = tid; sid < n; sid += step) {
-        const int4 e = rec[sid];
-        if (e.x >= 0) sorted[off[e.x] + e.z] = make_int4(sid, e.y, e.w, 0);
+    for (int k = tid; k < n; k += step) {
+        const int4 e = rec[k];  // (bucket, id, rank in bucket, position)
+        const int i = (e.y / kSglSlots) % n_max;
+        sorted[(size_t)choff[e.x] * qt + e.z] = make_int4(e.y, i, e.w, e.x);
     }
     for (int b = tid; b < nbk; b += step) {
         const int cnt = hist[b];
-        for (int c = 0; c * qt < cnt; ++c)
-            items[choff[b] + c] = make_int4(b, off[b] + c * qt, min(qt, cnt - c * qt), 0);
+        const int nch = (cnt + qt - 1) / qt;
+        for (int c = 0; c < nch; ++c)
+            items[choff[b] + c] =
+                make_int4(b, (choff[b] + c) * qt, min(qt, cnt - c * qt), 0);
+        for (int x = cnt; x < nch * qt; ++x)
+            sorted[(size_t)choff[b] * qt + x] = make_int4(-1, 0, 0, b);
+    }
+}
+
+// The selection output of each (vision query, head): the union tiles' part
+// (slc_u, slc_lse) and the query's single-query pairs (slot ids qg kSglSlots +
+// z, z < n[qg]: sgl_o, sgl_lse), each the exact softmax over its keys,
+// combined with the weights 2^(lse_part - M) / sum over the parts; then
+// partial += sigmoid(g_slc) * o_slc (fp32) and the optional export.  Every
+// address follows from (group, query, slot), so all of a row's loads are
+// independent; one warp per (group, query), lane l holding dims 4l .. 4l + 3 of
+// each head (256-byte rows read whole by the warp), heads one after another;
+// the weights of head hl live in lane hl.
+struct SlcMergeArgs {
+    const int32_t *n;
+    const __half *sgl_o, *slc_u;
+    const float *sgl_lse, *slc_lse, *v_scale;
+};
+
+__device__ __forceinline__ float4 half4_to_float4(uint2 u) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+    const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <int RMAX>
+__global__ void __launch_bounds__(256) slc_merge_kernel(LayerParams p, SlcMergeArgs a) {
+    const Counts cn = *p.counts;
+    const int lane = threadIdx.x & 31;
+    const int r = p.r;
+    const float vsc = *a.v_scale;
+    const long long rows = (long long)p.h_kv * cn.n_vision;
+    for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < rows;
+         wid += ((long long)gridDim.x * blockDim.x) >> 5) {
+        const int g = (int)(wid / cn.n_vision), i = (int)(wid % cn.n_vision);
+        const int h0 = g * r;
+        const int t = p.vis[i];
+        const size_t qg = (size_t)g * p.n_max + i;
+        const size_t id0 = qg * kSglSlots;
+        // round trip 1: the pair count, every slot's log-sum-exp (slots past the
+        // count hold stale values and are masked after the load), the union's
+        // log-sum-exp and the gate, all independent (lane hl < r: head hl)
+        const int ns = a.n[qg];
+        float lu = -INFINITY, lz[kSglSlots], gl = 0.f;
+        if (lane < r) {
+            lu = a.slc_lse[(size_t)i * p.h_q + h0 + lane];
+            gl = p.gate[((size_t)t * p.h_q + h0 + lane) * 3 + 1];
+#pragma unroll
+            for (int z = 0; z < kSglSlots; ++z) lz[z] = a.sgl_lse[(id0 + z) * r + lane];
+        }
+        float mx = lu;
+#pragma unroll
+        for (int z = 0; z < kSglSlots; ++z) {
+            lz[z] = (lane < r && z < ns) ? lz[z] : -INFINITY;
+            mx = fmaxf(mx, lz[z]);
+        }
+        const float wu = lu == -INFINITY ? 0.f : exp2f(lu - mx);
+        float wsum = wu;
+#pragma unroll
+        for (int z = 0; z < kSglSlots; ++z) {
+            lz[z] = lz[z] == -INFINITY ? 0.f : exp2f(lz[z] - mx);
+            wsum += lz[z];
+        }
+        const float norm = wsum > 0.f ? vsc / wsum : 0.f;  // back to V's units
+        const float cu = wu * norm;
+#pragma unroll
+        for (int z = 0; z < kSglSlots; ++z) lz[z] *= norm;
+        gl = lane < r ? sigmoidf_(gl) : 0.f;
+        // round trip 2: the union part and the pairs of every head (no store in
+        // between, so the loads of consecutive heads overlap)
+        float4 acc[RMAX];
+#pragma unroll
+        for (int hl = 0; hl < RMAX; ++hl) {
+            acc[hl] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (hl >= r) continue;
+            const size_t prow = ((size_t)i * p.h_q + h0 + hl) * kD + 4 * lane;
+            const float c_u = __shfl_sync(0xffffffffu, cu, hl);
+            const float4 u = half4_to_float4(__ldcs(reinterpret_cast<const uint2 *>(a.slc_u + prow)));
+            acc[hl] = make_float4(c_u * u.x, c_u * u.y, c_u * u.z, c_u * u.w);
+#pragma unroll
+            for (int z = 0; z < kSglSlots; ++z) {
+                const float wz = __shfl_sync(0xffffffffu, lz[z], hl);
+                if (z < ns) {
+                    const float4 f = half4_to_float4(__ldcs(reinterpret_cast<const uint2 *>(
+                        a.sgl_o + ((id0 + z) * r + hl) * kD + 4 * lane)));
+                    acc[hl].x += wz * f.x;
+                    acc[hl].y += wz * f.y;
+                    acc[hl].z += wz * f.z;
+                    acc[hl].w += wz * f.w;
+                }
+            }
+        }
+        // round trip 3: partial += sigmoid(g_slc) o_slc for every head
+        float4 pv[RMAX];
+#pragma unroll
+        for (int hl = 0; hl < RMAX; ++hl)
+            if (hl < r)
+                pv[hl] = __ldcs(reinterpret_cast<const float4 *>(
+                    p.o_cmp_ws + ((size_t)i * p.h_q + h0 + hl) * kD + 4 * lane));
+#pragma unroll
+        for (int hl = 0; hl < RMAX; ++hl) {
+            const float gh = __shfl_sync(0xffffffffu, gl, hl);
+            if (hl >= r) continue;
+            const float4 o = acc[hl];
+            pv[hl].x += gh * o.x;
+            pv[hl].y += gh * o.y;
+            pv[hl].z += gh * o.z;
+            pv[hl].w += gh * o.w;
+            __stcs(reinterpret_cast<float4 *>(p.o_cmp_ws + ((size_t)i * p.h_q + h0 + hl) * kD +
+                                              4 * lane),
+                   pv[hl]);
+            if (p.dbg_o_slc) {
+                float *dbg = p.dbg_o_slc + ((size_t)t * p.h_q + h0 + hl) * kD + 4 * lane;
+                dbg[0] = o.x;
+                dbg[1] = o.y;
+                dbg[2] = o.z;
+                dbg[3] = o.w;
+            }
+        }
     }
 }
 
@@ -1590,19 +1699,16 @@ struct TcState {
     float *part;
     // single-query selection tiles (block 64): see TcParams and sgl_attn.h
     int sgl_on, sgl_nbt, sgl_cap;
-    int32_t *sgl_meta, *sgl_of, *sgl_n;
+    int32_t *sgl_meta, *sgl_n;
     int4 *sgl_rec, *sgl_sorted, *sgl_items;
-    __half *sgl_o;
-    float *sgl_lse, *sgl_scale;
+    __half *sgl_o, *slc_u;
+    float *sgl_lse, *slc_lse;
 };
 
-// Single-query pairs the workspace holds, per query and group on average;
-// beyond it items keep their single-query tiles in the union.
-constexpr int kSglPerQuery = 6;
 
 struct SglSizes {
     int on, nbt, nbk, cap;
-    size_t meta, rec, sorted, items, of, n, o, lse, scale, total;
+    size_t meta, rec, sorted, items, n, o, lse, u, ulse, total;
 };
 
 static SglSizes sgl_sizes(const vnsa_config &c) {
@@ -1613,17 +1719,19 @@ static SglSizes sgl_sizes(const vnsa_config &c) {
     const int r = c.h_q / c.h_kv;
     z.nbt = (c.n_max + kKeys - 1) / kKeys;
     z.nbk = c.h_kv * z.nbt;
-    z.cap = (int)std::min<long long>((long long)c.h_kv * c.n_max * kSglPerQuery, 1ll << 30);
+    const int qt = kRows / r;
+    z.cap = c.h_kv * c.n_max * kSglSlots;  // every (group, query, slot) id
+    const size_t chunks = (size_t)z.cap / qt + z.nbk + 1;
     z.meta = up256((size_t)(2 + 3 * z.nbk + 1) * 4);
     z.rec = up256((size_t)z.cap * 16);
-    z.sorted = up256((size_t)z.cap * 16);
-    z.items = up256(((size_t)z.cap / (kRows / r) + z.nbk + 1) * 16);
-    z.of = up256((size_t)c.h_kv * c.n_max * c.top_k * 4);
+    z.sorted = up256(chunks * qt * 16);
+    z.items = up256(chunks * 16);
     z.n = up256((size_t)c.h_kv * c.n_max * 4);
     z.o = up256((size_t)z.cap * r * kD * 2);
     z.lse = up256((size_t)z.cap * r * 4);
-    z.scale = up256((size_t)z.cap * r * 4);
-    z.total = z.meta + z.rec + z.sorted + z.items + z.of + z.n + z.o + z.lse + z.scale;
+    z.u = up256((size_t)c.n_max * c.h_q * kD * 2);
+    z.ulse = up256((size_t)c.n_max * c.h_q * 4);
+    z.total = z.meta + z.rec + z.sorted + z.items + z.n + z.o + z.lse + z.u + z.ulse;
     return z;
 }
 
@@ -1698,11 +1806,11 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
         st->sgl_rec = (int4 *)(q += z.meta);
         st->sgl_sorted = (int4 *)(q += z.rec);
         st->sgl_items = (int4 *)(q += z.sorted);
-        st->sgl_of = (int32_t *)(q += z.items);
-        st->sgl_n = (int32_t *)(q += z.of);
+        st->sgl_n = (int32_t *)(q += z.items);
         st->sgl_o = (__half *)(q += z.n);
         st->sgl_lse = (float *)(q += z.o);
-        st->sgl_scale = (float *)(q += z.lse);
+        st->slc_u = (__half *)(q += z.lse);
+        st->slc_lse = (float *)(q += z.u);
     }
     cudaError_t e = cudaSuccess;
     for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
@@ -1731,11 +1839,8 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     P.part_items = st->part_items;
     const bool sgl = st->sgl_on && c.block == kKeys;
     P.sgl_on = 0;  // set for the selection launch below
-    P.sgl_of = st->sgl_of;
-    P.sgl_n = st->sgl_n;
-    P.sgl_o = st->sgl_o;
-    P.sgl_lse = st->sgl_lse;
-    P.sgl_scale = st->sgl_scale;
+    P.slc_u = st->slc_u;
+    P.slc_lse = st->slc_lse;
     const int nb_rows = L.nb_max > 0 ? L.nb_max : 1;  // compression blocks
     if (!make_map(&P.tm_k, L.k, c.h_kv, L.n, false) ||
         !make_map(&P.tm_v, st->vh, c.h_kv, L.n, true) ||
@@ -1795,7 +1900,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     {
         const int words = ((c.n_max + kKeys - 1) / kKeys + 31) / 32 + 1;
         const int wpb = 4;
-        const size_t smem = (size_t)wpb * (2 * words + st->plan_max + 32) * 4;
+        const size_t smem = (size_t)wpb * (2 * words + 2 * st->plan_max + 32) * 4;
         if (smem > 48 * 1024) {
             e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem);
@@ -1812,7 +1917,6 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
             sa.cap = st->sgl_cap;
             sa.meta = st->sgl_meta;
             sa.rec = st->sgl_rec;
-            sa.of = st->sgl_of;
             sa.n = st->sgl_n;
         }
         union_kernel<<<st->num_sms * 8, wpb * 32, smem, s>>>(L, st->plan, st->plan_max, words, sa);
@@ -1822,7 +1926,8 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
             sgl_scan_kernel<<<1, 1024, 0, s>>>(st->sgl_meta, nbk, kRows / L.r);
             sgl_scatter_kernel<<<st->num_sms * 4, 256, 0, s>>>(st->sgl_meta, st->sgl_rec,
                                                                st->sgl_sorted, st->sgl_items, nbk,
-                                                               st->sgl_cap, kRows / L.r);
+                                                               st->sgl_cap, kRows / L.r,
+                                                               c.n_max);
             *launches += 2;
         }
     }
@@ -1838,7 +1943,6 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         sp.tm_v = P.tm_v;
         sp.tm_kc = P.tm_kc;
         sp.tm_vc = P.tm_vc;
-        sp.v_scale = st->v_scale;
         sp.counts = L.counts;
         sp.q = (const __nv_bfloat16 *)L.q;
         sp.h_q = c.h_q;
@@ -1850,7 +1954,6 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         sp.items = st->sgl_items;
         sp.o = st->sgl_o;
         sp.lse = st->sgl_lse;
-        sp.oscale = st->sgl_scale;
         sp.status = L.status;
         sp.wait_ns = L.wait_ns;
         if ((e = launch_sgl_attn(sp, st->num_sms, s)) != cudaSuccess) return e;
@@ -1858,6 +1961,16 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         P.sgl_on = 1;
         if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
         P.sgl_on = 0;
+        SlcMergeArgs ma;
+        ma.n = st->sgl_n;
+        ma.sgl_o = st->sgl_o;
+        ma.slc_u = st->slc_u;
+        ma.sgl_lse = st->sgl_lse;
+        ma.slc_lse = st->slc_lse;
+        ma.v_scale = st->v_scale;
+        if (L.r <= 8) slc_merge_kernel<8><<<st->num_sms * 16, 256, 0, s>>>(L, ma);
+        else slc_merge_kernel<16><<<st->num_sms * 16, 256, 0, s>>>(L, ma);
+        ++*launches;
     } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
         return e;
     }
