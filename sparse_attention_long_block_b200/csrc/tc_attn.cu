@@ -1451,114 +1451,114 @@ __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *s
 // z, z < n[qg]: sgl_o, sgl_lse), each the exact softmax over its keys,
 // combined with the weights 2^(lse_part - M) / sum over the parts; then
 // partial += sigmoid(g_slc) * o_slc (fp32) and the optional export.  Every
-// address follows from (group, query, slot), so all of a row's loads are
-// independent; one warp per (group, query), lane l holding dims 4l .. 4l + 3 of
-// each head (256-byte rows read whole by the warp), heads one after another;
-// the weights of head hl live in lane hl.
+// address follows from (group, query, slot), so a row's loads are independent.
+// One warp per (group, query); its r heads x 128 dims are cut into 16-dim
+// chunks, chunk c = lane + 32 k (head c / 8), so a warp's load instruction
+// covers four heads contiguously and each lane computes the weights of its
+// own (at most two) heads.
 struct SlcMergeArgs {
     const int32_t *n;
     const __half *sgl_o, *slc_u;
     const float *sgl_lse, *slc_lse, *v_scale;
 };
 
-__device__ __forceinline__ float4 half4_to_float4(uint2 u) {
+__device__ __forceinline__ void acc_half8(float (&acc)[8], uint4 u, float w) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&u);
-    const float2 a = __half22float2(h[0]), b = __half22float2(h[1]);
-    return make_float4(a.x, a.y, b.x, b.y);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(h[q]);
+        acc[2 * q] = fmaf(w, f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(w, f.y, acc[2 * q + 1]);
+    }
 }
 
-template <int RMAX>
 __global__ void __launch_bounds__(256) slc_merge_kernel(LayerParams p, SlcMergeArgs a) {
     const Counts cn = *p.counts;
     const int lane = threadIdx.x & 31;
-    const int r = p.r;
+    const int r = p.r, nv = cn.n_vision;
+    const int nchunk = r * (kD / 16);  // 16-dim chunks of a row (56 for 7 heads)
     const float vsc = *a.v_scale;
-    const long long rows = (long long)p.h_kv * cn.n_vision;
-    for (long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < rows;
-         wid += ((long long)gridDim.x * blockDim.x) >> 5) {
-        const int g = (int)(wid / cn.n_vision), i = (int)(wid % cn.n_vision);
+    const int rows = p.h_kv * nv;
+    for (int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < rows;
+         wid += (gridDim.x * blockDim.x) >> 5) {
+        const int g = wid / nv, i = wid - g * nv;
         const int h0 = g * r;
         const int t = p.vis[i];
         const size_t qg = (size_t)g * p.n_max + i;
         const size_t id0 = qg * kSglSlots;
-        // round trip 1: the pair count, every slot's log-sum-exp (slots past the
-        // count hold stale values and are masked after the load), the union's
-        // log-sum-exp and the gate, all independent (lane hl < r: head hl)
         const int ns = a.n[qg];
-        float lu = -INFINITY, lz[kSglSlots], gl = 0.f;
-        if (lane < r) {
-            lu = a.slc_lse[(size_t)i * p.h_q + h0 + lane];
-            gl = p.gate[((size_t)t * p.h_q + h0 + lane) * 3 + 1];
 #pragma unroll
-            for (int z = 0; z < kSglSlots; ++z) lz[z] = a.sgl_lse[(id0 + z) * r + lane];
-        }
-        float mx = lu;
+        for (int k = 0; k < 2; ++k) {
+            const int c = lane + 32 * k;
+            if (c >= nchunk) continue;
+            const int hl = c >> 3, d0 = (c & 7) * 16;
+            // weights of this chunk's head (slots past the count hold stale
+            // values and are masked after the load)
+            const float lu = a.slc_lse[(size_t)i * p.h_q + h0 + hl];
+            float lz[kSglSlots];
 #pragma unroll
-        for (int z = 0; z < kSglSlots; ++z) {
-            lz[z] = (lane < r && z < ns) ? lz[z] : -INFINITY;
-            mx = fmaxf(mx, lz[z]);
-        }
-        const float wu = lu == -INFINITY ? 0.f : exp2f(lu - mx);
-        float wsum = wu;
-#pragma unroll
-        for (int z = 0; z < kSglSlots; ++z) {
-            lz[z] = lz[z] == -INFINITY ? 0.f : exp2f(lz[z] - mx);
-            wsum += lz[z];
-        }
-        const float norm = wsum > 0.f ? vsc / wsum : 0.f;  // back to V's units
-        const float cu = wu * norm;
-#pragma unroll
-        for (int z = 0; z < kSglSlots; ++z) lz[z] *= norm;
-        gl = lane < r ? sigmoidf_(gl) : 0.f;
-        // round trip 2: the union part and the pairs of every head (no store in
-        // between, so the loads of consecutive heads overlap)
-        float4 acc[RMAX];
-#pragma unroll
-        for (int hl = 0; hl < RMAX; ++hl) {
-            acc[hl] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (hl >= r) continue;
-            const size_t prow = ((size_t)i * p.h_q + h0 + hl) * kD + 4 * lane;
-            const float c_u = __shfl_sync(0xffffffffu, cu, hl);
-            const float4 u = half4_to_float4(__ldcs(reinterpret_cast<const uint2 *>(a.slc_u + prow)));
-            acc[hl] = make_float4(c_u * u.x, c_u * u.y, c_u * u.z, c_u * u.w);
+            for (int z = 0; z < kSglSlots; ++z) lz[z] = a.sgl_lse[(id0 + z) * r + hl];
+            const size_t urow = ((size_t)i * p.h_q + h0 + hl) * kD + d0;
+            const uint4 *us = reinterpret_cast<const uint4 *>(a.slc_u + urow);
+            const uint4 u0 = __ldcs(us), u1 = __ldcs(us + 1);
+            uint4 pz[kSglSlots][2];
 #pragma unroll
             for (int z = 0; z < kSglSlots; ++z) {
-                const float wz = __shfl_sync(0xffffffffu, lz[z], hl);
                 if (z < ns) {
-                    const float4 f = half4_to_float4(__ldcs(reinterpret_cast<const uint2 *>(
-                        a.sgl_o + ((id0 + z) * r + hl) * kD + 4 * lane)));
-                    acc[hl].x += wz * f.x;
-                    acc[hl].y += wz * f.y;
-                    acc[hl].z += wz * f.z;
-                    acc[hl].w += wz * f.w;
+                    const uint4 *ps = reinterpret_cast<const uint4 *>(
+                        a.sgl_o + ((id0 + z) * r + hl) * kD + d0);
+                    pz[z][0] = __ldcs(ps);
+                    pz[z][1] = __ldcs(ps + 1);
                 }
             }
-        }
-        // round trip 3: partial += sigmoid(g_slc) o_slc for every head
-        float4 pv[RMAX];
+            const float gl = sigmoidf_(p.gate[((size_t)t * p.h_q + h0 + hl) * 3 + 1]);
+            float mx = lu;
 #pragma unroll
-        for (int hl = 0; hl < RMAX; ++hl)
-            if (hl < r)
-                pv[hl] = __ldcs(reinterpret_cast<const float4 *>(
-                    p.o_cmp_ws + ((size_t)i * p.h_q + h0 + hl) * kD + 4 * lane));
+            for (int z = 0; z < kSglSlots; ++z) {
+                lz[z] = z < ns ? lz[z] : -INFINITY;
+                mx = fmaxf(mx, lz[z]);
+            }
+            const float wu = lu == -INFINITY ? 0.f : exp2f(lu - mx);
+            float wsum = wu;
 #pragma unroll
-        for (int hl = 0; hl < RMAX; ++hl) {
-            const float gh = __shfl_sync(0xffffffffu, gl, hl);
-            if (hl >= r) continue;
-            const float4 o = acc[hl];
-            pv[hl].x += gh * o.x;
-            pv[hl].y += gh * o.y;
-            pv[hl].z += gh * o.z;
-            pv[hl].w += gh * o.w;
-            __stcs(reinterpret_cast<float4 *>(p.o_cmp_ws + ((size_t)i * p.h_q + h0 + hl) * kD +
-                                              4 * lane),
-                   pv[hl]);
+            for (int z = 0; z < kSglSlots; ++z) {
+                lz[z] = lz[z] == -INFINITY ? 0.f : exp2f(lz[z] - mx);
+                wsum += lz[z];
+            }
+            const float norm = wsum > 0.f ? vsc / wsum : 0.f;  // back to V's units
+            float acc0[8], acc1[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc0[e] = acc1[e] = 0.f;
+            acc_half8(acc0, u0, wu * norm);
+            acc_half8(acc1, u1, wu * norm);
+#pragma unroll
+            for (int z = 0; z < kSglSlots; ++z) {
+                if (z < ns) {
+                    acc_half8(acc0, pz[z][0], lz[z] * norm);
+                    acc_half8(acc1, pz[z][1], lz[z] * norm);
+                }
+            }
+            float4 *pr = reinterpret_cast<float4 *>(p.o_cmp_ws + urow);
+            float4 pv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pv[q] = __ldcs(pr + q);
+            const float *ac[2] = {acc0, acc1};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float *o4 = ac[q >> 1] + 4 * (q & 1);
+                pv[q].x = fmaf(gl, o4[0], pv[q].x);
+                pv[q].y = fmaf(gl, o4[1], pv[q].y);
+                pv[q].z = fmaf(gl, o4[2], pv[q].z);
+                pv[q].w = fmaf(gl, o4[3], pv[q].w);
+                __stcs(pr + q, pv[q]);
+            }
             if (p.dbg_o_slc) {
-                float *dbg = p.dbg_o_slc + ((size_t)t * p.h_q + h0 + hl) * kD + 4 * lane;
-                dbg[0] = o.x;
-                dbg[1] = o.y;
-                dbg[2] = o.z;
-                dbg[3] = o.w;
+                float *dbg = p.dbg_o_slc + ((size_t)t * p.h_q + h0 + hl) * kD + d0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    dbg[e] = acc0[e];
+                    dbg[8 + e] = acc1[e];
+                }
             }
         }
     }
@@ -1968,8 +1968,7 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         ma.sgl_lse = st->sgl_lse;
         ma.slc_lse = st->slc_lse;
         ma.v_scale = st->v_scale;
-        if (L.r <= 8) slc_merge_kernel<8><<<st->num_sms * 16, 256, 0, s>>>(L, ma);
-        else slc_merge_kernel<16><<<st->num_sms * 16, 256, 0, s>>>(L, ma);
+        slc_merge_kernel<<<st->num_sms * 16, 256, 0, s>>>(L, ma);
         ++*launches;
     } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
         return e;
