@@ -38,7 +38,15 @@ def test_v_scaled_by_powers_of_two_far_from_unit_range():
         assert np.array_equal(g["out"].astype(np.float64), base["out"].astype(np.float64) * scale)
         o = oracle.forward(oracle_params(wl), xs["q"], xs["k"], xs["v"], xs["is_vision"],
                            xs["gate"], xs["w_k"], xs["w_v"], want=("idx", "imp"))
-        check_selection(np.transpose(g["idx"][:, :nv], (1, 0, 2)), o["idx"][:nv],
-                        o["imp"][:nv], wl.top_k, block=wl.block, ranks=np.arange(nv))
-        err = float(np.abs(g["out"] - o["out"]).max()) / scale
+        gsel = np.transpose(g["idx"][:, :nv], (1, 0, 2))
+        swapped = check_selection(gsel, o["idx"][:nv], o["imp"][:nv], wl.top_k,
+                                  block=wl.block, ranks=np.arange(nv))
+        ref = o["out"].copy()
+        if swapped:  # near-tied blocks the kernel chose: the oracle on its selection
+            rows = np.nonzero(xs["is_vision"])[0][swapped].astype(np.int32)
+            o2 = oracle.forward(oracle_params(wl), xs["q"], xs["k"], xs["v"], xs["is_vision"],
+                                xs["gate"], xs["w_k"], xs["w_v"], rows=rows,
+                                forced_idx=gsel[swapped])
+            ref[rows] = o2["out"]
+        err = float(np.abs(g["out"] - ref).max()) / scale
         assert err <= 2e-2, (scale, err)
