@@ -64,19 +64,21 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
     if (m > 0 && ncand > m) {
         // 1. the lane's T largest candidate bit patterns, descending
         uint32_t t[4] = {0u, 0u, 0u, 0u};
+        // (every load of the lane's stripe is issued before the candidate test,
+        // so a batch of 16 is in flight at once; masked values count as 0)
         if (m <= 32) {
-#pragma unroll 8
+#pragma unroll 16
             for (int j = lane; j < c; j += 32) {
-                if (!is_cand(j)) continue;
-                const uint32_t kj = bits_of(load(j));
+                const float v = load(j);
+                const uint32_t kj = is_cand(j) ? bits_of(v) : 0u;
                 if (kj > t[0]) { t[1] = t[0]; t[0] = kj; }
                 else if (kj > t[1]) { t[1] = kj; }
             }
         } else {
-#pragma unroll 8
+#pragma unroll 16
             for (int j = lane; j < c; j += 32) {
-                if (!is_cand(j)) continue;
-                const uint32_t kj = bits_of(load(j));
+                const float v = load(j);
+                const uint32_t kj = is_cand(j) ? bits_of(v) : 0u;
                 if (kj <= t[3]) continue;
                 if (kj > t[0]) { t[3] = t[2]; t[2] = t[1]; t[1] = t[0]; t[0] = kj; }
                 else if (kj > t[1]) { t[3] = t[2]; t[2] = t[1]; t[1] = kj; }
@@ -104,7 +106,7 @@ __device__ __forceinline__ void topk_select_row(const float *row, int c, int own
         }
         // 2. survivors in block order
         int cnt = 0;
-#pragma unroll 4
+#pragma unroll 8
         for (int base = 0; base < c; base += 32) {
             const int j = base + lane;
             const float v = j < c ? load(j) : 0.f;
