@@ -193,6 +193,7 @@ __device__ __forceinline__ float *part_of(const DecodeParams &p, int br, int g, 
 
 // ---------------------------------------------------------------------------
 __global__ void decode_prep_kernel(DecodeParams p) {
+    wait_prior_grid();
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
     Counts cn = *p.counts;
     const int t = p.n - 1;
@@ -233,6 +234,7 @@ __global__ void decode_prep_kernel(DecodeParams p) {
 // go to s_cmp for the importance; the split's softmax state to the partials.
 template <typename T, int D, int R>
 __global__ void __launch_bounds__(kWarps * 32) decode_cmp_kernel(DecodeParams p) {
+    wait_prior_grid();
     constexpr int PER = D / 32;
     extern __shared__ float sm[];
     const Counts cn = *p.counts;
@@ -284,6 +286,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_cmp_kernel(DecodeParams p)
 // selection.
 template <int D>
 __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeParams p) {
+    wait_prior_grid();
     extern __shared__ float sm[];  // lse [16], split weights [16][kSplit], importance
     __shared__ uint64_t buf[128];
     const Counts cn = *p.counts;
@@ -324,6 +327,7 @@ __global__ void __launch_bounds__(1024) decode_select_kernel(DecodeParams p) {
 // a dense key a position.  Each split takes an even share of each key range.
 template <typename T, int D, int R>
 __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p) {
+    wait_prior_grid();
     constexpr int PER = D / 32;
     extern __shared__ float sm[];
     const Counts cn = *p.counts;
@@ -426,6 +430,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(DecodeParams p
 // window or text), the gates, the output row.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
+    wait_prior_grid();
     __shared__ float fw[3][kSplit];
     const Counts cn = *p.counts;
     const bool vision = cn.pad[1] != 0;
@@ -482,6 +487,25 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
     ((T *)p.out)[(size_t)h * D + e] = from_f<T>(o);
 }
 
+// A decode step is a chain of small dependent kernels; each is launched with
+// programmatic stream serialisation, so it is scheduled while the previous one
+// drains and waits for it in wait_prior_grid().
+template <typename Kern>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       const DecodeParams &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <typename T, int D, int R>
 cudaError_t launch_typed(const DecodeParams &p, cudaStream_t s, int *launches) {
     const size_t part_smem = (size_t)kWarps * R * (D + 2) * sizeof(float);
@@ -496,12 +520,16 @@ cudaError_t launch_typed(const DecodeParams &p, cudaStream_t s, int *launches) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem);
     if (e != cudaSuccess) return e;
     const dim3 split(kSplit, p.h_kv);
-    decode_cmp_kernel<T, D, R><<<split, kWarps * 32, part_smem, s>>>(p);
-    decode_select_kernel<D><<<p.h_kv, 1024, sel_smem, s>>>(p);
-    decode_attn_kernel<T, D, R><<<split, kWarps * 32, part_smem, s>>>(p);
-    decode_combine_kernel<T, D><<<p.h_q, D, 0, s>>>(p);
+    if (e == cudaSuccess)
+        e = launch_pdl(decode_cmp_kernel<T, D, R>, split, dim3(kWarps * 32), part_smem, s, p);
+    if (e == cudaSuccess)
+        e = launch_pdl(decode_select_kernel<D>, dim3(p.h_kv), dim3(1024), sel_smem, s, p);
+    if (e == cudaSuccess)
+        e = launch_pdl(decode_attn_kernel<T, D, R>, split, dim3(kWarps * 32), part_smem, s, p);
+    if (e == cudaSuccess)
+        e = launch_pdl(decode_combine_kernel<T, D>, dim3(p.h_q), dim3(D), 0, s, p);
     *launches += 4;
-    return cudaGetLastError();
+    return e;
 }
 
 template <typename T, int D>

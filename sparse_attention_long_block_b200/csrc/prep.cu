@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(256) pool_proj_kernel(
     constexpr int NPART = 256 / D;     // threads per output column
     constexpr int JBP = JB / NPART;    // blocks per thread in the projection
     __shared__ float mean[JB][D];
+    wait_prior_grid();
     const int nb = counts->nc;
     // from_pad: only the blocks from counts->pad[0] on (the block a decode
     // step completed, or none)
@@ -194,6 +195,7 @@ __global__ void __launch_bounds__(256) pool_mlp_kernel(
     constexpr int JBP = JB / NPART;
     __shared__ float mean[JB][D];
     __shared__ float hid[JB][kCmpMlpMaxHidden];
+    wait_prior_grid();
     const int nb = counts->nc;
     const int j0 = (from_pad ? counts->pad[0] : 0) + blockIdx.x * JB;
     if (j0 >= nb) return;
