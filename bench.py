@@ -753,7 +753,8 @@ def run_decode_bench(args, rank, world, local_rank):
 
 
 # the sources that define the tensor-core attention kernel and its launches
-ATTN_KERNEL_SOURCES = ("tc_attn.cu", "tc_attn.h", "tc_ptx.cuh", "common.cuh", "kernels.h")
+ATTN_KERNEL_SOURCES = ("tc_attn.cu", "tc_attn.h", "sgl_attn.cu", "sgl_attn.h", "tc_ptx.cuh",
+                       "common.cuh", "kernels.h", "config.h")
 
 
 def layer_build_id():
