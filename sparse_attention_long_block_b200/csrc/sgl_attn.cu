@@ -227,12 +227,8 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
             if (!ok) break;
         }
         ptx::tc_fence_after();
-        // Q K^T of this chunk is done, so its buffer takes chunk x + 2; the
-        // next chunk's rows (gathered one chunk ago) are handed to the MMA
+        // Q K^T of this chunk is done, so its buffer takes chunk x + 2
         gather(q_src(e_b), j & 1);
-        ptx::cp_async_wait<1>();
-        ptx::fence_proxy_async();
-        if (x + 1 < hi) ptx::mbar_arrive(sm.bar(B_Q_FULL + ((j + 1) & 1)));
 
         float m_run = -INFINITY, l_run = 0.f;
         uint32_t pk[32];
@@ -286,6 +282,12 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(sm.bar(B_P_FULL + (j & 1)));
+        // the next chunk's rows (gathered one chunk ago) go to the MMA now, after
+        // this chunk's softmax: the copies had that long to land, and the next
+        // Q K^T still runs while this chunk's P V and epilogue do
+        ptx::cp_async_wait<1>();
+        ptx::fence_proxy_async();
+        if (x + 1 < hi) ptx::mbar_arrive(sm.bar(B_Q_FULL + ((j + 1) & 1)));
         if (none) continue;  // no row of this warp writes anything
         {
             bool rr = ptx::mbar_wait(sm.bar(B_PV_DONE), j & 1, abort, P.status, P.wait_ns);

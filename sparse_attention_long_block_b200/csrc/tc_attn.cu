@@ -115,6 +115,11 @@ struct TcParams {
     int sgl_on;                // 1: the selection branch runs split this way
     __half *slc_u;             // [n_max][h_q][d] the union tiles' normalised output
     float *slc_lse;            // [n_max][h_q] their log-sum-exp (log2 units)
+    // With the split selection the merge kernel writes the output rows; the
+    // window epilogue then stores sig(g_swa) o_swa here ([n_max][h_q][d] fp16,
+    // in units of V / v_scale like the selection parts) instead of reading the
+    // partial (null: the window epilogue writes the rows).
+    __half *swa_part;
 };
 
 __host__ __device__ __forceinline__ int pow2_at_least(int r) {
@@ -572,7 +577,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     float *dbg = is_slc(MODE) ? L.dbg_o_slc : L.dbg_o_swa;
                     for (int e = 0; e < kD; ++e) {
                         if (dbg) dbg[prow + e] = 0.f;
-                        if (MODE == MODE_SWA)
+                        if (MODE == MODE_SWA && P.swa_part)
+                            P.swa_part[((size_t)rc.i * L.h_q + rc.h) * kD + e] = __float2half_rn(0.f);
+                        else if (MODE == MODE_SWA)
                             ((__nv_bfloat16 *)L.out)[prow + e] = __float2bfloat16_rn(part[e]);
                     }
                 }
@@ -946,6 +953,27 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
                 ptx::tmem_wait_ld();
                 if (!rc.valid) continue;
+                if (MODE == MODE_SWA && P.swa_part) {
+                    // the merge kernel adds this to the partial and the
+                    // selection and writes the row: store sig(g_swa) o_swa in
+                    // units of V / v_scale (|value| < 2^15, inside fp16)
+                    const float inv_u = l_run > 0.f ? 1.f / l_run : 0.f;
+                    __half *dst = P.swa_part + qrow + ch * 32;
+#pragma unroll
+                    for (int k = 0; k < 32; k += 8) {
+                        uint4 v;
+                        __half2 *h2 = reinterpret_cast<__half2 *>(&v);
+#pragma unroll
+                        for (int z = 0; z < 4; ++z)
+                            h2[z] = __floats2half2_rn(g * (o[k + 2 * z] * inv_u),
+                                                      g * (o[k + 2 * z + 1] * inv_u));
+                        __stcg(reinterpret_cast<uint4 *>(dst + k), v);
+                        if (dbg)
+                            for (int z = 0; z < 8; ++z)
+                                dbg[prow + ch * 32 + k + z] = l_run > 0.f ? o[k + z] * inv : 0.f;
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int k = 0; k < 32; k += 8) {
                     const float4 p0 = __ldcg(reinterpret_cast<const float4 *>(part + ch * 32 + k));
@@ -1449,8 +1477,9 @@ __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *s
 // The selection output of each (vision query, head): the union tiles' part
 // (slc_u, slc_lse) and the query's single-query pairs (slot ids qg kSglSlots +
 // z, z < n[qg]: sgl_o, sgl_lse), each the exact softmax over its keys,
-// combined with the weights 2^(lse_part - M) / sum over the parts; then
-// partial += sigmoid(g_slc) * o_slc (fp32) and the optional export.  Every
+// combined with the weights 2^(lse_part - M) / sum over the parts; then the
+// vision output row out = partial (compression) + sigmoid(g_slc) * o_slc +
+// swa_part (window), rounded once to bf16, and the optional export.  Every
 // address follows from (group, query, slot), so a row's loads are independent.
 // One warp per (group, query); its r heads x 128 dims are cut into 16-dim
 // chunks, chunk c = lane + 32 k (head c / 8), so a warp's load instruction
@@ -1460,6 +1489,7 @@ struct SlcMergeArgs {
     const int32_t *n;
     const __half *sgl_o, *slc_u;
     const float *sgl_lse, *slc_lse, *v_scale;
+    const __half *swa_part;  // sig(g_swa) o_swa / v_scale of the window pass
 };
 
 __device__ __forceinline__ void acc_half8(float (&acc)[8], uint4 u, float w) {
@@ -1538,20 +1568,43 @@ __global__ void __launch_bounds__(256) slc_merge_kernel(LayerParams p, SlcMergeA
                     acc_half8(acc1, pz[z][1], lz[z] * norm);
                 }
             }
-            float4 *pr = reinterpret_cast<float4 *>(p.o_cmp_ws + urow);
+            const float4 *pr = reinterpret_cast<const float4 *>(p.o_cmp_ws + urow);
+            const uint4 *sw = reinterpret_cast<const uint4 *>(a.swa_part + urow);
             float4 pv[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) pv[q] = __ldcs(pr + q);
+            const uint4 sw0 = __ldcs(sw), sw1 = __ldcs(sw + 1);
+            float wf[16];
+            {
+                const __half2 *h0 = reinterpret_cast<const __half2 *>(&sw0);
+                const __half2 *h1 = reinterpret_cast<const __half2 *>(&sw1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f0 = __half22float2(h0[q]), f1 = __half22float2(h1[q]);
+                    wf[2 * q] = f0.x * vsc;
+                    wf[2 * q + 1] = f0.y * vsc;
+                    wf[8 + 2 * q] = f1.x * vsc;
+                    wf[8 + 2 * q + 1] = f1.y * vsc;
+                }
+            }
+            const float4 *wv = reinterpret_cast<const float4 *>(wf);
             const float *ac[2] = {acc0, acc1};
+            uint4 ob[2];
+            __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(ob);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float *o4 = ac[q >> 1] + 4 * (q & 1);
-                pv[q].x = fmaf(gl, o4[0], pv[q].x);
-                pv[q].y = fmaf(gl, o4[1], pv[q].y);
-                pv[q].z = fmaf(gl, o4[2], pv[q].z);
-                pv[q].w = fmaf(gl, o4[3], pv[q].w);
-                __stcs(pr + q, pv[q]);
+                const float x0 = fmaf(gl, o4[0], pv[q].x) + wv[q].x;
+                const float x1 = fmaf(gl, o4[1], pv[q].y) + wv[q].y;
+                const float x2 = fmaf(gl, o4[2], pv[q].z) + wv[q].z;
+                const float x3 = fmaf(gl, o4[3], pv[q].w) + wv[q].w;
+                b2[2 * q] = __floats2bfloat162_rn(x0, x1);
+                b2[2 * q + 1] = __floats2bfloat162_rn(x2, x3);
             }
+            uint4 *orow = reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.out +
+                                                    ((size_t)t * p.h_q + h0 + hl) * kD + d0);
+            __stcs(orow, ob[0]);
+            __stcs(orow + 1, ob[1]);
             if (p.dbg_o_slc) {
                 float *dbg = p.dbg_o_slc + ((size_t)t * p.h_q + h0 + hl) * kD + d0;
 #pragma unroll
@@ -1703,12 +1756,13 @@ struct TcState {
     int4 *sgl_rec, *sgl_sorted, *sgl_items;
     __half *sgl_o, *slc_u;
     float *sgl_lse, *slc_lse;
+    __half *swa_part;
 };
 
 
 struct SglSizes {
     int on, nbt, nbk, cap;
-    size_t meta, rec, sorted, items, n, o, lse, u, ulse, total;
+    size_t meta, rec, sorted, items, n, o, lse, u, ulse, swa, total;
 };
 
 static SglSizes sgl_sizes(const vnsa_config &c) {
@@ -1731,7 +1785,8 @@ static SglSizes sgl_sizes(const vnsa_config &c) {
     z.lse = up256((size_t)z.cap * r * 4);
     z.u = up256((size_t)c.n_max * c.h_q * kD * 2);
     z.ulse = up256((size_t)c.n_max * c.h_q * 4);
-    z.total = z.meta + z.rec + z.sorted + z.items + z.n + z.o + z.lse + z.u + z.ulse;
+    z.swa = up256((size_t)c.n_max * c.h_q * kD * 2);
+    z.total = z.meta + z.rec + z.sorted + z.items + z.n + z.o + z.lse + z.u + z.ulse + z.swa;
     return z;
 }
 
@@ -1811,6 +1866,7 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
         st->sgl_lse = (float *)(q += z.o);
         st->slc_u = (__half *)(q += z.lse);
         st->slc_lse = (float *)(q += z.u);
+        st->swa_part = (__half *)(q += z.ulse);
     }
     cudaError_t e = cudaSuccess;
     for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
@@ -1961,6 +2017,17 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         P.sgl_on = 1;
         if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
         P.sgl_on = 0;
+    } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
+        return e;
+    }
+    end(VNSA_STAGE_SLC);
+    begin(VNSA_STAGE_SWA);
+    P.swa_part = sgl ? st->swa_part : nullptr;
+    if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
+    P.swa_part = nullptr;
+    if (sgl) {
+        // the selection output from its parts, and with the compression and
+        // window parts the vision output rows
         SlcMergeArgs ma;
         ma.n = st->sgl_n;
         ma.sgl_o = st->sgl_o;
@@ -1968,14 +2035,10 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         ma.sgl_lse = st->sgl_lse;
         ma.slc_lse = st->slc_lse;
         ma.v_scale = st->v_scale;
+        ma.swa_part = st->swa_part;
         slc_merge_kernel<<<st->num_sms * 16, 256, 0, s>>>(L, ma);
         ++*launches;
-    } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
-        return e;
     }
-    end(VNSA_STAGE_SLC);
-    begin(VNSA_STAGE_SWA);
-    if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
     end(VNSA_STAGE_SWA);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TEXT);
