@@ -21,8 +21,11 @@
 //
 //   warp 0     lane 0: TMA loads of each new tile's K and V (one stage)
 //   warp 1     lane 0: the MMAs
-//   warps 2-5  one thread per MMA row: the row's Q gathered by cp.async two
-//              chunks ahead into a double buffer, softmax, epilogue
+//   warps 2-5  one thread per MMA row: softmax and epilogue; each warp gathers
+//              its 32 rows' Q by cp.async two chunks ahead into a double
+//              buffer (half a warp per 256-byte row, so every 32-byte sector
+//              is read whole) and stores its rows' outputs through shared
+//              memory (eight 64-byte row pieces per instruction)
 #include <math.h>
 
 #include "sgl_attn.h"
@@ -40,8 +43,12 @@ constexpr uint32_t SM_Q = 0;         // 2 x [128 rows][128] bf16, 32 KB each
 constexpr uint32_t Q_BYTES = 32768;
 constexpr uint32_t SM_K = 65536;     // one K tile: 2 boxes of 64 keys x 64 d (16 KB)
 constexpr uint32_t SM_V = 81920;     // one V tile (16 KB)
-constexpr uint32_t SM_BAR = 98304;
+constexpr uint32_t SM_STG = 98304;   // per softmax warp: 32 rows x 64 B of output (+16 B pad)
+constexpr uint32_t STG_ROW = 80, STG_WARP = 32 * STG_ROW;
+constexpr uint32_t SM_BAR = SM_STG + 4 * STG_WARP;
 constexpr uint32_t SMEM_BYTES = SM_BAR + 256 + 1024;  // + alignment slack
+// two CTAs per SM: 2 x (SMEM_BYTES + 1 KB reserved) within the SM's 228 KB
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
 
 enum { B_Q_FULL = 0, B_KV_FULL = 2, B_KV_EMPTY = 3, B_S_FULL = 4, B_P_FULL = 6, B_PV_DONE = 8,
        B_FINAL = 9, B_COUNT = 10 };
@@ -180,30 +187,36 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
     auto entry = [&](int x) -> int4 {
         return (x < hi && slot < qt) ? P.sorted[(size_t)x * qt + slot] : make_int4(-1, 0, 0, 0);
     };
-    auto q_src = [&](const int4 &e) -> const __nv_bfloat16 * {
-        if (e.x < 0) return nullptr;
+    // the row's Q row index (token x h_q + head) in q, -1 for no pair
+    auto q_off = [&](const int4 &e) -> int {
+        if (e.x < 0) return -1;
         const int h = (e.w / P.nbt) * r + hl;
-        return P.q + ((size_t)e.z * P.h_q + h) * kD;
+        return e.z * P.h_q + h;
     };
-    // The row into Q buffer `buf`, 16-byte pieces in the 128-byte swizzled
-    // K-major layout of the MMA's A operand; a row without a pair is
-    // zero-filled.  One cp.async group per call.
-    auto gather = [&](const __nv_bfloat16 *src, int buf) {
+    // The warp's 32 rows into Q buffer `buf`, 16-byte pieces in the 128-byte
+    // swizzled K-major layout of the MMA's A operand; a row without a pair is
+    // zero-filled.  Each instruction copies two whole rows (lanes 0-15 one,
+    // 16-31 the next), so the sectors of a row are read in full and together.
+    // One cp.async group per call.
+    auto gather = [&](int off, int buf) {
         const uint32_t qb = sm.u32 + SM_Q + (uint32_t)buf * Q_BYTES;
-        const bool valid = src != nullptr;
+        const int c16 = lane & 15;
+        const uint32_t hf = (uint32_t)(c16 >> 3), c = (uint32_t)(c16 & 7);
 #pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16) {
-            const int hf = c16 >> 3, c = c16 & 7;
-            const uint32_t dst = qb + (uint32_t)hf * 16384u + (uint32_t)rho * 128u +
-                                 (uint32_t)((c ^ (rho & 7)) << 4);
-            ptx::cp_async16(dst, valid ? (const void *)(src + c16 * 8) : (const void *)P.q,
+        for (int z = 0; z < 16; ++z) {
+            const int t = 2 * z + (lane >> 4);  // row wq * 32 + t is lane t's
+            const int o = __shfl_sync(0xffffffffu, off, t);
+            const uint32_t row = (uint32_t)(wq * 32 + t);
+            const uint32_t dst = qb + hf * 16384u + row * 128u + ((c ^ (row & 7u)) << 4);
+            const bool valid = o >= 0;
+            ptx::cp_async16(dst, valid ? (const void *)(P.q + (size_t)o * kD + c16 * 8) : (const void *)P.q,
                             valid ? 16u : 0u);
         }
         ptx::cp_async_commit();
     };
     int4 e_a = entry(lo), e_b = entry(lo + 1), e_c = entry(lo + 2);
-    gather(q_src(e_a), 0);
-    gather(q_src(e_b), 1);
+    gather(q_off(e_a), 0);
+    gather(q_off(e_b), 1);
     ptx::cp_async_wait<1>();
     ptx::fence_proxy_async();
     if (hi > lo) ptx::mbar_arrive(sm.bar(B_Q_FULL));
@@ -228,7 +241,7 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
         }
         ptx::tc_fence_after();
         // Q K^T of this chunk is done, so its buffer takes chunk x + 2
-        gather(q_src(e_b), j & 1);
+        gather(q_off(e_b), j & 1);
 
         float m_run = -INFINITY, l_run = 0.f;
         uint32_t pk[32];
@@ -295,15 +308,17 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
             if (!ok) break;
         }
         ptx::tc_fence_after();
-        // epilogue: the normalised row in the scaled V's units (fp16)
+        // epilogue: the normalised row in the scaled V's units (fp16), 32
+        // columns at a time through the warp's staging rows, then stored by
+        // eight lanes' 64-byte pieces per instruction (whole sectors)
         const float mul = l_run > 0.f ? 1.f / l_run : 0.f;
-        __half *orow = P.o + ((size_t)sid * r + hl) * kD;
+        const int orow = hi_key >= 0 ? sid * r + hl : -1;  // output row, -1: none
+        uint8_t *stg = sm.base + SM_STG + (uint32_t)wq * STG_WARP;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
             float o[32];
             ptx::tmem_ld32(tmem + lane_base + TM_O + ch * 32, o);
             ptx::tmem_wait_ld();
-            if (hi_key < 0) continue;
 #pragma unroll
             for (int k = 0; k < 32; k += 8) {
                 uint4 v;
@@ -311,8 +326,18 @@ __device__ void rows(const SglParams &P, const Sm &sm, uint32_t tmem, int lo, in
 #pragma unroll
                 for (int z = 0; z < 4; ++z)
                     h2[z] = __floats2half2_rn(o[k + 2 * z] * mul, o[k + 2 * z + 1] * mul);
-                *reinterpret_cast<uint4 *>(orow + ch * 32 + k) = v;
+                *reinterpret_cast<uint4 *>(stg + lane * STG_ROW + k * 2) = v;
             }
+            __syncwarp();
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const int t = 8 * z + (lane >> 2), pc = lane & 3;
+                const int dst = __shfl_sync(0xffffffffu, orow, t);
+                const uint4 v = *reinterpret_cast<const uint4 *>(stg + t * STG_ROW + pc * 16);
+                if (dst >= 0)
+                    *reinterpret_cast<uint4 *>(P.o + (size_t)dst * kD + ch * 32 + pc * 8) = v;
+            }
+            __syncwarp();  // the staging rows are rewritten by the next columns
         }
         if (hi_key >= 0)
             P.lse[(size_t)sid * r + hl] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
