@@ -97,10 +97,11 @@ def executed_work(wl, is_vision, idx):
     tile (8 head slots), a statistics pass (QK^T) and an exact pass (QK^T + P V)
     over the visible blocks; selection: 18 queries (7 heads) against the union
     of the 64-key tiles their selected blocks reach (from idx [h_kv][N_v][k]);
-    with block 64 the tiles that only one of the 18 queries reaches run
+    with block 64 the tiles that only one or two of the 18 queries reach run
     tile-major instead, up to 18 such (query, tile) pairs per 128-row tile;
-    window and text: 18 queries against their key ranges.  (Up to 8 of a
-    query's single tiles, in tile order, leave the union.)"""
+    window and text: 18 queries against their key ranges.  (Up to 16 pairs
+    per query leave the union: its single-query tiles, then the two-query
+    tiles while both queries have room, each in tile order.)"""
     prod = 2.0 * 128 * 64 * wl.d
     vis = np.nonzero(is_vision)[0]
     txt = np.nonzero(is_vision == 0)[0]
@@ -123,20 +124,34 @@ def executed_work(wl, is_vision, idx):
         for g in range(wl.h_kv):
             sel = idx[g, q0:ql + 1]
             if wl.block == 64:
-                flat = sel.ravel()
-                u, cnt = np.unique(flat[flat >= 0], return_counts=True)
-                ones = set(u[cnt == 1].tolist())
-                # up to 8 single tiles per query (in tile order) leave the union
-                pairs = []
-                for row in sel:
-                    mine = sorted(j for j in row if j >= 0 and j in ones)
-                    pairs += mine[:8]
-                keep = len(u) - len(pairs)
+                # up to 16 pairs per query leave the union: its single-query
+                # tiles in tile order, then the two-query tiles in tile order
+                # while both queries have a slot left
+                who = {}
+                for qi, row in enumerate(sel):
+                    for j in row:
+                        if j >= 0:
+                            who.setdefault(int(j), []).append(qi)
+                used = [0] * len(sel)
+                pairs, leave = [], 0
+                for j in sorted(who):
+                    if len(who[j]) == 1 and used[who[j][0]] < 16:
+                        used[who[j][0]] += 1
+                        pairs.append(j)
+                        leave += 1
+                for j in sorted(who):
+                    qs = who[j]
+                    if len(qs) == 2 and used[qs[0]] < 16 and used[qs[1]] < 16:
+                        used[qs[0]] += 1
+                        used[qs[1]] += 1
+                        pairs += [j, j]
+                        leave += 1
+                keep = len(who) - leave
                 if pairs and keep:
                     slc += 2 * keep
-                    single[g, pairs] += 1
+                    np.add.at(single[g], pairs, 1)
                 else:
-                    slc += 2 * len(u)
+                    slc += 2 * len(who)
                 continue
             # the 64-key tiles each selected block reaches, up to the query
             ok = sel >= 0

@@ -61,7 +61,7 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 constexpr int kTextSplitKeys = 8192;
 constexpr size_t kTextPartBytes = 256ull << 20;
 constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
-constexpr int kSglSlots = 8;         // single-query pairs per (group, query) at most
+constexpr int kSglSlots = 16;        // tile-major pairs per (group, query) at most
 
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
 constexpr uint32_t SM_KV = 32768;                             // K ring, then V ring
@@ -1306,15 +1306,23 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         __syncwarp();
         int tot = min(total, plan_max);
         if (sg.on) {
-            // Tiles that exactly one query of the item reaches leave the plan for
-            // the tile-major pass (sgl_attn.cu): up to kSglSlots of them per query,
-            // in tile order (the rest stay), and only while at least one tile
-            // stays.  The pair (vision query i of group g, slot s) has the id
-            // (g n_max + i) kSglSlots + s, so the selection epilogue finds a
-            // query's pairs without a lookup.
+            // Tiles that one or two queries of the item reach leave the plan for
+            // the tile-major pass (sgl_attn.cu) as (query, tile) pairs: a 128-row
+            // union tile costs the same whatever number of its rows attend, and
+            // a pair costs a gathered Q row block, an output row block and its
+            // merge, which is less for one or two queries and more for three.
+            // Up to kSglSlots pairs per query: first its single-query tiles in
+            // tile order, then the two-query tiles in tile order while both
+            // queries have a slot left (the rest stay), and only while at least
+            // one tile stays.  The pair (vision query i of group g, slot s) has
+            // the id (g n_max + i) kSglSlots + s, so the merge finds a query's
+            // pairs without a lookup.  sslot[x]: -1 (stays), the slot of a
+            // single-query tile, or 32 + slot of the lower query + 32 x slot
+            // of the higher one.
             qcnt[lane] = 0u;
             __syncwarp();
-            int npair = 0;
+            int npair = 0;   // pairs
+            int nleave = 0;  // tiles that leave
             for (int xb = 0; xb < tot; xb += 32) {
                 const int x = xb + lane;
                 const uint32_t m = x < tot ? qm[x] : 0u;
@@ -1329,8 +1337,28 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
                 if (x < tot) sslot[x] = pair ? slot : -1;
                 npair += __popc(__ballot_sync(0xffffffffu, pair));
             }
+            nleave = npair;
             __syncwarp();
-            if (npair >= tot) {  // every tile would leave: the item keeps them all
+            // two-query tiles, in tile order; one lane assigns (a few dozen
+            // per item), so a tile takes both slots or none and no slot is
+            // left unused below a query's count
+            if (lane == 0) {
+                for (int x = 0; x < tot; ++x) {
+                    const uint32_t m = qm[x];
+                    if (__popc(m) != 2) continue;
+                    const int qa = __ffs(m) - 1, qb = 31 - __clz(m);
+                    if (qcnt[qa] >= (uint32_t)kSglSlots || qcnt[qb] >= (uint32_t)kSglSlots) continue;
+                    sslot[x] = 32 + (int)qcnt[qa] + 32 * (int)qcnt[qb];
+                    ++qcnt[qa];
+                    ++qcnt[qb];
+                    npair += 2;
+                    ++nleave;
+                }
+            }
+            npair = __shfl_sync(0xffffffffu, npair, 0);
+            nleave = __shfl_sync(0xffffffffu, nleave, 0);
+            __syncwarp();
+            if (nleave >= tot) {  // every tile would leave: the item keeps them all
                 for (int x = lane; x < tot; x += 32) sslot[x] = -1;
                 npair = 0;
             }
@@ -1353,24 +1381,33 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
                     const int tl = x < tot ? out[1 + x] : 0;
                     const int sl = x < tot ? sslot[x] : -1;
                     const bool pair = sl >= 0;
+                    const bool dbl = sl >= 32;
                     const bool keep = x < tot && !pair;
                     // every lane holds its entry before any entry is moved down
                     const unsigned bk = __ballot_sync(0xffffffffu, keep);
                     const unsigned bp = __ballot_sync(0xffffffffu, pair);
+                    const unsigned bd = __ballot_sync(0xffffffffu, dbl);
                     if (keep) {
                         const int pos = kept + __popc(bk & lt);
                         out[1 + pos] = tl;
                         qm[pos] = m;
                     }
                     if (pair) {
-                        const int i = q0 + __ffs(m) - 1;
-                        const int id = (g * p.n_max + i) * kSglSlots + sl;
                         const int bucket = g * sg.nbt + tl;
-                        const int lp = atomicAdd(&sg.meta[2 + bucket], 1);
-                        sg.rec[base + si + __popc(bp & lt)] = make_int4(bucket, id, lp, p.vis[i]);
+                        const int at = base + si + __popc(bp & lt) + __popc(bd & lt);
+                        const int lp = atomicAdd(&sg.meta[2 + bucket], dbl ? 2 : 1);
+                        const int i = q0 + __ffs(m) - 1;
+                        const int s0 = dbl ? (sl - 32) & 31 : sl;
+                        sg.rec[at] = make_int4(bucket, (g * p.n_max + i) * kSglSlots + s0, lp, p.vis[i]);
+                        if (dbl) {
+                            const int i2 = q0 + 31 - __clz(m);
+                            const int s1 = (sl - 32) >> 5;
+                            sg.rec[at + 1] = make_int4(bucket, (g * p.n_max + i2) * kSglSlots + s1,
+                                                       lp + 1, p.vis[i2]);
+                        }
                     }
                     kept += __popc(bk);
-                    si += __popc(bp);
+                    si += __popc(bp) + __popc(bd);
                     __syncwarp();
                 }
                 tot = kept;
@@ -1522,32 +1559,34 @@ __global__ void __launch_bounds__(256) slc_merge_kernel(LayerParams p, SlcMergeA
             const int c = lane + 32 * k;
             if (c >= nchunk) continue;
             const int hl = c >> 3, d0 = (c & 7) * 16;
-            // weights of this chunk's head (slots past the count hold stale
-            // values and are masked after the load)
+            // weights of this chunk's head (slots past the count are not read)
             const float lu = a.slc_lse[(size_t)i * p.h_q + h0 + hl];
             float lz[kSglSlots];
 #pragma unroll
-            for (int z = 0; z < kSglSlots; ++z) lz[z] = a.sgl_lse[(id0 + z) * r + hl];
+            for (int z = 0; z < kSglSlots; ++z)
+                lz[z] = z < ns ? a.sgl_lse[(id0 + z) * r + hl] : -INFINITY;
             const size_t urow = ((size_t)i * p.h_q + h0 + hl) * kD + d0;
             const uint4 *us = reinterpret_cast<const uint4 *>(a.slc_u + urow);
             const uint4 u0 = __ldcs(us), u1 = __ldcs(us + 1);
-            uint4 pz[kSglSlots][2];
+            // the first half of the slots' outputs in flight with the weights
+            constexpr int kHalf = kSglSlots / 2;
+            uint4 pz[kHalf][2];
+            auto load_half = [&](int zb) {
 #pragma unroll
-            for (int z = 0; z < kSglSlots; ++z) {
-                if (z < ns) {
-                    const uint4 *ps = reinterpret_cast<const uint4 *>(
-                        a.sgl_o + ((id0 + z) * r + hl) * kD + d0);
-                    pz[z][0] = __ldcs(ps);
-                    pz[z][1] = __ldcs(ps + 1);
+                for (int z = 0; z < kHalf; ++z) {
+                    if (zb + z < ns) {
+                        const uint4 *ps = reinterpret_cast<const uint4 *>(
+                            a.sgl_o + ((id0 + zb + z) * r + hl) * kD + d0);
+                        pz[z][0] = __ldcs(ps);
+                        pz[z][1] = __ldcs(ps + 1);
+                    }
                 }
-            }
+            };
+            load_half(0);
             const float gl = sigmoidf_(p.gate[((size_t)t * p.h_q + h0 + hl) * 3 + 1]);
             float mx = lu;
 #pragma unroll
-            for (int z = 0; z < kSglSlots; ++z) {
-                lz[z] = z < ns ? lz[z] : -INFINITY;
-                mx = fmaxf(mx, lz[z]);
-            }
+            for (int z = 0; z < kSglSlots; ++z) mx = fmaxf(mx, lz[z]);
             const float wu = lu == -INFINITY ? 0.f : exp2f(lu - mx);
             float wsum = wu;
 #pragma unroll
@@ -1562,10 +1601,20 @@ __global__ void __launch_bounds__(256) slc_merge_kernel(LayerParams p, SlcMergeA
             acc_half8(acc0, u0, wu * norm);
             acc_half8(acc1, u1, wu * norm);
 #pragma unroll
-            for (int z = 0; z < kSglSlots; ++z) {
+            for (int z = 0; z < kHalf; ++z) {
                 if (z < ns) {
                     acc_half8(acc0, pz[z][0], lz[z] * norm);
                     acc_half8(acc1, pz[z][1], lz[z] * norm);
+                }
+            }
+            if (ns > kHalf) {
+                load_half(kHalf);
+#pragma unroll
+                for (int z = 0; z < kHalf; ++z) {
+                    if (kHalf + z < ns) {
+                        acc_half8(acc0, pz[z][0], lz[kHalf + z] * norm);
+                        acc_half8(acc1, pz[z][1], lz[kHalf + z] * norm);
+                    }
                 }
             }
             const float4 *pr = reinterpret_cast<const float4 *>(p.o_cmp_ws + urow);

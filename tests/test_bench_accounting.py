@@ -57,7 +57,7 @@ def test_algorithmic_pairs_match_enumeration(wl, mask):
     assert got["topk_bytes"] == 4.0 * wl.h_kv * want["cmp"] + 4.0 * wl.h_kv * nv * wl.top_k
 
 
-def test_selection_executed_work_splits_single_query_tiles():
+def test_selection_executed_work_splits_one_and_two_query_tiles():
     # one group, 7 heads (18 queries per 128-row tile), block 64, two items
     wl = Workload("acct_split", 36 * 64, 0, h_q=7, h_kv=1, d=128, top_k=3, window=64)
     isv = np.ones(wl.n, np.uint8)
@@ -68,14 +68,32 @@ def test_selection_executed_work_splits_single_query_tiles():
     idx[0, 18:36, 1] = np.arange(1, 19)   # item 1: the same 18 tiles, one query each
     idx[0, 0, 2] = 30                     # item 0: tile 30 reached by queries 0 and 1
     idx[0, 1, 2] = 30
+    idx[0, 18:21, 2] = 31                 # item 1: tile 31 reached by three queries
     ex = bench.executed_work(wl, isv, idx)
     prod = 2.0 * 128 * 64 * wl.d
-    # items 0, 1 keep 2 and 1 union tiles; the 36 single-query pairs fall into
-    # 18 (group, tile) buckets of 2 pairs, one tile-major tile each; the other
-    # items (queries 36 ..) reach block 0 only
+    # item 0 keeps block 0's tile, item 1 block 0's and tile 31; the 36
+    # single-query pairs fall into 18 (group, tile) buckets of 2 pairs and the
+    # two-query tile 30 adds a bucket of 2 pairs: one tile-major tile each; the
+    # other items (queries 36 ..) reach block 0 only
     n_items = -(-nv // 18)
-    union_tiles = 2 + 1 + (n_items - 2) * 1
-    assert ex["slc"] == 2 * prod * (union_tiles + 18)
+    union_tiles = 1 + 2 + (n_items - 2) * 1
+    assert ex["slc"] == 2 * prod * (union_tiles + 19)
+    # a query with more than 16 pairs: its 17th single-query tile stays, and so
+    # does a two-query tile of a query without a free slot
+    wl2 = Workload("acct_cap", 64 * 64, 0, h_q=7, h_kv=1, d=128, top_k=20, window=64)
+    isv2 = np.ones(wl2.n, np.uint8)
+    idx2 = -np.ones((1, wl2.n_vision, 20), np.int32)
+    idx2[0, :, 0] = 0
+    q = 2600                                # own block 40; item 144 (queries 2592 ..)
+    idx2[0, q, 1:18] = np.arange(1, 18)     # 17 tiles reached by this query alone
+    idx2[0, q, 18] = 30                     # and a tile shared with the next query
+    idx2[0, q + 1, 1] = 30
+    ex2 = bench.executed_work(wl2, isv2, idx2)
+    prod2 = 2.0 * 128 * 64 * wl2.d
+    n_items2 = -(-wl2.n_vision // 18)
+    # item 144 keeps block 0's tile, the 17th single tile and tile 30; 16
+    # pairs leave, one bucket each
+    assert ex2["slc"] == 2 * prod2 * ((n_items2 - 1) + 3 + 16)
     # an item whose tiles all serve one query keeps them all (the plan cannot
     # be empty), so nothing leaves for the tile-major pass
     idx1 = -np.ones((1, nv, 3), np.int32)
