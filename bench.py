@@ -71,9 +71,12 @@ def algorithmic_work(wl, is_vision):
     txt = np.nonzero(is_vision == 0)[0]
     nv = len(vis)
     B = wl.block
+    st = wl.stride or B  # compression stride (overlapping blocks when below B)
     i = np.arange(nv, dtype=np.int64)
     nb = nv // B
-    c = np.minimum((i + 1) // B, nb)
+    c = np.minimum((i + 1) // B, nb)  # complete selection blocks
+    nc = (nv - B) // st + 1 if nv >= B else 0
+    cc = np.where(i >= B - 1, np.minimum(nc, (i - B + 1) // st + 1), 0)  # visible cmp blocks
     own = i // B
     n_sel = np.minimum(wl.top_k, c + (own >= c).astype(np.int64))
     slc_tokens = B * (n_sel - 1) + (i % B + 1)
@@ -81,11 +84,12 @@ def algorithmic_work(wl, is_vision):
     f = 4.0 * wl.d * wl.h_q
     es = 2 if wl.dtype == "bf16" else 4
     return {
-        "cmp": f * float(c.sum()),
+        "cmp": f * float(cc.sum()),
         "slc": f * float(slc_tokens.sum()),
         "swa": f * float(swa_tokens.sum()),
         "text": f * float((txt.astype(np.int64) + 1).sum()),
-        "pool_bytes": float(2 * nb * B * wl.h_kv * wl.d * es + 2 * nb * wl.h_kv * wl.d * es),
+        "pool_bytes": float(2 * (min(nv, (nc - 1) * st + B) if nc else 0) * wl.h_kv * wl.d * es
+                            + 2 * nc * wl.h_kv * wl.d * es),
         "topk_bytes": float(4 * wl.h_kv * int(c.sum()) + 4 * wl.h_kv * nv * wl.top_k),
     }
 
@@ -112,9 +116,12 @@ def executed_work(wl, is_vision, idx):
         rpad *= 2
     qc, qt = 128 // rpad, 128 // r
     cmp = slc = swa = text = 0.0
+    B, st = wl.block, wl.stride or wl.block
+    nc = (nv - B) // st + 1 if nv >= B else 0
     for q0 in range(0, nv, qc):
         ql = min(nv, q0 + qc) - 1
-        t = -(-min((ql + 1) // wl.block, nb) // 64)
+        vis_c = min(nc, (ql - B + 1) // st + 1) if ql >= B - 1 else 0
+        t = -(-vis_c // 64)
         cmp += 3 * t
     single = np.zeros((wl.h_kv, (nv + 63) // 64 + 1), np.int64)  # pairs per (group, tile)
     for q0 in range(0, nv, qt):
@@ -394,6 +401,8 @@ def main():
                          "through the gate perceptron, and compression uses its perceptron")
     ap.add_argument("--gate-hidden", type=int, default=256)
     ap.add_argument("--cmp-hidden", type=int, default=128)
+    ap.add_argument("--cmp-stride", type=int, default=0,
+                    help="compression stride below the block size (overlapping blocks); 0: the block")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -420,6 +429,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
 
     wl = replica_workload(args.workload, rank)
+    if args.cmp_stride:
+        wl = wl.with_(stride=args.cmp_stride)
     x = generate(wl)
     td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     dev = torch.device("cuda", local_rank)
@@ -431,7 +442,7 @@ def main():
     out = torch.empty_like(q)
     layer = binding.Layer(n_max=wl.n, h_q=wl.h_q, h_kv=wl.h_kv, d=wl.d, block=wl.block,
                           top_k=wl.top_k, window=wl.window, w_k=torch.from_numpy(x["w_k"]),
-                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype)
+                          w_v=torch.from_numpy(x["w_v"]), dtype=wl.dtype, stride=wl.stride)
     stream = torch.cuda.current_stream()
     gm = None
     if args.mlp:
@@ -502,7 +513,7 @@ def main():
     executed = None
     if wl.dtype == "bf16" and wl.d == 128:
         dbg, tens = binding.make_debug(wl.n, wl.h_q, wl.h_kv, wl.d, wl.top_k, wl.block,
-                                       dtype=td, want=("idx",))
+                                       dtype=td, want=("idx",), stride=wl.stride)
         layer.forward(q, k, v, isv, gate, out=out, dbg=dbg, stream=stream)
         torch.cuda.synchronize()
         nvis = int(x["is_vision"].sum())
@@ -627,7 +638,8 @@ def main():
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": wl.name, "tokens": wl.n, "n_vision": wl.n_vision,
                        "n_text": wl.n_text, "h_q": wl.h_q, "h_kv": wl.h_kv, "d": wl.d,
-                       "block": wl.block, "top_k": wl.top_k, "window": wl.window,
+                       "block": wl.block, "cmp_stride": wl.stride or wl.block,
+                       "top_k": wl.top_k, "window": wl.window,
                        "attention": "dense (all tokens text)" if wl.dense else "hybrid",
                        "kernels": layer.path(),
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

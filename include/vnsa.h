@@ -117,8 +117,10 @@ typedef enum vnsa_stage {
     VNSA_STAGE_POOL = 1,      /* block mean-pool + projection -> K_cmp, V_cmp       */
     VNSA_STAGE_CMP = 2,       /* compression attention + importance                 */
     VNSA_STAGE_TOPK = 3,      /* block selection                                    */
-    VNSA_STAGE_SLC = 4,       /* selection attention                                */
-    VNSA_STAGE_SWA = 5,       /* sliding window + gate combine + vision output      */
+    VNSA_STAGE_SLC = 4,       /* selection attention (block 64, tensor cores: with  */
+                              /* the merge that writes the vision output rows)      */
+    VNSA_STAGE_SWA = 5,       /* sliding window (other configurations: + gate       */
+                              /* combine + vision output)                           */
     VNSA_STAGE_TEXT = 6,      /* dense text GQA                                     */
     VNSA_NUM_STAGES = 7
 } vnsa_stage;

@@ -239,6 +239,7 @@ __device__ __forceinline__ int item_tiles(const Item &it) {
 
 __device__ __forceinline__ bool kind_has_pv(int kind) { return kind != K_STATS; }
 
+
 // ---------------------------------------------------------------------------
 struct Smem {
     uint8_t *base;
@@ -523,7 +524,9 @@ __device__ __forceinline__ uint64_t sel_coverage(const int32_t *sel, int &cur, i
     return cov;
 }
 
-template <int MODE>
+// RPAD: the compression mode's head slots per query (4, 8 or 16), fixed per
+// instantiation so that each compression kernel carries one importance reduce
+template <int MODE, int RPAD>
 __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
@@ -865,13 +868,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                                       ? L.imp + ((size_t)it.g * L.n_max + iq) * L.imp_stride + key0
                                       : nullptr;
                     const int lim = cq - key0;  // valid columns of this tile for the query
-                    switch (w.rpad) {
-                        case 1: imp_reduce_store<1>(sv, lane, irow, lim); break;
-                        case 2: imp_reduce_store<2>(sv, lane, irow, lim); break;
-                        case 4: imp_reduce_store<4>(sv, lane, irow, lim); break;
-                        case 8: imp_reduce_store<8>(sv, lane, irow, lim); break;
-                        default: imp_reduce_store<16>(sv, lane, irow, lim); break;
-                    }
+                    imp_reduce_store<RPAD>(sv, lane, irow, lim);
                 }
             }
             if (!ok) break;
@@ -1038,7 +1035,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
     }
 }
 
-template <int MODE>
+template <int MODE, int RPAD = 8>
 __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_constant__ TcParams P) {
     extern __shared__ uint8_t smem_raw[];
     const LayerParams &L = P.L;
@@ -1106,7 +1103,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
         if (lane == 0) run_mma<MODE>(P, w, sm, tmem);
         __syncwarp();
     } else {
-        run_softmax<MODE>(P, w, sm, tmem);
+        run_softmax<MODE, RPAD>(P, w, sm, tmem);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1339,24 +1336,32 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
             }
             nleave = npair;
             __syncwarp();
-            // two-query tiles, in tile order; one lane assigns (a few dozen
+            // two-query tiles, one after the other in tile order (a few dozen
             // per item), so a tile takes both slots or none and no slot is
-            // left unused below a query's count
-            if (lane == 0) {
-                for (int x = 0; x < tot; ++x) {
-                    const uint32_t m = qm[x];
-                    if (__popc(m) != 2) continue;
-                    const int qa = __ffs(m) - 1, qb = 31 - __clz(m);
-                    if (qcnt[qa] >= (uint32_t)kSglSlots || qcnt[qb] >= (uint32_t)kSglSlots) continue;
-                    sslot[x] = 32 + (int)qcnt[qa] + 32 * (int)qcnt[qb];
-                    ++qcnt[qa];
-                    ++qcnt[qb];
-                    npair += 2;
-                    ++nleave;
+            // left unused below a query's count; lane q holds query q's count
+            uint32_t myc = qcnt[lane];
+            for (int xb = 0; xb < tot; xb += 32) {
+                const int x = xb + lane;
+                const uint32_t m = x < tot ? qm[x] : 0u;
+                unsigned two = __ballot_sync(0xffffffffu, x < tot && __popc(m) == 2);
+                int mine = -1;
+                while (two) {  // the same tiles on every lane
+                    const int b = __ffs(two) - 1;
+                    two &= two - 1;
+                    const uint32_t mb = __shfl_sync(0xffffffffu, m, b);
+                    const int qa = __ffs(mb) - 1, qb = 31 - __clz(mb);
+                    const uint32_t ca = __shfl_sync(0xffffffffu, myc, qa);
+                    const uint32_t cb = __shfl_sync(0xffffffffu, myc, qb);
+                    if (ca < (uint32_t)kSglSlots && cb < (uint32_t)kSglSlots) {
+                        if (lane == qa || lane == qb) ++myc;
+                        if (lane == b) mine = 32 + (int)ca + 32 * (int)cb;
+                        npair += 2;
+                        ++nleave;
+                    }
                 }
+                if (mine >= 0) sslot[x] = mine;
             }
-            npair = __shfl_sync(0xffffffffu, npair, 0);
-            nleave = __shfl_sync(0xffffffffu, nleave, 0);
+            qcnt[lane] = myc;
             __syncwarp();
             if (nleave >= tot) {  // every tile would leave: the item keeps them all
                 for (int x = lane; x < tot; x += 32) sslot[x] = -1;
@@ -1918,7 +1923,8 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
         st->swa_part = (__half *)(q += z.ulse);
     }
     cudaError_t e = cudaSuccess;
-    for (auto fn : {tc_attn_kernel<MODE_CMP>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
+    for (auto fn : {tc_attn_kernel<MODE_CMP, 4>, tc_attn_kernel<MODE_CMP, 8>,
+                    tc_attn_kernel<MODE_CMP, 16>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
                     tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>})
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -1971,7 +1977,14 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
             if (!make_map_q(&P.tm_q, L.q, c.h_q, L.n, rq, kRows / rq)) return cudaErrorInvalidValue;
         }
         switch (mode) {
-            case MODE_CMP: tc_attn_kernel<MODE_CMP><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
+            case MODE_CMP:  // head slots per query: 4, 8 or 16 (4 to 16 heads per KV head)
+                if (pow2_at_least(L.r) == 4)
+                    tc_attn_kernel<MODE_CMP, 4><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                else if (pow2_at_least(L.r) == 8)
+                    tc_attn_kernel<MODE_CMP, 8><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                else
+                    tc_attn_kernel<MODE_CMP, 16><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                break;
             case MODE_SLC: tc_attn_kernel<MODE_SLC><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             case MODE_SLC_UNALIGNED:
                 tc_attn_kernel<MODE_SLC_UNALIGNED><<<grid, kThreads, SMEM_BYTES, s>>>(P);
@@ -1992,6 +2005,16 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     if ((e = attn(MODE_CMP)) != cudaSuccess) return e;
     end(VNSA_STAGE_CMP);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (sgl) {
+        // the window pass writes only its own gated part here (the selection
+        // merge writes the rows), so it needs neither the top-k nor the
+        // selection
+        begin(VNSA_STAGE_SWA);
+        P.swa_part = st->swa_part;
+        if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
+        P.swa_part = nullptr;
+        end(VNSA_STAGE_SWA);
+    }
     begin(VNSA_STAGE_TOPK);
     if (L.stride != L.block) {
         // overlapping compression blocks: their importance onto the selection blocks
@@ -2040,8 +2063,9 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_SLC);
     if (sgl) {
-        // single-query tiles tile-major, then the union tiles, whose epilogue
-        // merges each query's pairs into its selection output
+        // the (query, tile) pairs tile-major, the union tiles, then the merge
+        // of both into the selection output, which with the compression
+        // partial and the window part gives the vision output rows
         SglParams sp;
         memset(&sp, 0, sizeof(sp));
         sp.tm_k = P.tm_k;
@@ -2066,17 +2090,6 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         P.sgl_on = 1;
         if ((e = attn(MODE_SLC)) != cudaSuccess) return e;
         P.sgl_on = 0;
-    } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
-        return e;
-    }
-    end(VNSA_STAGE_SLC);
-    begin(VNSA_STAGE_SWA);
-    P.swa_part = sgl ? st->swa_part : nullptr;
-    if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
-    P.swa_part = nullptr;
-    if (sgl) {
-        // the selection output from its parts, and with the compression and
-        // window parts the vision output rows
         SlcMergeArgs ma;
         ma.n = st->sgl_n;
         ma.sgl_o = st->sgl_o;
@@ -2087,8 +2100,16 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
         ma.swa_part = st->swa_part;
         slc_merge_kernel<<<st->num_sms * 16, 256, 0, s>>>(L, ma);
         ++*launches;
+    } else if ((e = attn(c.block % kKeys == 0 ? MODE_SLC : MODE_SLC_UNALIGNED)) != cudaSuccess) {
+        return e;
     }
-    end(VNSA_STAGE_SWA);
+    end(VNSA_STAGE_SLC);
+    if (!sgl) {
+        // the window epilogue adds its part to the partial and writes the rows
+        begin(VNSA_STAGE_SWA);
+        if ((e = attn(MODE_SWA)) != cudaSuccess) return e;
+        end(VNSA_STAGE_SWA);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     begin(VNSA_STAGE_TEXT);
     if ((e = attn(MODE_TEXT)) != cudaSuccess) return e;

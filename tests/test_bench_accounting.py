@@ -25,16 +25,20 @@ def _pairs_by_enumeration(wl, x):
     vis = np.nonzero(isv)[0]
     txt = np.nonzero(isv == 0)[0]
     B = wl.block
+    st = wl.stride or B
+    cmp = slc = swa = imp = 0
     nb = len(vis) // B
-    cmp = slc = swa = 0
+    # compression blocks: start c s, tokens [c s, c s + B) all vision ranks
+    starts = [c for c in range(0, len(vis)) if c % st == 0 and c + B <= len(vis)]
     for i, t in enumerate(vis):
-        cmp += min((i + 1) // B, nb)
+        cmp += sum(1 for c0 in starts if c0 + B - 1 <= i)
+        imp += min((i + 1) // B, nb)  # selection blocks with an importance
         swa += min(wl.window, i + 1)
         row = o["idx"][t, 0]  # group 0; every group selects as many keys
         for j in row[row >= 0]:
             slc += sum(1 for u in range(j * B, j * B + B) if u <= i)
     text = int((txt + 1).sum())
-    return {"cmp": cmp, "slc": slc, "swa": swa, "text": text}
+    return {"cmp": cmp, "slc": slc, "swa": swa, "text": text, "imp": imp}
 
 
 @pytest.mark.parametrize("wl,mask", [
@@ -42,6 +46,8 @@ def _pairs_by_enumeration(wl, x):
     (Workload("acct64", 700, 60, h_q=8, h_kv=2, d=64, top_k=5, window=100, seed=3), "mix"),
     (Workload("acct36", 520, 40, h_q=8, h_kv=2, d=64, top_k=6, window=90, block=36,
               frame=36, seed=4), None),
+    (Workload("acct_s16", 600, 30, h_q=8, h_kv=2, d=64, top_k=5, window=80, stride=16,
+              seed=5), "mix"),
 ])
 def test_algorithmic_pairs_match_enumeration(wl, mask):
     isv = interleaved_mask(wl.n_vision, wl.n_text, seed=2) if mask else None
@@ -51,10 +57,10 @@ def test_algorithmic_pairs_match_enumeration(wl, mask):
     f = 4.0 * wl.d * wl.h_q
     for name in ("cmp", "slc", "swa", "text"):
         assert got[name] == f * want[name], name
-    # top-k reads one fp32 importance per visible (group, query, block) and
-    # writes top_k int32 per (group, query)
+    # top-k reads one fp32 importance per complete (group, query, selection
+    # block) and writes top_k int32 per (group, query)
     nv = int(x["is_vision"].sum())
-    assert got["topk_bytes"] == 4.0 * wl.h_kv * want["cmp"] + 4.0 * wl.h_kv * nv * wl.top_k
+    assert got["topk_bytes"] == 4.0 * wl.h_kv * want["imp"] + 4.0 * wl.h_kv * nv * wl.top_k
 
 
 def test_selection_executed_work_splits_one_and_two_query_tiles():
