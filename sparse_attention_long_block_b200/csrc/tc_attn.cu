@@ -120,6 +120,7 @@ struct TcParams {
     // in units of V / v_scale like the selection parts) instead of reading the
     // partial (null: the window epilogue writes the rows).
     __half *swa_part;
+    int exact_kind;            // K_EXACT (a run-time value, for the exact pass's segment)
 };
 
 __host__ __device__ __forceinline__ int pow2_at_least(int r) {
@@ -184,7 +185,7 @@ struct Item {
     int key_lo;     // SWA window start (vision rank) / TEXT split start (position)
 };
 
-template <int MODE>
+template <int MODE, int PASS = 0>
 __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int item) {
     const LayerParams &L = P.L;
     Item it;
@@ -207,12 +208,14 @@ __device__ __forceinline__ Item make_item(const TcParams &P, const Work &w, int 
     it.seg_tiles[1] = 0;
     it.seg_kind[1] = K_EXACT;
     if (MODE == MODE_CMP) {
+        // PASS 0: both segments; 1: the statistics pass alone; 2: the exact
+        // pass alone (its log-sum-exp from pass 1)
         const int c_last = cmp_visible(ql, L.block, L.stride, w.nb);
         const int t = (c_last + kKeys - 1) / kKeys;
-        it.nseg = 2;
-        it.seg_kind[0] = K_STATS;
+        it.nseg = PASS == 0 ? 2 : 1;
+        it.seg_kind[0] = PASS == 2 ? P.exact_kind : K_STATS;
         it.seg_tiles[0] = t;
-        it.seg_tiles[1] = t;
+        it.seg_tiles[1] = PASS == 0 ? t : 0;
     } else if (is_slc(MODE)) {
         it.nseg = 1;
         it.seg_kind[0] = K_SLC;
@@ -278,7 +281,7 @@ __device__ __forceinline__ int tile_key0(const TcParams &P, const Item &it, int 
 // every item, in order, each lane with its own ring and waits: a K stage is
 // free once its Q K^T is done, a V stage only after its P V, so the K loads
 // run ahead.  Lane 0 also prefetches the tiles kPrefetch ahead into L2.
-template <int MODE>
+template <int MODE, int PASS = 0>
 __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, int lane) {
     if (lane > 1) return;
     const LayerParams &L = P.L;
@@ -302,7 +305,7 @@ __device__ void run_producer(const TcParams &P, const Work &w, const Smem &sm, i
     uint32_t nq = 0;  // Q tiles loaded (lane 0, TMA path)
     const int qrows = MODE == MODE_CMP ? w.rpad : L.r;  // MMA rows per query
     for (int item = blockIdx.x; item < w.items; item += gridDim.x) {
-        const Item it = make_item<MODE>(P, w, item);
+        const Item it = make_item<MODE, PASS>(P, w, item);
         const int xc = it.g * kD;
         if (is_k && w.q_tma && item_tiles(it) > 0) {
             // the item's Q rows (query, head) are one box of the [n][h_q][d]
@@ -370,7 +373,7 @@ drain:
 
 // ---------------------------------------------------------------------------
 // MMA issuer (one thread).
-template <int MODE>
+template <int MODE, int PASS = 0>
 __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
@@ -403,7 +406,7 @@ __device__ void run_mma(const TcParams &P, const Work &w, const Smem &sm, uint32
         return true;
     };
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
-        const Item it = make_item<MODE>(P, w, item);
+        const Item it = make_item<MODE, PASS>(P, w, item);
         if (item_tiles(it) == 0) continue;
         if (!ptx::mbar_wait(sm.bar(B_Q_FULL), nitems & 1, abort, L.status, L.wait_ns)) { ok = false; break; }
         ++nitems;
@@ -526,7 +529,7 @@ __device__ __forceinline__ uint64_t sel_coverage(const int32_t *sel, int &cur, i
 
 // RPAD: the compression mode's head slots per query (4, 8 or 16), fixed per
 // instantiation so that each compression kernel carries one importance reduce
-template <int MODE, int RPAD>
+template <int MODE, int RPAD, int PASS = 0>
 __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, uint32_t tmem) {
     const LayerParams &L = P.L;
     volatile int *abort = sm.abort_flag();
@@ -540,7 +543,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
     uint32_t gt = 0, npv = 0, gphase = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < w.items; item += gridDim.x) {
-        const Item it = make_item<MODE>(P, w, item);
+        const Item it = make_item<MODE, PASS>(P, w, item);
         RowCtx rc;
         rc.qi = rho / w.rpad;
         rc.hl = rho % w.rpad;
@@ -554,8 +557,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         }
         rc.c_vis = cmp_visible(rc.i, L.block, L.stride, w.nb);
         if (item_tiles(it) == 0) {
-            // nothing attended: empty branch outputs
-            if (rc.valid) {
+            // nothing attended: empty branch outputs (the exact pass writes
+            // those of the compression branch)
+            if (rc.valid && !(MODE == MODE_CMP && PASS == 1)) {
                 float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
                 const size_t prow = ((size_t)rc.t * L.h_q + rc.h) * kD;
                 if (MODE == MODE_CMP) {
@@ -621,7 +625,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             }
         }
         if (item + (int)gridDim.x < w.items) {
-            const Item nx = make_item<MODE>(P, w, item + gridDim.x);
+            const Item nx = make_item<MODE, PASS>(P, w, item + gridDim.x);
             const int qn = rho / w.rpad, hn = rho % w.rpad;
             if (qn < nx.nq && hn < L.r) {
                 const int tn = (MODE == MODE_TEXT) ? L.txt[nx.q0 + qn] : L.vis[nx.q0 + qn];
@@ -659,7 +663,10 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         const int32_t *my_sel = plan_s + kPlanSmem + min(rc.qi, w.qt - 1) * L.top_k;
         int sel_cur = 0;
 
-        float lse2 = -INFINITY;                 // CMP: from the stats segment
+        // CMP: from the statistics segment (pass 2: from pass 1, log2 units)
+        float lse2 = (MODE == MODE_CMP && PASS == 2 && rc.valid)
+                         ? L.lse[(size_t)rc.i * L.h_q + rc.h]
+                         : -INFINITY;
         float m_run = -INFINITY, l_run = 0.f;   // running max / sum (log2 units)
         for (int s = 0; ok && s < it.nseg; ++s) {
             const int kind = it.seg_kind[s];
@@ -876,6 +883,12 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                 lse2 = (m_run == -INFINITY || l_run <= 0.f) ? -INFINITY : m_run + log2f(l_run);
         }
         if (!ok) break;
+        if (MODE == MODE_CMP && PASS == 1) {
+            // the statistics pass hands the exact pass its log-sum-exp (log2
+            // units; the exact pass's epilogue stores it in natural units)
+            if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2;
+            continue;
+        }
         // ---- epilogue: wait for the item's last P V (#npv-1)
         {
             bool r = ptx::mbar_wait(sm.bar(B_PV_DONE + ((npv - 1) & 1)), ((npv - 1) >> 1) & 1,
@@ -1035,7 +1048,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
     }
 }
 
-template <int MODE, int RPAD = 8>
+template <int MODE, int RPAD = 8, int PASS = 0>
 __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_constant__ TcParams P) {
     extern __shared__ uint8_t smem_raw[];
     const LayerParams &L = P.L;
@@ -1098,12 +1111,12 @@ __global__ void __launch_bounds__(kThreads, 2) tc_attn_kernel(const __grid_const
     const uint32_t tmem = *sm.tmem_slot();
 
     if (warp == 0) {
-        run_producer<MODE>(P, w, sm, lane);
+        run_producer<MODE, PASS>(P, w, sm, lane);
     } else if (warp == 1) {
-        if (lane == 0) run_mma<MODE>(P, w, sm, tmem);
+        if (lane == 0) run_mma<MODE, PASS>(P, w, sm, tmem);
         __syncwarp();
     } else {
-        run_softmax<MODE, RPAD>(P, w, sm, tmem);
+        run_softmax<MODE, RPAD, PASS>(P, w, sm, tmem);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -1923,9 +1936,11 @@ cudaError_t tc_create(const vnsa_config &c, void *ws, TcState **out) {
         st->swa_part = (__half *)(q += z.ulse);
     }
     cudaError_t e = cudaSuccess;
-    for (auto fn : {tc_attn_kernel<MODE_CMP, 4>, tc_attn_kernel<MODE_CMP, 8>,
-                    tc_attn_kernel<MODE_CMP, 16>, tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>,
-                    tc_attn_kernel<MODE_TEXT>, tc_attn_kernel<MODE_SLC_UNALIGNED>})
+    for (auto fn : {tc_attn_kernel<MODE_CMP, 4, 1>, tc_attn_kernel<MODE_CMP, 4, 2>,
+                    tc_attn_kernel<MODE_CMP, 8, 1>, tc_attn_kernel<MODE_CMP, 8, 2>,
+                    tc_attn_kernel<MODE_CMP, 16, 1>, tc_attn_kernel<MODE_CMP, 16, 2>,
+                    tc_attn_kernel<MODE_SLC>, tc_attn_kernel<MODE_SWA>, tc_attn_kernel<MODE_TEXT>,
+                    tc_attn_kernel<MODE_SLC_UNALIGNED>})
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e == cudaSuccess) e = sgl_prepare();
@@ -1943,6 +1958,9 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
     const vnsa_config &c = st->cfg;
     TcParams P;
     memset(&P, 0, sizeof(P));
+    // a kernel argument rather than a constant: with the kind fixed at compile
+    // time the exact pass's register allocation spills
+    P.exact_kind = K_EXACT;
     P.L = L;
     P.plan = st->plan;
     P.plan_max = st->plan_max;
@@ -1977,13 +1995,21 @@ cudaError_t tc_forward(TcState *st, const LayerParams &L, cudaStream_t s, cudaEv
             if (!make_map_q(&P.tm_q, L.q, c.h_q, L.n, rq, kRows / rq)) return cudaErrorInvalidValue;
         }
         switch (mode) {
-            case MODE_CMP:  // head slots per query: 4, 8 or 16 (4 to 16 heads per KV head)
-                if (pow2_at_least(L.r) == 4)
-                    tc_attn_kernel<MODE_CMP, 4><<<grid, kThreads, SMEM_BYTES, s>>>(P);
-                else if (pow2_at_least(L.r) == 8)
-                    tc_attn_kernel<MODE_CMP, 8><<<grid, kThreads, SMEM_BYTES, s>>>(P);
-                else
-                    tc_attn_kernel<MODE_CMP, 16><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+            case MODE_CMP:
+                // head slots per query 4, 8 or 16 (4 to 16 heads per KV head);
+                // the statistics pass, then the exact pass, as two launches so
+                // that each kernel carries only its pass's code
+                if (pow2_at_least(L.r) == 4) {
+                    tc_attn_kernel<MODE_CMP, 4, 1><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                    tc_attn_kernel<MODE_CMP, 4, 2><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                } else if (pow2_at_least(L.r) == 8) {
+                    tc_attn_kernel<MODE_CMP, 8, 1><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                    tc_attn_kernel<MODE_CMP, 8, 2><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                } else {
+                    tc_attn_kernel<MODE_CMP, 16, 1><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                    tc_attn_kernel<MODE_CMP, 16, 2><<<grid, kThreads, SMEM_BYTES, s>>>(P);
+                }
+                ++*launches;
                 break;
             case MODE_SLC: tc_attn_kernel<MODE_SLC><<<grid, kThreads, SMEM_BYTES, s>>>(P); break;
             case MODE_SLC_UNALIGNED:

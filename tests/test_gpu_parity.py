@@ -1,9 +1,9 @@
 """GPU parity: the CUDA layer (through the C ABI) against the fp64 oracle.
 
 Sizes: the tiny fp32 workload and the 8K layer in full; the 36K, 64K and 128K
-workloads at their full size on stratified rows (first rows, every 97th row,
-both sides of block boundaries, text rows), in the launch configuration the
-benchmark times.  Edge cases: ragged vision counts, interleaved masks, no
+workloads and the largest call the library takes (262,144 tokens) at their full
+size on stratified rows (first rows, every 97th row, both sides of block
+boundaries, text rows), in the launch configuration the benchmark times.  Edge cases: ragged vision counts, interleaved masks, no
 complete block, text only, vision only, single token, full budgets, forced
 blocks off, 4/1 heads with d 64 in bf16 and 28/4 heads in fp32.
 """
@@ -50,6 +50,17 @@ def test_long_128k_sampled_rows():
     wl = WORKLOADS["long_128k"]
     x = generate(wl)
     rows = stratified_rows(x["is_vision"], every=1021, first=96, max_text=32)
+    compare_layer(wl, x, rows=rows, want_branches=False)
+
+
+def test_max_tokens_sampled_rows():
+    # the largest call the library takes (262,144 tokens: 261,120 vision + 1,024
+    # text, 4,080 blocks), the long-context recipe; sampled rows on both sides
+    # of block boundaries, the last rows and the text rows
+    wl = Workload("max_256k", 261120, 1024, top_k=32, window=512, ar1=True, seed=9)
+    assert wl.n == 262144
+    x = generate(wl)
+    rows = stratified_rows(x["is_vision"], every=4099, first=64, max_text=16)
     compare_layer(wl, x, rows=rows, want_branches=False)
 
 
