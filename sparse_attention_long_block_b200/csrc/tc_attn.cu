@@ -618,7 +618,9 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
         // next item, so that neither waits on DRAM when it is needed
         if (rc.valid) {
             ptx::prefetch_l2(L.gate + ((size_t)rc.t * L.h_q + rc.h) * 3);
-            if (is_slc(MODE) || MODE == MODE_SWA) {
+            // the partial, where the epilogue reads it (not with the split
+            // selection, whose merge kernel adds the parts)
+            if ((is_slc(MODE) && !P.sgl_on) || (MODE == MODE_SWA && !P.swa_part)) {
                 const float *part = L.o_cmp_ws + ((size_t)rc.i * L.h_q + rc.h) * kD;
 #pragma unroll
                 for (int z = 0; z < kD; z += 32) ptx::prefetch_l2(part + z);
