@@ -3,13 +3,14 @@
 // Method: "VideoNSA: Native Sparse Attention Scales Video Understanding" (paper
 // notes), section "Method": each vision query attends to the tokens of the
 // blocks it selected.  The union pass of tc_attn.cu attends, for 128 MMA rows
-// (consecutive queries x the heads of one GQA group), the 64-key tiles that two
-// or more of those queries selected.  A tile that only one of them selected
-// would cost a whole 128-row tile of tensor work for 7 useful rows, so the
-// union kernel hands such (query, tile) pairs to this pass instead.  Here the
-// pairs are grouped by tile (bucket = group x tile): a chunk is up to 128 / r
-// pairs of one tile, and a thread block takes a contiguous range of chunks,
-// so a tile's K/V is loaded once and serves every chunk of it in the range.
+// (consecutive queries x the heads of one GQA group), the 64-key tiles that
+// three or more of those queries selected.  A tile that only one or two of
+// them selected would cost a whole 128-row tile of tensor work for 7 or 14
+// useful rows, so the union kernel hands such (query, tile) pairs to this
+// pass instead.  Here the pairs are grouped by tile (bucket = group x tile):
+// a chunk is up to 128 / r pairs of one tile, and a thread block takes a
+// contiguous range of chunks, so a tile's K/V is loaded once and serves every
+// chunk of it in the range.
 //
 // Per chunk: S = Q K^T (M 128, N 64, K 128, bf16), the softmax of each row over
 // the tile's keys at or before its query, P (fp16) back into TMEM, O = P V

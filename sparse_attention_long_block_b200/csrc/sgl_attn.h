@@ -1,7 +1,7 @@
 // sgl_attn.h -- the tile-major pass of the selection branch: (query, tile)
-// pairs in which a query is the only one of its 128-row item that reaches a
-// 64-key tile, grouped by tile, attended with the tile's K/V held in shared
-// memory while the pairs' query rows stream through.
+// pairs of the 64-key tiles that only one or two queries of a 128-row item
+// reach, grouped by tile, attended with the tile's K/V held in shared memory
+// while the pairs' query rows stream through.
 #pragma once
 
 #include <cuda.h>

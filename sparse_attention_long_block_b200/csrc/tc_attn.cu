@@ -108,10 +108,10 @@ struct TcParams {
     float *part;               // TEXT partials: [item][128][kPartStride]
     int part_items;
     int mode;
-    // Selection tiles that a single query of an item reaches (block 64 only):
-    // the union kernel takes them out of the item's plan and records each
-    // (query, tile) pair; the tile-major pass (sgl_attn.cu) attends them, and
-    // the selection epilogue merges each query's pairs into its output.
+    // Selection tiles that one or two queries of an item reach (block 64
+    // only): the union kernel takes them out of the item's plan and records
+    // each (query, tile) pair; the tile-major pass (sgl_attn.cu) attends them,
+    // and the merge kernel combines each query's pairs with its union part.
     int sgl_on;                // 1: the selection branch runs split this way
     __half *slc_u;             // [n_max][h_q][d] the union tiles' normalised output
     float *slc_lse;            // [n_max][h_q] their log-sum-exp (log2 units)
@@ -573,8 +573,8 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
                     pr[kD] = -INFINITY;
                     pr[kD + 1] = 0.f;
                 } else if (MODE == MODE_SLC && P.sgl_on) {
-                    // no union tile (nor single-query pair: the union keeps at
-                    // least one tile of an item that has any)
+                    // no union tile (nor pair: the union keeps at least one
+                    // tile of an item that has any)
                     for (int e = 0; e < kD; e += 8)
                         *reinterpret_cast<uint4 *>(P.slc_u + ((size_t)rc.i * L.h_q + rc.h) * kD +
                                                    e) = make_uint4(0u, 0u, 0u, 0u);
@@ -928,7 +928,7 @@ __device__ void run_softmax(const TcParams &P, const Work &w, const Smem &sm, ui
             if (rc.valid) L.lse[(size_t)rc.i * L.h_q + rc.h] = lse2 * kLn2;
         } else if (MODE == MODE_SLC && P.sgl_on) {
             // The selection softmax of this row is split into the union's tiles
-            // and the query's single-query pairs (the tile-major pass); the
+            // and the query's (query, tile) pairs (the tile-major pass); the
             // merge kernel combines them.  Here: the union part, normalised, in
             // the units of the scaled V copy (fp16: a convex combination of
             // values below 2^15), and its log-sum-exp (log2 units).
@@ -1229,8 +1229,8 @@ __device__ __forceinline__ void sel_tiles(int j, int B, int i, int &t0, int &t1)
     t1 = (int)(min(a + B - 1, (long long)i) / kKeys);
 }
 
-// Where single-query tiles go (SglArgs.on): pair records, the per-bucket
-// counts, and each query's list of its pairs.
+// Where the tiles that leave the union go (SglArgs.on): pair records, the
+// per-bucket counts, and each query's pair count.
 struct SglArgs {
     int on, nbt, cap;
     int32_t *meta;  // [0] pairs, [1] items, [2, 2 + h_kv*nbt) pairs per bucket
@@ -1246,7 +1246,7 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
     uint32_t *bm = sh + (size_t)warp * (2 * words + 2 * plan_max + 32);
     uint32_t *pre = bm + words;
     uint32_t *qm = pre + words;
-    uint32_t *qcnt = qm + plan_max;  // per query of the item: its single-query tiles
+    uint32_t *qcnt = qm + plan_max;  // per query of the item: its pair slots taken
     int *sslot = (int *)(qcnt + 32); // per tile: its pair slot, -1 if it stays
     const Counts cn = *p.counts;
     const int qt = kRows / p.r;
@@ -1446,7 +1446,7 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
     }
 }
 
-// Offsets of the single-query pairs grouped by bucket (group, tile) and of the
+// Offsets of the (query, tile) pairs grouped by bucket (group, tile) and of the
 // tile-major pass's chunks (qt pairs of one bucket): exclusive prefix sums
 // over the bucket counts, one block.
 __global__ void __launch_bounds__(1024) sgl_scan_kernel(int32_t *meta, int nbk, int qt) {
@@ -1532,7 +1532,7 @@ __global__ void sgl_scatter_kernel(const int32_t *meta, const int4 *rec, int4 *s
 }
 
 // The selection output of each (vision query, head): the union tiles' part
-// (slc_u, slc_lse) and the query's single-query pairs (slot ids qg kSglSlots +
+// (slc_u, slc_lse) and the query's (query, tile) pairs (slot ids qg kSglSlots +
 // z, z < n[qg]: sgl_o, sgl_lse), each the exact softmax over its keys,
 // combined with the weights 2^(lse_part - M) / sum over the parts; then the
 // vision output row out = partial (compression) + sigmoid(g_slc) * o_slc +
@@ -1819,7 +1819,7 @@ struct TcState {
     float *v_scale;     // [2] their powers of two
     int32_t *plan;
     float *part;
-    // single-query selection tiles (block 64): see TcParams and sgl_attn.h
+    // selection tiles of one or two queries (block 64): see TcParams and sgl_attn.h
     int sgl_on, sgl_nbt, sgl_cap;
     int32_t *sgl_meta, *sgl_n;
     int4 *sgl_rec, *sgl_sorted, *sgl_items;
