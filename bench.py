@@ -101,11 +101,12 @@ def executed_work(wl, is_vision, idx):
     tile (8 head slots), a statistics pass (QK^T) and an exact pass (QK^T + P V)
     over the visible blocks; selection: 18 queries (7 heads) against the union
     of the 64-key tiles their selected blocks reach (from idx [h_kv][N_v][k]);
-    with block 64 the tiles that only one or two of the 18 queries reach run
-    tile-major instead, up to 18 such (query, tile) pairs per 128-row tile;
-    window and text: 18 queries against their key ranges.  (Up to 16 pairs
-    per query leave the union: its single-query tiles, then the two-query
-    tiles while both queries have room, each in tile order.)"""
+    with block 64 the tiles that only one, two or three of the 18 queries
+    reach run tile-major instead, up to 18 such (query, tile) pairs per
+    128-row tile; window and text: 18 queries against their key ranges.  (Up
+    to 16 pairs per query leave the union: its single-query tiles, then the
+    two-query and the three-query tiles while each of their queries has room,
+    each in tile order.)"""
     prod = 2.0 * 128 * 64 * wl.d
     vis = np.nonzero(is_vision)[0]
     txt = np.nonzero(is_vision == 0)[0]
@@ -132,8 +133,9 @@ def executed_work(wl, is_vision, idx):
             sel = idx[g, q0:ql + 1]
             if wl.block == 64:
                 # up to 16 pairs per query leave the union: its single-query
-                # tiles in tile order, then the two-query tiles in tile order
-                # while both queries have a slot left
+                # tiles in tile order, then the two-query and then the
+                # three-query tiles in tile order while each of the tile's
+                # queries has a slot left
                 who = {}
                 for qi, row in enumerate(sel):
                     for j in row:
@@ -146,13 +148,14 @@ def executed_work(wl, is_vision, idx):
                         used[who[j][0]] += 1
                         pairs.append(j)
                         leave += 1
-                for j in sorted(who):
-                    qs = who[j]
-                    if len(qs) == 2 and used[qs[0]] < 16 and used[qs[1]] < 16:
-                        used[qs[0]] += 1
-                        used[qs[1]] += 1
-                        pairs += [j, j]
-                        leave += 1
+                for share in (2, 3):
+                    for j in sorted(who):
+                        qs = who[j]
+                        if len(qs) == share and all(used[q] < 16 for q in qs):
+                            for q in qs:
+                                used[q] += 1
+                            pairs += [j] * share
+                            leave += 1
                 keep = len(who) - leave
                 if pairs and keep:
                     slc += 2 * keep

@@ -62,6 +62,7 @@ constexpr int kTextSplitKeys = 8192;
 constexpr size_t kTextPartBytes = 256ull << 20;
 constexpr int kPartStride = kD + 2;  // floats per partial row: O, m, l
 constexpr int kSglSlots = 16;        // tile-major pairs per (group, query) at most
+constexpr int kSglShare = 3;         // tiles of at most this many queries leave the union
 
 constexpr uint32_t SM_Q = 0;                                  // 2 x [128][64] bf16
 constexpr uint32_t SM_KV = 32768;                             // K ring, then V ring
@@ -1318,19 +1319,20 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
         __syncwarp();
         int tot = min(total, plan_max);
         if (sg.on) {
-            // Tiles that one or two queries of the item reach leave the plan for
-            // the tile-major pass (sgl_attn.cu) as (query, tile) pairs: a 128-row
-            // union tile costs the same whatever number of its rows attend, and
-            // a pair costs a gathered Q row block, an output row block and its
-            // merge, which is less for one or two queries and more for three.
-            // Up to kSglSlots pairs per query: first its single-query tiles in
-            // tile order, then the two-query tiles in tile order while both
-            // queries have a slot left (the rest stay), and only while at least
-            // one tile stays.  The pair (vision query i of group g, slot s) has
-            // the id (g n_max + i) kSglSlots + s, so the merge finds a query's
-            // pairs without a lookup.  sslot[x]: -1 (stays), the slot of a
-            // single-query tile, or 32 + slot of the lower query + 32 x slot
-            // of the higher one.
+            // Tiles that at most kSglShare queries of the item reach leave the
+            // plan for the tile-major pass (sgl_attn.cu) as (query, tile) pairs:
+            // a 128-row union tile costs the same whatever number of its rows
+            // attend, and a pair costs a gathered Q row block, an output row
+            // block and its merge, which is about a union tile's cost for three
+            // queries.  Up to kSglSlots pairs per query: first its single-query
+            // tiles in tile order, then the two-query and then the three-query
+            // tiles in tile order while each of the tile's queries has a slot
+            // left (the rest stay), and only while at least one tile stays.
+            // The pair (vision query i of group g, slot s) has the id
+            // (g n_max + i) kSglSlots + s, so the merge finds a query's pairs
+            // without a lookup.  sslot[x]: -1 (stays), the slot of a
+            // single-query tile, or 32 + the slots of the tile's queries in
+            // 5-bit fields, lowest query first.
             qcnt[lane] = 0u;
             __syncwarp();
             int npair = 0;   // pairs
@@ -1351,30 +1353,37 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
             }
             nleave = npair;
             __syncwarp();
-            // two-query tiles, one after the other in tile order (a few dozen
-            // per item), so a tile takes both slots or none and no slot is
-            // left unused below a query's count; lane q holds query q's count
+            // then the tiles of two, then of three queries, each kind one tile
+            // after the other in tile order (a few dozen per item), so a tile
+            // takes all its slots or none and no slot is left unused below a
+            // query's count; lane q holds query q's count
             uint32_t myc = qcnt[lane];
-            for (int xb = 0; xb < tot; xb += 32) {
-                const int x = xb + lane;
-                const uint32_t m = x < tot ? qm[x] : 0u;
-                unsigned two = __ballot_sync(0xffffffffu, x < tot && __popc(m) == 2);
-                int mine = -1;
-                while (two) {  // the same tiles on every lane
-                    const int b = __ffs(two) - 1;
-                    two &= two - 1;
-                    const uint32_t mb = __shfl_sync(0xffffffffu, m, b);
-                    const int qa = __ffs(mb) - 1, qb = 31 - __clz(mb);
-                    const uint32_t ca = __shfl_sync(0xffffffffu, myc, qa);
-                    const uint32_t cb = __shfl_sync(0xffffffffu, myc, qb);
-                    if (ca < (uint32_t)kSglSlots && cb < (uint32_t)kSglSlots) {
-                        if (lane == qa || lane == qb) ++myc;
-                        if (lane == b) mine = 32 + (int)ca + 32 * (int)cb;
-                        npair += 2;
-                        ++nleave;
+            for (int want = 2; want <= kSglShare; ++want) {
+                for (int xb = 0; xb < tot; xb += 32) {
+                    const int x = xb + lane;
+                    const uint32_t m = x < tot ? qm[x] : 0u;
+                    unsigned sel = __ballot_sync(0xffffffffu, x < tot && __popc(m) == want);
+                    int mine = -1;
+                    while (sel) {  // the same tiles on every lane
+                        const int b = __ffs(sel) - 1;
+                        sel &= sel - 1;
+                        const uint32_t mb = __shfl_sync(0xffffffffu, m, b);
+                        bool room = true;
+                        int v = 0, sh = 0;
+                        for (uint32_t mm = mb; mm; mm &= mm - 1, sh += 5) {
+                            const uint32_t cq = __shfl_sync(0xffffffffu, myc, __ffs(mm) - 1);
+                            room = room && cq < (uint32_t)kSglSlots;
+                            v |= (int)cq << sh;
+                        }
+                        if (room) {
+                            if ((mb >> lane) & 1u) ++myc;
+                            if (lane == b) mine = 32 + v;
+                            npair += want;
+                            ++nleave;
+                        }
                     }
+                    if (mine >= 0) sslot[x] = mine;
                 }
-                if (mine >= 0) sslot[x] = mine;
             }
             qcnt[lane] = myc;
             __syncwarp();
@@ -1401,12 +1410,18 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
                     const int tl = x < tot ? out[1 + x] : 0;
                     const int sl = x < tot ? sslot[x] : -1;
                     const bool pair = sl >= 0;
-                    const bool dbl = sl >= 32;
                     const bool keep = x < tot && !pair;
+                    // pairs of this tile (one per query) and their offset in the batch
+                    const int cnt = pair ? (sl >= 32 ? __popc(m) : 1) : 0;
+                    int incl = cnt;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    const int all = __shfl_sync(0xffffffffu, incl, 31);
                     // every lane holds its entry before any entry is moved down
                     const unsigned bk = __ballot_sync(0xffffffffu, keep);
-                    const unsigned bp = __ballot_sync(0xffffffffu, pair);
-                    const unsigned bd = __ballot_sync(0xffffffffu, dbl);
                     if (keep) {
                         const int pos = kept + __popc(bk & lt);
                         out[1 + pos] = tl;
@@ -1414,20 +1429,19 @@ __global__ void union_kernel(LayerParams p, int32_t *plan, int plan_max, int wor
                     }
                     if (pair) {
                         const int bucket = g * sg.nbt + tl;
-                        const int at = base + si + __popc(bp & lt) + __popc(bd & lt);
-                        const int lp = atomicAdd(&sg.meta[2 + bucket], dbl ? 2 : 1);
-                        const int i = q0 + __ffs(m) - 1;
-                        const int s0 = dbl ? (sl - 32) & 31 : sl;
-                        sg.rec[at] = make_int4(bucket, (g * p.n_max + i) * kSglSlots + s0, lp, p.vis[i]);
-                        if (dbl) {
-                            const int i2 = q0 + 31 - __clz(m);
-                            const int s1 = (sl - 32) >> 5;
-                            sg.rec[at + 1] = make_int4(bucket, (g * p.n_max + i2) * kSglSlots + s1,
-                                                       lp + 1, p.vis[i2]);
+                        const int at = base + si + incl - cnt;
+                        const int lp = atomicAdd(&sg.meta[2 + bucket], cnt);
+                        const int v = sl >= 32 ? sl - 32 : sl;  // 5-bit slot fields
+                        uint32_t mm = m;
+                        for (int e = 0; e < cnt; ++e, mm &= mm - 1) {
+                            const int i = q0 + __ffs(mm) - 1;
+                            const int se = (v >> (5 * e)) & 31;
+                            sg.rec[at + e] = make_int4(bucket, (g * p.n_max + i) * kSglSlots + se,
+                                                       lp + e, p.vis[i]);
                         }
                     }
                     kept += __popc(bk);
-                    si += __popc(bp) + __popc(bd);
+                    si += all;
                     __syncwarp();
                 }
                 tot = kept;

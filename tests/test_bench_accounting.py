@@ -5,8 +5,9 @@ The roofline numerator is the algorithmic work: 4 d H_q flops per attended
 attend, key by key, and check the benchmark's closed-form counts against them
 (compression: visible blocks; selection: the keys of the selected blocks at or
 before the query; window: min(w, i + 1); text: t + 1).  They also check the
-executed-work count of the selection branch when tiles that one query of an
-item reaches run tile-major (up to 18 such pairs of one tile per 128-row tile).
+executed-work count of the selection branch when tiles that one to three
+queries of an item reach run tile-major (up to 18 such pairs of one tile per
+128-row tile).
 """
 import numpy as np
 import pytest
@@ -63,7 +64,7 @@ def test_algorithmic_pairs_match_enumeration(wl, mask):
     assert got["topk_bytes"] == 4.0 * wl.h_kv * want["imp"] + 4.0 * wl.h_kv * nv * wl.top_k
 
 
-def test_selection_executed_work_splits_one_and_two_query_tiles():
+def test_selection_executed_work_splits_one_to_three_query_tiles():
     # one group, 7 heads (18 queries per 128-row tile), block 64, two items
     wl = Workload("acct_split", 36 * 64, 0, h_q=7, h_kv=1, d=128, top_k=3, window=64)
     isv = np.ones(wl.n, np.uint8)
@@ -75,15 +76,17 @@ def test_selection_executed_work_splits_one_and_two_query_tiles():
     idx[0, 0, 2] = 30                     # item 0: tile 30 reached by queries 0 and 1
     idx[0, 1, 2] = 30
     idx[0, 18:21, 2] = 31                 # item 1: tile 31 reached by three queries
+    idx[0, 21:25, 2] = 32                 # item 1: tile 32 reached by four queries
     ex = bench.executed_work(wl, isv, idx)
     prod = 2.0 * 128 * 64 * wl.d
-    # item 0 keeps block 0's tile, item 1 block 0's and tile 31; the 36
-    # single-query pairs fall into 18 (group, tile) buckets of 2 pairs and the
-    # two-query tile 30 adds a bucket of 2 pairs: one tile-major tile each; the
-    # other items (queries 36 ..) reach block 0 only
+    # item 0 keeps block 0's tile, item 1 block 0's and tile 32; the 36
+    # single-query pairs fall into 18 (group, tile) buckets of 2 pairs, the
+    # two-query tile 30 and the three-query tile 31 add a bucket of 2 and one of
+    # 3 pairs: one tile-major tile each; the other items (queries 36 ..) reach
+    # block 0 only
     n_items = -(-nv // 18)
     union_tiles = 1 + 2 + (n_items - 2) * 1
-    assert ex["slc"] == 2 * prod * (union_tiles + 19)
+    assert ex["slc"] == 2 * prod * (union_tiles + 20)
     # a query with more than 16 pairs: its 17th single-query tile stays, and so
     # does a two-query tile of a query without a free slot
     wl2 = Workload("acct_cap", 64 * 64, 0, h_q=7, h_kv=1, d=128, top_k=20, window=64)

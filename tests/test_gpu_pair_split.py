@@ -1,10 +1,10 @@
 """The selection branch's split between union tiles and tile-major (query,
 tile) pairs, driven by caller selections built to reach every case of the
 split: queries with more single-query tiles than pair slots (the rest stay in
-the union), tiles that two queries of an item share (they leave when both
-queries have a slot left, else they stay), tiles that three or more queries
-share (they stay), and a last item of one query, whose every tile could leave
-(it keeps them all).  The selection output and the layer output of those queries are
+the union), tiles that two or three queries of an item share (they leave when
+each of their queries has a slot left, else they stay), tiles that more
+queries share (block 0 and the queries' own blocks: they stay), and a last
+item of one query, whose every tile could leave (it keeps them all).  The selection output and the layer output of those queries are
 compared with the fp64 oracle given the same selection ("VideoNSA: Native
 Sparse Attention Scales Video Understanding", paper notes, section "Method":
 each query attends to the tokens of its selected blocks; the split only
